@@ -1,0 +1,494 @@
+#!/usr/bin/env python
+"""Benchmark of the routed mixture-of-experts FFN layer (libmoe.so) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
+
+Default workload (--config 1): MoE-layer decode, hidden 7168, inter 2048,
+256 routed experts + 1 shared, top-8, sigmoid gating, T=1 token, all experts
+resident in HBM.  One step = one moe_forward (router, permutation, gate/up +
+SwiGLU, down, combine).  The L2 is flushed (a 256 MiB write) before every step
+and only the forward is timed, with CUDA events on the forward's stream.
+--config 2 (T=64), 3 (T=4096 prefill) and 4 (8-layer expert streaming with a
+12e9-byte cache) run the other workloads.
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs an independent
+replica on its own GPU (the layer has no cross-GPU exchange in this build), and
+`value` is the tokens of all ranks over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from routed_expert_ffn_forward_b200 import synth  # noqa: E402
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ----------------------------------------------------------------------------- helpers
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={CLOCK_FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception as e:  # no nvidia-smi: report nothing rather than fail
+            log("clock sampler unavailable:", e)
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.15)
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+            self.f.close()
+
+    def summary(self) -> dict | None:
+        if not self.proc:
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            p = [q.strip() for q in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx.append(float(p[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_traffic(kernel: str) -> float | None:
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
+    kernel's source has not changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["sha256"]:
+        return None
+    return float(d["bytes_per_launch"])
+
+
+def algorithmic_bytes(cfg, ids: np.ndarray, which: str) -> float:
+    """Bytes a kernel must move at least once per launch for this routing.
+    gate_up: gate+up weights of every active expert, x rows, h writes (fp32).
+    forward: every active expert's weights, the router weight, x and out."""
+    T = ids.shape[0]
+    active = len(np.unique(ids)) + cfg.n_shared
+    nb_h, nb_i = cfg.hidden // 256, (cfg.inter + 255) // 256
+    gate = cfg.inter * nb_h * 144
+    down = cfg.hidden * nb_i * 144
+    pairs = T * (cfg.top_k + cfg.n_shared)
+    if which == "gate_up":
+        return active * 2 * gate + T * cfg.hidden * 2 + pairs * cfg.inter * 4
+    if which == "down":
+        return active * down + pairs * cfg.inter * 4 + pairs * cfg.hidden * 4
+    return active * (2 * gate + down) + cfg.n_experts * cfg.hidden * 4 + 2 * T * cfg.hidden * 2
+
+
+def flops(cfg, T: int) -> float:
+    return 2.0 * T * (cfg.top_k + cfg.n_shared) * 3 * cfg.hidden * cfg.inter
+
+
+# ----------------------------------------------------------------------------- CPU oracle baseline
+def oracle_sample_rate(cfg, n_tokens: int, budget_s: float) -> dict:
+    """Time the oracle (as it stands) on a bounded sample: whole tokens of the
+    workload, one after another, until the budget is used (at least one)."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import moe_ref as ref
+    layer = dict(router_w=synth.router_weight(cfg), router_b=synth.router_bias(cfg),
+                 experts=lambda e: synth.expert_tensors(cfg, 0, e))
+    x = synth.activations(cfg, tokens=max(n_tokens, 1))
+    done, t0 = 0, time.perf_counter()
+    with threadpool_limits(limits=1):
+        while done < n_tokens and (done == 0 or time.perf_counter() - t0 < budget_s):
+            ref.moe_forward(x[done:done + 1], layer, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter)
+            done += 1
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} token(s) of the workload's layer through the fp64 numpy oracle "
+                      f"(full routing + {cfg.top_k}+{cfg.n_shared} experts each), BLAS limited to 1 thread",
+            "seconds": dt}
+
+
+_EXPERT_CACHE: dict = {}
+
+
+def oracle_unit(cfg, step: int, rows_frac: float, ref, x64, l64):
+    """One reference step: the oracle's expert FFN for token 0 restricted to one
+    256-feature block of one of its experts (gate/up rows of that block, the
+    down column block; rows_frac < 1 also subsamples rows).  Returns the
+    fraction of one token's expert work it covers."""
+    k, S = cfg.top_k, cfg.n_shared
+    ids = ref.topk_ids(l64[:1], k)[0].tolist() + [cfg.n_experts + s for s in range(S)]
+    e = ids[step % len(ids)]
+    nb_i = (cfg.inter + 255) // 256
+    b = (step // len(ids)) % nb_i
+    if e not in _EXPERT_CACHE:
+        _EXPERT_CACHE[e] = synth.expert_tensors(cfg, 0, e)
+    g, u, d = _EXPERT_CACHE[e]
+    r = max(1, int(round(min(256, cfg.inter - 256 * b) * rows_frac)))
+    rows = slice(256 * b, 256 * b + r)
+    wg, wu = ref.q4k_dequant(g[rows]), ref.q4k_dequant(u[rows])
+    h = ref.silu(wg @ x64[0]) * (wu @ x64[0])
+    ro = max(1, int(round(cfg.hidden * rows_frac)))
+    wd = ref.q4k_dequant(d[:ro, 144 * b:144 * (b + 1)])[:, :r]
+    _ = wd @ h
+    total_blocks = len(ids) * (2 * cfg.inter * (cfg.hidden // 256) + cfg.hidden * nb_i)
+    return (2 * r * (cfg.hidden // 256) + ro) / total_blocks
+
+
+def run_reference(args, cfg) -> dict:
+    """--impl reference: the oracle on the host cores, same metric and config."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import moe_ref as ref
+    layer = dict(router_w=synth.router_weight(cfg), router_b=synth.router_bias(cfg))
+    x = synth.activations(cfg, tokens=1)
+    x64 = ref.bf16_to_f64(x)
+    budget = 150.0
+    rows_frac = min(1.0, budget / max(1, args.steps + args.warmup) / 0.09)
+    fracs, times = [], []
+    with threadpool_limits(limits=1):
+        for step in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            l64 = ref.router_logits(x64, layer["router_w"], layer["router_b"])
+            f = oracle_unit(cfg, step, rows_frac, ref, x64, l64)
+            dt = time.perf_counter() - t0
+            if step >= args.warmup:
+                fracs.append(f)
+                times.append(dt)
+    tokens = float(np.sum(fracs))
+    secs = float(np.sum(times))
+    value = tokens / secs
+    sample = (f"per step: router logits for one token plus one 256-feature block of one of its "
+              f"{cfg.top_k + cfg.n_shared} experts (gate/up rows x{rows_frac:.3f}, down rows x{rows_frac:.3f}); "
+              f"value = fraction of a token's expert work per second")
+    return {"metric": "moe_layer_decode_tokens_per_s", "value": value, "unit": "tokens/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_json(cfg, args),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def config_json(cfg, args) -> dict:
+    return {"workload": cfg.name, "hidden": cfg.hidden, "inter": cfg.inter, "experts": cfg.n_experts,
+            "top_k": cfg.top_k, "shared": cfg.n_shared, "tokens": cfg.tokens, "quant": "Q4_K",
+            "gating": "softmax-topk" if cfg.gating == 0 else "sigmoid-renorm",
+            "layers": cfg.n_layers, "cache_bytes": cfg.cache_bytes,
+            "l2": "flushed before every step (256 MiB write)" if args.config != 4 else
+                  "not flushed; working set 51 GB streamed through a 12e9 B cache",
+            "parallelism": f"replicas x{args.gpus}"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, cfg, rank: int, world: int, local_rank: int) -> dict | None:
+    import torch
+
+    from routed_expert_ffn_forward_b200 import build, moe
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    peaks = measured_peaks()
+    if args.config == 4:
+        return run_streaming(args, cfg, rank, world, local_rank, peaks)
+    moe.moe_set_cache_bytes(moe.SIZE_MAX)
+    t0 = time.time()
+    L = layer_from_config(cfg)
+    log(f"[rank {rank}] layer ready in {time.time() - t0:.1f}s")
+    T = cfg.tokens
+    n_pool = 16 if T > 1 else 64
+    xs = [synth.activations(cfg, 0, i, tokens=T) for i in range(n_pool)]
+    x_dev = torch.from_numpy(np.stack(xs).view(np.int16)).view(torch.bfloat16).to(dev)
+    out = torch.empty((T, cfg.hidden), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    # routing of every pool entry (for the algorithmic byte counts)
+    ids_pool = []
+    for i in range(n_pool):
+        L.forward(x_dev[i], out)
+        ids_pool.append(L.routing(T)[0].cpu().numpy())
+    torch.cuda.synchronize()
+
+    def step(i, prof_events):
+        flush.zero_()
+        s, e = prof_events
+        s.record(stream)
+        L.forward(x_dev[i % n_pool], out, stream.cuda_stream)
+        e.record(stream)
+
+    for i in range(args.warmup):
+        step(i, (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    moe.moe_reset_profile()
+    moe.moe_set_profiling(True)
+    st0 = moe.moe_get_stats()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            step(i, evs[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    moe.moe_set_profiling(False)
+    st1 = moe.moe_get_stats()
+    prof = moe.moe_get_profile()
+    step_ms = [s.elapsed_time(e) for s, e in evs]
+    total_ms = max_over_ranks(float(np.sum(step_ms)), world, dev)
+    launches = st1["launches"] - st0["launches"]
+
+    # e2e: the same forward through moe_forward_host, host buffers in and out
+    xh = torch.from_numpy(np.stack(xs).view(np.int16)).view(torch.bfloat16).pin_memory()
+    oh = torch.empty((T, cfg.hidden), dtype=torch.bfloat16).pin_memory()
+    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(min(args.warmup, 3)):
+        moe.moe_forward_host(L.handle, xh[i].data_ptr(), oh.data_ptr(), T, stream.cuda_stream)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        s, e = e2e_evs[i]
+        s.record(stream)
+        moe.moe_forward_host(L.handle, xh[i % n_pool].data_ptr(), oh.data_ptr(), T, stream.cuda_stream)
+        e.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(float(np.sum([s.elapsed_time(e) for s, e in e2e_evs])), world, dev)
+    L.destroy()
+
+    tokens_total = T * args.steps * world
+    value = tokens_total / (total_ms / 1e3)
+    # roofline of the dominant kernel
+    ids_cycle = [ids_pool[i % n_pool] for i in range(args.steps)]
+    if args.config == 3:
+        kern = "gate_up"
+        fl = np.mean([flops(cfg, T) * 2 / 3 for _ in ids_cycle])
+        avg_ms = prof["ms"][kern] / max(1, prof["launches"][kern])
+        achieved = fl / (avg_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "kernel": kern, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": kernel_traffic(kern), "peak_source": peaks["source"]}
+    else:
+        kern = "gate_up"
+        ab = float(np.mean([algorithmic_bytes(cfg, ids, kern) for ids in ids_cycle]))
+        avg_ms = prof["ms"][kern] / max(1, prof["launches"][kern])
+        achieved = ab / (avg_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": kernel_traffic(kern), "algorithmic_bytes": ab,
+                "peak_source": peaks["source"]}
+    fwd_bytes = float(np.mean([algorithmic_bytes(cfg, ids, "forward") for ids in ids_cycle]))
+    fwd_ms = total_ms / args.steps
+    kernels = {k: {"avg_us": 1e3 * prof["ms"][k] / max(1, prof["launches"][k]),
+                   "share": prof["ms"][k] / max(1e-12, sum(prof["ms"][q] for q in moe.KERNELS[:6]))}
+               for k in moe.KERNELS[:6]}
+    if args.config == 3:
+        metric, unit = "moe_layer_prefill_tokens_per_s", "tokens/s"
+    else:
+        metric, unit = "moe_layer_decode_tokens_per_s", "tokens/s"
+    res = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": fwd_ms, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_json(cfg, args),
+           "roofline": roof,
+           "forward_hbm": {"algorithmic_bytes": fwd_bytes, "achieved_gbs": fwd_bytes / (fwd_ms / 1e3) / 1e9,
+                           "frac": fwd_bytes / (fwd_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+           "prefill_tflops": flops(cfg, T) / (fwd_ms / 1e3) / 1e12 if args.config == 3 else None,
+           "kernels": kernels,
+           "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": T * cfg.hidden * 2, "d2h_bytes_per_step": T * cfg.hidden * 2,
+                   "api": "moe_forward_host (pinned host x and out)"},
+           "gpu_launches": launches, "clocks": clk.summary()}
+    return res
+
+
+def run_streaming(args, cfg, rank, world, local_rank, peaks) -> dict:
+    """Config 4: 8 stacked layers streamed through a 12e9-byte cache; each step
+    runs layers 0..7 on one token with the trace's routing and prefetches the
+    next layer's experts one layer ahead."""
+    import torch
+
+    from routed_expert_ffn_forward_b200 import moe
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    h2d_peak = h2d_probe(dev)
+    moe.moe_set_cache_bytes(cfg.cache_bytes)
+    t0 = time.time()
+    layers = [layer_from_config(cfg, l) for l in range(cfg.n_layers)]
+    log(f"[rank {rank}] {cfg.n_layers} layers ready in {time.time() - t0:.1f}s")
+    trace = synth.streaming_trace(cfg)
+    n_steps = args.warmup + args.steps
+    assert n_steps <= cfg.steps, f"trace has {cfg.steps} steps"
+    xs = np.stack([synth.activations(cfg, l, s, tokens=1) for s in range(n_steps) for l in range(cfg.n_layers)])
+    x_dev = torch.from_numpy(xs.view(np.int16)).view(torch.bfloat16).to(dev).view(n_steps, cfg.n_layers, 1, -1)
+    out = torch.empty((1, cfg.hidden), dtype=torch.bfloat16, device=dev)
+    prefetch = not args.no_prefetch
+
+    def run_step(s):
+        for l in range(cfg.n_layers):
+            if prefetch:
+                nl, ns = (l + 1, s) if l + 1 < cfg.n_layers else (0, s + 1)
+                if ns < n_steps:
+                    layers[nl].prefetch(trace[ns, nl])
+            layers[l].forward_routed(x_dev[s, l], trace[s, l][None], out, stream.cuda_stream)
+
+    for s in range(args.warmup):
+        run_step(s)
+    torch.cuda.synchronize()
+    moe.moe_reset_stats()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        for s in range(args.warmup, n_steps):
+            run_step(s)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    st = moe.moe_get_stats()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    for L in layers:
+        L.destroy()
+    moe.moe_set_cache_bytes(moe.SIZE_MAX)
+    secs = ms / 1e3
+    h2d_gbs = st["h2d_bytes"] / secs / 1e9
+    lookups = st["cache_hits"] + st["cache_misses"]
+    return {"metric": "moe_streaming_decode_tokens_per_s", "value": args.steps * world / secs, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": config_json(cfg, args),
+            "roofline": {"bound": "h2d", "achieved": h2d_gbs, "peak": h2d_peak, "unit": "GB/s",
+                         "frac": h2d_gbs / h2d_peak, "traffic": None,
+                         "peak_source": "pinned cudaMemcpyAsync H2D probe, 256 MiB, best of 10"},
+            "cache": {"hit_rate": st["cache_hits"] / max(1, lookups), "misses_per_step": st["cache_misses"] / args.steps,
+                      "prefetches_per_step": st["prefetches"] / args.steps, "h2d_gb_per_step": st["h2d_bytes"] / args.steps / 1e9,
+                      "slots": st["cache_slots"], "prefetch": prefetch},
+            "gpu_launches": st["launches"], "clocks": clk.summary()}
+
+
+def h2d_probe(dev) -> float:
+    import torch
+    src = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    best = 0.0
+    for _ in range(10):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        dst.copy_(src, non_blocking=True)
+        e.record()
+        torch.cuda.synchronize()
+        best = max(best, src.numel() / (s.elapsed_time(e) / 1e3) / 1e9)
+    return best
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+_PG = None
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int, dev) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=1, choices=[1, 2, 3, 4])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefetch", action="store_true")
+    args = ap.parse_args()
+    cfg = synth.CONFIGS[args.config]
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, cfg)), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    res = run_ours(args, cfg, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config in (1, 2):
+        res["cpu_baseline"] = oracle_sample_rate(cfg, n_tokens=cfg.tokens, budget_s=20.0)
+    elif rank == 0 and not args.no_cpu_baseline and world == 1:
+        res["cpu_baseline"] = oracle_sample_rate(synth.CONFIGS[1], n_tokens=3, budget_s=20.0) | {
+            "sample": "decode tokens of the config-1 layer (the oracle's cost per token is the same per expert)"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,197 @@
+/*
+ * moe.h -- C ABI of libmoe.so: the routed mixture-of-experts FFN layer on B200.
+ *
+ * The layer (LayerStoRm README, "TL;DR"): each token activates only a few of
+ * the layer's experts, picked by a router; the full expert set lives in pinned
+ * host RAM and the GPU's memory is a cache in front of it, with the activated
+ * experts streamed in and overlapped with compute.  Weights are GGUF Q4_K
+ * ("Get a model": UD-Q4_K_XL GGUF weights); the architecture is the
+ * DeepSeek-V3 MoE ("References"): routed experts plus always-on shared experts.
+ *
+ * One forward computes, for every token t of x[T,H]:
+ *   l[e]   = sum_h x[t,h] * Wr[e,h] + b[e]                       router logits
+ *   S_t    = the top_k largest l[e] (ties to the lower index)      top-k routing
+ *   w_j    = softmax(l[S_t])_j             (MOE_GATE_SOFTMAX_TOPK)
+ *          = sig(l_j) / sum sig(l[S_t])    (MOE_GATE_SIGMOID_RENORM)
+ *   y_e    = W_d,e ( silu(W_g,e x) * (W_u,e x) )                  SwiGLU expert
+ *   out[t] = bf16_rne( sum_j w_j y_(S_t[j]) + sum_s y_(shared s) ) combine
+ * The combine runs in a fixed order with no atomics, so results are identical
+ * run to run (the pages' "Notes": a deterministic expert-parallel combine).
+ *
+ * Conventions for every call:
+ *  - Every call returns a moe_status and never aborts.  On failure
+ *    moe_last_error() returns a message (thread-local, valid until the next
+ *    call on that thread).  A CUDA error maps to MOE_ERR_CUDA.
+ *  - "device pointer" means memory of the GPU that was current when the layer
+ *    was created; calls must be made with that GPU current.  "host pointer"
+ *    means CPU memory.  A `stream` argument is a cudaStream_t passed as void*
+ *    (NULL = the legacy default stream).
+ *  - Calls on one layer are not thread-safe; calls on different layers are.
+ *
+ * Q4_K weight layout (public GGUF k-quant format): a matrix of R rows and C
+ * input columns is R rows of ceil(C/256) consecutive 144-byte super-blocks.
+ * A super-block holds 256 weights: fp16 d, fp16 dmin, 12 bytes packing eight
+ * 6-bit scales and mins, and 128 bytes of 4-bit quants; weight = d*sc*q - dmin*m.
+ * When C is not a multiple of 256 the last block of each row is padded; the
+ * padded weights are read but multiply zeros and never contribute.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_layer* moe_layer_t; /* opaque, owned by the library */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,     /* bad shape, null pointer, wrong memory kind */
+  MOE_ERR_UNSUPPORTED = -2,     /* a quant type or size this build cannot run */
+  MOE_ERR_OOM = -3,             /* device or pinned allocation failed */
+  MOE_ERR_CUDA = -4,            /* a CUDA runtime call failed */
+  MOE_ERR_CACHE_TOO_SMALL = -5, /* one call needs more experts than cache slots */
+  MOE_ERR_NOT_READY = -6        /* router or experts not set yet */
+} moe_status;
+
+typedef enum { MOE_Q4_K = 12 } moe_quant; /* GGUF type id; the only one supported */
+
+typedef enum {
+  MOE_GATE_SOFTMAX_TOPK = 0,  /* softmax over the top_k selected logits */
+  MOE_GATE_SIGMOID_RENORM = 1 /* sigmoid of the selected logits, renormalised to 1 */
+} moe_gating;
+
+typedef struct {
+  uint64_t forwards;        /* moe_forward* calls that launched work */
+  uint64_t tokens;          /* sum of T over those calls */
+  uint64_t decode_calls;    /* calls that took the decode path (T <= 64) */
+  uint64_t prefill_calls;   /* calls that took the prefill path (T > 64) */
+  uint64_t cache_hits;      /* streamed experts found in the cache */
+  uint64_t cache_misses;    /* streamed experts fetched on demand */
+  uint64_t prefetches;      /* experts fetched by moe_prefetch */
+  uint64_t evictions;       /* cache slots reused for another expert */
+  uint64_t h2d_bytes;       /* bytes copied host -> device into the cache */
+  uint64_t cache_slots;     /* slots of the streaming cache (0: none) */
+  uint64_t slot_bytes;      /* bytes per cache slot */
+  uint64_t launches;        /* kernels launched by the library */
+} moe_stats;
+
+/* Per-kernel device time of profiled forwards, summed (milliseconds, from CUDA
+ * events recorded on the forward's stream right before and after each kernel). */
+enum {
+  MOE_K_ROUTER = 0,  /* router logits */
+  MOE_K_TOPK = 1,    /* top-k + gating */
+  MOE_K_PERMUTE = 2, /* counting-sort permutation */
+  MOE_K_GATE_UP = 3, /* gate/up projections + SwiGLU */
+  MOE_K_DOWN = 4,    /* down projection */
+  MOE_K_COMBINE = 5, /* weighted combine */
+  MOE_K_FORWARD = 6, /* whole forward, first kernel start to last kernel end */
+  MOE_K_COUNT = 7
+};
+typedef struct {
+  uint64_t forwards;             /* forwards profiled */
+  double ms[MOE_K_COUNT];        /* summed device time per MOE_K_* */
+  uint64_t launches[MOE_K_COUNT];/* launches per MOE_K_* */
+} moe_profile;
+
+/* Size in bytes of one expert (gate + up + down) in Q4_K.  0 on bad args. */
+size_t moe_expert_bytes(int hidden, int inter, moe_quant quant);
+
+/* Create a layer on the current GPU.
+ * hidden: H, multiple of 256, <= 16384.  inter: I, >= 1, <= 16384 (any value;
+ * the down rows are padded to whole super-blocks).  n_experts: E, 1..1024.
+ * top_k: 1..min(32, E).  n_shared: S, 0..8 always-on experts (weight 1).
+ * quant must be MOE_Q4_K.  *out receives the handle.
+ * Errors: INVALID_ARG (shape out of range, out == NULL), UNSUPPORTED (quant),
+ * CUDA/OOM (small device allocations). */
+moe_status moe_layer_create(int hidden, int inter, int n_experts, int top_k,
+                            int n_shared, moe_quant quant, moe_layer_t* out);
+
+/* Destroy a layer: waits for its outstanding work, frees its device memory and
+ * drops its experts from the shared cache.  NULL is a no-op. */
+moe_status moe_layer_destroy(moe_layer_t layer);
+
+/* Router weights: W fp32 [E, H] row-major and bias fp32 [E] (NULL = zero),
+ * host or device pointers; both are copied, so the caller keeps ownership.
+ * The bias is added to the logits and used for both selection and weights. */
+moe_status moe_set_router(moe_layer_t layer, const float* W, const float* bias,
+                          moe_gating gating);
+
+/* Expert weights: three arrays of E+S host pointers (routed experts 0..E-1,
+ * then the shared ones), each to one Q4_K matrix: gate [I, H], up [I, H],
+ * down [H, I].  The memory must be pinned (cudaHostAlloc/cudaHostRegister) and
+ * stay valid and unchanged until the layer is destroyed: it is borrowed, not
+ * copied, and cache misses are copied from it later.  In resident mode (see
+ * moe_set_cache_bytes) every expert is uploaded to device memory here, and the
+ * call returns when the upload is done.
+ * Errors: INVALID_ARG (NULL entry or a pointer that is not pinned host memory),
+ * OOM (resident copy does not fit). */
+moe_status moe_set_experts(moe_layer_t layer, const void* const* gate,
+                           const void* const* up, const void* const* down);
+
+/* Device memory budget for experts, shared by every layer on this GPU.
+ * SIZE_MAX (the default) = resident mode: each layer keeps all its experts in
+ * device memory, forwards never wait on the host and can be captured in a CUDA
+ * graph.  Any other value = streaming mode for layers registered afterwards:
+ * floor(bytes / slot_bytes) slots form an LRU cache in front of pinned host
+ * RAM; misses are copied with cudaMemcpyAsync on an internal copy-engine
+ * stream and compute waits on per-slot events.  Changing the budget empties
+ * the streaming cache (it waits for the GPU first). */
+moe_status moe_set_cache_bytes(size_t bytes);
+
+/* Forward: x bf16 [T, H] and out bf16 [T, H], device pointers, row-major.
+ * T >= 0 (T = 0 returns at once).  T <= 64 takes the decode path, larger T the
+ * prefill path.  Work is enqueued on `stream`; in resident mode the call does
+ * not wait for the GPU.  In streaming mode it reads the routing back to the
+ * host (one stream synchronisation) to resolve cache misses before the expert
+ * kernels are launched.  out must not overlap x. */
+moe_status moe_forward(moe_layer_t layer, const void* x, void* out, int T, void* stream);
+
+/* Forward with the routing given: forced_ids int32 [T, top_k] on the HOST
+ * (validated: every id in 0..E-1).  The gate weights are the gating function
+ * of the router logits at these ids.  In streaming mode no synchronisation is
+ * needed: the cache is resolved from the host ids before anything launches. */
+moe_status moe_forward_routed(moe_layer_t layer, const void* x, void* out, int T,
+                              const int32_t* forced_ids, void* stream);
+
+/* Forward on HOST buffers: copies x (host, bf16 [T, H]) in, runs moe_forward
+ * and copies out (host, bf16 [T, H]) back, all on `stream`; returns once the
+ * copies are enqueued (synchronise the stream before reading out).  Pinned
+ * buffers make the copies asynchronous. */
+moe_status moe_forward_host(moe_layer_t layer, const void* x_host, void* out_host,
+                            int T, void* stream);
+
+/* Routing of the last forward: ids int32 [T, top_k] and weights fp32
+ * [T, top_k] (either may be NULL), copied on `stream` to device or host
+ * memory.  ids[t] are ordered by decreasing logit. */
+moe_status moe_get_routing(moe_layer_t layer, int32_t* ids, float* weights, void* stream);
+
+/* Router logits of the last forward, fp32 [T, E], copied on `stream`. */
+moe_status moe_get_logits(moe_layer_t layer, float* logits, void* stream);
+
+/* Streaming mode: start fetching the given experts (host array of n ids in
+ * 0..E+S-1) into the cache now, on the copy stream, so a later forward finds
+ * them ready.  A no-op for resident layers and for experts already cached. */
+moe_status moe_prefetch(moe_layer_t layer, const int32_t* ids, int n);
+
+moe_status moe_get_stats(moe_stats* out);
+moe_status moe_reset_stats(void);
+
+/* Profiling (global, off by default): when on, every forward records CUDA
+ * events around each of its kernels.  moe_get_profile waits for the recorded
+ * events, adds their times into *out and forgets them; moe_reset_profile
+ * drops recorded events without waiting. */
+moe_status moe_set_profiling(int enable);
+moe_status moe_get_profile(moe_profile* out);
+moe_status moe_reset_profile(void);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

@@ -1,0 +1,741 @@
+// Host runtime of libmoe.so: the C ABI of include/moe.h.
+//
+// A layer owns its router weights, a device table of expert weight pointers
+// and per-call scratch.  Experts live either in a per-layer resident copy
+// (cache budget SIZE_MAX) or in the device-wide streaming cache: an arena of
+// fixed-size slots with a host-side LRU, filled from pinned host RAM by
+// cudaMemcpyAsync on an internal copy-engine stream (LayerStoRm README,
+// "TL;DR": GPU memory is a cache in front of the expert set pinned in host RAM,
+// activated experts are streamed in, overlapped with compute).
+//
+// Ordering without host waits: a slot's `ready` event is recorded on the copy
+// stream after its fill, and compute waits on it; a slot's `used` event is
+// recorded on the compute stream after the kernels that read it, and a later
+// fill of that slot waits on it before overwriting.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <list>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "moe_internal.h"
+
+using namespace moe;
+
+namespace {
+
+thread_local std::string g_err;
+
+moe_status fail(moe_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+#define CUDA_TRY(call)                                                                       \
+  do {                                                                                       \
+    cudaError_t e_ = (call);                                                                 \
+    if (e_ != cudaSuccess)                                                                   \
+      return fail(e_ == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA, "%s: %s", #call, \
+                  cudaGetErrorString(e_));                                                   \
+  } while (0)
+
+#define MOE_TRY(call)               \
+  do {                              \
+    moe_status s_ = (call);         \
+    if (s_ != MOE_OK) return s_;    \
+  } while (0)
+
+constexpr int kMaxTokens = 32768;
+
+std::mutex g_mu;            // guards the cache, the stats and the budget
+moe_stats g_stats{};
+size_t g_cache_bytes = SIZE_MAX;
+uint32_t g_next_layer_id = 1;
+
+struct Slot {
+  uint64_t key = UINT64_MAX;  // (layer id << 32) | expert, UINT64_MAX = empty
+  cudaEvent_t ready = nullptr;
+  cudaEvent_t used = nullptr;
+  bool ready_rec = false, used_rec = false;
+  uint64_t epoch = 0;         // last forward that needs this slot
+  std::list<int>::iterator lru;
+};
+
+struct Cache {
+  int device = -1;
+  size_t slot_bytes = 0;
+  int n_slots = 0;
+  uint8_t* arena = nullptr;
+  std::vector<Slot> slots;
+  std::list<int> lru;  // front = most recently used
+  std::unordered_map<uint64_t, int> where;
+  cudaStream_t copy = nullptr;
+  uint64_t epoch = 0;
+};
+Cache* g_cache = nullptr;
+
+// Profiling: events recorded around each kernel of a forward (start/end pairs
+// for MOE_K_ROUTER..MOE_K_COMBINE), resolved by moe_get_profile.
+constexpr int kProfKernels = MOE_K_FORWARD;  // kernels with their own pair
+struct ProfRec {
+  cudaEvent_t ev[2 * kProfKernels];
+  bool used[kProfKernels];
+};
+bool g_profiling = false;
+std::vector<ProfRec> g_prof_pending;
+std::vector<cudaEvent_t> g_prof_pool;
+
+cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+void cache_free(Cache* c) {
+  if (!c) return;
+  for (auto& s : c->slots) {
+    if (s.ready) cudaEventDestroy(s.ready);
+    if (s.used) cudaEventDestroy(s.used);
+  }
+  if (c->arena) cudaFree(c->arena);
+  if (c->copy) cudaStreamDestroy(c->copy);
+  delete c;
+}
+
+}  // namespace
+
+struct moe_layer {
+  uint32_t id = 0;
+  int device = 0;
+  Shape s{};
+  size_t gate_bytes = 0, down_bytes = 0, expert_bytes = 0;
+  moe_gating gating = MOE_GATE_SIGMOID_RENORM;
+  bool router_set = false, experts_set = false, resident = false;
+  float* d_W = nullptr;
+  float* d_b = nullptr;
+  std::vector<const uint8_t*> host;     // (E+S)*3 borrowed pinned pointers
+  uint8_t* d_resident = nullptr;        // resident copy of all experts
+  const uint8_t** d_wptr = nullptr;     // device table (E+S)*3 of weight pointers
+  cudaStream_t copy = nullptr;          // resident uploads
+  // scratch
+  int T_cap = 0;
+  void* scratch = nullptr;
+  Work wk{};
+  __nv_bfloat16* xbuf = nullptr;
+  __nv_bfloat16* obuf = nullptr;
+  int32_t* h_ids = nullptr;             // pinned, for reading routing back
+  int last_T = 0;
+};
+
+namespace {
+
+moe_status check_device(const moe_layer* L) {
+  int dev = -1;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev != L->device)
+    return fail(MOE_ERR_INVALID_ARG, "layer lives on device %d but device %d is current", L->device, dev);
+  return MOE_OK;
+}
+
+size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// Grow the per-call scratch to hold T tokens (power of two, at least 64).
+moe_status ensure_scratch(moe_layer* L, int T) {
+  if (T <= L->T_cap) return MOE_OK;
+  int cap = 64;
+  while (cap < T) cap <<= 1;
+  const Shape& s = L->s;
+  const size_t P = (size_t)cap * (s.k + s.S);
+  const size_t ES = (size_t)(s.E + s.S);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += align256(bytes); return o; };
+  const size_t o_logits = take((size_t)cap * s.E * 4), o_ids = take((size_t)cap * s.k * 4),
+               o_w = take((size_t)cap * s.k * 4), o_forced = take((size_t)cap * s.k * 4),
+               o_counts = take(ES * 4), o_offsets = take((ES + 1) * 4), o_perm = take(P * 4),
+               o_inv = take(P * 4), o_act = take(ES * 4), o_nact = take(4), o_ticket = take(4),
+               o_h = take(P * s.I_pad * 4), o_y = take(P * s.H * 4),
+               o_x = take((size_t)cap * s.H * 2), o_o = take((size_t)cap * s.H * 2);
+  if (L->scratch) {
+    CUDA_TRY(cudaDeviceSynchronize());
+    cudaFree(L->scratch);
+    L->scratch = nullptr;
+    L->T_cap = 0;
+  }
+  if (L->h_ids) {
+    cudaFreeHost(L->h_ids);
+    L->h_ids = nullptr;
+  }
+  CUDA_TRY(cudaMalloc(&L->scratch, off));
+  CUDA_TRY(cudaMallocHost(&L->h_ids, (size_t)cap * s.k * 4));
+  uint8_t* b = static_cast<uint8_t*>(L->scratch);
+  L->wk.logits = reinterpret_cast<float*>(b + o_logits);
+  L->wk.ids = reinterpret_cast<int*>(b + o_ids);
+  L->wk.w = reinterpret_cast<float*>(b + o_w);
+  L->wk.forced = reinterpret_cast<int*>(b + o_forced);
+  L->wk.counts = reinterpret_cast<int*>(b + o_counts);
+  L->wk.offsets = reinterpret_cast<int*>(b + o_offsets);
+  L->wk.perm = reinterpret_cast<int*>(b + o_perm);
+  L->wk.inv = reinterpret_cast<int*>(b + o_inv);
+  L->wk.act = reinterpret_cast<int*>(b + o_act);
+  L->wk.n_act = reinterpret_cast<int*>(b + o_nact);
+  L->wk.ticket = reinterpret_cast<unsigned*>(b + o_ticket);
+  L->wk.h = reinterpret_cast<float*>(b + o_h);
+  L->wk.y = reinterpret_cast<float*>(b + o_y);
+  L->xbuf = reinterpret_cast<__nv_bfloat16*>(b + o_x);
+  L->obuf = reinterpret_cast<__nv_bfloat16*>(b + o_o);
+  // zero everything once: the ticket must start at 0 and the padded columns of
+  // h (I..I_pad) are never written and must read as 0
+  CUDA_TRY(cudaMemset(L->scratch, 0, off));
+  CUDA_TRY(cudaDeviceSynchronize());
+  L->T_cap = cap;
+  return MOE_OK;
+}
+
+// Build (or rebuild) the streaming cache so its slots hold `slot_bytes`.
+// Caller holds g_mu.
+moe_status ensure_cache(int device, size_t slot_bytes) {
+  if (g_cache && g_cache->device == device && g_cache->slot_bytes >= slot_bytes) return MOE_OK;
+  if (g_cache) {
+    CUDA_TRY(cudaDeviceSynchronize());
+    cache_free(g_cache);
+    g_cache = nullptr;
+    g_stats.cache_slots = 0;
+    g_stats.slot_bytes = 0;
+  }
+  if (g_cache_bytes == SIZE_MAX) return fail(MOE_ERR_INVALID_ARG, "no streaming budget set");
+  const size_t n = g_cache_bytes / slot_bytes;
+  if (n == 0)
+    return fail(MOE_ERR_CACHE_TOO_SMALL, "cache budget %zu B holds no %zu-byte expert", g_cache_bytes,
+                slot_bytes);
+  Cache* c = new Cache();
+  c->device = device;
+  c->slot_bytes = slot_bytes;
+  c->n_slots = (int)n;
+  cudaError_t e = cudaMalloc(&c->arena, n * slot_bytes);
+  if (e != cudaSuccess) {
+    cache_free(c);
+    return fail(MOE_ERR_OOM, "cache arena of %zu slots x %zu B: %s", n, slot_bytes, cudaGetErrorString(e));
+  }
+  e = cudaStreamCreateWithFlags(&c->copy, cudaStreamNonBlocking);
+  c->slots.resize(n);
+  for (size_t i = 0; i < n && e == cudaSuccess; ++i) {
+    e = cudaEventCreateWithFlags(&c->slots[i].ready, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->slots[i].used, cudaEventDisableTiming);
+    c->slots[i].lru = c->lru.insert(c->lru.end(), (int)i);
+  }
+  if (e != cudaSuccess) {
+    cache_free(c);
+    return fail(MOE_ERR_CUDA, "cache setup: %s", cudaGetErrorString(e));
+  }
+  g_cache = c;
+  g_stats.cache_slots = n;
+  g_stats.slot_bytes = slot_bytes;
+  return MOE_OK;
+}
+
+uint64_t slot_key(const moe_layer* L, int e) { return ((uint64_t)L->id << 32) | (uint32_t)e; }
+
+// Make sure expert e of L is in the cache (or on its way there).  Returns the
+// slot.  `pin_epoch` != 0 marks the slot as needed by the current forward so
+// that later misses of the same forward cannot evict it.  Caller holds g_mu.
+moe_status cache_fetch(moe_layer* L, int e, uint64_t pin_epoch, bool prefetch, int* slot_out) {
+  Cache* c = g_cache;
+  const uint64_t key = slot_key(L, e);
+  auto it = c->where.find(key);
+  int s;
+  if (it != c->where.end()) {
+    s = it->second;
+    if (!prefetch) g_stats.cache_hits++;
+  } else {
+    // victim: least recently used slot not needed by the current forward
+    int victim = -1;
+    for (auto r = c->lru.rbegin(); r != c->lru.rend(); ++r) {
+      if (c->slots[*r].epoch != c->epoch || c->epoch == 0) {
+        victim = *r;
+        break;
+      }
+    }
+    if (victim < 0)
+      return fail(MOE_ERR_CACHE_TOO_SMALL, "one forward needs more than the %d cache slots", c->n_slots);
+    s = victim;
+    Slot& sl = c->slots[s];
+    if (sl.key != UINT64_MAX) {
+      c->where.erase(sl.key);
+      g_stats.evictions++;
+    }
+    if (sl.used_rec) CUDA_TRY(cudaStreamWaitEvent(c->copy, sl.used, 0));
+    uint8_t* dst = c->arena + (size_t)s * c->slot_bytes;
+    const uint8_t* const* hp = &L->host[3 * (size_t)e];
+    CUDA_TRY(cudaMemcpyAsync(dst, hp[0], L->gate_bytes, cudaMemcpyHostToDevice, c->copy));
+    CUDA_TRY(cudaMemcpyAsync(dst + L->gate_bytes, hp[1], L->gate_bytes, cudaMemcpyHostToDevice, c->copy));
+    CUDA_TRY(cudaMemcpyAsync(dst + 2 * L->gate_bytes, hp[2], L->down_bytes, cudaMemcpyHostToDevice, c->copy));
+    CUDA_TRY(cudaEventRecord(sl.ready, c->copy));
+    sl.ready_rec = true;
+    sl.key = key;
+    c->where[key] = s;
+    g_stats.h2d_bytes += L->expert_bytes;
+    if (prefetch)
+      g_stats.prefetches++;
+    else
+      g_stats.cache_misses++;
+  }
+  Slot& sl = c->slots[s];
+  c->lru.erase(sl.lru);
+  sl.lru = c->lru.insert(c->lru.begin(), s);
+  if (pin_epoch) sl.epoch = pin_epoch;
+  *slot_out = s;
+  return MOE_OK;
+}
+
+// Streaming: bring every expert a forward needs into the cache, make `st`
+// wait for their fills and point the device table at their slots.
+// Caller holds g_mu until the `used` events of these slots are recorded.
+moe_status resolve_experts(moe_layer* L, const int32_t* ids, int n, cudaStream_t st,
+                           std::vector<int>* used_slots) {
+  const Shape& s = L->s;
+  std::vector<char> need(s.E + s.S, 0);
+  for (int i = 0; i < n; ++i) need[ids[i]] = 1;
+  for (int j = 0; j < s.S; ++j) need[s.E + j] = 1;
+  MOE_TRY(ensure_cache(L->device, L->expert_bytes));
+  Cache* c = g_cache;
+  c->epoch++;
+  PtrUpdate u{};
+  for (int e = 0; e < s.E + s.S; ++e) {
+    if (!need[e]) continue;
+    int slot;
+    MOE_TRY(cache_fetch(L, e, c->epoch, false, &slot));
+    if (c->slots[slot].ready_rec) CUDA_TRY(cudaStreamWaitEvent(st, c->slots[slot].ready, 0));
+    used_slots->push_back(slot);
+    u.expert[u.n] = e;
+    u.base[u.n] = c->arena + (size_t)slot * c->slot_bytes;
+    if (++u.n == PtrUpdate::kMax) {
+      CUDA_TRY(launch_set_ptrs(L->d_wptr, u, L->gate_bytes, st));
+      g_stats.launches++;
+      u.n = 0;
+    }
+  }
+  if (u.n) {
+    CUDA_TRY(launch_set_ptrs(L->d_wptr, u, L->gate_bytes, st));
+    g_stats.launches++;
+  }
+  return MOE_OK;
+}
+
+moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int32_t* forced,
+                        cudaStream_t st) {
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "null layer");
+  if (T < 0 || T > kMaxTokens) return fail(MOE_ERR_INVALID_ARG, "T=%d outside 0..%d", T, kMaxTokens);
+  if (T > 0 && (!x || !out)) return fail(MOE_ERR_INVALID_ARG, "null x or out");
+  if (!L->router_set) return fail(MOE_ERR_NOT_READY, "router not set");
+  if (!L->experts_set) return fail(MOE_ERR_NOT_READY, "experts not set");
+  MOE_TRY(check_device(L));
+  const Shape& s = L->s;
+  if (forced) {
+    for (int i = 0; i < T * s.k; ++i)
+      if (forced[i] < 0 || forced[i] >= s.E)
+        return fail(MOE_ERR_INVALID_ARG, "forced id %d at %d outside 0..%d", forced[i], i, s.E - 1);
+  }
+  if (T == 0) return MOE_OK;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 15)
+    return fail(MOE_ERR_INVALID_ARG, "x and out must be 16-byte aligned");
+  MOE_TRY(ensure_scratch(L, T));
+  const Work& wk = L->wk;
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  // one kernel launch, optionally bracketed by profiling events
+  ProfRec pr{};
+  bool prof;
+  {
+    std::lock_guard<std::mutex> lk0(g_mu);
+    prof = g_profiling;
+    if (prof)
+      for (int i = 0; i < 2 * kProfKernels; ++i) pr.ev[i] = prof_event();
+  }
+  int n_launch = 0;
+#define MOE_KERNEL(kid, call)                                    \
+  do {                                                           \
+    if (prof) CUDA_TRY(cudaEventRecord(pr.ev[2 * (kid)], st));   \
+    CUDA_TRY(call);                                              \
+    if (prof) CUDA_TRY(cudaEventRecord(pr.ev[2 * (kid) + 1], st)); \
+    if (prof) pr.used[kid] = true;                               \
+    ++n_launch;                                                  \
+  } while (0)
+  MOE_KERNEL(MOE_K_ROUTER, launch_router_logits(xb, L->d_W, L->d_b, wk.logits, T, s.H, s.E, st));
+  if (forced)
+    CUDA_TRY(cudaMemcpyAsync(wk.forced, forced, (size_t)T * s.k * 4, cudaMemcpyHostToDevice, st));
+  MOE_KERNEL(MOE_K_TOPK, launch_topk(wk.logits, T, s.E, s.k, (int)L->gating, forced ? wk.forced : nullptr,
+                                     wk.ids, wk.w, st));
+  // Streaming: the cache lock is held from resolving the experts until the
+  // slots' `used` events are recorded, so no other forward can evict a slot
+  // between this forward's fill-wait and its last read.
+  std::unique_lock<std::mutex> lk(g_mu, std::defer_lock);
+  std::vector<int> used;
+  if (!L->resident) {
+    const int32_t* hid = forced;
+    if (!hid) {
+      CUDA_TRY(cudaMemcpyAsync(L->h_ids, wk.ids, (size_t)T * s.k * 4, cudaMemcpyDeviceToHost, st));
+      CUDA_TRY(cudaStreamSynchronize(st));
+      hid = L->h_ids;
+    }
+    lk.lock();
+    MOE_TRY(resolve_experts(L, hid, T * s.k, st, &used));
+  }
+  MOE_KERNEL(MOE_K_PERMUTE, launch_permute(wk.ids, T, s, wk, st));
+  MOE_KERNEL(MOE_K_GATE_UP, launch_gate_up_simt(L->d_wptr, xb, s, wk, st));
+  MOE_KERNEL(MOE_K_DOWN, launch_down_simt(L->d_wptr, s, wk, st));
+  MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st));
+#undef MOE_KERNEL
+  {
+    if (!lk.owns_lock()) lk.lock();
+    if (prof) g_prof_pending.push_back(pr);
+    g_stats.launches += (uint64_t)n_launch;
+    if (!used.empty() && g_cache) {
+      for (int slot : used) {
+        CUDA_TRY(cudaEventRecord(g_cache->slots[slot].used, st));
+        g_cache->slots[slot].used_rec = true;
+      }
+    }
+    g_stats.forwards++;
+    g_stats.tokens += (uint64_t)T;
+    if (T <= kDecodeMaxT)
+      g_stats.decode_calls++;
+    else
+      g_stats.prefill_calls++;
+  }
+  L->last_T = T;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_expert_bytes(int hidden, int inter, moe_quant quant) {
+  if (quant != MOE_Q4_K || hidden <= 0 || inter <= 0 || hidden % kQK) return 0;
+  const size_t nbh = hidden / kQK, nbi = (inter + kQK - 1) / kQK;
+  return 2 * (size_t)inter * nbh * kQBytes + (size_t)hidden * nbi * kQBytes;
+}
+
+moe_status moe_layer_create(int hidden, int inter, int n_experts, int top_k, int n_shared,
+                            moe_quant quant, moe_layer_t* out) {
+  g_err.clear();
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (quant != MOE_Q4_K) return fail(MOE_ERR_UNSUPPORTED, "quant type %d (only Q4_K=12)", (int)quant);
+  if (hidden <= 0 || hidden > 16384 || hidden % kQK)
+    return fail(MOE_ERR_INVALID_ARG, "hidden=%d must be a multiple of 256 in 256..16384", hidden);
+  if (inter <= 0 || inter > 16384) return fail(MOE_ERR_INVALID_ARG, "inter=%d outside 1..16384", inter);
+  if (n_experts <= 0 || n_experts > 1024)
+    return fail(MOE_ERR_INVALID_ARG, "n_experts=%d outside 1..1024", n_experts);
+  if (top_k <= 0 || top_k > 32 || top_k > n_experts)
+    return fail(MOE_ERR_INVALID_ARG, "top_k=%d outside 1..min(32, E)", top_k);
+  if (n_shared < 0 || n_shared > 8) return fail(MOE_ERR_INVALID_ARG, "n_shared=%d outside 0..8", n_shared);
+  moe_layer* L = new moe_layer();
+  Shape& s = L->s;
+  s.H = hidden;
+  s.I = inter;
+  s.E = n_experts;
+  s.k = top_k;
+  s.S = n_shared;
+  s.nbh = hidden / kQK;
+  s.nbi = (inter + kQK - 1) / kQK;
+  s.I_pad = s.nbi * kQK;
+  L->gate_bytes = (size_t)inter * s.nbh * kQBytes;
+  L->down_bytes = (size_t)hidden * s.nbi * kQBytes;
+  L->expert_bytes = 2 * L->gate_bytes + L->down_bytes;
+  cudaError_t e = cudaGetDevice(&L->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&s.n_sm, cudaDevAttrMultiProcessorCount, L->device);
+  if (e == cudaSuccess) e = cudaMalloc(&L->d_wptr, sizeof(void*) * 3 * (size_t)(s.E + s.S));
+  if (e == cudaSuccess) e = cudaMemset(L->d_wptr, 0, sizeof(void*) * 3 * (size_t)(s.E + s.S));
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->copy, cudaStreamNonBlocking);
+  if (e != cudaSuccess) {
+    moe_layer_destroy(L);
+    return fail(e == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA, "layer setup: %s",
+                cudaGetErrorString(e));
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    L->id = g_next_layer_id++;
+  }
+  *out = L;
+  return MOE_OK;
+}
+
+moe_status moe_layer_destroy(moe_layer_t L) {
+  g_err.clear();
+  if (!L) return MOE_OK;
+  cudaDeviceSynchronize();
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_cache) {
+      for (int e = 0; e < L->s.E + L->s.S; ++e) {
+        auto it = g_cache->where.find(slot_key(L, e));
+        if (it != g_cache->where.end()) {
+          g_cache->slots[it->second].key = UINT64_MAX;
+          g_cache->where.erase(it);
+        }
+      }
+    }
+  }
+  if (L->d_W) cudaFree(L->d_W);
+  if (L->d_b) cudaFree(L->d_b);
+  if (L->d_resident) cudaFree(L->d_resident);
+  if (L->d_wptr) cudaFree(L->d_wptr);
+  if (L->scratch) cudaFree(L->scratch);
+  if (L->h_ids) cudaFreeHost(L->h_ids);
+  if (L->copy) cudaStreamDestroy(L->copy);
+  delete L;
+  return MOE_OK;
+}
+
+moe_status moe_set_router(moe_layer_t L, const float* W, const float* bias, moe_gating gating) {
+  g_err.clear();
+  if (!L || !W) return fail(MOE_ERR_INVALID_ARG, "null layer or W");
+  if (gating != MOE_GATE_SOFTMAX_TOPK && gating != MOE_GATE_SIGMOID_RENORM)
+    return fail(MOE_ERR_INVALID_ARG, "gating=%d", (int)gating);
+  MOE_TRY(check_device(L));
+  const size_t wb = (size_t)L->s.E * L->s.H * sizeof(float);
+  if (!L->d_W) CUDA_TRY(cudaMalloc(&L->d_W, wb));
+  CUDA_TRY(cudaMemcpy(L->d_W, W, wb, cudaMemcpyDefault));
+  if (bias) {
+    if (!L->d_b) CUDA_TRY(cudaMalloc(&L->d_b, (size_t)L->s.E * sizeof(float)));
+    CUDA_TRY(cudaMemcpy(L->d_b, bias, (size_t)L->s.E * sizeof(float), cudaMemcpyDefault));
+  } else if (L->d_b) {
+    cudaFree(L->d_b);
+    L->d_b = nullptr;
+  }
+  L->gating = gating;
+  L->router_set = true;
+  return MOE_OK;
+}
+
+moe_status moe_set_experts(moe_layer_t L, const void* const* gate, const void* const* up,
+                           const void* const* down) {
+  g_err.clear();
+  if (!L || !gate || !up || !down) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  MOE_TRY(check_device(L));
+  const int n = L->s.E + L->s.S;
+  std::vector<const uint8_t*> host(3 * (size_t)n);
+  for (int e = 0; e < n; ++e) {
+    const void* p[3] = {gate[e], up[e], down[e]};
+    for (int m = 0; m < 3; ++m) {
+      if (!p[m]) return fail(MOE_ERR_INVALID_ARG, "expert %d matrix %d is NULL", e, m);
+      cudaPointerAttributes a{};
+      cudaError_t err = cudaPointerGetAttributes(&a, p[m]);
+      if (err != cudaSuccess || a.type != cudaMemoryTypeHost) {
+        cudaGetLastError();
+        return fail(MOE_ERR_INVALID_ARG, "expert %d matrix %d is not pinned host memory", e, m);
+      }
+      host[3 * (size_t)e + m] = static_cast<const uint8_t*>(p[m]);
+    }
+  }
+  size_t budget;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    budget = g_cache_bytes;
+  }
+  L->host = std::move(host);
+  L->experts_set = false;
+  if (budget == SIZE_MAX) {
+    // resident: one device copy of every expert, uploaded now
+    if (!L->d_resident) CUDA_TRY(cudaMalloc(&L->d_resident, (size_t)n * L->expert_bytes));
+    std::vector<const uint8_t*> table(3 * (size_t)n);
+    for (int e = 0; e < n; ++e) {
+      uint8_t* dst = L->d_resident + (size_t)e * L->expert_bytes;
+      const size_t sz[3] = {L->gate_bytes, L->gate_bytes, L->down_bytes};
+      const size_t off[3] = {0, L->gate_bytes, 2 * L->gate_bytes};
+      for (int m = 0; m < 3; ++m) {
+        CUDA_TRY(cudaMemcpyAsync(dst + off[m], L->host[3 * (size_t)e + m], sz[m], cudaMemcpyHostToDevice,
+                                 L->copy));
+        table[3 * (size_t)e + m] = dst + off[m];
+      }
+    }
+    CUDA_TRY(cudaMemcpyAsync(L->d_wptr, table.data(), sizeof(void*) * table.size(), cudaMemcpyHostToDevice,
+                             L->copy));
+    CUDA_TRY(cudaStreamSynchronize(L->copy));
+    L->resident = true;
+  } else {
+    if (L->d_resident) {
+      CUDA_TRY(cudaDeviceSynchronize());
+      cudaFree(L->d_resident);
+      L->d_resident = nullptr;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    MOE_TRY(ensure_cache(L->device, L->expert_bytes));
+    L->resident = false;
+  }
+  L->experts_set = true;
+  return MOE_OK;
+}
+
+moe_status moe_set_cache_bytes(size_t bytes) {
+  g_err.clear();
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_cache) {
+    CUDA_TRY(cudaDeviceSynchronize());
+    cache_free(g_cache);
+    g_cache = nullptr;
+    g_stats.cache_slots = 0;
+    g_stats.slot_bytes = 0;
+  }
+  g_cache_bytes = bytes;
+  return MOE_OK;
+}
+
+moe_status moe_forward(moe_layer_t L, const void* x, void* out, int T, void* stream) {
+  g_err.clear();
+  return forward_impl(L, x, out, T, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_routed(moe_layer_t L, const void* x, void* out, int T, const int32_t* forced_ids,
+                              void* stream) {
+  g_err.clear();
+  if (T > 0 && !forced_ids) return fail(MOE_ERR_INVALID_ARG, "forced_ids is NULL");
+  return forward_impl(L, x, out, T, forced_ids, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_host(moe_layer_t L, const void* x_host, void* out_host, int T, void* stream) {
+  g_err.clear();
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "null layer");
+  if (T < 0 || T > kMaxTokens) return fail(MOE_ERR_INVALID_ARG, "T=%d outside 0..%d", T, kMaxTokens);
+  if (T == 0) return MOE_OK;
+  if (!x_host || !out_host) return fail(MOE_ERR_INVALID_ARG, "null x or out");
+  MOE_TRY(check_device(L));
+  MOE_TRY(ensure_scratch(L, T));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)T * L->s.H * 2;
+  CUDA_TRY(cudaMemcpyAsync(L->xbuf, x_host, bytes, cudaMemcpyHostToDevice, st));
+  MOE_TRY(forward_impl(L, L->xbuf, L->obuf, T, nullptr, st));
+  CUDA_TRY(cudaMemcpyAsync(out_host, L->obuf, bytes, cudaMemcpyDeviceToHost, st));
+  return MOE_OK;
+}
+
+moe_status moe_get_routing(moe_layer_t L, int32_t* ids, float* weights, void* stream) {
+  g_err.clear();
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "null layer");
+  if (L->last_T == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n = (size_t)L->last_T * L->s.k * 4;
+  if (ids) CUDA_TRY(cudaMemcpyAsync(ids, L->wk.ids, n, cudaMemcpyDefault, st));
+  if (weights) CUDA_TRY(cudaMemcpyAsync(weights, L->wk.w, n, cudaMemcpyDefault, st));
+  return MOE_OK;
+}
+
+moe_status moe_get_logits(moe_layer_t L, float* logits, void* stream) {
+  g_err.clear();
+  if (!L || !logits) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  if (L->last_T == 0) return MOE_OK;
+  CUDA_TRY(cudaMemcpyAsync(logits, L->wk.logits, (size_t)L->last_T * L->s.E * 4, cudaMemcpyDefault,
+                           static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_prefetch(moe_layer_t L, const int32_t* ids, int n) {
+  g_err.clear();
+  if (!L || (n > 0 && !ids) || n < 0) return fail(MOE_ERR_INVALID_ARG, "bad argument");
+  if (!L->experts_set) return fail(MOE_ERR_NOT_READY, "experts not set");
+  if (L->resident || n == 0) return MOE_OK;
+  MOE_TRY(check_device(L));
+  for (int i = 0; i < n; ++i)
+    if (ids[i] < 0 || ids[i] >= L->s.E + L->s.S)
+      return fail(MOE_ERR_INVALID_ARG, "prefetch id %d outside 0..%d", ids[i], L->s.E + L->s.S - 1);
+  std::lock_guard<std::mutex> lk(g_mu);
+  MOE_TRY(ensure_cache(L->device, L->expert_bytes));
+  for (int i = 0; i < n; ++i) {
+    int slot;
+    MOE_TRY(cache_fetch(L, ids[i], 0, true, &slot));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_get_stats(moe_stats* out) {
+  g_err.clear();
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "null out");
+  std::lock_guard<std::mutex> lk(g_mu);
+  *out = g_stats;
+  return MOE_OK;
+}
+
+moe_status moe_reset_stats(void) {
+  g_err.clear();
+  std::lock_guard<std::mutex> lk(g_mu);
+  const uint64_t slots = g_stats.cache_slots, sb = g_stats.slot_bytes;
+  g_stats = moe_stats{};
+  g_stats.cache_slots = slots;
+  g_stats.slot_bytes = sb;
+  return MOE_OK;
+}
+
+moe_status moe_set_profiling(int enable) {
+  g_err.clear();
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_profiling = enable != 0;
+  return MOE_OK;
+}
+
+moe_status moe_get_profile(moe_profile* out) {
+  g_err.clear();
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "null out");
+  std::vector<ProfRec> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    recs.swap(g_prof_pending);
+  }
+  moe_status st = MOE_OK;
+  for (auto& r : recs) {
+    int first = -1, last = -1;
+    for (int kid = 0; kid < kProfKernels; ++kid) {
+      if (!r.used[kid]) continue;
+      if (first < 0) first = kid;
+      last = kid;
+      float ms = 0.f;
+      cudaError_t e = cudaEventSynchronize(r.ev[2 * kid + 1]);
+      if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.ev[2 * kid], r.ev[2 * kid + 1]);
+      if (e != cudaSuccess) {
+        st = fail(MOE_ERR_CUDA, "profile events: %s", cudaGetErrorString(e));
+        continue;
+      }
+      out->ms[kid] += ms;
+      out->launches[kid]++;
+    }
+    if (first >= 0) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, r.ev[2 * first], r.ev[2 * last + 1]) == cudaSuccess) {
+        out->ms[MOE_K_FORWARD] += ms;
+        out->launches[MOE_K_FORWARD]++;
+      }
+      out->forwards++;
+    }
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (auto& r : recs)
+    for (auto e : r.ev) g_prof_pool.push_back(e);
+  return st;
+}
+
+moe_status moe_reset_profile(void) {
+  g_err.clear();
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (auto& r : g_prof_pending)
+    for (auto e : r.ev) g_prof_pool.push_back(e);
+  g_prof_pending.clear();
+  return MOE_OK;
+}
+
+const char* moe_last_error(void) { return g_err.c_str(); }
+
+}  // extern "C"

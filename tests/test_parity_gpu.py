@@ -1,0 +1,158 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle, on the
+same seeded inputs.  Small shapes are compared element by element over every
+token; the full-size configurations compare router ids over every token and
+outputs over sampled tokens (the oracle computes those rows one by one)."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+from oracle import moe_ref as ref
+from routed_expert_ffn_forward_b200 import build, moe, synth
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="session")
+def torch():
+    import torch as _t
+    if not _t.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    moe.lib()
+    moe.moe_set_cache_bytes(moe.SIZE_MAX)
+    return _t
+
+
+def oracle_layer(cfg, layer_index=0):
+    return dict(router_w=synth.router_weight(cfg, layer_index), router_b=synth.router_bias(cfg, layer_index),
+                experts=lambda e: synth.expert_tensors(cfg, layer_index, e))
+
+
+def to_dev(torch, bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def to_bits(torch, t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def run_gpu(torch, cfg, T, layer_index=0, layer=None):
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    L = layer or layer_from_config(cfg, layer_index)
+    x = synth.activations(cfg, layer_index, tokens=T)
+    out = L.forward(to_dev(torch, x))
+    ids, w = L.routing(T)
+    logits = L.logits(T)
+    torch.cuda.synchronize()
+    res = dict(x=x, out=to_bits(torch, out), ids=ids.cpu().numpy(), w=w.cpu().numpy(),
+               logits=logits.cpu().numpy())
+    if layer is None:
+        L.destroy()
+    return res
+
+
+def check_against_oracle(cfg, g, sample=None, layer_index=0):
+    """Index rule on every token, outputs on `sample` tokens (all if None)."""
+    ol = oracle_layer(cfg, layer_index)
+    x = g["x"]
+    T = x.shape[0]
+    l64 = ref.router_logits(ref.bf16_to_f64(x), ol["router_w"], ol["router_b"])
+    np.testing.assert_allclose(g["logits"], l64, rtol=0, atol=1e-4 * max(1.0, np.abs(l64).max()))
+    near = pu.check_ids(g["ids"], l64, cfg.top_k)
+    toks = np.arange(T) if sample is None else np.asarray(sample)
+    # weights of the GPU's picks, by the oracle's gating of its own logits
+    w_or = ref.gate_weights(l64, g["ids"].astype(np.int64), cfg.gating)
+    np.testing.assert_allclose(g["w"], w_or, rtol=1e-5, atol=1e-6)
+    forced = np.where(near[:, None], g["ids"], ref.topk_ids(l64, cfg.top_k))
+    r = ref.moe_forward(x, ol, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter, forced_ids=forced,
+                        token_subset=toks)
+    return pu.check_outputs(g["out"][toks], r["out_bf16"], cfg.name)
+
+
+# ------------------------------------------------------------------ small shapes, every token
+C0 = synth.CONFIGS[0]
+SMALL = {
+    "c0": C0,
+    "c0_shared_sigmoid_bias": dataclasses.replace(C0, n_shared=1, gating=1, zipf_s=1.1, seed=11),
+    "k_equals_E": dataclasses.replace(C0, top_k=16, seed=12),
+    "ragged_inter": dataclasses.replace(C0, hidden=512, inter=300, n_experts=40, top_k=5, n_shared=2,
+                                        gating=1, seed=13, router_std=1 / 512 ** 0.5),
+    "k1_E1": dataclasses.replace(C0, n_experts=1, top_k=1, seed=14),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+@pytest.mark.parametrize("T", [1, 4, 17, 64, 65, 200])
+def test_small_every_token(torch, name, T):
+    cfg = SMALL[name]
+    g = run_gpu(torch, cfg, T)
+    check_against_oracle(cfg, g)
+
+
+def test_zero_tokens(torch):
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    L = layer_from_config(C0)
+    x = torch.empty((0, C0.hidden), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((0, C0.hidden), dtype=torch.bfloat16, device="cuda")
+    moe.moe_forward(L.handle, x.data_ptr(), out.data_ptr(), 0, None)
+    L.destroy()
+
+
+# ------------------------------------------------------------------ full-size configurations
+def test_c1_decode_every_token(torch):
+    cfg = synth.CONFIGS[1]
+    g = run_gpu(torch, cfg, cfg.tokens)
+    check_against_oracle(cfg, g)
+
+
+def test_c2_batched_decode_sampled(torch):
+    cfg = synth.CONFIGS[2]
+    g = run_gpu(torch, cfg, cfg.tokens)
+    counts = np.bincount(g["ids"].ravel(), minlength=cfg.n_experts)
+    assert (counts > 10).sum() >= 1 and (counts.max() <= cfg.tokens)
+    check_against_oracle(cfg, g, sample=[0, 1, 17, 31, 42, 63])
+
+
+def test_c3_prefill_sampled(torch):
+    cfg = synth.CONFIGS[3]
+    g = run_gpu(torch, cfg, cfg.tokens)
+    check_against_oracle(cfg, g, sample=[0, 1777, 4095])
+
+
+def test_deterministic_and_host_path(torch):
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    cfg = synth.CONFIGS[2]
+    L = layer_from_config(cfg)
+    x = synth.activations(cfg)
+    xd = to_dev(torch, x)
+    a = to_bits(torch, L.forward(xd))
+    b = to_bits(torch, L.forward(xd))
+    np.testing.assert_array_equal(a, b)
+    xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    moe.moe_forward_host(L.handle, xh.data_ptr(), oh.data_ptr(), cfg.tokens, None)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(oh.view(torch.int16).numpy().view(np.uint16), a)
+    L.destroy()
+
+
+def test_forced_routing(torch):
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    cfg = SMALL["c0_shared_sigmoid_bias"]
+    L = layer_from_config(cfg)
+    x = synth.activations(cfg, tokens=5)
+    forced = np.array([[0, 1], [15, 14], [3, 3], [7, 2], [9, 0]], dtype=np.int32)
+    out = to_bits(torch, L.forward_routed(to_dev(torch, x), forced))
+    ids, w = L.routing(5)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(ids.cpu().numpy(), forced)
+    r = ref.moe_forward(x, oracle_layer(cfg), cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter,
+                        forced_ids=forced)
+    np.testing.assert_allclose(w.cpu().numpy(), r["w"], rtol=1e-5)
+    pu.check_outputs(out, r["out_bf16"], "forced")
+    with pytest.raises(moe.MoEError) as ei:
+        L.forward_routed(to_dev(torch, x), np.full((5, 2), 16, dtype=np.int32))
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    L.destroy()
