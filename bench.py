@@ -460,8 +460,13 @@ def main():
     ap.add_argument("--config", type=int, default=1, choices=[1, 2, 3, 4])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefetch", action="store_true")
+    ap.add_argument("--small", action="store_true",
+                    help="32 routed experts instead of 256 (same per-launch work at T=1; for ncu captures)")
     args = ap.parse_args()
     cfg = synth.CONFIGS[args.config]
+    if args.small:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, n_experts=32, name=cfg.name + " [32 experts]")
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

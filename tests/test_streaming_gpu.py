@@ -1,0 +1,201 @@
+"""Expert streaming through the device cache (GPU).
+
+Streamed layers must give bit-identical outputs to resident layers (same
+kernels, same arithmetic; only where the weights come from differs), and the
+cache's hit/miss/eviction counts must match a host-side model of its LRU
+policy step by step.  A small cache forces evictions every step.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+from oracle import moe_ref as ref
+from routed_expert_ffn_forward_b200 import build, moe, synth
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch as _t
+    if not _t.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    moe.moe_set_cache_bytes(moe.SIZE_MAX)
+    yield _t
+    moe.moe_set_cache_bytes(moe.SIZE_MAX)
+
+
+class LRUModel:
+    """Host model of the cache policy: slots start in order 0..n-1 (front =
+    most recent); a miss takes the least recently used slot not needed by the
+    current forward; a forward touches its experts in ascending order, shared
+    experts last; prefetch misses avoid the last forward's slots."""
+
+    def __init__(self, n_slots):
+        self.order = list(range(n_slots))          # front = MRU
+        self.key = [None] * n_slots
+        self.epoch_of = [0] * n_slots
+        self.epoch = 0
+        self.hits = self.misses = self.prefetches = self.evictions = 0
+
+    def _touch(self, s):
+        self.order.remove(s)
+        self.order.insert(0, s)
+
+    def _fetch(self, key, pin, prefetch):
+        if key in self.key:
+            s = self.key.index(key)
+            if not prefetch:
+                self.hits += 1
+        else:
+            s = next(s for s in reversed(self.order) if self.epoch == 0 or self.epoch_of[s] != self.epoch)
+            if self.key[s] is not None:
+                self.evictions += 1
+            self.key[s] = key
+            if prefetch:
+                self.prefetches += 1
+            else:
+                self.misses += 1
+        self._touch(s)
+        if pin:
+            self.epoch_of[s] = self.epoch
+
+    def forward(self, layer, experts):
+        self.epoch += 1
+        for e in sorted(set(experts)):
+            self._fetch((layer, e), True, False)
+
+    def prefetch(self, layer, experts):
+        for e in experts:
+            self._fetch((layer, e), False, True)
+
+
+def to_dev(torch, bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def run_trace(torch, cfg, layers, trace, steps, prefetch, model=None):
+    outs = []
+    for s in range(steps):
+        for l in range(cfg.n_layers):
+            if prefetch:
+                nl, ns = (l + 1, s) if l + 1 < cfg.n_layers else (0, s + 1)
+                if ns < steps:
+                    layers[nl].prefetch(trace[ns, nl])
+                    if model:
+                        model.prefetch(nl, trace[ns, nl].tolist())
+            x = synth.activations(cfg, l, s, tokens=1)
+            out = layers[l].forward_routed(to_dev(torch, x), trace[s, l][None])
+            if model:
+                model.forward(l, trace[s, l].tolist() + [cfg.n_experts + j for j in range(cfg.n_shared)])
+            outs.append(out.view(torch.int16).cpu().numpy().view(np.uint16))
+    torch.cuda.synchronize()
+    return outs
+
+
+SMALL = dataclasses.replace(synth.CONFIGS[0], name="streaming small", n_shared=1, gating=1, n_layers=3,
+                            steps=14, seed=21)
+
+
+@pytest.mark.parametrize("prefetch", [False, True])
+@pytest.mark.parametrize("slots", [4, 7, 40])
+def test_streaming_matches_resident_and_lru_model(torch, prefetch, slots):
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    cfg = SMALL
+    trace = synth.streaming_trace(cfg)
+    moe.moe_set_cache_bytes(moe.SIZE_MAX)
+    res = [layer_from_config(cfg, l) for l in range(cfg.n_layers)]
+    want = run_trace(torch, cfg, res, trace, cfg.steps, prefetch=False)
+    for L in res:
+        L.destroy()
+    eb = moe.moe_expert_bytes(cfg.hidden, cfg.inter)
+    moe.moe_set_cache_bytes(slots * eb + 7)
+    try:
+        layers = [layer_from_config(cfg, l) for l in range(cfg.n_layers)]
+        moe.moe_reset_stats()
+        model = LRUModel(slots)
+        got = run_trace(torch, cfg, layers, trace, cfg.steps, prefetch=prefetch, model=model)
+        st = moe.moe_get_stats()
+        for L in layers:
+            L.destroy()
+    finally:
+        moe.moe_set_cache_bytes(moe.SIZE_MAX)
+    for a, b in zip(got, want):
+        np.testing.assert_array_equal(a, b)
+    assert st["cache_slots"] == slots and st["slot_bytes"] == eb
+    assert (st["cache_hits"], st["cache_misses"], st["prefetches"], st["evictions"]) == \
+        (model.hits, model.misses, model.prefetches, model.evictions)
+    assert st["h2d_bytes"] == (model.misses + model.prefetches) * eb
+    if slots < cfg.n_layers * (cfg.n_experts + 1):
+        assert model.evictions > 0
+
+
+def test_streaming_c1_shapes_against_oracle(torch):
+    """Full-size expert shapes (hidden 7168, inter 2048), 32 experts per layer,
+    2 layers through a 12-slot cache; unrouted forward (routing read back to the
+    host) and a check of one streamed token against the oracle."""
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    cfg = dataclasses.replace(synth.CONFIGS[4], n_experts=32, n_layers=2, steps=6, seed=41)
+    eb = moe.moe_expert_bytes(cfg.hidden, cfg.inter)
+    moe.moe_set_cache_bytes(12 * eb)
+    try:
+        layers = [layer_from_config(cfg, l) for l in range(cfg.n_layers)]
+        moe.moe_reset_stats()
+        outs = []
+        for s in range(3):
+            for l in range(cfg.n_layers):
+                x = synth.activations(cfg, l, s, tokens=2)
+                o = layers[l].forward(to_dev(torch, x))
+                ids, _ = layers[l].routing(2)
+                outs.append((l, x, o.view(torch.int16).cpu().numpy().view(np.uint16), ids.cpu().numpy()))
+        st = moe.moe_get_stats()
+        for L in layers:
+            L.destroy()
+    finally:
+        moe.moe_set_cache_bytes(moe.SIZE_MAX)
+    assert st["cache_misses"] > 0 and st["evictions"] > 0
+    l, x, o, ids = outs[-1]
+    layer = dict(router_w=synth.router_weight(cfg, l), router_b=synth.router_bias(cfg, l),
+                 experts=lambda e: synth.expert_tensors(cfg, l, e))
+    l64 = ref.router_logits(ref.bf16_to_f64(x), layer["router_w"], layer["router_b"])
+    near = pu.check_ids(ids, l64, cfg.top_k)
+    forced = np.where(near[:, None], ids, ref.topk_ids(l64, cfg.top_k))
+    r = ref.moe_forward(x, layer, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter, forced_ids=forced)
+    pu.check_outputs(o, r["out_bf16"], "streamed c1 shapes")
+
+
+def test_cache_too_small_is_an_error(torch):
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    cfg = SMALL
+    eb = moe.moe_expert_bytes(cfg.hidden, cfg.inter)
+    moe.moe_set_cache_bytes(2 * eb)        # k + S = 3 experts per token
+    try:
+        L = layer_from_config(cfg, 0)
+        x = synth.activations(cfg, 0, 0, tokens=1)
+        with pytest.raises(moe.MoEError) as ei:
+            L.forward_routed(to_dev(torch, x), np.array([[0, 1]], dtype=np.int32))
+        assert ei.value.status == moe.MOE_ERR_CACHE_TOO_SMALL
+        L.destroy()
+        with pytest.raises(moe.MoEError) as ei:
+            moe.moe_set_cache_bytes(eb - 1)
+            layer_from_config(cfg, 0)
+        assert ei.value.status == moe.MOE_ERR_CACHE_TOO_SMALL
+    finally:
+        moe.moe_set_cache_bytes(moe.SIZE_MAX)
+
+
+def test_unpinned_host_memory_is_rejected(torch):
+    cfg = SMALL
+    h = moe.moe_layer_create(cfg.hidden, cfg.inter, cfg.n_experts, cfg.top_k, cfg.n_shared)
+    buf = np.zeros(moe.moe_expert_bytes(cfg.hidden, cfg.inter), dtype=np.uint8)   # pageable
+    p = [buf.ctypes.data] * (cfg.n_experts + cfg.n_shared)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_set_experts(h, p, p, p)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_forward(h, 16, 16, 1, None)
+    assert ei.value.status == moe.MOE_ERR_NOT_READY
+    moe.moe_layer_destroy(h)
