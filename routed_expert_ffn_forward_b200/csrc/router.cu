@@ -4,6 +4,7 @@
 #include <cfloat>
 
 #include "moe_internal.h"
+#include "topk.cuh"
 
 namespace moe {
 namespace {
@@ -51,84 +52,16 @@ router_logits_kernel(const __nv_bfloat16* __restrict__ x, const float* __restric
     if (lane == i && i < nt) logits[(size_t)(t0 + i) * E + e] = acc[i] + bias;
 }
 
-// (value, index) ordering of the top-k: larger logit first, equal logits to the
-// lower expert index.  `ok` false means "no candidate".
-struct Cand {
-  float v;
-  int e;
-  bool ok;
-};
-__device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
-  if (a.ok != b.ok) return a.ok;
-  if (!a.ok) return false;
-  return a.v > b.v || (a.v == b.v && a.e < b.e);
-}
-
-// One warp per token.  Lane l holds logits l, l+32, ...; k rounds of a warp
-// arg-max pick the experts in decreasing order.  Lane r keeps round r's pick.
+// One warp per token.
 template <int PL>
 __global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int k, int gating,
                             const int* __restrict__ forced, int* __restrict__ ids,
                             float* __restrict__ w) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= T) return;
-  const float* lt = logits + (size_t)t * E;
-  int my_e = 0;
-  float my_l = 0.f;
-  if (forced) {
-    if (lane < k) {
-      my_e = forced[(size_t)t * k + lane];
-      my_l = lt[my_e];
-    }
-  } else {
-    float v[PL];
-    bool taken[PL];
-#pragma unroll
-    for (int i = 0; i < PL; ++i) {
-      const int e = lane + 32 * i;
-      taken[i] = e >= E;
-      v[i] = taken[i] ? 0.f : lt[e];
-    }
-    for (int r = 0; r < k; ++r) {
-      Cand c{0.f, 0, false};
-#pragma unroll
-      for (int i = 0; i < PL; ++i) {
-        const Cand d{v[i], lane + 32 * i, !taken[i]};
-        if (better(d, c)) c = d;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        Cand d;
-        d.v = __shfl_xor_sync(0xffffffffu, c.v, o);
-        d.e = __shfl_xor_sync(0xffffffffu, c.e, o);
-        d.ok = __shfl_xor_sync(0xffffffffu, (int)c.ok, o);
-        if (better(d, c)) c = d;
-      }
-      if (lane == r) {
-        my_e = c.e;
-        my_l = c.v;
-      }
-      if ((c.e & 31) == lane) {
-#pragma unroll
-        for (int i = 0; i < PL; ++i)
-          if (i == (c.e >> 5)) taken[i] = true;
-      }
-    }
-  }
-  // gating over the k picks (lanes >= k contribute zero)
-  float m = lane < k ? my_l : -FLT_MAX;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float z = 0.f;
-  if (lane < k) z = gating == 0 ? expf(my_l - m) : 1.0f / (1.0f + expf(-my_l));
-  float sum = z;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane < k) {
-    ids[(size_t)t * k + lane] = my_e;
-    w[(size_t)t * k + lane] = z / sum;
-  }
+  warp_topk_gate<PL>(logits + (size_t)t * E, E, k, gating, forced ? forced + (size_t)t * k : nullptr,
+                     ids + (size_t)t * k, w + (size_t)t * k);
 }
 
 }  // namespace

@@ -129,18 +129,19 @@ def test_streaming_matches_resident_and_lru_model(torch, prefetch, slots):
     assert (st["cache_hits"], st["cache_misses"], st["prefetches"], st["evictions"]) == \
         (model.hits, model.misses, model.prefetches, model.evictions)
     assert st["h2d_bytes"] == (model.misses + model.prefetches) * eb
-    if slots < cfg.n_layers * (cfg.n_experts + 1):
+    touched = len({k for k in model.key if k is not None}) + model.evictions
+    if touched > slots:
         assert model.evictions > 0
 
 
 def test_streaming_c1_shapes_against_oracle(torch):
     """Full-size expert shapes (hidden 7168, inter 2048), 32 experts per layer,
-    2 layers through a 12-slot cache; unrouted forward (routing read back to the
+    2 layers through a 20-slot cache (2 tokens need at most 17 experts); unrouted forward (routing read back to the
     host) and a check of one streamed token against the oracle."""
     from routed_expert_ffn_forward_b200.layer import layer_from_config
     cfg = dataclasses.replace(synth.CONFIGS[4], n_experts=32, n_layers=2, steps=6, seed=41)
     eb = moe.moe_expert_bytes(cfg.hidden, cfg.inter)
-    moe.moe_set_cache_bytes(12 * eb)
+    moe.moe_set_cache_bytes(20 * eb)
     try:
         layers = [layer_from_config(cfg, l) for l in range(cfg.n_layers)]
         moe.moe_reset_stats()
