@@ -119,6 +119,13 @@ void cache_free(Cache* c) {
 
 }  // namespace
 
+// Error reporting for entry points defined in other files of the library.
+int moe::report_error(int status, const char* msg) {
+  g_err = msg;
+  return status;
+}
+void moe::clear_error() { g_err.clear(); }
+
 struct moe_layer {
   uint32_t id = 0;
   int device = 0;

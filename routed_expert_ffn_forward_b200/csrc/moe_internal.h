@@ -61,6 +61,10 @@ struct PtrUpdate {
 cudaError_t launch_set_ptrs(const uint8_t** table, const PtrUpdate& u, size_t gate_bytes,
                             cudaStream_t st);
 
+// Set / clear the thread-local message returned by moe_last_error().
+int report_error(int status, const char* msg);
+void clear_error();
+
 // ---- device helpers -------------------------------------------------------
 #ifdef __CUDACC__
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }

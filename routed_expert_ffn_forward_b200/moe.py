@@ -34,7 +34,7 @@ EXPORTS = ("moe_expert_bytes", "moe_layer_create", "moe_layer_destroy", "moe_set
            "moe_set_experts", "moe_set_cache_bytes", "moe_forward", "moe_forward_routed",
            "moe_forward_host", "moe_get_routing", "moe_get_logits", "moe_prefetch",
            "moe_get_stats", "moe_reset_stats", "moe_set_profiling", "moe_get_profile",
-           "moe_reset_profile", "moe_last_error")
+           "moe_reset_profile", "moe_route_noalloc", "moe_last_error")
 
 KERNELS = ("router", "topk", "permute", "gate_up", "down", "combine", "forward")
 
@@ -93,6 +93,7 @@ def lib() -> ctypes.CDLL:
             "moe_set_profiling": (_I, [_I]),
             "moe_get_profile": (_I, [ctypes.POINTER(moe_profile)]),
             "moe_reset_profile": (_I, []),
+            "moe_route_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
             "moe_last_error": (ctypes.c_char_p, []),
         }
         for name, (res, args) in sig.items():
@@ -187,6 +188,11 @@ def moe_get_profile() -> dict:
 
 def moe_reset_profile() -> None:
     _check(lib().moe_reset_profile())
+
+
+def moe_route_noalloc(x: int, W: int, bias: int | None, T: int, H: int, E: int, top_k: int, gating: int,
+                      ids: int, weights: int, stream: int | None = None) -> None:
+    _check(lib().moe_route_noalloc(x, W, bias or None, T, H, E, top_k, gating, ids, weights, stream or None))
 
 
 def moe_last_error() -> str:
