@@ -177,6 +177,13 @@ moe_status moe_get_logits(moe_layer_t layer, float* logits, void* stream);
  * them ready.  A no-op for resident layers and for experts already cached. */
 moe_status moe_prefetch(moe_layer_t layer, const int32_t* ids, int n);
 
+/* Wait for all work on the layer's GPU, then report whether one of the layer's
+ * kernels gave up on a bounded wait (a shared-memory pipeline barrier that did
+ * not complete within its time limit; the kernel then stops early and its
+ * output is invalid).  Returns MOE_ERR_CUDA with a message in that case and
+ * clears the record; MOE_OK otherwise. */
+moe_status moe_check(moe_layer_t layer);
+
 moe_status moe_get_stats(moe_stats* out);
 moe_status moe_reset_stats(void);
 

@@ -3,6 +3,7 @@
 // then the shared experts, with no atomics: the result does not depend on
 // scheduling (LayerStoRm README, "Notes": a deterministic expert combine).
 #include "moe_internal.h"
+#include "ptx.cuh"
 
 namespace moe {
 namespace {
@@ -10,6 +11,9 @@ namespace {
 __global__ void combine_kernel(const float* __restrict__ y, const float* __restrict__ w,
                                const int* __restrict__ inv, int H, int k, int S,
                                __nv_bfloat16* __restrict__ out) {
+  // launched as a programmatic dependent of the down kernel on the decode path:
+  // wait for it (a no-op when launched normally)
+  ptx::pdl_wait();
   const int t = blockIdx.y;
   const int o = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (o >= H) return;
@@ -42,11 +46,24 @@ __global__ void combine_kernel(const float* __restrict__ y, const float* __restr
 
 }  // namespace
 
-cudaError_t launch_combine(const Work& wk, int T, const Shape& s, __nv_bfloat16* out, cudaStream_t st) {
+cudaError_t launch_combine(const Work& wk, int T, const Shape& s, __nv_bfloat16* out, cudaStream_t st, bool pdl) {
   const int threads = 128;
   dim3 grid((s.H / 4 + threads - 1) / threads, T);
-  combine_kernel<<<grid, threads, 0, st>>>(wk.y, wk.w, wk.inv, s.H, s.k, s.S, out);
-  return cudaGetLastError();
+  if (!pdl) {
+    combine_kernel<<<grid, threads, 0, st>>>(wk.y, wk.w, wk.inv, s.H, s.k, s.S, out);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, (const float*)wk.y, (const float*)wk.w, (const int*)wk.inv, s.H,
+                            s.k, s.S, out);
 }
 
 }  // namespace moe

@@ -81,8 +81,10 @@ struct Cache {
   std::unordered_map<uint64_t, int> where;
   cudaStream_t copy = nullptr;
   uint64_t epoch = 0;
+  uint64_t gen = 0;  // changes whenever the arena is (re)allocated
 };
 Cache* g_cache = nullptr;
+uint64_t g_cache_gen = 0;
 
 // Profiling: events recorded around each kernel of a forward (start/end pairs
 // for MOE_K_ROUTER..MOE_K_COMBINE), resolved by moe_get_profile.
@@ -138,6 +140,10 @@ struct moe_layer {
   std::vector<const uint8_t*> host;     // (E+S)*3 borrowed pinned pointers
   uint8_t* d_resident = nullptr;        // resident copy of all experts
   const uint8_t** d_wptr = nullptr;     // device table (E+S)*3 of weight pointers
+  CUtensorMap* d_tmaps = nullptr;       // [slots][3] TMA maps (resident: one slot per expert)
+  size_t n_tmap_slots = 0;
+  int* d_slot_of = nullptr;             // [E+S] expert -> slot of d_tmaps
+  uint64_t cache_gen = 0;               // streaming: cache arena the maps point into
   cudaStream_t copy = nullptr;          // resident uploads
   // scratch
   int T_cap = 0;
@@ -176,7 +182,11 @@ moe_status ensure_scratch(moe_layer* L, int T) {
                o_counts = take(ES * 4), o_offsets = take((ES + 1) * 4), o_perm = take(P * 4),
                o_inv = take(P * 4), o_act = take(ES * 4), o_nact = take(4), o_ticket = take(4),
                o_h = take(P * s.I_pad * 4), o_y = take(P * s.H * 4),
-               o_x = take((size_t)cap * s.H * 2), o_o = take((size_t)cap * s.H * 2);
+               o_x = take((size_t)cap * s.H * 2), o_o = take((size_t)cap * s.H * 2),
+               o_xq = take((size_t)cap * s.H * 2), o_xsc = take((size_t)cap * (s.H / 32) * 8),
+               o_hq = take(P * s.I_pad * 2), o_hsc = take(P * (s.I_pad / 32) * 8), o_act1 = take(ES * 4),
+               o_act2 = take(ES * 4), o_nact1 = take(4), o_nact2 = take(4), o_tcnt = take((size_t)(s.H / 64) * 4),
+               o_err = take(4);
   if (L->scratch) {
     CUDA_TRY(cudaDeviceSynchronize());
     cudaFree(L->scratch);
@@ -205,6 +215,18 @@ moe_status ensure_scratch(moe_layer* L, int T) {
   L->wk.y = reinterpret_cast<float*>(b + o_y);
   L->xbuf = reinterpret_cast<__nv_bfloat16*>(b + o_x);
   L->obuf = reinterpret_cast<__nv_bfloat16*>(b + o_o);
+  L->wk.xq = reinterpret_cast<int8_t*>(b + o_xq);
+  L->wk.xq_plane = (size_t)cap * s.H;
+  L->wk.xsc = reinterpret_cast<float2*>(b + o_xsc);
+  L->wk.hq = reinterpret_cast<int8_t*>(b + o_hq);
+  L->wk.hq_plane = P * s.I_pad;
+  L->wk.hsc = reinterpret_cast<float2*>(b + o_hsc);
+  L->wk.act1 = reinterpret_cast<int*>(b + o_act1);
+  L->wk.act2 = reinterpret_cast<int*>(b + o_act2);
+  L->wk.n_act1 = reinterpret_cast<int*>(b + o_nact1);
+  L->wk.n_act2 = reinterpret_cast<int*>(b + o_nact2);
+  L->wk.tile_cnt = reinterpret_cast<unsigned*>(b + o_tcnt);
+  L->wk.err = reinterpret_cast<unsigned*>(b + o_err);
   // zero everything once: the ticket must start at 0 and the padded columns of
   // h (I..I_pad) are never written and must read as 0
   CUDA_TRY(cudaMemset(L->scratch, 0, off));
@@ -249,6 +271,7 @@ moe_status ensure_cache(int device, size_t slot_bytes) {
     cache_free(c);
     return fail(MOE_ERR_CUDA, "cache setup: %s", cudaGetErrorString(e));
   }
+  c->gen = ++g_cache_gen;
   g_cache = c;
   g_stats.cache_slots = n;
   g_stats.slot_bytes = slot_bytes;
@@ -309,6 +332,36 @@ moe_status cache_fetch(moe_layer* L, int e, uint64_t pin_epoch, bool prefetch, i
   return MOE_OK;
 }
 
+// TMA maps for every slot the layer's experts can occupy: `n_slots` expert
+// images `stride` bytes apart from `arena`.
+moe_status build_maps(moe_layer* L, const uint8_t* arena, size_t stride, size_t n_slots) {
+  std::vector<CUtensorMap> maps(3 * n_slots);
+  for (size_t i = 0; i < n_slots; ++i) {
+    if (encode_expert_maps(&maps[3 * i], arena + i * stride, L->s.H, L->s.I) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for slot %zu", i);
+  }
+  if (L->n_tmap_slots < n_slots) {
+    if (L->d_tmaps) {
+      CUDA_TRY(cudaDeviceSynchronize());
+      cudaFree(L->d_tmaps);
+      L->d_tmaps = nullptr;
+      L->n_tmap_slots = 0;
+    }
+    CUDA_TRY(cudaMalloc(&L->d_tmaps, sizeof(CUtensorMap) * maps.size()));
+    L->n_tmap_slots = n_slots;
+  }
+  CUDA_TRY(cudaMemcpy(L->d_tmaps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice));
+  return MOE_OK;
+}
+
+// Streaming layers: point the maps at the current cache arena.  Caller holds g_mu.
+moe_status refresh_stream_maps(moe_layer* L) {
+  if (L->cache_gen == g_cache->gen) return MOE_OK;
+  MOE_TRY(build_maps(L, g_cache->arena, g_cache->slot_bytes, (size_t)g_cache->n_slots));
+  L->cache_gen = g_cache->gen;
+  return MOE_OK;
+}
+
 // Streaming: bring every expert a forward needs into the cache, make `st`
 // wait for their fills and point the device table at their slots.
 // Caller holds g_mu until the `used` events of these slots are recorded.
@@ -319,6 +372,7 @@ moe_status resolve_experts(moe_layer* L, const int32_t* ids, int n, cudaStream_t
   for (int i = 0; i < n; ++i) need[ids[i]] = 1;
   for (int j = 0; j < s.S; ++j) need[s.E + j] = 1;
   MOE_TRY(ensure_cache(L->device, L->expert_bytes));
+  MOE_TRY(refresh_stream_maps(L));
   Cache* c = g_cache;
   c->epoch++;
   PtrUpdate u{};
@@ -329,15 +383,16 @@ moe_status resolve_experts(moe_layer* L, const int32_t* ids, int n, cudaStream_t
     if (c->slots[slot].ready_rec) CUDA_TRY(cudaStreamWaitEvent(st, c->slots[slot].ready, 0));
     used_slots->push_back(slot);
     u.expert[u.n] = e;
+    u.slot[u.n] = slot;
     u.base[u.n] = c->arena + (size_t)slot * c->slot_bytes;
     if (++u.n == PtrUpdate::kMax) {
-      CUDA_TRY(launch_set_ptrs(L->d_wptr, u, L->gate_bytes, st));
+      CUDA_TRY(launch_set_ptrs(L->d_wptr, L->d_slot_of, u, L->gate_bytes, st));
       g_stats.launches++;
       u.n = 0;
     }
   }
   if (u.n) {
-    CUDA_TRY(launch_set_ptrs(L->d_wptr, u, L->gate_bytes, st));
+    CUDA_TRY(launch_set_ptrs(L->d_wptr, L->d_slot_of, u, L->gate_bytes, st));
     g_stats.launches++;
   }
   return MOE_OK;
@@ -381,11 +436,25 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     if (prof) pr.used[kid] = true;                               \
     ++n_launch;                                                  \
   } while (0)
-  MOE_KERNEL(MOE_K_ROUTER, launch_router_logits(xb, L->d_W, L->d_b, wk.logits, T, s.H, s.E, st));
+  // decode path (few tokens): kernels specialised for one row per expert when
+  // T == 1; activation slots of the down kernel must fit in shared memory
+  const int max_tok = T == 1 ? 1 : kD1MaxTok;
+  const size_t act_slot = (size_t)max_tok * (2 * (size_t)s.I_pad + (size_t)(s.I_pad / 32) * 8);
+  const size_t x_stage = 2 * (size_t)T * s.H + (size_t)T * (s.H / 32) * 8;
+  const bool stage_x = max_tok == 1 && gate_up_d1_smem(1, x_stage) <= kMaxDecodeSmem;
+  const bool fast = T <= kD1MaxTok && down_d1_smem(max_tok, act_slot) <= kMaxDecodeSmem;
   if (forced)
     CUDA_TRY(cudaMemcpyAsync(wk.forced, forced, (size_t)T * s.k * 4, cudaMemcpyHostToDevice, st));
-  MOE_KERNEL(MOE_K_TOPK, launch_topk(wk.logits, T, s.E, s.k, (int)L->gating, forced ? wk.forced : nullptr,
-                                     wk.ids, wk.w, st));
+  if (fast) {
+    RouteArgs ra{xb, L->d_W, L->d_b, forced ? wk.forced : nullptr, T, s.H, s.E, s.k, s.S, (int)L->gating,
+                 wk.logits, wk.ids, wk.w, wk.counts, wk.offsets, wk.perm, wk.inv, wk.act1, wk.n_act1, wk.act2,
+                 wk.n_act2, wk.n_act, wk.xq, wk.xq_plane, wk.xsc, wk.ticket};
+    MOE_KERNEL(MOE_K_ROUTER, launch_route_decode(ra, st));
+  } else {
+    MOE_KERNEL(MOE_K_ROUTER, launch_router_logits(xb, L->d_W, L->d_b, wk.logits, T, s.H, s.E, st));
+    MOE_KERNEL(MOE_K_TOPK, launch_topk(wk.logits, T, s.E, s.k, (int)L->gating, forced ? wk.forced : nullptr,
+                                       wk.ids, wk.w, st));
+  }
   // Streaming: the cache lock is held from resolving the experts until the
   // slots' `used` events are recorded, so no other forward can evict a slot
   // between this forward's fill-wait and its last read.
@@ -401,10 +470,48 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     lk.lock();
     MOE_TRY(resolve_experts(L, hid, T * s.k, st, &used));
   }
-  MOE_KERNEL(MOE_K_PERMUTE, launch_permute(wk.ids, T, s, wk, st));
-  MOE_KERNEL(MOE_K_GATE_UP, launch_gate_up_simt(L->d_wptr, xb, s, wk, st));
-  MOE_KERNEL(MOE_K_DOWN, launch_down_simt(L->d_wptr, s, wk, st));
-  MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st));
+  if (fast) {
+    DecodeArgs da{};
+    da.tmaps = L->d_tmaps;
+    da.slot_of = L->d_slot_of;
+    da.act = wk.act1;
+    da.n_act = wk.n_act1;
+    da.n_act_total = wk.n_act;
+    da.counts = wk.counts;
+    da.offsets = wk.offsets;
+    da.perm = wk.perm;
+    da.inv = wk.inv;
+    da.w = wk.w;
+    da.kS = s.k + s.S;
+    da.T = T;
+    da.k = s.k;
+    da.S = s.S;
+    da.H = s.H;
+    da.I = s.I;
+    da.I_pad = s.I_pad;
+    da.nbh = s.nbh;
+    da.nbi = s.nbi;
+    da.xq = wk.xq;
+    da.xq_plane = wk.xq_plane;
+    da.xsc = wk.xsc;
+    da.hq = wk.hq;
+    da.hq_plane = wk.hq_plane;
+    da.hsc = wk.hsc;
+    da.y = wk.y;
+    da.out = static_cast<__nv_bfloat16*>(out);
+    da.tile_cnt = wk.tile_cnt;
+    da.err = wk.err;
+    da.stage_x = stage_x ? 1 : 0;
+    da.act_slot_bytes = act_slot;
+    MOE_KERNEL(MOE_K_GATE_UP, launch_gate_up_d1(da, max_tok, s.n_sm, st));
+    MOE_KERNEL(MOE_K_DOWN, launch_down_d1(da, max_tok, s.n_sm, st));
+    MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true));
+  } else {
+    MOE_KERNEL(MOE_K_PERMUTE, launch_permute(wk.ids, T, s, wk, st));
+    MOE_KERNEL(MOE_K_GATE_UP, launch_gate_up_simt(L->d_wptr, xb, s, wk, st));
+    MOE_KERNEL(MOE_K_DOWN, launch_down_simt(L->d_wptr, s, wk, st));
+    MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st));
+  }
 #undef MOE_KERNEL
   {
     if (!lk.owns_lock()) lk.lock();
@@ -468,6 +575,8 @@ moe_status moe_layer_create(int hidden, int inter, int n_experts, int top_k, int
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&s.n_sm, cudaDevAttrMultiProcessorCount, L->device);
   if (e == cudaSuccess) e = cudaMalloc(&L->d_wptr, sizeof(void*) * 3 * (size_t)(s.E + s.S));
   if (e == cudaSuccess) e = cudaMemset(L->d_wptr, 0, sizeof(void*) * 3 * (size_t)(s.E + s.S));
+  if (e == cudaSuccess) e = cudaMalloc(&L->d_slot_of, sizeof(int) * (size_t)(s.E + s.S));
+  if (e == cudaSuccess) e = cudaMemset(L->d_slot_of, 0, sizeof(int) * (size_t)(s.E + s.S));
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->copy, cudaStreamNonBlocking);
   if (e != cudaSuccess) {
     moe_layer_destroy(L);
@@ -502,6 +611,8 @@ moe_status moe_layer_destroy(moe_layer_t L) {
   if (L->d_b) cudaFree(L->d_b);
   if (L->d_resident) cudaFree(L->d_resident);
   if (L->d_wptr) cudaFree(L->d_wptr);
+  if (L->d_tmaps) cudaFree(L->d_tmaps);
+  if (L->d_slot_of) cudaFree(L->d_slot_of);
   if (L->scratch) cudaFree(L->scratch);
   if (L->h_ids) cudaFreeHost(L->h_ids);
   if (L->copy) cudaStreamDestroy(L->copy);
@@ -574,6 +685,10 @@ moe_status moe_set_experts(moe_layer_t L, const void* const* gate, const void* c
     CUDA_TRY(cudaMemcpyAsync(L->d_wptr, table.data(), sizeof(void*) * table.size(), cudaMemcpyHostToDevice,
                              L->copy));
     CUDA_TRY(cudaStreamSynchronize(L->copy));
+    MOE_TRY(build_maps(L, L->d_resident, L->expert_bytes, (size_t)n));
+    std::vector<int> ident(n);
+    for (int e = 0; e < n; ++e) ident[e] = e;
+    CUDA_TRY(cudaMemcpy(L->d_slot_of, ident.data(), sizeof(int) * n, cudaMemcpyHostToDevice));
     L->resident = true;
   } else {
     if (L->d_resident) {
@@ -583,6 +698,8 @@ moe_status moe_set_experts(moe_layer_t L, const void* const* gate, const void* c
     }
     std::lock_guard<std::mutex> lk(g_mu);
     MOE_TRY(ensure_cache(L->device, L->expert_bytes));
+    L->cache_gen = 0;
+    MOE_TRY(refresh_stream_maps(L));
     L->resident = false;
   }
   L->experts_set = true;
@@ -665,6 +782,21 @@ moe_status moe_prefetch(moe_layer_t L, const int32_t* ids, int n) {
   for (int i = 0; i < n; ++i) {
     int slot;
     MOE_TRY(cache_fetch(L, ids[i], 0, true, &slot));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_check(moe_layer_t L) {
+  g_err.clear();
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "null layer");
+  MOE_TRY(check_device(L));
+  CUDA_TRY(cudaDeviceSynchronize());
+  if (!L->scratch) return MOE_OK;
+  unsigned flags = 0;
+  CUDA_TRY(cudaMemcpy(&flags, L->wk.err, sizeof flags, cudaMemcpyDeviceToHost));
+  if (flags) {
+    CUDA_TRY(cudaMemset(L->wk.err, 0, sizeof flags));
+    return fail(MOE_ERR_CUDA, "a kernel of this layer gave up waiting (flags 0x%x)", flags);
   }
   return MOE_OK;
 }

@@ -5,6 +5,7 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -14,6 +15,8 @@ namespace moe {
 constexpr int kQK = 256;        // weights per Q4_K super-block
 constexpr int kQBytes = 144;    // bytes per Q4_K super-block
 constexpr int kDecodeMaxT = 64; // T <= this takes the decode path
+constexpr int kD1MaxTok = 4;    // experts with <= this many rows use the per-sub-block decode kernels
+constexpr int kTileRows = 64;   // weight rows per decode work unit
 
 // Pointers to one layer's per-call scratch (device memory owned by the layer).
 struct Work {
@@ -30,7 +33,76 @@ struct Work {
   unsigned* ticket;   // [1] last-block-done counter of the permutation kernel
   float* h;           // [P, I_pad] SwiGLU activations, padded columns are zero
   float* y;           // [P, H] expert outputs
+  // decode path: activations as 16-bit fixed point per 32-element run,
+  // x = (256*hi + lo) * 2^-s, in two byte planes (hi s8, then lo u8), with
+  // (2^-s, sum of the represented values) per run
+  int8_t* xq;         // [2][T_cap, H]
+  size_t xq_plane;    // T_cap * H
+  float2* xsc;        // [T, H/32]
+  int8_t* hq;         // [2][P_cap, I_pad] SwiGLU output
+  size_t hq_plane;    // P_cap * I_pad
+  float2* hsc;        // [P, I_pad/32]
+  int* act1;          // experts with 1..kD1MaxTok rows
+  int* n_act1;
+  int* act2;          // experts with more rows
+  int* n_act2;
+  unsigned* tile_cnt; // [ceil(H/64)] finished expert units per output row tile
+  unsigned* err;      // device-side error flags (timeouts)
 };
+
+struct RouteArgs {
+  const __nv_bfloat16* x;
+  const float* W;
+  const float* b;
+  const int* forced;   // device [T, k] or null
+  int T, H, E, k, S, gating;
+  float* logits;
+  int *ids;
+  float* w;
+  int *counts, *offsets, *perm, *inv;
+  int *act1, *n_act1, *act2, *n_act2, *n_act;
+  int8_t* xq;
+  size_t xq_plane;
+  float2* xsc;
+  unsigned* ticket;
+};
+cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st);
+
+// Arguments of the decode expert kernels.
+struct DecodeArgs {
+  const CUtensorMap* tmaps;  // [slots][3] maps of gate, up, down (2-D, 8-byte elements)
+  const int* slot_of;        // [E+S] expert -> slot
+  const int* act;            // experts this kernel handles
+  const int* n_act;
+  const int* n_act_total;    // all experts with rows (units per output row tile)
+  const int *counts, *offsets, *perm, *inv;
+  const float* w;
+  int kS, T, k, S;
+  int H, I, I_pad, nbh, nbi;
+  const int8_t* xq;
+  size_t xq_plane;
+  const float2* xsc;
+  int8_t* hq;
+  size_t hq_plane;
+  float2* hsc;
+  float* y;
+  __nv_bfloat16* out;
+  unsigned* tile_cnt;
+  unsigned* err;
+  int stage_x;            // gate/up: copy x (all T tokens) to shared memory once per CTA
+  size_t act_slot_bytes;  // down: bytes of one activation slot (2 * max_tok * I_pad + scales)
+};
+constexpr size_t kMaxDecodeSmem = 227 * 1024;
+// max_tok: 1 (every expert has one row, T == 1) or kD1MaxTok
+cudaError_t launch_gate_up_d1(const DecodeArgs& a, int max_tok, int n_sm, cudaStream_t st);
+cudaError_t launch_down_d1(const DecodeArgs& a, int max_tok, int n_sm, cudaStream_t st);
+size_t gate_up_d1_smem(int max_tok, size_t x_stage_bytes);
+size_t down_d1_smem(int max_tok, size_t act_slot_bytes);
+
+// Tensor maps of one expert's Q4_K matrices at `base` (gate, up, down), boxes
+// of 64 rows x 2 (gate/up) or 4 (down) super-blocks.
+cudaError_t encode_expert_maps(CUtensorMap* maps3, const uint8_t* base, int H, int I);
+size_t route_decode_smem(int H, int T, int E, int k, int S);
 
 struct Shape {
   int H, I, E, k, S;
@@ -49,16 +121,18 @@ cudaError_t launch_permute(const int* ids, int T, const Shape& s, const Work& wk
 cudaError_t launch_gate_up_simt(const uint8_t* const* wptr, const __nv_bfloat16* x, const Shape& s,
                                 const Work& wk, cudaStream_t st);
 cudaError_t launch_down_simt(const uint8_t* const* wptr, const Shape& s, const Work& wk, cudaStream_t st);
-cudaError_t launch_combine(const Work& wk, int T, const Shape& s, __nv_bfloat16* out, cudaStream_t st);
+cudaError_t launch_combine(const Work& wk, int T, const Shape& s, __nv_bfloat16* out, cudaStream_t st,
+                           bool pdl = false);
 
 // Streaming cache: point experts at their cache slots (device pointer table).
 struct PtrUpdate {
   static constexpr int kMax = 64;
   int n;
   int expert[kMax];
+  int slot[kMax];
   const uint8_t* base[kMax];
 };
-cudaError_t launch_set_ptrs(const uint8_t** table, const PtrUpdate& u, size_t gate_bytes,
+cudaError_t launch_set_ptrs(const uint8_t** table, int* slot_of, const PtrUpdate& u, size_t gate_bytes,
                             cudaStream_t st);
 
 // Set / clear the thread-local message returned by moe_last_error().
@@ -84,6 +158,56 @@ __device__ __forceinline__ void q4k_scale_min(const uint8_t* sb, int j, int& sc,
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+
+// Called by a full warp with one value per lane (a 32-element run): writes
+// this lane's value as 16-bit fixed point x ~ (256*hi + lo) * 2^-s, with s
+// chosen so the run's largest magnitude lands in [2^13, 2^14), and returns in
+// run_sc (2^-s, sum of the represented values) of the run.
+__device__ __forceinline__ void quant_run16(float v, int8_t& hi, uint8_t& lo, float2& run_sc) {
+  float m = fabsf(v);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  int e = 0;
+  if (m > 0.f && m < 3.0e38f) e = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;
+  e = max(-100, min(100, e));
+  const float scale = __uint_as_float((uint32_t)(127 + 13 - e) << 23);
+  const float inv = __uint_as_float((uint32_t)(127 - 13 + e) << 23);
+  const int xi = __float2int_rn(v * scale);  // |xi| <= 2^14
+  hi = (int8_t)(xi >> 8);
+  lo = (uint8_t)(xi & 0xFF);
+  int s = xi;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  run_sc = make_float2(inv, (float)s * inv);
+}
+
+// Exclusive scan of one int per thread over a block of any size <= 1024;
+// returns the prefix and writes the block total.  s_warp: 32 ints of shared memory.
+__device__ __forceinline__ int block_exclusive_scan_1024(int v, int* total, int* s_warp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int wv = lane < nw ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, wv, o);
+      if (lane >= o) wv += n;
+    }
+    if (lane < nw) s_warp[lane] = wv;
+  }
+  __syncthreads();
+  const int before = warp ? s_warp[warp - 1] : 0;
+  *total = s_warp[nw - 1];
+  __syncthreads();
+  return before + incl - v;
+}
 #endif
 
 }  // namespace moe

@@ -25,7 +25,9 @@ __device__ __forceinline__ bool topk_better(const TopkCand& a, const TopkCand& b
 // experts in decreasing order and lane r keeps round r's pick.  With `forced`
 // (k ids) the picks are given.  Gating over the k picks: softmax (gating 0) or
 // sigmoid renormalised to sum 1 (gating 1).  Writes ids[0..k) and w[0..k).
-template <int PL>
+// kL2 reads the logits through L2 only (they were written by other CTAs of the
+// same kernel).
+template <int PL, bool kL2 = false>
 __device__ __forceinline__ void warp_topk_gate(const float* __restrict__ lt, int E, int k, int gating,
                                                const int* __restrict__ forced, int* __restrict__ ids,
                                                float* __restrict__ w) {
@@ -35,7 +37,7 @@ __device__ __forceinline__ void warp_topk_gate(const float* __restrict__ lt, int
   if (forced) {
     if (lane < k) {
       my_e = forced[lane];
-      my_l = lt[my_e];
+      my_l = kL2 ? __ldcg(lt + my_e) : lt[my_e];
     }
   } else {
     float v[PL];
@@ -44,7 +46,7 @@ __device__ __forceinline__ void warp_topk_gate(const float* __restrict__ lt, int
     for (int i = 0; i < PL; ++i) {
       const int e = lane + 32 * i;
       taken[i] = e >= E;
-      v[i] = taken[i] ? 0.f : lt[e];
+      v[i] = taken[i] ? 0.f : (kL2 ? __ldcg(lt + e) : lt[e]);
     }
     for (int r = 0; r < k; ++r) {
       TopkCand c{0.f, 0, false};

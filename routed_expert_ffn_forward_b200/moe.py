@@ -33,7 +33,7 @@ SIZE_MAX = (1 << 64) - 1
 EXPORTS = ("moe_expert_bytes", "moe_layer_create", "moe_layer_destroy", "moe_set_router",
            "moe_set_experts", "moe_set_cache_bytes", "moe_forward", "moe_forward_routed",
            "moe_forward_host", "moe_get_routing", "moe_get_logits", "moe_prefetch",
-           "moe_get_stats", "moe_reset_stats", "moe_set_profiling", "moe_get_profile",
+           "moe_check", "moe_get_stats", "moe_reset_stats", "moe_set_profiling", "moe_get_profile",
            "moe_reset_profile", "moe_route_noalloc", "moe_last_error")
 
 KERNELS = ("router", "topk", "permute", "gate_up", "down", "combine", "forward")
@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
             "moe_get_routing": (_I, [_P, _P, _P, _P]),
             "moe_get_logits": (_I, [_P, _P, _P]),
             "moe_prefetch": (_I, [_P, _P, _I]),
+            "moe_check": (_I, [_P]),
             "moe_get_stats": (_I, [ctypes.POINTER(moe_stats)]),
             "moe_reset_stats": (_I, []),
             "moe_set_profiling": (_I, [_I]),
@@ -164,6 +165,10 @@ def moe_get_logits(layer: int, logits: int, stream: int | None = None) -> None:
 
 def moe_prefetch(layer: int, ids_host: int, n: int) -> None:
     _check(lib().moe_prefetch(layer, ids_host, n))
+
+
+def moe_check(layer: int) -> None:
+    _check(lib().moe_check(layer))
 
 
 def moe_get_stats() -> dict:

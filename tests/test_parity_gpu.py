@@ -46,6 +46,7 @@ def run_gpu(torch, cfg, T, layer_index=0, layer=None):
     ids, w = L.routing(T)
     logits = L.logits(T)
     torch.cuda.synchronize()
+    moe.moe_check(L.handle)   # no kernel gave up on a bounded wait
     res = dict(x=x, out=to_bits(torch, out), ids=ids.cpu().numpy(), w=w.cpu().numpy(),
                logits=logits.cpu().numpy())
     if layer is None:
