@@ -450,6 +450,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
                  wk.logits, wk.ids, wk.w, wk.counts, wk.offsets, wk.perm, wk.inv, wk.act1, wk.n_act1, wk.act2,
                  wk.n_act2, wk.n_act, wk.xq, wk.xq_plane, wk.xsc, wk.ticket};
     MOE_KERNEL(MOE_K_ROUTER, launch_route_decode(ra, st));
+    ++n_launch;  // route = logits kernel + finishing kernel
   } else {
     MOE_KERNEL(MOE_K_ROUTER, launch_router_logits(xb, L->d_W, L->d_b, wk.logits, T, s.H, s.E, st));
     MOE_KERNEL(MOE_K_TOPK, launch_topk(wk.logits, T, s.E, s.k, (int)L->gating, forced ? wk.forced : nullptr,

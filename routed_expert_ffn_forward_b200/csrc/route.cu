@@ -1,14 +1,18 @@
-// Decode-path routing in one launch (T <= 64): router logits, top-k + gating,
-// the counting-sort permutation, the lists of active experts, and the fp16
-// fixed-point copy of x that the expert kernels read.
+// Decode-path routing (T <= 64): two kernels chained with programmatic
+// dependent launch.
 //
-// One CTA per expert computes that expert's logits for every token (all 1024
-// threads share the row, four tokens at a time).  Independently
-// of routing, every CTA also converts a slice of x: each 32-element run of x
-// becomes 16-bit fixed point with its own power-of-two scale, stored as a
-// high-byte and a low-byte plane, with the run's scale and sum.
-// The last CTA to finish (a ticket counter) does the top-k for all tokens and
-// the stable permutation in shared memory.
+// route_logits_kernel: one CTA per expert computes that expert's logits for
+// every token (256 threads share the row, four tokens at a time, partial sums
+// reduced in a fixed order).  Independently of routing, every CTA also
+// converts a slice of x: each 32-element run becomes 16-bit fixed point with
+// its own power-of-two scale (a high-byte and a low-byte plane), with the
+// run's scale and sum -- the form the expert kernels read.
+//
+// route_finish_kernel: one CTA does the top-k + gating of every token (a warp
+// per token) and the stable counting-sort permutation of the T*k picks.  With
+// few picks (N = T*k <= 2048) each pick's sorted position is found by counting
+// the picks before it in (expert, token, slot) order, so no pass over all E
+// expert counters is needed; only experts with rows get counts and offsets.
 #include "moe_internal.h"
 #include "ptx.cuh"
 #include "topk.cuh"
@@ -16,21 +20,19 @@
 namespace moe {
 namespace {
 
-constexpr int kRouteThreads = 256;
+constexpr int kLogitThreads = 256;
+constexpr int kFinishThreads = 256;
 
-
-template <int PL>
-__global__ void __launch_bounds__(kRouteThreads) route_decode_kernel(RouteArgs a) {
-  extern __shared__ float4 smem_f4[];
-  __shared__ float s_red[kRouteThreads / 32][4];
+__global__ void __launch_bounds__(kLogitThreads) route_logits_kernel(RouteArgs a) {
+  __shared__ float s_red[kLogitThreads / 32][4];
   const int e = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, T = a.T, E = a.E;
-  // the first kernel of a forward: let the expert kernel start launching now
+  // the first kernel of a forward: let the finishing kernel start launching now
   ptx::pdl_launch_dependents();
 
   // (1) x prep: 16-bit fixed point per 32-element run, with the run scales
   const int runs_per_tok = H / 32;
-  for (int run = e + gridDim.x * warp; run < T * runs_per_tok; run += gridDim.x * (kRouteThreads / 32)) {
+  for (int run = e + gridDim.x * warp; run < T * runs_per_tok; run += gridDim.x * (kLogitThreads / 32)) {
     const int t = run / runs_per_tok, r = run - t * runs_per_tok;
     const int h = r * 32 + lane;
     float2 rsc;
@@ -42,15 +44,14 @@ __global__ void __launch_bounds__(kRouteThreads) route_decode_kernel(RouteArgs a
     if (lane == 0) a.xsc[(size_t)t * runs_per_tok + r] = rsc;
   }
 
-  // (2) logits of expert e: every thread takes 4-element pieces of the row
-  // (h = 4*tid + 4096*i) for up to 4 tokens at a time; partial sums are
-  // reduced in a fixed order (warp xor tree, then warps in index order).
+  // (2) logits of expert e: thread takes 4-element pieces h = 4*tid + 1024*i
   const float4* wrow = reinterpret_cast<const float4*>(a.W + (size_t)e * H);
   const float bias = a.b ? a.b[e] : 0.f;
   for (int t0 = 0; t0 < T; t0 += 4) {
     const int nt = min(4, T - t0);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int q = tid; q < H / 4; q += kRouteThreads) {
+#pragma unroll 4
+    for (int q = tid; q < H / 4; q += kLogitThreads) {
       const float4 w4 = __ldg(wrow + q);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -72,110 +73,127 @@ __global__ void __launch_bounds__(kRouteThreads) route_decode_kernel(RouteArgs a
     __syncthreads();
     if (warp == 0 && lane < nt) {
       float v = 0.f;
-      for (int w = 0; w < kRouteThreads / 32; ++w) v += s_red[w][lane];
+#pragma unroll
+      for (int w = 0; w < kLogitThreads / 32; ++w) v += s_red[w][lane];
       a.logits[(size_t)(t0 + lane) * E + e] = v + bias;
     }
     __syncthreads();
   }
+}
 
-  // (4) the last CTA finishes the routing
-  __shared__ bool s_last;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  const int k = a.k, S = a.S, kS = k + S, N = T * k, ES = E + S;
-  int* s_ids = reinterpret_cast<int*>(smem_f4);   // [N]
-  float* s_wt = reinterpret_cast<float*>(s_ids + N);
-  int* s_cnt = reinterpret_cast<int*>(s_wt + N);  // [ES]
-  int* s_off = s_cnt + ES;                        // [ES + 1]
-  __shared__ int s_scan[32];
-  __syncthreads();
-
-  // top-k + gating, one warp per token (logits read from L2: other CTAs wrote them)
-  for (int t = warp; t < T; t += kRouteThreads / 32)
-    warp_topk_gate<PL, true>(a.logits + (size_t)t * E, E, k, a.gating, a.forced ? a.forced + (size_t)t * k : nullptr,
-                             s_ids + (size_t)t * k, s_wt + (size_t)t * k);
-  for (int i = tid; i < ES; i += kRouteThreads) s_cnt[i] = i < E ? 0 : T;
-  __syncthreads();
-  for (int i = tid; i < N; i += kRouteThreads) {
-    atomicAdd(&s_cnt[s_ids[i]], 1);
-    a.ids[i] = s_ids[i];
-    a.w[i] = s_wt[i];
-  }
-  __syncthreads();
-  // exclusive scan of the counts (routed experts, then shared) and the active lists
-  int base = 0, base1 = 0, base2 = 0;
-  for (int c0 = 0; c0 < ES; c0 += kRouteThreads) {
-    const int i = c0 + tid;
-    const int cnt = i < ES ? s_cnt[i] : 0;
-    const int small = (cnt > 0 && cnt <= kD1MaxTok) ? 1 : 0, big = cnt > kD1MaxTok ? 1 : 0;
-    // three scans share s_scan: do them one after another
-    int tot;
-    const int pre = block_exclusive_scan_1024(cnt, &tot, s_scan);
-    if (i < ES) {
-      s_off[i] = base + pre;
-      a.counts[i] = cnt;
-      a.offsets[i] = base + pre;
-    }
-    base += tot;
-    const int p1 = block_exclusive_scan_1024(small, &tot, s_scan);
-    if (small) a.act1[base1 + p1] = i;
-    base1 += tot;
-    const int p2 = block_exclusive_scan_1024(big, &tot, s_scan);
-    if (big) a.act2[base2 + p2] = i;
-    base2 += tot;
-  }
+template <int PL>
+__global__ void __launch_bounds__(kFinishThreads) route_finish_kernel(RouteArgs a) {
+  extern __shared__ int s_ids[];          // [N]
+  __shared__ int s_cnt_small, s_cnt_big;  // distinct routed experts with <= / > kD1MaxTok rows
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int T = a.T, E = a.E, k = a.k, S = a.S, kS = k + S, N = T * k;
+  int* s_first = s_ids + N;               // [N] 1 if pick i is its expert's first pick
+  int* s_count = s_first + N;             // [N] rows of pick i's expert
+  ptx::pdl_wait();                        // the logits
+  ptx::pdl_launch_dependents();
   if (tid == 0) {
-    a.offsets[ES] = base;
-    *a.n_act1 = base1;
-    *a.n_act2 = base2;
-    *a.n_act = base1 + base2;
+    s_cnt_small = 0;
+    s_cnt_big = 0;
+  }
+  // top-k + gating, one warp per token
+  for (int t = warp; t < T; t += kFinishThreads / 32)
+    warp_topk_gate<PL, true>(a.logits + (size_t)t * E, E, k, a.gating, a.forced ? a.forced + (size_t)t * k : nullptr,
+                             s_ids + t * k, a.w + (size_t)t * k);
+  __syncthreads();
+  // per pick: rows of its expert, whether it is the expert's first pick
+  for (int i = tid; i < N; i += kFinishThreads) {
+    const int ex = s_ids[i];
+    int cnt = 0, before = 0;
+    for (int j = 0; j < N; ++j) {
+      const int kj = s_ids[j];
+      cnt += kj == ex;
+      before += (kj == ex) & (j < i);
+    }
+    s_first[i] = before == 0;
+    s_count[i] = cnt;
+    a.ids[i] = ex;
   }
   __syncthreads();
-  // stable scatter: rank of pick i among the earlier picks of the same expert
-  for (int i = tid; i < N; i += kRouteThreads) {
+  // sorted positions: picks of smaller experts first, then earlier picks of
+  // the same expert; first picks also place their expert in the active lists
+  for (int i = tid; i < N; i += kFinishThreads) {
     const int ex = s_ids[i];
-    int rank = 0;
-    for (int j = 0; j < i; ++j) rank += s_ids[j] == ex;
+    int lt = 0, eq_before = 0, d_small = 0, d_big = 0;
+    for (int j = 0; j < N; ++j) {
+      const int kj = s_ids[j];
+      lt += kj < ex;
+      eq_before += (kj == ex) & (j < i);
+      const bool distinct_lt = (kj < ex) & (s_first[j] != 0);
+      d_small += distinct_lt & (s_count[j] <= kD1MaxTok);
+      d_big += distinct_lt & (s_count[j] > kD1MaxTok);
+    }
     const int t = i / k, j = i - t * k;
-    const int r = s_off[ex] + rank;
+    const int r = lt + eq_before;
     a.perm[r] = t * kS + j;
     a.inv[t * kS + j] = r;
+    if (s_first[i]) {
+      a.counts[ex] = s_count[i];
+      a.offsets[ex] = lt;
+      if (s_count[i] <= kD1MaxTok) {
+        a.act1[d_small] = ex;
+        atomicAdd(&s_cnt_small, 1);
+      } else {
+        a.act2[d_big] = ex;
+        atomicAdd(&s_cnt_big, 1);
+      }
+    }
   }
-  for (int i = tid; i < T * S; i += kRouteThreads) {
+  // shared experts: all T tokens, after the routed rows
+  for (int i = tid; i < T * S; i += kFinishThreads) {
     const int s = i / T, t = i - s * T;
     const int r = N + s * T + t;
     a.perm[r] = t * kS + k + s;
     a.inv[t * kS + k + s] = r;
   }
-  if (tid == 0) *a.ticket = 0u;
+  __syncthreads();
+  if (tid < S) {
+    const int ex = E + tid;
+    a.counts[ex] = T;
+    a.offsets[ex] = N + tid * T;
+    if (T <= kD1MaxTok)
+      a.act1[s_cnt_small + tid] = ex;
+    else
+      a.act2[s_cnt_big + tid] = ex;
+  }
+  if (tid == 0) {
+    const int n1 = s_cnt_small + (T <= kD1MaxTok ? S : 0), n2 = s_cnt_big + (T <= kD1MaxTok ? 0 : S);
+    *a.n_act1 = n1;
+    *a.n_act2 = n2;
+    *a.n_act = n1 + n2;
+    a.offsets[E + S] = T * kS;
+  }
 }
 
 }  // namespace
 
 size_t route_decode_smem(int H, int T, int E, int k, int S) {
   (void)H;
-  return (size_t)T * k * 8 + (size_t)(E + S) * 4 + (size_t)(E + S + 1) * 4;
+  (void)E;
+  (void)S;
+  return (size_t)T * k * 3 * sizeof(int);
 }
 
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st) {
-  const size_t smem = route_decode_smem(a.H, a.T, a.E, a.k, a.S);
-  const int pl = (a.E + 31) / 32;
-  cudaError_t err;
-  if (pl <= 8) {
-    err = cudaFuncSetAttribute(route_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    route_decode_kernel<8><<<a.E, kRouteThreads, smem, st>>>(a);
-  } else {
-    err = cudaFuncSetAttribute(route_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    route_decode_kernel<32><<<a.E, kRouteThreads, smem, st>>>(a);
-  }
-  return cudaGetLastError();
+  route_logits_kernel<<<a.E, kLogitThreads, 0, st>>>(a);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kFinishThreads);
+  cfg.dynamicSmemBytes = route_decode_smem(a.H, a.T, a.E, a.k, a.S);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if ((a.E + 31) / 32 <= 8) return cudaLaunchKernelEx(&cfg, route_finish_kernel<8>, a);
+  return cudaLaunchKernelEx(&cfg, route_finish_kernel<32>, a);
 }
 
 }  // namespace moe
