@@ -339,15 +339,15 @@ def run_ours(args, cfg, rank: int, world: int, local_rank: int) -> dict | None:
     fwd_bytes = float(np.mean([algorithmic_bytes(cfg, ids, "forward") for ids in ids_cycle]))
     fwd_ms = total_ms / args.steps
     kernels = {k: {"avg_us": 1e3 * prof["ms"][k] / max(1, prof["launches"][k]),
-                   "share": prof["ms"][k] / max(1e-12, sum(prof["ms"][q] for q in moe.KERNELS[:6]))}
-               for k in moe.KERNELS[:6]}
+                   "share": prof["ms"][k] / max(1e-12, sum(prof["ms"][q] for q in moe.KERNELS[:-1]))}
+               for k in moe.KERNELS[:-1]}
     if args.config == 3:
         metric, unit = "moe_layer_prefill_tokens_per_s", "tokens/s"
     else:
         metric, unit = "moe_layer_decode_tokens_per_s", "tokens/s"
     res = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": fwd_ms, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "bf16" if cfg.tokens <= 4 else "f32", "data": "synthetic",
+           "vs_baseline": None, "dtype": "int8" if cfg.tokens <= 4 else "f16", "data": "synthetic",
            "config": config_json(cfg, args), "roofline": roof,
            "forward_hbm": {"algorithmic_bytes": fwd_bytes, "achieved_gbs": fwd_bytes / (fwd_ms / 1e3) / 1e9,
                            "frac": fwd_bytes / (fwd_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
@@ -413,7 +413,7 @@ def run_streaming(args, cfg, rank, world, local_rank, peaks) -> dict:
     lookups = st["cache_hits"] + st["cache_misses"]
     return {"metric": "moe_streaming_decode_tokens_per_s", "value": args.steps * world / secs, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": config_json(cfg, args),
             "roofline": {"bound": "h2d", "achieved": h2d_gbs, "peak": h2d_peak, "unit": "GB/s",
                          "frac": h2d_gbs / h2d_peak, "traffic": None,

@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
       uint32_t phase = 0;
       for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
         const int ai = unit / tiles, rt = unit - ai * tiles;
-        const CUtensorMap* mg = a.tmaps + 3 * __ldcg(a.slot_of + __ldcg(a.act + ai));
+        const CUtensorMap* mg = a.tmaps + kMapsPerSlot * __ldcg(a.slot_of + __ldcg(a.act + ai));
         for (int st = 0; st < n_st; ++st) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
             flag_error(a.err, 1u);
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) down_d1_kernel(DecodeArgs a) {
       for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
         const int ai = unit / tiles, rt = unit - ai * tiles;
         const int e = __ldcg(a.act + ai);
-        const CUtensorMap* md = a.tmaps + 3 * __ldcg(a.slot_of + e) + 2;
+        const CUtensorMap* md = a.tmaps + kMapsPerSlot * __ldcg(a.slot_of + e) + 2;
         // weights first: they do not depend on the gate/up kernel
         for (int st = 0; st < n_st; ++st) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {

@@ -86,12 +86,13 @@ struct Cache {
 Cache* g_cache = nullptr;
 uint64_t g_cache_gen = 0;
 
-// Profiling: events recorded around each kernel of a forward (start/end pairs
-// for MOE_K_ROUTER..MOE_K_COMBINE), resolved by moe_get_profile.
-constexpr int kProfKernels = MOE_K_FORWARD;  // kernels with their own pair
+// Profiling: events recorded around each kernel launch of a forward, in launch
+// order, each range attributed to one MOE_K_* step; resolved by moe_get_profile.
+constexpr int kProfRanges = 12;              // launches per forward at most
 struct ProfRec {
-  cudaEvent_t ev[2 * kProfKernels];
-  bool used[kProfKernels];
+  int n = 0;
+  int kid[kProfRanges];
+  cudaEvent_t ev[2 * kProfRanges];
 };
 bool g_profiling = false;
 std::vector<ProfRec> g_prof_pending;
@@ -140,7 +141,7 @@ struct moe_layer {
   std::vector<const uint8_t*> host;     // (E+S)*3 borrowed pinned pointers
   uint8_t* d_resident = nullptr;        // resident copy of all experts
   const uint8_t** d_wptr = nullptr;     // device table (E+S)*3 of weight pointers
-  CUtensorMap* d_tmaps = nullptr;       // [slots][3] TMA maps (resident: one slot per expert)
+  CUtensorMap* d_tmaps = nullptr;       // [slots][kMapsPerSlot] TMA maps (resident: one slot per expert)
   size_t n_tmap_slots = 0;
   int* d_slot_of = nullptr;             // [E+S] expert -> slot of d_tmaps
   uint64_t cache_gen = 0;               // streaming: cache arena the maps point into
@@ -153,6 +154,7 @@ struct moe_layer {
   __nv_bfloat16* obuf = nullptr;
   int32_t* h_ids = nullptr;             // pinned, for reading routing back
   int last_T = 0;
+  CUtensorMap x16_map{}, h16_map{};     // B operands of the prefill GEMMs (over the scratch)
 };
 
 namespace {
@@ -186,7 +188,9 @@ moe_status ensure_scratch(moe_layer* L, int T) {
                o_xq = take((size_t)cap * s.H * 2), o_xsc = take((size_t)cap * (s.H / 32) * 8),
                o_hq = take(P * s.I_pad * 2), o_hsc = take(P * (s.I_pad / 32) * 8), o_act1 = take(ES * 4),
                o_act2 = take(ES * 4), o_nact1 = take(4), o_nact2 = take(4), o_tcnt = take((size_t)(s.H / 64) * 4),
-               o_err = take(4);
+               o_err = take(4), o_tiles = take(prefill_max_tiles((int)ES, P) * 16), o_ntiles = take(4),
+               o_x16 = take(P * s.H * 2), o_rinv = take(P * 4), o_h16 = take(P * s.I_pad * 2), o_hinv = take(P * 4),
+               o_hmax = take(P * 4);
   if (L->scratch) {
     CUDA_TRY(cudaDeviceSynchronize());
     cudaFree(L->scratch);
@@ -227,8 +231,18 @@ moe_status ensure_scratch(moe_layer* L, int T) {
   L->wk.n_act2 = reinterpret_cast<int*>(b + o_nact2);
   L->wk.tile_cnt = reinterpret_cast<unsigned*>(b + o_tcnt);
   L->wk.err = reinterpret_cast<unsigned*>(b + o_err);
-  // zero everything once: the ticket must start at 0 and the padded columns of
-  // h (I..I_pad) are never written and must read as 0
+  L->wk.tiles = reinterpret_cast<int4*>(b + o_tiles);
+  L->wk.n_tiles = reinterpret_cast<int*>(b + o_ntiles);
+  L->wk.x16 = reinterpret_cast<__half*>(b + o_x16);
+  L->wk.rinv = reinterpret_cast<float*>(b + o_rinv);
+  L->wk.h16 = reinterpret_cast<__half*>(b + o_h16);
+  L->wk.hinv = reinterpret_cast<float*>(b + o_hinv);
+  L->wk.hmax = reinterpret_cast<unsigned*>(b + o_hmax);
+  if (encode_act16(&L->x16_map, L->wk.x16, P, s.H) != cudaSuccess ||
+      encode_act16(&L->h16_map, L->wk.h16, P, s.I_pad) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activation maps");
+  // zero everything once: the ticket and hmax must start at 0 and the padded
+  // columns of h (I..I_pad) are never written and must read as 0
   CUDA_TRY(cudaMemset(L->scratch, 0, off));
   CUDA_TRY(cudaDeviceSynchronize());
   L->T_cap = cap;
@@ -335,9 +349,9 @@ moe_status cache_fetch(moe_layer* L, int e, uint64_t pin_epoch, bool prefetch, i
 // TMA maps for every slot the layer's experts can occupy: `n_slots` expert
 // images `stride` bytes apart from `arena`.
 moe_status build_maps(moe_layer* L, const uint8_t* arena, size_t stride, size_t n_slots) {
-  std::vector<CUtensorMap> maps(3 * n_slots);
+  std::vector<CUtensorMap> maps(kMapsPerSlot * n_slots);
   for (size_t i = 0; i < n_slots; ++i) {
-    if (encode_expert_maps(&maps[3 * i], arena + i * stride, L->s.H, L->s.I) != cudaSuccess)
+    if (encode_expert_maps(&maps[kMapsPerSlot * i], arena + i * stride, L->s.H, L->s.I) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for slot %zu", i);
   }
   if (L->n_tmap_slots < n_slots) {
@@ -425,16 +439,19 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     std::lock_guard<std::mutex> lk0(g_mu);
     prof = g_profiling;
     if (prof)
-      for (int i = 0; i < 2 * kProfKernels; ++i) pr.ev[i] = prof_event();
+      for (int i = 0; i < 2 * kProfRanges; ++i) pr.ev[i] = prof_event();
   }
   int n_launch = 0;
-#define MOE_KERNEL(kid, call)                                    \
-  do {                                                           \
-    if (prof) CUDA_TRY(cudaEventRecord(pr.ev[2 * (kid)], st));   \
-    CUDA_TRY(call);                                              \
-    if (prof) CUDA_TRY(cudaEventRecord(pr.ev[2 * (kid) + 1], st)); \
-    if (prof) pr.used[kid] = true;                               \
-    ++n_launch;                                                  \
+#define MOE_KERNEL(k_id, call)                                          \
+  do {                                                                  \
+    const bool rec_ = prof && pr.n < kProfRanges;                       \
+    if (rec_) CUDA_TRY(cudaEventRecord(pr.ev[2 * pr.n], st));           \
+    CUDA_TRY(call);                                                     \
+    if (rec_) {                                                         \
+      CUDA_TRY(cudaEventRecord(pr.ev[2 * pr.n + 1], st));               \
+      pr.kid[pr.n++] = (k_id);                                          \
+    }                                                                   \
+    ++n_launch;                                                         \
   } while (0)
   // decode path (few tokens): kernels specialised for one row per expert when
   // T == 1; activation slots of the down kernel must fit in shared memory
@@ -450,7 +467,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
                  wk.logits, wk.ids, wk.w, wk.counts, wk.offsets, wk.perm, wk.inv, wk.act1, wk.n_act1, wk.act2,
                  wk.n_act2, wk.n_act, wk.xq, wk.xq_plane, wk.xsc, wk.ticket};
     MOE_KERNEL(MOE_K_ROUTER, launch_route_decode(ra, st));
-    ++n_launch;  // route = logits kernel + finishing kernel
+    ++n_launch;  // route = logits kernel + finishing kernel (one profiled range)
   } else {
     MOE_KERNEL(MOE_K_ROUTER, launch_router_logits(xb, L->d_W, L->d_b, wk.logits, T, s.H, s.E, st));
     MOE_KERNEL(MOE_K_TOPK, launch_topk(wk.logits, T, s.E, s.k, (int)L->gating, forced ? wk.forced : nullptr,
@@ -508,10 +525,34 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     MOE_KERNEL(MOE_K_DOWN, launch_down_d1(da, max_tok, s.n_sm, st));
     MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true));
   } else {
+    // prefill: tensor-core GEMMs over tiles of up to 256 rows of one expert
+    const int kS = s.k + s.S, P = T * kS;
     MOE_KERNEL(MOE_K_PERMUTE, launch_permute(wk.ids, T, s, wk, st));
-    MOE_KERNEL(MOE_K_GATE_UP, launch_gate_up_simt(L->d_wptr, xb, s, wk, st));
-    MOE_KERNEL(MOE_K_DOWN, launch_down_simt(L->d_wptr, s, wk, st));
-    MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st));
+    MOE_KERNEL(MOE_K_PERMUTE, launch_build_tiles(wk, st));
+    MOE_KERNEL(MOE_K_PREP, launch_gather_rows(xb, wk, P, kS, s.H, st));
+    GemmArgs ga{};
+    ga.wmaps = L->d_tmaps;
+    ga.slot_of = L->d_slot_of;
+    ga.tiles = wk.tiles;
+    ga.n_tiles = wk.n_tiles;
+    ga.ft = (s.I + 127) / 128;
+    ga.nkb = s.nbh;
+    ga.rinv = wk.rinv;
+    ga.out = wk.h;
+    ga.out_ld = s.I_pad;
+    ga.out_rows = s.I;
+    ga.hmax = wk.hmax;
+    ga.err = wk.err;
+    MOE_KERNEL(MOE_K_GATE_UP, launch_prefill_gemm(0, L->x16_map, ga, s.n_sm, st));
+    MOE_KERNEL(MOE_K_PREP, launch_convert_h(wk, P, s.I, s.I_pad, st));
+    ga.ft = s.H / 256;
+    ga.nkb = s.nbi;
+    ga.rinv = wk.hinv;
+    ga.out = wk.y;
+    ga.out_ld = s.H;
+    ga.out_rows = s.H;
+    MOE_KERNEL(MOE_K_DOWN, launch_prefill_gemm(1, L->h16_map, ga, s.n_sm, st));
+    MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true));
   }
 #undef MOE_KERNEL
   {
@@ -797,7 +838,11 @@ moe_status moe_check(moe_layer_t L) {
   CUDA_TRY(cudaMemcpy(&flags, L->wk.err, sizeof flags, cudaMemcpyDeviceToHost));
   if (flags) {
     CUDA_TRY(cudaMemset(L->wk.err, 0, sizeof flags));
-    return fail(MOE_ERR_CUDA, "a kernel of this layer gave up waiting (flags 0x%x)", flags);
+    return fail(MOE_ERR_CUDA,
+                "%s (flags 0x%x)",
+                (flags & 0xFFu) || (flags & ~0x1FFu) ? "a kernel of this layer gave up waiting"
+                                                      : "a Q4_K weight exceeds the fp16 range of the prefill GEMMs",
+                flags);
   }
   return MOE_OK;
 }
@@ -837,24 +882,20 @@ moe_status moe_get_profile(moe_profile* out) {
   }
   moe_status st = MOE_OK;
   for (auto& r : recs) {
-    int first = -1, last = -1;
-    for (int kid = 0; kid < kProfKernels; ++kid) {
-      if (!r.used[kid]) continue;
-      if (first < 0) first = kid;
-      last = kid;
+    for (int i = 0; i < r.n; ++i) {
       float ms = 0.f;
-      cudaError_t e = cudaEventSynchronize(r.ev[2 * kid + 1]);
-      if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.ev[2 * kid], r.ev[2 * kid + 1]);
+      cudaError_t e = cudaEventSynchronize(r.ev[2 * i + 1]);
+      if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.ev[2 * i], r.ev[2 * i + 1]);
       if (e != cudaSuccess) {
         st = fail(MOE_ERR_CUDA, "profile events: %s", cudaGetErrorString(e));
         continue;
       }
-      out->ms[kid] += ms;
-      out->launches[kid]++;
+      out->ms[r.kid[i]] += ms;
+      out->launches[r.kid[i]]++;
     }
-    if (first >= 0) {
+    if (r.n > 0) {
       float ms = 0.f;
-      if (cudaEventElapsedTime(&ms, r.ev[2 * first], r.ev[2 * last + 1]) == cudaSuccess) {
+      if (cudaEventElapsedTime(&ms, r.ev[0], r.ev[2 * r.n - 1]) == cudaSuccess) {
         out->ms[MOE_K_FORWARD] += ms;
         out->launches[MOE_K_FORWARD]++;
       }

@@ -48,6 +48,14 @@ struct Work {
   int* n_act2;
   unsigned* tile_cnt; // [ceil(H/64)] finished expert units per output row tile
   unsigned* err;      // device-side error flags (timeouts)
+  // prefill path (tensor-core GEMMs)
+  int4* tiles;        // [max tiles] (expert, n0, count, r0): up to 256 rows of one expert
+  int* n_tiles;
+  __half* x16;        // [P_cap, H] activations of each row, fp16 scaled by 1/rinv, K order (0,2,1,3)
+  float* rinv;        // [P]
+  __half* h16;        // [P_cap, I_pad] SwiGLU output, fp16 scaled by 1/hinv, same K order
+  float* hinv;        // [P]
+  unsigned* hmax;     // [P] max |h| of each row (float bits), reset after use
 };
 
 struct RouteArgs {
@@ -70,7 +78,7 @@ cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st);
 
 // Arguments of the decode expert kernels.
 struct DecodeArgs {
-  const CUtensorMap* tmaps;  // [slots][3] maps of gate, up, down (2-D, 8-byte elements)
+  const CUtensorMap* tmaps;  // [slots][kMapsPerSlot] maps of gate, up, down (2-D, 8-byte elements)
   const int* slot_of;        // [E+S] expert -> slot
   const int* act;            // experts this kernel handles
   const int* n_act;
@@ -99,9 +107,36 @@ cudaError_t launch_down_d1(const DecodeArgs& a, int max_tok, int n_sm, cudaStrea
 size_t gate_up_d1_smem(int max_tok, size_t x_stage_bytes);
 size_t down_d1_smem(int max_tok, size_t act_slot_bytes);
 
-// Tensor maps of one expert's Q4_K matrices at `base` (gate, up, down), boxes
-// of 64 rows x 2 (gate/up) or 4 (down) super-blocks.
-cudaError_t encode_expert_maps(CUtensorMap* maps3, const uint8_t* base, int H, int I);
+// Tensor maps of one expert's Q4_K matrices at `base`, kMapsPerSlot of them:
+// [0..2] gate, up, down with boxes of 64 rows x 2 (gate/up) or 4 (down)
+// super-blocks (decode kernels); [3..5] gate, up, down with boxes of 128 rows x
+// 1 super-block (prefill GEMMs).
+constexpr int kMapsPerSlot = 6;
+cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, int H, int I);
+// 2-D map over a row-major fp16 matrix [rows, cols] with 128B-swizzled boxes
+// of 256 rows x 64 columns (cols a multiple of 64).
+cudaError_t encode_act16(CUtensorMap* map, const __half* base, size_t rows, int cols);
+
+// Prefill GEMMs (tcgen05): mode 0 gate/up -> h (+ hmax), mode 1 down -> y.
+struct GemmArgs {
+  const CUtensorMap* wmaps;  // [slots][kMapsPerSlot]
+  const int* slot_of;        // [E+S] expert -> slot
+  const int4* tiles;
+  const int* n_tiles;
+  int ft;                    // feature blocks per tile: ceil(I/128) (mode 0), H/256 (mode 1)
+  int nkb;                   // super-blocks along K: H/256 (mode 0), I_pad/256 (mode 1)
+  const float* rinv;         // [P] inverse activation scale of each row
+  float* out;                // h [P, I_pad] or y [P, H]
+  int out_ld, out_rows;      // row pitch (floats); features stored (mode 0: I)
+  unsigned* hmax;            // mode 0
+  unsigned* err;
+};
+size_t prefill_gemm_smem();
+size_t prefill_max_tiles(int n_experts_total, size_t pairs);
+cudaError_t launch_build_tiles(const Work& wk, cudaStream_t st);
+cudaError_t launch_gather_rows(const __nv_bfloat16* x, const Work& wk, int P, int kS, int H, cudaStream_t st);
+cudaError_t launch_convert_h(const Work& wk, int P, int I, int I_pad, cudaStream_t st);
+cudaError_t launch_prefill_gemm(int mode, const CUtensorMap& bmap, const GemmArgs& a, int n_sm, cudaStream_t st);
 size_t route_decode_smem(int H, int T, int E, int k, int S);
 
 struct Shape {

@@ -1,0 +1,551 @@
+// Prefill path (T > 4): grouped GEMMs on the 5th-generation tensor cores
+// (tcgen05.mma, fp32 accumulators in tensor memory) over Q4_K weights.
+//
+// A work unit is (tile, feature block): a tile is up to 256 consecutive rows
+// of one expert in the expert-sorted order, a feature block 256 weight rows
+// (gate/up: 128 gate rows + the same 128 up rows; down: 256 output rows).
+// The weights are the A operand as two M = 128 halves, the tile's activation
+// rows the B operand (N <= 256), so one dequantisation of a weight tile
+// serves up to 256 rows and the two accumulators fill all 512 TMEM columns.
+//
+//   warp 0      producer of raw Q4_K tiles (2-D TMA, 128 rows x 1 super-block)
+//   warp 1      producer of activation tiles (2-D TMA, 128B-swizzled fp16,
+//               256 rows x 64 columns)
+//   warp 2      TMEM allocation; one thread issues tcgen05.mma M128 N<=256 K16
+//               and tcgen05.commit
+//   warps 3-6   dequantise Q4_K to fp16 straight into the UMMA 128B-swizzled
+//               K-major layout, one weight row per thread
+//   warps 7-14  epilogue: tcgen05.ld of the accumulators (a warp reads the TMEM
+//               lane quarter warp % 4; two warps per quarter split the columns)
+//
+// Numerics: activations are fp16 scaled per row by a power of two (largest
+// magnitude in [2^14, 2^15), 1/scale kept in `rinv`); weights are fp16 scaled
+// by 2^8 (sub-block scale and min rounded to fp16, one rounding per weight);
+// products accumulate in fp32 and the epilogue undoes both scales.  A weight
+// that would not fit fp16 after the 2^8 scale sets error bit 256.
+//
+// K order: within every group of four K elements both operands are stored in
+// the order (0, 2, 1, 3), so two quant nibbles of one 32-bit word become one
+// fp16x2 register without byte shuffles; the dot product is unchanged.
+#include "moe_internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kGM = 128;                       // rows of one A half (MMA M)
+constexpr int kGN = 256;                       // activation rows per tile (max MMA N)
+constexpr int kRawBytes = kGM * kQBytes;       // one A half, one super-block: 18432
+constexpr int kABytes = kGM * 64 * 2;          // one A half, 64 K as fp16: 16384
+constexpr int kBBytes = kGN * 64 * 2;          // 256 rows x 64 K as fp16: 32768
+constexpr int kNR = 2;                         // raw super-block stages
+constexpr int kNS = 2;                         // A/B stages (64 K each)
+constexpr int kDeqWarps = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kFirstDeq = 3, kFirstEpi = kFirstDeq + kDeqWarps;
+constexpr int kGemmThreads = (kFirstEpi + kEpiWarps) * 32;  // 480
+constexpr float kWScale = 256.f, kWScaleInv = 1.f / 256.f;
+constexpr float kWMax = 60000.f;               // largest |weight| * 2^8 accepted
+
+constexpr size_t kSmemRaw = (size_t)kNR * 2 * kRawBytes;
+constexpr size_t kSmemA = (size_t)kNS * 2 * kABytes;
+constexpr size_t kSmemB = (size_t)kNS * kBBytes;
+constexpr size_t kSmemBar = 8 * (2 * kNR + 3 * kNS + 2 + 1) + 16;
+constexpr size_t kGemmSmem = 1024 + kSmemRaw + kSmemA + kSmemB + kSmemBar;
+static_assert(kGemmSmem <= 227 * 1024, "GEMM shared memory");
+
+// Scales (d*sc) and mins (dmin*m) of sub-blocks 2c (lo) and 2c+1 (hi) of a
+// Q4_K block whose first 16 bytes are `hdr` (fp16 d, fp16 dmin, 12 scale bytes).
+__device__ __forceinline__ void block_scales(uint4 hdr, int c, float& s_lo, float& s_hi, float& m_lo,
+                                             float& m_hi) {
+  const float d = __half2float(__ushort_as_half((unsigned short)(hdr.x & 0xFFFFu)));
+  const float dmin = __half2float(__ushort_as_half((unsigned short)(hdr.x >> 16)));
+  const uint32_t sh = 16u * (uint32_t)(c & 1);
+  const uint32_t s0 = hdr.y >> sh, s1 = hdr.z >> sh, s2 = hdr.w >> sh;
+  uint32_t vsc, vm;
+  if (c < 2) {
+    vsc = s0 & 0x3F3Fu;
+    vm = s1 & 0x3F3Fu;
+  } else {
+    vsc = (s2 & 0x0F0Fu) | ((s0 >> 2) & 0x3030u);
+    vm = ((s2 >> 4) & 0x0F0Fu) | ((s1 >> 2) & 0x3030u);
+  }
+  s_lo = d * (float)(vsc & 0xFFu);
+  s_hi = d * (float)((vsc >> 8) & 0xFFu);
+  m_lo = dmin * (float)(vm & 0xFFu);
+  m_hi = dmin * (float)((vm >> 8) & 0xFFu);
+}
+
+// fp16x2 (1024 + a, 1024 + b) -> (a * s - m, b * s - m), `nm` = -m
+__device__ __forceinline__ uint32_t deq2(uint32_t t, __half2 s, __half2 nm) {
+  const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&t), __float2half2_rn(1024.f));
+  const __half2 v = __hfma2(q, s, nm);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* raw) {
+  const uint32_t pad = (1024u - (ptx::smem_u32(raw) & 1023u)) & 1023u;
+  return raw + pad;
+}
+
+// Column-wise max over the 32 lanes of a warp: v[i] is this lane's value of
+// column i; the result (v[0] afterwards) is the max of column `lane`.
+// Reduce-scatter butterfly: 31 shuffles instead of 32 x 5.
+__device__ __forceinline__ float colmax32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < o; ++j) {
+      const float send = up ? v[j] : v[j + o];
+      const float keep = up ? v[j + o] : v[j];
+      v[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+    }
+  }
+  return v[0];
+}
+
+// kMode 0: gate/up, out = h (fp32 [P, ld]) = silu(g) * u, hmax[pair] = max |h|.
+// kMode 1: down,    out = y (fp32 [P, ld]).
+template <int kMode>
+__global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
+                                                                    const GemmArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint8_t* s_rawbuf = sm;                       // [kNR][2][kRawBytes]
+  uint8_t* s_a = s_rawbuf + kSmemRaw;           // [kNS][2][kABytes]
+  uint8_t* s_b = s_a + kSmemA;                  // [kNS][kBBytes]
+  uint64_t* raw_full = reinterpret_cast<uint64_t*>(s_b + kSmemB);
+  uint64_t* raw_empty = raw_full + kNR;
+  uint64_t* a_full = raw_empty + kNR;
+  uint64_t* b_full = a_full + kNS;
+  uint64_t* ab_empty = b_full + kNS;
+  uint64_t* acc_full = ab_empty + kNS;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNR; ++i) {
+      ptx::mbar_init(&raw_full[i], 1);
+      ptx::mbar_init(&raw_empty[i], kDeqWarps);
+    }
+    for (int i = 0; i < kNS; ++i) {
+      ptx::mbar_init(&a_full[i], kDeqWarps);
+      ptx::mbar_init(&b_full[i], 1);
+      ptx::mbar_init(&ab_empty[i], 1);
+    }
+    ptx::mbar_init(acc_full, 1);
+    ptx::mbar_init(acc_empty, kEpiWarps);
+    ptx::mbar_init(drain, 1);
+    ptx::fence_barrier_init();
+  }
+  if (warp == 2) ptx::tmem_alloc(s_tmem, 512);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  ptx::pdl_wait();  // tiles, activations and scales of the previous kernels
+  ptx::pdl_launch_dependents();
+
+  const int ft = a.ft;
+  const int n_units = __ldcg(a.n_tiles) * ft;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ raw weight tiles
+    if (lane == 0) {
+      int rs = 0;
+      uint32_t rph = 0, issued = 0, last_ph = 0;
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const int4 tl = __ldcg(a.tiles + u / ft);  // (expert, n0, count, r0)
+        const int f = u % ft;
+        const CUtensorMap* wm = a.wmaps + kMapsPerSlot * __ldcg(a.slot_of + tl.x) + 3;
+        const CUtensorMap* m0 = kMode == 0 ? wm : wm + 2;
+        const CUtensorMap* m1 = kMode == 0 ? wm + 1 : wm + 2;
+        const int y0 = kMode == 0 ? f * kGM : f * 2 * kGM;
+        const int y1 = kMode == 0 ? f * kGM : f * 2 * kGM + kGM;
+        for (int kb = 0; kb < a.nkb; ++kb) {
+          if (!ptx::mbar_wait(&raw_empty[rs], rph ^ 1u)) {
+            atomicOr(a.err, 16u);
+            goto raw_drain;
+          }
+          ptx::mbar_arrive_expect_tx(&raw_full[rs], 2 * kRawBytes);
+          ptx::tma_load_2d(s_rawbuf + (2 * rs) * kRawBytes, m0, kb * 18, y0, &raw_full[rs]);
+          ptx::tma_load_2d(s_rawbuf + (2 * rs + 1) * kRawBytes, m1, kb * 18, y1, &raw_full[rs]);
+          issued |= 1u << rs;
+          last_ph = (last_ph & ~(1u << rs)) | (rph << rs);
+          if (++rs == kNR) { rs = 0; rph ^= 1u; }
+        }
+      }
+    raw_drain:
+      // never leave with a copy into shared memory in flight
+      for (int i = 0; i < kNR; ++i)
+        if ((issued >> i) & 1u) ptx::mbar_wait(&raw_full[i], (last_ph >> i) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ activation tiles
+    if (lane == 0) {
+      int bs = 0;
+      uint32_t bph = 0, issued = 0, last_ph = 0;
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const int4 tl = __ldcg(a.tiles + u / ft);
+        const int row = tl.w + tl.y;
+        for (int kb = 0; kb < a.nkb; ++kb) {
+          for (int s = 0; s < 4; ++s) {
+            if (!ptx::mbar_wait(&ab_empty[bs], bph ^ 1u)) {
+              atomicOr(a.err, 16u);
+              goto b_drain;
+            }
+            ptx::mbar_arrive_expect_tx(&b_full[bs], kBBytes);
+            ptx::tma_load_2d(s_b + bs * kBBytes, &bmap, kb * 256 + s * 64, row, &b_full[bs]);
+            issued |= 1u << bs;
+            last_ph = (last_ph & ~(1u << bs)) | (bph << bs);
+            if (++bs == kNS) { bs = 0; bph ^= 1u; }
+          }
+        }
+      }
+    b_drain:
+      for (int i = 0; i < kNS; ++i)
+        if ((issued >> i) & 1u) ptx::mbar_wait(&b_full[i], (last_ph >> i) & 1u);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int as = 0;
+      uint32_t aph = 0, eph = 0;
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const int4 tl = __ldcg(a.tiles + u / ft);
+        const uint32_t idesc = ptx::umma_idesc_f16(kGM, min(kGN, (tl.z + 15) & ~15));
+        if (!ptx::mbar_wait(acc_empty, eph ^ 1u)) {
+          atomicOr(a.err, 32u);
+          break;
+        }
+        eph ^= 1u;
+        ptx::tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < a.nkb && ok; ++kb) {
+          for (int s = 0; s < 4; ++s) {
+            if (!ptx::mbar_wait(&a_full[as], aph) || !ptx::mbar_wait(&b_full[as], aph)) {
+              atomicOr(a.err, 32u);
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t a0 = ptx::smem_u32(s_a + (2 * as) * kABytes);
+            const uint32_t b0 = ptx::smem_u32(s_b + as * kBBytes);
+#pragma unroll
+            for (int k16 = 0; k16 < 4; ++k16) {
+              const uint64_t bd = ptx::umma_desc_sw128(b0 + 32 * k16);
+              const bool acc = (kb | s | k16) != 0;
+              ptx::umma_f16(tmem, ptx::umma_desc_sw128(a0 + 32 * k16), bd, idesc, acc);
+              ptx::umma_f16(tmem + kGN, ptx::umma_desc_sw128(a0 + kABytes + 32 * k16), bd, idesc, acc);
+            }
+            ptx::umma_commit(&ab_empty[as]);
+            if (++as == kNS) { as = 0; aph ^= 1u; }
+          }
+        }
+        if (!ok) break;
+        ptx::umma_commit(acc_full);
+      }
+      // wait for every MMA this thread issued before TMEM is released
+      ptx::umma_commit(drain);
+      if (!ptx::mbar_wait(drain, 0)) atomicOr(a.err, 32u);
+    }
+  } else if (warp < kFirstEpi) {
+    // ------------------------------------------------------------ dequantisers
+    const int r = threadIdx.x - kFirstDeq * 32;  // weight row of each A half, 0..127
+    int rs = 0, as = 0;
+    uint32_t rph = 0, aph = 0;
+    bool bad = false;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      for (int kb = 0; kb < a.nkb; ++kb) {
+        if (!ptx::mbar_wait(&raw_full[rs], rph)) {
+          atomicOr(a.err, 64u);
+          goto done;
+        }
+        for (int s = 0; s < 4; ++s) {
+          if (!ptx::mbar_wait(&ab_empty[as], aph ^ 1u)) {
+            atomicOr(a.err, 64u);
+            goto done;
+          }
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            const uint8_t* row = s_rawbuf + (2 * rs + m) * kRawBytes + r * kQBytes;
+            const uint4 hdr = *reinterpret_cast<const uint4*>(row);
+            const uint4 qa = *reinterpret_cast<const uint4*>(row + 16 + 32 * s);
+            const uint4 qb = *reinterpret_cast<const uint4*>(row + 32 + 32 * s);
+            float s_lo, s_hi, m_lo, m_hi;
+            block_scales(hdr, s, s_lo, s_hi, m_lo, m_hi);
+            bad |= !(fmaxf(15.f * fmaxf(s_lo, s_hi), fmaxf(m_lo, m_hi)) * kWScale < kWMax);
+            const __half2 sl = __float2half2_rn(s_lo * kWScale), nl = __float2half2_rn(-m_lo * kWScale);
+            const __half2 sh = __float2half2_rn(s_hi * kWScale), nh = __float2half2_rn(-m_hi * kWScale);
+            const uint32_t w[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+            uint8_t* arow = s_a + (2 * as + m) * kABytes + r * 128;
+            // low nibbles: K 0..31 (chunks 0..3), high nibbles: K 32..63 (chunks 4..7)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t w0 = w[2 * j], w1 = w[2 * j + 1];
+              uint4 lo, hi;
+              lo.x = deq2((w0 & 0x000F000Fu) | 0x64006400u, sl, nl);
+              lo.y = deq2(((w0 >> 8) & 0x000F000Fu) | 0x64006400u, sl, nl);
+              lo.z = deq2((w1 & 0x000F000Fu) | 0x64006400u, sl, nl);
+              lo.w = deq2(((w1 >> 8) & 0x000F000Fu) | 0x64006400u, sl, nl);
+              hi.x = deq2(((w0 >> 4) & 0x000F000Fu) | 0x64006400u, sh, nh);
+              hi.y = deq2(((w0 >> 12) & 0x000F000Fu) | 0x64006400u, sh, nh);
+              hi.z = deq2(((w1 >> 4) & 0x000F000Fu) | 0x64006400u, sh, nh);
+              hi.w = deq2(((w1 >> 12) & 0x000F000Fu) | 0x64006400u, sh, nh);
+              *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = lo;
+              *reinterpret_cast<uint4*>(arow + (((j + 4) ^ (r & 7)) << 4)) = hi;
+            }
+          }
+          ptx::fence_proxy_async();  // generic-proxy stores -> visible to the tensor cores
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&a_full[as]);
+          if (++as == kNS) { as = 0; aph ^= 1u; }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&raw_empty[rs]);
+        if (++rs == kNR) { rs = 0; rph ^= 1u; }
+      }
+    }
+    if (bad) atomicOr(a.err, 256u);
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                      // TMEM lane quarter this warp may read
+    const int half = (warp - kFirstEpi) >> 2;    // which 32-column chunks
+    const int mrow = q * 32 + lane;              // row of the A halves
+    uint32_t fph = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      const int4 tl = __ldcg(a.tiles + u / ft);
+      const int f = u % ft;
+      const bool ok = ptx::mbar_wait(acc_full, fph);
+      __syncwarp();
+      if (!ok) {
+        atomicOr(a.err, 128u);
+        goto done;
+      }
+      fph ^= 1u;
+      ptx::tc_fence_after();
+      const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+      const int pair0 = tl.w + tl.y;
+      for (int c0 = 32 * half; c0 < tl.z; c0 += 64) {
+        float v0[32], v1[32];
+        ptx::tmem_ld32(tq + c0, v0);
+        ptx::tmem_ld32(tq + kGN + c0, v1);
+        const int nc = min(32, tl.z - c0);
+        if (kMode == 0) {
+          const int feat = f * kGM + mrow;
+          const bool frow = feat < a.out_rows;
+          float* outp = a.out + (size_t)(pair0 + c0) * a.out_ld + feat;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float inv = __ldg(a.rinv + pair0 + c0 + min(i, nc - 1)) * kWScaleInv;
+            const float hv = silu_f(v0[i] * inv) * (v1[i] * inv);
+            if (i < nc && frow) outp[(size_t)i * a.out_ld] = hv;
+            v0[i] = (i < nc && frow) ? fabsf(hv) : 0.f;
+          }
+          const float mx = colmax32(v0, lane);
+          if (lane < nc) atomicMax(a.hmax + pair0 + c0 + lane, __float_as_uint(mx));
+        } else {
+          const int orow = f * 2 * kGM + mrow;
+          float* outp = a.out + (size_t)(pair0 + c0) * a.out_ld + orow;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (i < nc) {
+              const float inv = __ldg(a.rinv + pair0 + c0 + i) * kWScaleInv;
+              outp[(size_t)i * a.out_ld] = v0[i] * inv;
+              outp[(size_t)i * a.out_ld + kGM] = v1[i] * inv;
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(acc_empty);
+    }
+  }
+done:
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- helper kernels
+// Tiles: each expert with rows, in chunks of kGN rows: (expert, n0, count, r0).
+// One block; experts are taken 1024 at a time with a block scan of their tile counts.
+__global__ void __launch_bounds__(1024) build_tiles_kernel(const int* __restrict__ act, const int* __restrict__ n_act,
+                                                           const int* __restrict__ counts,
+                                                           const int* __restrict__ offsets, int4* __restrict__ tiles,
+                                                           int* __restrict__ n_tiles) {
+  __shared__ int s_warp[32];
+  ptx::pdl_wait();
+  const int na = __ldcg(n_act);
+  int base = 0;
+  for (int c0 = 0; c0 < na; c0 += blockDim.x) {
+    const int i = c0 + threadIdx.x;
+    int e = 0, c = 0, r0 = 0, nt = 0;
+    if (i < na) {
+      e = __ldcg(act + i);
+      c = __ldcg(counts + e);
+      r0 = __ldcg(offsets + e);
+      nt = (c + kGN - 1) / kGN;
+    }
+    int tot;
+    const int pos = base + block_exclusive_scan_1024(nt, &tot, s_warp);
+    for (int j = 0; j < nt; ++j) tiles[pos + j] = make_int4(e, j * kGN, min(kGN, c - j * kGN), r0);
+    base += tot;
+  }
+  if (threadIdx.x == 0) *n_tiles = base;
+}
+
+// Power of two p with max * p in [2^14, 2^15) (1 for max == 0 or not finite); *inv = 1/p.
+__device__ __forceinline__ float row_scale(float mx, float* inv) {
+  int e = 0;
+  if (mx > 0.f && mx < 3.0e38f) e = (int)((__float_as_uint(mx) >> 23) & 0xFFu) - 127;
+  e = max(-110, min(110, e));
+  *inv = __uint_as_float((uint32_t)(127 - 14 + e) << 23);
+  return __uint_as_float((uint32_t)(127 + 14 - e) << 23);
+}
+
+__device__ __forceinline__ float block_max(float m, float* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float v = s_red[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) v = fmaxf(v, s_red[w]);
+  return v;
+}
+
+// 4 floats -> 4 fp16 in the order (0, 2, 1, 3)
+__device__ __forceinline__ uint2 pack4_swz(float a0, float a1, float a2, float a3) {
+  const __half2 p = __floats2half2_rn(a0, a2), q = __floats2half2_rn(a1, a3);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(&p), *reinterpret_cast<const uint32_t*>(&q));
+}
+
+constexpr int kRowThreads = 256;
+constexpr int kRowMaxVec = 16;  // 4-element vectors per thread: rows up to 16384
+
+// Row r of the expert-sorted order: token perm[r] / kS of x as scaled fp16 (x16[r, :]), rinv[r] = 1/scale.
+__global__ void __launch_bounds__(kRowThreads) gather_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                  const int* __restrict__ perm, int kS, int H,
+                                                                  __half* __restrict__ x16,
+                                                                  float* __restrict__ rinv) {
+  __shared__ float s_red[kRowThreads / 32];
+  ptx::pdl_wait();
+  const int r = blockIdx.x;
+  const uint2* src = reinterpret_cast<const uint2*>(x + (size_t)(__ldg(perm + r) / kS) * H);
+  uint2 v[kRowMaxVec];
+  float m = 0.f;
+  const int nv = H / 4;
+#pragma unroll
+  for (int j = 0; j < kRowMaxVec; ++j) {
+    const int c = threadIdx.x + j * kRowThreads;
+    v[j] = c < nv ? __ldg(src + c) : make_uint2(0u, 0u);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(v[j].x)), fabsf(bf16hi(v[j].x))),
+                       fmaxf(fabsf(bf16lo(v[j].y)), fabsf(bf16hi(v[j].y)))));
+  }
+  float inv;
+  const float sc = row_scale(block_max(m, s_red), &inv);
+  uint2* dst = reinterpret_cast<uint2*>(x16 + (size_t)r * H);
+#pragma unroll
+  for (int j = 0; j < kRowMaxVec; ++j) {
+    const int c = threadIdx.x + j * kRowThreads;
+    if (c < nv)
+      dst[c] = pack4_swz(bf16lo(v[j].x) * sc, bf16hi(v[j].x) * sc, bf16lo(v[j].y) * sc, bf16hi(v[j].y) * sc);
+  }
+  if (threadIdx.x == 0) rinv[r] = inv;
+}
+
+// h (fp32 [P, I_pad], columns >= I unwritten) -> scaled fp16 h16 with zero
+// padding, hinv[r] = 1/scale from hmax[r]; hmax[r] is reset for the next forward.
+__global__ void __launch_bounds__(kRowThreads) convert_h_kernel(const float* __restrict__ h,
+                                                                unsigned* __restrict__ hmax, int I, int I_pad,
+                                                                __half* __restrict__ h16,
+                                                                float* __restrict__ hinv) {
+  __shared__ float s_sc[2];
+  ptx::pdl_wait();
+  const int r = blockIdx.x;
+  if (threadIdx.x == 0) {
+    float inv;
+    s_sc[0] = row_scale(__uint_as_float(__ldcg(hmax + r)), &inv);
+    s_sc[1] = inv;
+    hmax[r] = 0u;
+  }
+  __syncthreads();
+  const float sc = s_sc[0];
+  const float4* src = reinterpret_cast<const float4*>(h + (size_t)r * I_pad);
+  uint2* dst = reinterpret_cast<uint2*>(h16 + (size_t)r * I_pad);
+  for (int c = threadIdx.x; c < I_pad / 4; c += kRowThreads) {
+    float4 f = __ldcg(src + c);
+    const int i = 4 * c;
+    if (i + 3 >= I) {
+      f.x = i < I ? f.x : 0.f;
+      f.y = i + 1 < I ? f.y : 0.f;
+      f.z = i + 2 < I ? f.z : 0.f;
+      f.w = 0.f;
+    }
+    dst[c] = pack4_swz(f.x * sc, f.y * sc, f.z * sc, f.w * sc);
+  }
+  if (threadIdx.x == 0) hinv[r] = s_sc[1];
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+}  // namespace
+
+size_t prefill_gemm_smem() { return kGemmSmem; }
+
+size_t prefill_max_tiles(int n_experts_total, size_t pairs) { return (size_t)n_experts_total + pairs / kGN + 1; }
+
+cudaError_t launch_build_tiles(const Work& wk, cudaStream_t st) {
+  return launch_pdl(build_tiles_kernel, dim3(1), dim3(1024), 0, st, (const int*)wk.act, (const int*)wk.n_act,
+                    (const int*)wk.counts, (const int*)wk.offsets, wk.tiles, wk.n_tiles);
+}
+
+cudaError_t launch_gather_rows(const __nv_bfloat16* x, const Work& wk, int P, int kS, int H, cudaStream_t st) {
+  if (H / 4 > kRowThreads * kRowMaxVec) return cudaErrorInvalidValue;
+  return launch_pdl(gather_rows_kernel, dim3(P), dim3(kRowThreads), 0, st, x, (const int*)wk.perm, kS, H, wk.x16,
+                    wk.rinv);
+}
+
+cudaError_t launch_convert_h(const Work& wk, int P, int I, int I_pad, cudaStream_t st) {
+  return launch_pdl(convert_h_kernel, dim3(P), dim3(kRowThreads), 0, st, (const float*)wk.h, wk.hmax, I, I_pad,
+                    wk.h16, wk.hinv);
+}
+
+cudaError_t launch_prefill_gemm(int mode, const CUtensorMap& bmap, const GemmArgs& a, int n_sm, cudaStream_t st) {
+  static uint64_t attr_done[2] = {0, 0};  // per mode, one bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  auto kern = mode == 0 ? q4k_gemm_kernel<0> : q4k_gemm_kernel<1>;
+  if (!(attr_done[mode & 1] & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
+    if (e != cudaSuccess) return e;
+    attr_done[mode & 1] |= bit;
+  }
+  return launch_pdl(kern, dim3(n_sm), dim3(kGemmThreads), kGemmSmem, st, bmap, a);
+}
+
+}  // namespace moe

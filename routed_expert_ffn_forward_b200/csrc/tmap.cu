@@ -2,8 +2,10 @@
 //
 // A matrix of R rows and nb super-blocks per row is viewed as a 2-D array of
 // 8-byte elements, nb*18 wide and R high (row pitch nb*144 bytes, a multiple
-// of 16).  A box is 64 rows by SB super-blocks (SB*18 elements, SB*144 bytes);
-// boxes past the last row or block read zeros, which decode to zero weights.
+// of 16).  A box is 64 or 128 rows by SB super-blocks (SB*18 elements, SB*144
+// bytes); boxes past the last row or block read zeros, which decode to zero
+// weights.  Activation matrices of the prefill GEMMs are fp16 [rows, cols]
+// with 128-byte-swizzled boxes of 256 rows x 64 columns.
 #include <mutex>
 
 #include "moe_internal.h"
@@ -28,12 +30,12 @@ EncodeFn encode_fn() {
   return fn;
 }
 
-cudaError_t encode_q4k(CUtensorMap* m, const uint8_t* base, int rows, int nb, int box_blocks) {
+cudaError_t encode_q4k(CUtensorMap* m, const uint8_t* base, int rows, int nb, int box_blocks, int box_rows) {
   EncodeFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   const cuuint64_t dims[2] = {(cuuint64_t)nb * 18, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)nb * kQBytes};
-  const cuuint32_t box[2] = {(cuuint32_t)box_blocks * 18, (cuuint32_t)kTileRows};
+  const cuuint32_t box[2] = {(cuuint32_t)box_blocks * 18, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -43,13 +45,29 @@ cudaError_t encode_q4k(CUtensorMap* m, const uint8_t* base, int rows, int nb, in
 
 }  // namespace
 
-cudaError_t encode_expert_maps(CUtensorMap* maps3, const uint8_t* base, int H, int I) {
+cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, int H, int I) {
   const int nbh = H / kQK, nbi = (I + kQK - 1) / kQK;
   const size_t gate_bytes = (size_t)I * nbh * kQBytes;
-  cudaError_t e = encode_q4k(&maps3[0], base, I, nbh, 2);
-  if (e == cudaSuccess) e = encode_q4k(&maps3[1], base + gate_bytes, I, nbh, 2);
-  if (e == cudaSuccess) e = encode_q4k(&maps3[2], base + 2 * gate_bytes, H, nbi, 4);
+  const uint8_t* mats[3] = {base, base + gate_bytes, base + 2 * gate_bytes};
+  const int rows[3] = {I, I, H}, nb[3] = {nbh, nbh, nbi};
+  cudaError_t e = cudaSuccess;
+  for (int m = 0; m < 3 && e == cudaSuccess; ++m) e = encode_q4k(&maps[m], mats[m], rows[m], nb[m], m < 2 ? 2 : 4, kTileRows);
+  for (int m = 0; m < 3 && e == cudaSuccess; ++m) e = encode_q4k(&maps[3 + m], mats[m], rows[m], nb[m], 1, 128);
   return e;
+}
+
+cudaError_t encode_act16(CUtensorMap* map, const __half* base, size_t rows, int cols) {
+  EncodeFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  if (cols % 64 || rows == 0) return cudaErrorInvalidValue;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 256};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 }  // namespace moe

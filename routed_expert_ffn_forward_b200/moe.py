@@ -36,7 +36,7 @@ EXPORTS = ("moe_expert_bytes", "moe_layer_create", "moe_layer_destroy", "moe_set
            "moe_check", "moe_get_stats", "moe_reset_stats", "moe_set_profiling", "moe_get_profile",
            "moe_reset_profile", "moe_route_noalloc", "moe_last_error")
 
-KERNELS = ("router", "topk", "permute", "gate_up", "down", "combine", "forward")
+KERNELS = ("router", "topk", "permute", "gate_up", "down", "combine", "prep", "forward")
 
 
 class moe_stats(ctypes.Structure):
@@ -49,7 +49,8 @@ class moe_stats(ctypes.Structure):
 
 
 class moe_profile(ctypes.Structure):
-    _fields_ = [("forwards", ctypes.c_uint64), ("ms", ctypes.c_double * 7), ("launches", ctypes.c_uint64 * 7)]
+    _fields_ = [("forwards", ctypes.c_uint64), ("ms", ctypes.c_double * len(KERNELS)),
+                ("launches", ctypes.c_uint64 * len(KERNELS))]
 
     def as_dict(self) -> dict:
         return {"forwards": int(self.forwards),
