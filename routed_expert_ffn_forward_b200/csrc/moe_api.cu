@@ -138,6 +138,8 @@ struct moe_layer {
   bool router_set = false, experts_set = false, resident = false;
   float* d_W = nullptr;
   float* d_b = nullptr;
+  __nv_bfloat16* d_Wp = nullptr;        // router weight as three bf16 planes [3][E][H]
+  CUtensorMap wp_map{};                 // over d_Wp, for the tensor-core router
   std::vector<const uint8_t*> host;     // (E+S)*3 borrowed pinned pointers
   uint8_t* d_resident = nullptr;        // resident copy of all experts
   const uint8_t** d_wptr = nullptr;     // device table (E+S)*3 of weight pointers
@@ -190,7 +192,7 @@ moe_status ensure_scratch(moe_layer* L, int T) {
                o_act2 = take(ES * 4), o_nact1 = take(4), o_nact2 = take(4), o_tcnt = take((size_t)(s.H / 64) * 4),
                o_err = take(4), o_tiles = take(prefill_max_tiles((int)ES, P) * 16), o_ntiles = take(4),
                o_x16 = take(P * s.H * 2), o_rinv = take(P * 4), o_h16 = take(P * s.I_pad * 2), o_hinv = take(P * 4),
-               o_hmax = take(P * 4);
+               o_hmax = take(P * 4), o_rpart = take(router_part_floats(cap, s.E, s.n_sm) * 4);
   if (L->scratch) {
     CUDA_TRY(cudaDeviceSynchronize());
     cudaFree(L->scratch);
@@ -238,6 +240,7 @@ moe_status ensure_scratch(moe_layer* L, int T) {
   L->wk.h16 = reinterpret_cast<__half*>(b + o_h16);
   L->wk.hinv = reinterpret_cast<float*>(b + o_hinv);
   L->wk.hmax = reinterpret_cast<unsigned*>(b + o_hmax);
+  L->wk.rpart = reinterpret_cast<float*>(b + o_rpart);
   if (encode_act16(&L->x16_map, L->wk.x16, P, s.H) != cudaSuccess ||
       encode_act16(&L->h16_map, L->wk.h16, P, s.I_pad) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activation maps");
@@ -469,9 +472,21 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     MOE_KERNEL(MOE_K_ROUTER, launch_route_decode(ra, st));
     ++n_launch;  // route = logits kernel + finishing kernel (one profiled range)
   } else {
-    MOE_KERNEL(MOE_K_ROUTER, launch_router_logits(xb, L->d_W, L->d_b, wk.logits, T, s.H, s.E, st));
+    // router on the tensor cores: split-K partial logits, summed in split order by top-k
+    CUtensorMap xmap;
+    if (encode_sw128_16(&xmap, xb, true, (size_t)T, s.H, 128) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
+    RouterGemmArgs rg{};
+    rg.T = T;
+    rg.E = s.E;
+    rg.nsplit = router_gemm_splits(T, s.E, s.H, s.n_sm);
+    rg.nk_split = s.H / 64 / rg.nsplit;
+    rg.part = wk.rpart;
+    rg.split_stride = (size_t)T * s.E;
+    rg.err = wk.err;
+    MOE_KERNEL(MOE_K_ROUTER, launch_router_gemm(xmap, L->wp_map, rg, st));
     MOE_KERNEL(MOE_K_TOPK, launch_topk(wk.logits, T, s.E, s.k, (int)L->gating, forced ? wk.forced : nullptr,
-                                       wk.ids, wk.w, st));
+                                       wk.ids, wk.w, st, wk.rpart, rg.nsplit, rg.split_stride, L->d_b));
   }
   // Streaming: the cache lock is held from resolving the experts until the
   // slots' `used` events are recorded, so no other forward can evict a slot
@@ -651,6 +666,7 @@ moe_status moe_layer_destroy(moe_layer_t L) {
   }
   if (L->d_W) cudaFree(L->d_W);
   if (L->d_b) cudaFree(L->d_b);
+  if (L->d_Wp) cudaFree(L->d_Wp);
   if (L->d_resident) cudaFree(L->d_resident);
   if (L->d_wptr) cudaFree(L->d_wptr);
   if (L->d_tmaps) cudaFree(L->d_tmaps);
@@ -678,6 +694,12 @@ moe_status moe_set_router(moe_layer_t L, const float* W, const float* bias, moe_
     cudaFree(L->d_b);
     L->d_b = nullptr;
   }
+  // bf16 planes of W for the tensor-core router (T > 4)
+  if (!L->d_Wp) CUDA_TRY(cudaMalloc(&L->d_Wp, 3 * (size_t)L->s.E * L->s.H * sizeof(__nv_bfloat16)));
+  CUDA_TRY(launch_split_router(L->d_W, L->s.E, L->s.H, L->d_Wp, nullptr));
+  CUDA_TRY(cudaDeviceSynchronize());
+  if (encode_sw128_16(&L->wp_map, L->d_Wp, true, 3 * (size_t)L->s.E, L->s.H, 128) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the router planes");
   L->gating = gating;
   L->router_set = true;
   return MOE_OK;

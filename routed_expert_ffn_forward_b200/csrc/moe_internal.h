@@ -2,6 +2,7 @@
 // libmoe.so.  Nothing here is part of the C ABI (include/moe.h).
 #pragma once
 
+#include <algorithm>
 #include <cstddef>
 #include <cstdint>
 
@@ -56,6 +57,7 @@ struct Work {
   __half* h16;        // [P_cap, I_pad] SwiGLU output, fp16 scaled by 1/hinv, same K order
   float* hinv;        // [P]
   unsigned* hmax;     // [P] max |h| of each row (float bits), reset after use
+  float* rpart;       // router partial logits [splits][T][E]
 };
 
 struct RouteArgs {
@@ -113,9 +115,26 @@ size_t down_d1_smem(int max_tok, size_t act_slot_bytes);
 // 1 super-block (prefill GEMMs).
 constexpr int kMapsPerSlot = 6;
 cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, int H, int I);
-// 2-D map over a row-major fp16 matrix [rows, cols] with 128B-swizzled boxes
-// of 256 rows x 64 columns (cols a multiple of 64).
-cudaError_t encode_act16(CUtensorMap* map, const __half* base, size_t rows, int cols);
+// 2-D map over a row-major 16-bit matrix [rows, cols] (fp16 or bf16) with
+// 128B-swizzled boxes of box_rows rows x 64 columns (cols a multiple of 64).
+cudaError_t encode_sw128_16(CUtensorMap* map, const void* base, bool bf16, size_t rows, int cols, int box_rows);
+inline cudaError_t encode_act16(CUtensorMap* map, const __half* base, size_t rows, int cols) {
+  return encode_sw128_16(map, base, false, rows, cols, 256);
+}
+
+// Router logits on the tensor cores (T > 4): partial sums per K split.
+struct RouterGemmArgs {
+  int T, E;
+  int nsplit, nk_split;     // K splits; 64-wide K steps per split
+  float* part;              // [nsplit][T][E]
+  size_t split_stride;      // floats between splits
+  unsigned* err;
+};
+int router_gemm_splits(int T, int E, int H, int n_sm);
+size_t router_part_floats(int T_cap, int E, int n_sm);
+cudaError_t launch_split_router(const float* W, int E, int H, __nv_bfloat16* planes, cudaStream_t st);
+cudaError_t launch_router_gemm(const CUtensorMap& xmap, const CUtensorMap& wmap, const RouterGemmArgs& a,
+                               cudaStream_t st);
 
 // Prefill GEMMs (tcgen05): mode 0 gate/up -> h (+ hmax), mode 1 down -> y.
 struct GemmArgs {
@@ -150,8 +169,13 @@ struct Shape {
 // ---- kernels (one launch helper per kernel; all enqueue on `st`) ----------
 cudaError_t launch_router_logits(const __nv_bfloat16* x, const float* W, const float* b,
                                  float* logits, int T, int H, int E, cudaStream_t st);
-cudaError_t launch_topk(const float* logits, int T, int E, int k, int gating,
-                        const int* forced, int* ids, float* w, cudaStream_t st);
+// Top-k + gating.  With `part` (nsplit slices of partial logits, split_stride
+// floats apart) the logits are first summed in split order, the bias added and
+// the result written to `logits`.
+cudaError_t launch_topk(float* logits, int T, int E, int k, int gating,
+                        const int* forced, int* ids, float* w, cudaStream_t st,
+                        const float* part = nullptr, int nsplit = 0, size_t split_stride = 0,
+                        const float* bias = nullptr);
 cudaError_t launch_permute(const int* ids, int T, const Shape& s, const Work& wk, cudaStream_t st);
 cudaError_t launch_gate_up_simt(const uint8_t* const* wptr, const __nv_bfloat16* x, const Shape& s,
                                 const Work& wk, cudaStream_t st);

@@ -64,6 +64,31 @@ __global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int 
                      ids + (size_t)t * k, w + (size_t)t * k);
 }
 
+// One block per token: the block sums the token's logits over the K splits in
+// split order and adds the bias (writing them to `logits` and shared memory),
+// then warp 0 selects and gates.
+constexpr int kSumThreads = 128;
+template <int PL>
+__global__ void __launch_bounds__(kSumThreads)
+    topk_sum_kernel(float* __restrict__ logits, int E, int k, int gating, const int* __restrict__ forced,
+                    int* __restrict__ ids, float* __restrict__ w, const float* __restrict__ part, int nsplit,
+                    size_t split_stride, const float* __restrict__ bias) {
+  __shared__ float s_l[32 * PL];
+  const int t = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += kSumThreads) {
+    const float* p = part + (size_t)t * E + e;
+    float v = p[0];
+    for (int s = 1; s < nsplit; ++s) v += p[(size_t)s * split_stride];
+    v += bias ? bias[e] : 0.f;
+    logits[(size_t)t * E + e] = v;
+    s_l[e] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32)
+    warp_topk_gate<PL>(s_l, E, k, gating, forced ? forced + (size_t)t * k : nullptr, ids + (size_t)t * k,
+                       w + (size_t)t * k);
+}
+
 }  // namespace
 
 cudaError_t launch_router_logits(const __nv_bfloat16* x, const float* W, const float* b,
@@ -73,11 +98,21 @@ cudaError_t launch_router_logits(const __nv_bfloat16* x, const float* W, const f
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk(const float* logits, int T, int E, int k, int gating, const int* forced,
-                        int* ids, float* w, cudaStream_t st) {
+cudaError_t launch_topk(float* logits, int T, int E, int k, int gating, const int* forced,
+                        int* ids, float* w, cudaStream_t st, const float* part, int nsplit, size_t split_stride,
+                        const float* bias) {
+  const int pl = (E + 31) / 32;
+  if (part) {
+    if (pl <= 8)
+      topk_sum_kernel<8><<<T, kSumThreads, 0, st>>>(logits, E, k, gating, forced, ids, w, part, nsplit,
+                                                    split_stride, bias);
+    else
+      topk_sum_kernel<32><<<T, kSumThreads, 0, st>>>(logits, E, k, gating, forced, ids, w, part, nsplit,
+                                                     split_stride, bias);
+    return cudaGetLastError();
+  }
   const int warps = 8;
   const int grid = (T + warps - 1) / warps;
-  const int pl = (E + 31) / 32;
   if (pl <= 8)
     topk_kernel<8><<<grid, warps * 32, 0, st>>>(logits, T, E, k, gating, forced, ids, w);
   else

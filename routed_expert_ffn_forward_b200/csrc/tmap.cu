@@ -4,8 +4,8 @@
 // 8-byte elements, nb*18 wide and R high (row pitch nb*144 bytes, a multiple
 // of 16).  A box is 64 or 128 rows by SB super-blocks (SB*18 elements, SB*144
 // bytes); boxes past the last row or block read zeros, which decode to zero
-// weights.  Activation matrices of the prefill GEMMs are fp16 [rows, cols]
-// with 128-byte-swizzled boxes of 256 rows x 64 columns.
+// weights.  16-bit operand matrices of the tensor-core GEMMs (activations,
+// router planes) use 128-byte-swizzled boxes of 64 columns.
 #include <mutex>
 
 #include "moe_internal.h"
@@ -56,15 +56,16 @@ cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, int H, in
   return e;
 }
 
-cudaError_t encode_act16(CUtensorMap* map, const __half* base, size_t rows, int cols) {
+cudaError_t encode_sw128_16(CUtensorMap* map, const void* base, bool bf16, size_t rows, int cols, int box_rows) {
   EncodeFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
-  if (cols % 64 || rows == 0) return cudaErrorInvalidValue;
+  if (cols % 64 || rows == 0 || box_rows <= 0 || box_rows > 256) return cudaErrorInvalidValue;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, 256};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(base), dims, strides, box, estr,
+  const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                        const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
