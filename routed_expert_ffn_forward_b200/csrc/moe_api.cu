@@ -192,7 +192,7 @@ moe_status ensure_scratch(moe_layer* L, int T) {
                o_act2 = take(ES * 4), o_nact1 = take(4), o_nact2 = take(4), o_tcnt = take((size_t)(s.H / 64) * 4),
                o_err = take(4), o_tiles = take(prefill_max_tiles((int)ES, P) * 16), o_ntiles = take(4),
                o_x16 = take(P * s.H * 2), o_rinv = take(P * 4), o_h16 = take(P * s.I_pad * 2), o_hinv = take(P * 4),
-               o_hmax = take(P * 4), o_rpart = take(router_part_floats(cap, s.E, s.n_sm) * 4);
+               o_rpart = take(router_part_floats(cap, s.E, s.n_sm) * 4);
   if (L->scratch) {
     CUDA_TRY(cudaDeviceSynchronize());
     cudaFree(L->scratch);
@@ -239,13 +239,11 @@ moe_status ensure_scratch(moe_layer* L, int T) {
   L->wk.rinv = reinterpret_cast<float*>(b + o_rinv);
   L->wk.h16 = reinterpret_cast<__half*>(b + o_h16);
   L->wk.hinv = reinterpret_cast<float*>(b + o_hinv);
-  L->wk.hmax = reinterpret_cast<unsigned*>(b + o_hmax);
   L->wk.rpart = reinterpret_cast<float*>(b + o_rpart);
   if (encode_act16(&L->x16_map, L->wk.x16, P, s.H) != cudaSuccess ||
       encode_act16(&L->h16_map, L->wk.h16, P, s.I_pad) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activation maps");
-  // zero everything once: the ticket and hmax must start at 0 and the padded
-  // columns of h (I..I_pad) are never written and must read as 0
+  // zero everything once: the ticket must start at 0
   CUDA_TRY(cudaMemset(L->scratch, 0, off));
   CUDA_TRY(cudaDeviceSynchronize());
   L->T_cap = cap;
@@ -556,7 +554,6 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     ga.out = wk.h;
     ga.out_ld = s.I_pad;
     ga.out_rows = s.I;
-    ga.hmax = wk.hmax;
     ga.err = wk.err;
     MOE_KERNEL(MOE_K_GATE_UP, launch_prefill_gemm(0, L->x16_map, ga, s.n_sm, st));
     MOE_KERNEL(MOE_K_PREP, launch_convert_h(wk, P, s.I, s.I_pad, st));

@@ -56,7 +56,6 @@ struct Work {
   float* rinv;        // [P]
   __half* h16;        // [P_cap, I_pad] SwiGLU output, fp16 scaled by 1/hinv, same K order
   float* hinv;        // [P]
-  unsigned* hmax;     // [P] max |h| of each row (float bits), reset after use
   float* rpart;       // router partial logits [splits][T][E]
 };
 
@@ -118,8 +117,12 @@ cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, int H, in
 // 2-D map over a row-major 16-bit matrix [rows, cols] (fp16 or bf16) with
 // 128B-swizzled boxes of box_rows rows x 64 columns (cols a multiple of 64).
 cudaError_t encode_sw128_16(CUtensorMap* map, const void* base, bool bf16, size_t rows, int cols, int box_rows);
+// box_cols 64 (128B swizzle) or 32 (64B swizzle)
+cudaError_t encode_swz_16(CUtensorMap* map, const void* base, bool bf16, size_t rows, int cols, int box_rows,
+                          int box_cols);
+// B operands of the prefill GEMMs: boxes of 256 rows x 32 columns, 64B swizzle
 inline cudaError_t encode_act16(CUtensorMap* map, const __half* base, size_t rows, int cols) {
-  return encode_sw128_16(map, base, false, rows, cols, 256);
+  return encode_swz_16(map, base, false, rows, cols, 256, 32);
 }
 
 // Router logits on the tensor cores (T > 4): partial sums per K split.
@@ -136,7 +139,7 @@ cudaError_t launch_split_router(const float* W, int E, int H, __nv_bfloat16* pla
 cudaError_t launch_router_gemm(const CUtensorMap& xmap, const CUtensorMap& wmap, const RouterGemmArgs& a,
                                cudaStream_t st);
 
-// Prefill GEMMs (tcgen05): mode 0 gate/up -> h (+ hmax), mode 1 down -> y.
+// Prefill GEMMs (tcgen05): mode 0 gate/up -> h, mode 1 down -> y.
 struct GemmArgs {
   const CUtensorMap* wmaps;  // [slots][kMapsPerSlot]
   const int* slot_of;        // [E+S] expert -> slot
@@ -147,7 +150,6 @@ struct GemmArgs {
   const float* rinv;         // [P] inverse activation scale of each row
   float* out;                // h [P, I_pad] or y [P, H]
   int out_ld, out_rows;      // row pitch (floats); features stored (mode 0: I)
-  unsigned* hmax;            // mode 0
   unsigned* err;
 };
 size_t prefill_gemm_smem();

@@ -7,16 +7,22 @@
 // The weights are the A operand as two M = 128 halves, the tile's activation
 // rows the B operand (N <= 256), so one dequantisation of a weight tile
 // serves up to 256 rows and the two accumulators fill all 512 TMEM columns.
+// K advances in steps of 32 (one Q4_K sub-block) through a 4-deep ring of
+// 64B-swizzled A/B stages.
 //
-//   warp 0      producer of raw Q4_K tiles (2-D TMA, 128 rows x 1 super-block)
-//   warp 1      producer of activation tiles (2-D TMA, 128B-swizzled fp16,
-//               256 rows x 64 columns)
+//   warp 0      producer of raw Q4_K tiles (2-D TMA, 128 rows x 1 super-block,
+//               both A halves, two super-blocks in flight)
+//   warp 1      producer of activation tiles (2-D TMA, 64B-swizzled fp16,
+//               256 rows x 32 columns)
 //   warp 2      TMEM allocation; one thread issues tcgen05.mma M128 N<=256 K16
 //               and tcgen05.commit
-//   warps 3-6   dequantise Q4_K to fp16 straight into the UMMA 128B-swizzled
-//               K-major layout, one weight row per thread
-//   warps 7-14  epilogue: tcgen05.ld of the accumulators (a warp reads the TMEM
-//               lane quarter warp % 4; two warps per quarter split the columns)
+//   warps 3-10  dequantise Q4_K to fp16 straight into the UMMA 64B-swizzled
+//               K-major layout: warps 3-6 the first A half, 7-10 the second,
+//               one weight row per thread
+//   warps 11-18 epilogue: tcgen05.ld of the accumulators (a warp reads the TMEM
+//               lane quarter warp % 4; two warps per quarter split the columns),
+//               SwiGLU with the fast exp and divide intrinsics (relative error
+//               ~1e-6, far below the fp16 rounding of the operands)
 //
 // Numerics: activations are fp16 scaled per row by a power of two (largest
 // magnitude in [2^14, 2^15), 1/scale kept in `rinv`); weights are fp16 scaled
@@ -36,14 +42,14 @@ namespace {
 constexpr int kGM = 128;                       // rows of one A half (MMA M)
 constexpr int kGN = 256;                       // activation rows per tile (max MMA N)
 constexpr int kRawBytes = kGM * kQBytes;       // one A half, one super-block: 18432
-constexpr int kABytes = kGM * 64 * 2;          // one A half, 64 K as fp16: 16384
-constexpr int kBBytes = kGN * 64 * 2;          // 256 rows x 64 K as fp16: 32768
+constexpr int kABytes = kGM * 32 * 2;          // one A half, 32 K as fp16: 8192
+constexpr int kBBytes = kGN * 32 * 2;          // 256 rows x 32 K as fp16: 16384
 constexpr int kNR = 2;                         // raw super-block stages
-constexpr int kNS = 2;                         // A/B stages (64 K each)
-constexpr int kDeqWarps = 4;
+constexpr int kNS = 4;                         // A/B stages (32 K each); even, a chunk fills two
+constexpr int kDeqWarps = 8;
 constexpr int kEpiWarps = 8;
 constexpr int kFirstDeq = 3, kFirstEpi = kFirstDeq + kDeqWarps;
-constexpr int kGemmThreads = (kFirstEpi + kEpiWarps) * 32;  // 480
+constexpr int kGemmThreads = (kFirstEpi + kEpiWarps) * 32;  // 608
 constexpr float kWScale = 256.f, kWScaleInv = 1.f / 256.f;
 constexpr float kWMax = 60000.f;               // largest |weight| * 2^8 accepted
 
@@ -54,31 +60,35 @@ constexpr size_t kSmemBar = 8 * (2 * kNR + 3 * kNS + 2 + 1) + 16;
 constexpr size_t kGemmSmem = 1024 + kSmemRaw + kSmemA + kSmemB + kSmemBar;
 static_assert(kGemmSmem <= 227 * 1024, "GEMM shared memory");
 
-// Scales (d*sc) and mins (dmin*m) of sub-blocks 2c (lo) and 2c+1 (hi) of a
-// Q4_K block whose first 16 bytes are `hdr` (fp16 d, fp16 dmin, 12 scale bytes).
-__device__ __forceinline__ void block_scales(uint4 hdr, int c, float& s_lo, float& s_hi, float& m_lo,
-                                             float& m_hi) {
-  const float d = __half2float(__ushort_as_half((unsigned short)(hdr.x & 0xFFFFu)));
-  const float dmin = __half2float(__ushort_as_half((unsigned short)(hdr.x >> 16)));
+// fp16x2 scale pair (s_lo, s_hi) = 2^8 * d * (sc_2c, sc_2c+1) and min pair
+// (nm_lo, nm_hi) = -2^8 * dmin * (m_2c, m_2c+1) of chunk c of a Q4_K block
+// whose first 16 bytes are `hdr` (fp16 d, fp16 dmin, 12 scale bytes).  All
+// in fp16 arithmetic: the 6-bit fields become fp16 integers through the 1024
+// exponent trick, and d * sc rounds once, as a float product converted to
+// fp16 would.  `d2s`/`nm2s` are (2^8 d, 2^8 d) and (-2^8 dmin, -2^8 dmin).
+__device__ __forceinline__ void chunk_scales(uint4 hdr, int c, __half2 d2s, __half2 nm2s, __half2& s2, __half2& nm2) {
   const uint32_t sh = 16u * (uint32_t)(c & 1);
-  const uint32_t s0 = hdr.y >> sh, s1 = hdr.z >> sh, s2 = hdr.w >> sh;
+  const uint32_t s0 = hdr.y >> sh, s1 = hdr.z >> sh, s2w = hdr.w >> sh;
   uint32_t vsc, vm;
   if (c < 2) {
     vsc = s0 & 0x3F3Fu;
     vm = s1 & 0x3F3Fu;
   } else {
-    vsc = (s2 & 0x0F0Fu) | ((s0 >> 2) & 0x3030u);
-    vm = ((s2 >> 4) & 0x0F0Fu) | ((s1 >> 2) & 0x3030u);
+    vsc = (s2w & 0x0F0Fu) | ((s0 >> 2) & 0x3030u);
+    vm = ((s2w >> 4) & 0x0F0Fu) | ((s1 >> 2) & 0x3030u);
   }
-  s_lo = d * (float)(vsc & 0xFFu);
-  s_hi = d * (float)((vsc >> 8) & 0xFFu);
-  m_lo = dmin * (float)(vm & 0xFFu);
-  m_hi = dmin * (float)((vm >> 8) & 0xFFu);
+  // bytes (f0, f1) -> fp16x2 (1024 + f0, 1024 + f1)
+  const uint32_t tsc = __byte_perm(vsc, 0x64u, 0x4140u), tm = __byte_perm(vm, 0x64u, 0x4140u);
+  const __half2 k1024 = __float2half2_rn(1024.f);
+  const __half2 sc = __hsub2(*reinterpret_cast<const __half2*>(&tsc), k1024);
+  const __half2 mm = __hsub2(*reinterpret_cast<const __half2*>(&tm), k1024);
+  s2 = __hmul2(d2s, sc);
+  nm2 = __hmul2(nm2s, mm);
 }
 
-// fp16x2 (1024 + a, 1024 + b) -> (a * s - m, b * s - m), `nm` = -m
-__device__ __forceinline__ uint32_t deq2(uint32_t t, __half2 s, __half2 nm) {
-  const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&t), __float2half2_rn(1024.f));
+// fp16x2 (o + a, o + b) -> (a * s - m, b * s - m), `off` = (o, o), `nm` = -m
+__device__ __forceinline__ uint32_t deq2(uint32_t t, __half2 off, __half2 s, __half2 nm) {
+  const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&t), off);
   const __half2 v = __hfma2(q, s, nm);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
@@ -88,24 +98,65 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* raw) {
   return raw + pad;
 }
 
-// Column-wise max over the 32 lanes of a warp: v[i] is this lane's value of
-// column i; the result (v[0] afterwards) is the max of column `lane`.
-// Reduce-scatter butterfly: 31 shuffles instead of 32 x 5.
-__device__ __forceinline__ float colmax32(float (&v)[32], int lane) {
+// Epilogue of unit u, run by the epilogue warps: warp w reads TMEM lane
+// quarter w % 4 and the 32-column chunks (w - first epilogue warp) / 4 + 2j.
+// Returns false (error flag set) if the accumulators never became ready.
+template <int kMode>
+__device__ __forceinline__ bool gemm_epilogue(const GemmArgs& a, uint32_t tmem, uint64_t* acc_full,
+                                              uint64_t* acc_empty, int u, uint32_t& fph, int wk, int warp,
+                                              int lane) {
+  const int4 tl = __ldcg(a.tiles + u / a.ft);
+  const int f = u % a.ft;
+  const int q = warp & 3;                      // TMEM lane quarter this warp may read
+  const int sub = wk >> 2;                     // 0..kEpiWarps/4-1
+  const int mrow = q * 32 + lane;              // row of the A halves
+  const bool ok = ptx::mbar_wait(acc_full, fph);
+  __syncwarp();
+  if (!ok) {
+    atomicOr(a.err, 128u);
+    return false;
+  }
+  fph ^= 1u;
+  ptx::tc_fence_after();
+  const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+  const int pair0 = tl.w + tl.y;
+  for (int c0 = 32 * sub; c0 < tl.z; c0 += 32 * (kEpiWarps / 4)) {
+    const int nc = min(32, tl.z - c0);
+    // lane i holds the inverse scale of column c0 + i
+    const float my_inv = __ldg(a.rinv + pair0 + c0 + min(lane, nc - 1)) * kWScaleInv;
+    uint32_t r0[32], r1[32];
+    ptx::tmem_ld32x2(tq + c0, tq + kGN + c0, r0, r1);
+    if (kMode == 0) {
+      const int feat = f * kGM + mrow;
+      const bool frow = feat < a.out_rows;
+      float* outp = a.out + (size_t)(pair0 + c0) * a.out_ld + feat;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const bool up = (lane & o) != 0;
+      for (int i = 0; i < 32; ++i) {
+        const float inv = __shfl_sync(0xffffffffu, my_inv, i);
+        const float g = __uint_as_float(r0[i]) * inv, up = __uint_as_float(r1[i]) * inv;
+        const float hv = __fdividef(g, 1.f + __expf(-g)) * up;   // silu(g) * up
+        if (i < nc && frow) outp[(size_t)i * a.out_ld] = hv;
+      }
+    } else {
+      const int orow = f * 2 * kGM + mrow;
+      float* outp = a.out + (size_t)(pair0 + c0) * a.out_ld + orow;
 #pragma unroll
-    for (int j = 0; j < o; ++j) {
-      const float send = up ? v[j] : v[j + o];
-      const float keep = up ? v[j + o] : v[j];
-      v[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+      for (int i = 0; i < 32; ++i) {
+        const float inv = __shfl_sync(0xffffffffu, my_inv, i);
+        if (i < nc) {
+          outp[(size_t)i * a.out_ld] = __uint_as_float(r0[i]) * inv;
+          outp[(size_t)i * a.out_ld + kGM] = __uint_as_float(r1[i]) * inv;
+        }
+      }
     }
   }
-  return v[0];
+  ptx::tc_fence_before();
+  __syncwarp();
+  if (lane == 0) ptx::mbar_arrive(acc_empty);
+  return true;
 }
 
-// kMode 0: gate/up, out = h (fp32 [P, ld]) = silu(g) * u, hmax[pair] = max |h|.
+// kMode 0: gate/up, out = h (fp32 [P, ld]) = silu(g) * u.
 // kMode 1: down,    out = y (fp32 [P, ld]).
 template <int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
@@ -191,18 +242,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
       for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
         const int4 tl = __ldcg(a.tiles + u / ft);
         const int row = tl.w + tl.y;
-        for (int kb = 0; kb < a.nkb; ++kb) {
-          for (int s = 0; s < 4; ++s) {
-            if (!ptx::mbar_wait(&ab_empty[bs], bph ^ 1u)) {
-              atomicOr(a.err, 16u);
-              goto b_drain;
-            }
-            ptx::mbar_arrive_expect_tx(&b_full[bs], kBBytes);
-            ptx::tma_load_2d(s_b + bs * kBBytes, &bmap, kb * 256 + s * 64, row, &b_full[bs]);
-            issued |= 1u << bs;
-            last_ph = (last_ph & ~(1u << bs)) | (bph << bs);
-            if (++bs == kNS) { bs = 0; bph ^= 1u; }
+        for (int ks = 0; ks < a.nkb * 8; ++ks) {
+          if (!ptx::mbar_wait(&ab_empty[bs], bph ^ 1u)) {
+            atomicOr(a.err, 16u);
+            goto b_drain;
           }
+          ptx::mbar_arrive_expect_tx(&b_full[bs], kBBytes);
+          ptx::tma_load_2d(s_b + bs * kBBytes, &bmap, ks * 32, row, &b_full[bs]);
+          issued |= 1u << bs;
+          last_ph = (last_ph & ~(1u << bs)) | (bph << bs);
+          if (++bs == kNS) { bs = 0; bph ^= 1u; }
         }
       }
     b_drain:
@@ -224,26 +273,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
         eph ^= 1u;
         ptx::tc_fence_after();
         bool ok = true;
-        for (int kb = 0; kb < a.nkb && ok; ++kb) {
-          for (int s = 0; s < 4; ++s) {
-            if (!ptx::mbar_wait(&a_full[as], aph) || !ptx::mbar_wait(&b_full[as], aph)) {
-              atomicOr(a.err, 32u);
-              ok = false;
-              break;
-            }
-            ptx::tc_fence_after();
-            const uint32_t a0 = ptx::smem_u32(s_a + (2 * as) * kABytes);
-            const uint32_t b0 = ptx::smem_u32(s_b + as * kBBytes);
-#pragma unroll
-            for (int k16 = 0; k16 < 4; ++k16) {
-              const uint64_t bd = ptx::umma_desc_sw128(b0 + 32 * k16);
-              const bool acc = (kb | s | k16) != 0;
-              ptx::umma_f16(tmem, ptx::umma_desc_sw128(a0 + 32 * k16), bd, idesc, acc);
-              ptx::umma_f16(tmem + kGN, ptx::umma_desc_sw128(a0 + kABytes + 32 * k16), bd, idesc, acc);
-            }
-            ptx::umma_commit(&ab_empty[as]);
-            if (++as == kNS) { as = 0; aph ^= 1u; }
+        for (int ks = 0; ks < a.nkb * 8; ++ks) {
+          if (!ptx::mbar_wait(&a_full[as], aph) || !ptx::mbar_wait(&b_full[as], aph)) {
+            atomicOr(a.err, 32u);
+            ok = false;
+            break;
           }
+          ptx::tc_fence_after();
+          const uint32_t a0 = ptx::smem_u32(s_a + (2 * as) * kABytes);
+          const uint32_t b0 = ptx::smem_u32(s_b + as * kBBytes);
+#pragma unroll
+          for (int k16 = 0; k16 < 2; ++k16) {
+            const uint64_t bd = ptx::umma_desc_sw64(b0 + 32 * k16);
+            const bool acc = (ks | k16) != 0;
+            ptx::umma_f16(tmem, ptx::umma_desc_sw64(a0 + 32 * k16), bd, idesc, acc);
+            ptx::umma_f16(tmem + kGN, ptx::umma_desc_sw64(a0 + kABytes + 32 * k16), bd, idesc, acc);
+          }
+          ptx::umma_commit(&ab_empty[as]);
+          if (++as == kNS) { as = 0; aph ^= 1u; }
         }
         if (!ok) break;
         ptx::umma_commit(acc_full);
@@ -254,7 +301,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
     }
   } else if (warp < kFirstEpi) {
     // ------------------------------------------------------------ dequantisers
-    const int r = threadIdx.x - kFirstDeq * 32;  // weight row of each A half, 0..127
+    const int m = (warp - kFirstDeq) >> 2;                    // A half
+    const int r = ((warp - kFirstDeq) & 3) * 32 + lane;       // weight row of the half, 0..127
+    const uint32_t sw = (uint32_t)((r >> 1) & 3);             // 64B swizzle of row r
+    const __half2 off_lo = __float2half2_rn(1024.f), off_hi = __float2half2_rn(64.f);
+    const __half2 kWScale2 = __float2half2_rn(kWScale), kNegWScale2 = __float2half2_rn(-kWScale);
     int rs = 0, as = 0;
     uint32_t rph = 0, aph = 0;
     bool bad = false;
@@ -264,45 +315,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
           atomicOr(a.err, 64u);
           goto done;
         }
-        for (int s = 0; s < 4; ++s) {
-          if (!ptx::mbar_wait(&ab_empty[as], aph ^ 1u)) {
-            atomicOr(a.err, 64u);
-            goto done;
-          }
+        const uint8_t* row = s_rawbuf + (2 * rs + m) * kRawBytes + r * kQBytes;
+        const uint4 hdr = *reinterpret_cast<const uint4*>(row);
+        // (d, d) and (dmin, dmin) scaled by 2^8 (exact); a block whose d or dmin could
+        // take a weight past kWMax (with the largest 6-bit scale) is flagged
+        const uint32_t dd = __byte_perm(hdr.x, 0u, 0x1010u), mm = __byte_perm(hdr.x, 0u, 0x3232u);
+        const __half2 d2 = *reinterpret_cast<const __half2*>(&dd), dm2 = *reinterpret_cast<const __half2*>(&mm);
+        bad |= !(__hlt(__habs(__low2half(d2)), __float2half_rn(kWMax / (kWScale * 63.f * 15.f))) &&
+                 __hlt(__habs(__low2half(dm2)), __float2half_rn(kWMax / (kWScale * 63.f))));
+        const __half2 d2s = __hmul2(d2, kWScale2), nm2s = __hmul2(dm2, kNegWScale2);
+        for (int c = 0; c < 4; ++c) {
+          // chunk c: 32 quant bytes; low nibbles are sub-block 2c, high nibbles 2c+1
+          const uint4 qa = *reinterpret_cast<const uint4*>(row + 16 + 32 * c);
+          const uint4 qb = *reinterpret_cast<const uint4*>(row + 32 + 32 * c);
+          const uint32_t w[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+          __half2 s2, nm2;
+          chunk_scales(hdr, c, d2s, nm2s, s2, nm2);
 #pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const uint8_t* row = s_rawbuf + (2 * rs + m) * kRawBytes + r * kQBytes;
-            const uint4 hdr = *reinterpret_cast<const uint4*>(row);
-            const uint4 qa = *reinterpret_cast<const uint4*>(row + 16 + 32 * s);
-            const uint4 qb = *reinterpret_cast<const uint4*>(row + 32 + 32 * s);
-            float s_lo, s_hi, m_lo, m_hi;
-            block_scales(hdr, s, s_lo, s_hi, m_lo, m_hi);
-            bad |= !(fmaxf(15.f * fmaxf(s_lo, s_hi), fmaxf(m_lo, m_hi)) * kWScale < kWMax);
-            const __half2 sl = __float2half2_rn(s_lo * kWScale), nl = __float2half2_rn(-m_lo * kWScale);
-            const __half2 sh = __float2half2_rn(s_hi * kWScale), nh = __float2half2_rn(-m_hi * kWScale);
-            const uint32_t w[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-            uint8_t* arow = s_a + (2 * as + m) * kABytes + r * 128;
-            // low nibbles: K 0..31 (chunks 0..3), high nibbles: K 32..63 (chunks 4..7)
+          for (int nib = 0; nib < 2; ++nib) {
+            if (!ptx::mbar_wait(&ab_empty[as], aph ^ 1u)) {
+              atomicOr(a.err, 64u);
+              goto done;
+            }
+            const __half2 sc = nib ? __high2half2(s2) : __low2half2(s2);
+            const __half2 nm = nib ? __high2half2(nm2) : __low2half2(nm2);
+            const __half2 off = nib ? off_hi : off_lo;
+            // low nibbles as 1024 + q (mask 0x000F), high nibbles as 64 + q (mask 0x00F0)
+            const uint32_t mask = nib ? 0x00F000F0u : 0x000F000Fu;
+            const uint32_t magic = nib ? 0x54005400u : 0x64006400u;
+            uint8_t* arow = s_a + (2 * as + m) * kABytes + r * 64;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint32_t w0 = w[2 * j], w1 = w[2 * j + 1];
-              uint4 lo, hi;
-              lo.x = deq2((w0 & 0x000F000Fu) | 0x64006400u, sl, nl);
-              lo.y = deq2(((w0 >> 8) & 0x000F000Fu) | 0x64006400u, sl, nl);
-              lo.z = deq2((w1 & 0x000F000Fu) | 0x64006400u, sl, nl);
-              lo.w = deq2(((w1 >> 8) & 0x000F000Fu) | 0x64006400u, sl, nl);
-              hi.x = deq2(((w0 >> 4) & 0x000F000Fu) | 0x64006400u, sh, nh);
-              hi.y = deq2(((w0 >> 12) & 0x000F000Fu) | 0x64006400u, sh, nh);
-              hi.z = deq2(((w1 >> 4) & 0x000F000Fu) | 0x64006400u, sh, nh);
-              hi.w = deq2(((w1 >> 12) & 0x000F000Fu) | 0x64006400u, sh, nh);
-              *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = lo;
-              *reinterpret_cast<uint4*>(arow + (((j + 4) ^ (r & 7)) << 4)) = hi;
+              uint4 o;
+              o.x = deq2((w0 & mask) | magic, off, sc, nm);
+              o.y = deq2(((w0 >> 8) & mask) | magic, off, sc, nm);
+              o.z = deq2((w1 & mask) | magic, off, sc, nm);
+              o.w = deq2(((w1 >> 8) & mask) | magic, off, sc, nm);
+              *reinterpret_cast<uint4*>(arow + ((j ^ sw) << 4)) = o;
             }
+            ptx::fence_proxy_async();  // generic-proxy stores -> visible to the tensor cores
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&a_full[as]);
+            if (++as == kNS) { as = 0; aph ^= 1u; }
           }
-          ptx::fence_proxy_async();  // generic-proxy stores -> visible to the tensor cores
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&a_full[as]);
-          if (++as == kNS) { as = 0; aph ^= 1u; }
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&raw_empty[rs]);
@@ -312,58 +368,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
     if (bad) atomicOr(a.err, 256u);
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;                      // TMEM lane quarter this warp may read
-    const int half = (warp - kFirstEpi) >> 2;    // which 32-column chunks
-    const int mrow = q * 32 + lane;              // row of the A halves
     uint32_t fph = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-      const int4 tl = __ldcg(a.tiles + u / ft);
-      const int f = u % ft;
-      const bool ok = ptx::mbar_wait(acc_full, fph);
-      __syncwarp();
-      if (!ok) {
-        atomicOr(a.err, 128u);
-        goto done;
-      }
-      fph ^= 1u;
-      ptx::tc_fence_after();
-      const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
-      const int pair0 = tl.w + tl.y;
-      for (int c0 = 32 * half; c0 < tl.z; c0 += 64) {
-        float v0[32], v1[32];
-        ptx::tmem_ld32(tq + c0, v0);
-        ptx::tmem_ld32(tq + kGN + c0, v1);
-        const int nc = min(32, tl.z - c0);
-        if (kMode == 0) {
-          const int feat = f * kGM + mrow;
-          const bool frow = feat < a.out_rows;
-          float* outp = a.out + (size_t)(pair0 + c0) * a.out_ld + feat;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float inv = __ldg(a.rinv + pair0 + c0 + min(i, nc - 1)) * kWScaleInv;
-            const float hv = silu_f(v0[i] * inv) * (v1[i] * inv);
-            if (i < nc && frow) outp[(size_t)i * a.out_ld] = hv;
-            v0[i] = (i < nc && frow) ? fabsf(hv) : 0.f;
-          }
-          const float mx = colmax32(v0, lane);
-          if (lane < nc) atomicMax(a.hmax + pair0 + c0 + lane, __float_as_uint(mx));
-        } else {
-          const int orow = f * 2 * kGM + mrow;
-          float* outp = a.out + (size_t)(pair0 + c0) * a.out_ld + orow;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (i < nc) {
-              const float inv = __ldg(a.rinv + pair0 + c0 + i) * kWScaleInv;
-              outp[(size_t)i * a.out_ld] = v0[i] * inv;
-              outp[(size_t)i * a.out_ld + kGM] = v1[i] * inv;
-            }
-          }
-        }
-      }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(acc_empty);
-    }
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x)
+      if (!gemm_epilogue<kMode>(a, tmem, acc_full, acc_empty, u, fph, warp - kFirstEpi, warp, lane)) goto done;
   }
 done:
   ptx::tc_fence_before();
@@ -462,37 +469,45 @@ __global__ void __launch_bounds__(kRowThreads) gather_rows_kernel(const __nv_bfl
   if (threadIdx.x == 0) rinv[r] = inv;
 }
 
-// h (fp32 [P, I_pad], columns >= I unwritten) -> scaled fp16 h16 with zero
-// padding, hinv[r] = 1/scale from hmax[r]; hmax[r] is reset for the next forward.
-__global__ void __launch_bounds__(kRowThreads) convert_h_kernel(const float* __restrict__ h,
-                                                                unsigned* __restrict__ hmax, int I, int I_pad,
+// h (fp32 [P, I_pad], columns >= I unwritten) -> fp16 h16 scaled by the power
+// of two that puts the row's largest magnitude in [2^14, 2^15), padding
+// zeroed, K order (0, 2, 1, 3); hinv[r] = 1/scale.
+__global__ void __launch_bounds__(kRowThreads) convert_h_kernel(const float* __restrict__ h, int I, int I_pad,
                                                                 __half* __restrict__ h16,
                                                                 float* __restrict__ hinv) {
-  __shared__ float s_sc[2];
+  __shared__ float s_red[kRowThreads / 32];
   ptx::pdl_wait();
   const int r = blockIdx.x;
-  if (threadIdx.x == 0) {
-    float inv;
-    s_sc[0] = row_scale(__uint_as_float(__ldcg(hmax + r)), &inv);
-    s_sc[1] = inv;
-    hmax[r] = 0u;
-  }
-  __syncthreads();
-  const float sc = s_sc[0];
   const float4* src = reinterpret_cast<const float4*>(h + (size_t)r * I_pad);
-  uint2* dst = reinterpret_cast<uint2*>(h16 + (size_t)r * I_pad);
-  for (int c = threadIdx.x; c < I_pad / 4; c += kRowThreads) {
-    float4 f = __ldcg(src + c);
-    const int i = 4 * c;
-    if (i + 3 >= I) {
-      f.x = i < I ? f.x : 0.f;
-      f.y = i + 1 < I ? f.y : 0.f;
-      f.z = i + 2 < I ? f.z : 0.f;
-      f.w = 0.f;
+  float4 v[kRowMaxVec];
+  float m = 0.f;
+  const int nv = I_pad / 4;
+#pragma unroll
+  for (int j = 0; j < kRowMaxVec; ++j) {
+    const int c = threadIdx.x + j * kRowThreads;
+    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (c < nv) {
+      f = __ldcg(src + c);
+      const int i = 4 * c;
+      if (i + 3 >= I) {
+        f.x = i < I ? f.x : 0.f;
+        f.y = i + 1 < I ? f.y : 0.f;
+        f.z = i + 2 < I ? f.z : 0.f;
+        f.w = 0.f;
+      }
     }
-    dst[c] = pack4_swz(f.x * sc, f.y * sc, f.z * sc, f.w * sc);
+    v[j] = f;
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w))));
   }
-  if (threadIdx.x == 0) hinv[r] = s_sc[1];
+  float inv;
+  const float sc = row_scale(block_max(m, s_red), &inv);
+  uint2* dst = reinterpret_cast<uint2*>(h16 + (size_t)r * I_pad);
+#pragma unroll
+  for (int j = 0; j < kRowMaxVec; ++j) {
+    const int c = threadIdx.x + j * kRowThreads;
+    if (c < nv) dst[c] = pack4_swz(v[j].x * sc, v[j].y * sc, v[j].z * sc, v[j].w * sc);
+  }
+  if (threadIdx.x == 0) hinv[r] = inv;
 }
 
 template <typename... KArgs, typename... Args>
@@ -529,8 +544,9 @@ cudaError_t launch_gather_rows(const __nv_bfloat16* x, const Work& wk, int P, in
 }
 
 cudaError_t launch_convert_h(const Work& wk, int P, int I, int I_pad, cudaStream_t st) {
-  return launch_pdl(convert_h_kernel, dim3(P), dim3(kRowThreads), 0, st, (const float*)wk.h, wk.hmax, I, I_pad,
-                    wk.h16, wk.hinv);
+  if (I_pad / 4 > kRowThreads * kRowMaxVec) return cudaErrorInvalidValue;
+  return launch_pdl(convert_h_kernel, dim3(P), dim3(kRowThreads), 0, st, (const float*)wk.h, I, I_pad, wk.h16,
+                    wk.hinv);
 }
 
 cudaError_t launch_prefill_gemm(int mode, const CUtensorMap& bmap, const GemmArgs& a, int n_sm, cudaStream_t st) {
