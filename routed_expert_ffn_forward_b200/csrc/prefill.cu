@@ -110,7 +110,7 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmArgs& a, uint32_t tmem, 
   const int q = warp & 3;                      // TMEM lane quarter this warp may read
   const int sub = wk >> 2;                     // 0..kEpiWarps/4-1
   const int mrow = q * 32 + lane;              // row of the A halves
-  const bool ok = ptx::mbar_wait(acc_full, fph);
+  const bool ok = ptx::mbar_wait_sleep(acc_full, fph, 200);
   __syncwarp();
   if (!ok) {
     atomicOr(a.err, 128u);
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
         const int y0 = kMode == 0 ? f * kGM : f * 2 * kGM;
         const int y1 = kMode == 0 ? f * kGM : f * 2 * kGM + kGM;
         for (int kb = 0; kb < a.nkb; ++kb) {
-          if (!ptx::mbar_wait(&raw_empty[rs], rph ^ 1u)) {
+          if (!ptx::mbar_wait_sleep(&raw_empty[rs], rph ^ 1u, 100)) {
             atomicOr(a.err, 16u);
             goto raw_drain;
           }
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
         const int4 tl = __ldcg(a.tiles + u / ft);
         const int row = tl.w + tl.y;
         for (int ks = 0; ks < a.nkb * 8; ++ks) {
-          if (!ptx::mbar_wait(&ab_empty[bs], bph ^ 1u)) {
+          if (!ptx::mbar_wait_sleep(&ab_empty[bs], bph ^ 1u, 50)) {
             atomicOr(a.err, 16u);
             goto b_drain;
           }
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
       for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
         const int4 tl = __ldcg(a.tiles + u / ft);
         const uint32_t idesc = ptx::umma_idesc_f16(kGM, min(kGN, (tl.z + 15) & ~15));
-        if (!ptx::mbar_wait(acc_empty, eph ^ 1u)) {
+        if (!ptx::mbar_wait_sleep(acc_empty, eph ^ 1u, 100)) {
           atomicOr(a.err, 32u);
           break;
         }
