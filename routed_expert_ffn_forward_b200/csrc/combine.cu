@@ -11,30 +11,43 @@ namespace {
 __global__ void combine_kernel(const float* __restrict__ y, const float* __restrict__ w,
                                const int* __restrict__ inv, int H, int k, int S,
                                __nv_bfloat16* __restrict__ out) {
-  // launched as a programmatic dependent of the down kernel on the decode path:
-  // wait for it (a no-op when launched normally)
+  constexpr int kMaxKS = 40;  // top_k + n_shared at most
+  __shared__ int s_row[kMaxKS];
+  __shared__ float s_w[kMaxKS];
+  // launched as a programmatic dependent of the down kernel: wait for it (a
+  // no-op when launched normally)
   ptx::pdl_wait();
-  const int t = blockIdx.y;
+  const int t = blockIdx.y, kS = k + S;
+  // the token's y rows and weights, once per block, so the y loads below are
+  // independent of each other
+  if (threadIdx.x < kS) {
+    s_row[threadIdx.x] = inv[t * kS + threadIdx.x];
+    s_w[threadIdx.x] = threadIdx.x < k ? w[(size_t)t * k + threadIdx.x] : 1.f;
+  }
+  __syncthreads();
   const int o = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (o >= H) return;
-  const int kS = k + S;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < k; ++j) {
-    const int r = inv[t * kS + j];
-    const float wj = w[(size_t)t * k + j];
-    const float4 v = *reinterpret_cast<const float4*>(y + (size_t)r * H + o);
-    acc.x = fmaf(wj, v.x, acc.x);
-    acc.y = fmaf(wj, v.y, acc.y);
-    acc.z = fmaf(wj, v.z, acc.z);
-    acc.w = fmaf(wj, v.w, acc.w);
-  }
-  for (int s = 0; s < S; ++s) {
-    const int r = inv[t * kS + k + s];
-    const float4 v = *reinterpret_cast<const float4*>(y + (size_t)r * H + o);
-    acc.x += v.x;
-    acc.y += v.y;
-    acc.z += v.z;
-    acc.w += v.w;
+  for (int j0 = 0; j0 < kS; j0 += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj)
+      if (j0 + jj < kS) v[jj] = *reinterpret_cast<const float4*>(y + (size_t)s_row[j0 + jj] * H + o);
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int j = j0 + jj;
+      if (j < k) {  // routed experts: weighted, in order
+        acc.x = fmaf(s_w[j], v[jj].x, acc.x);
+        acc.y = fmaf(s_w[j], v[jj].y, acc.y);
+        acc.z = fmaf(s_w[j], v[jj].z, acc.z);
+        acc.w = fmaf(s_w[j], v[jj].w, acc.w);
+      } else if (j < kS) {  // then the shared experts
+        acc.x += v[jj].x;
+        acc.y += v[jj].y;
+        acc.z += v[jj].z;
+        acc.w += v[jj].w;
+      }
+    }
   }
   __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
   __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
@@ -47,7 +60,7 @@ __global__ void combine_kernel(const float* __restrict__ y, const float* __restr
 }  // namespace
 
 cudaError_t launch_combine(const Work& wk, int T, const Shape& s, __nv_bfloat16* out, cudaStream_t st, bool pdl) {
-  const int threads = 128;
+  const int threads = 64;  // more, smaller blocks: the combine is latency-bound at small T
   dim3 grid((s.H / 4 + threads - 1) / threads, T);
   if (!pdl) {
     combine_kernel<<<grid, threads, 0, st>>>(wk.y, wk.w, wk.inv, s.H, s.k, s.S, out);

@@ -76,12 +76,18 @@ __device__ __forceinline__ RowScales decode_scales(uint4 hdr, int c) {
   return r;
 }
 
-__device__ __forceinline__ void load_row_block(const uint8_t* blk, int c, uint4& hdr, uint32_t* q) {
+// One row's block header and quant chunk c (32 bytes).  Rows sit 144*SB bytes
+// apart, so every 16-byte piece starts on a multiple of 8 banks: lanes of odd
+// row index g read the two halves in the opposite order, which puts the two
+// rows of an 8-lane phase on disjoint banks.
+__device__ __forceinline__ void load_row_block(const uint8_t* blk, int c, int g, uint4& hdr, uint32_t* q) {
   hdr = *reinterpret_cast<const uint4*>(blk);
-  const uint4 a = *reinterpret_cast<const uint4*>(blk + 16 + 32 * c);
-  const uint4 b = *reinterpret_cast<const uint4*>(blk + 32 + 32 * c);
-  q[0] = a.x; q[1] = a.y; q[2] = a.z; q[3] = a.w;
-  q[4] = b.x; q[5] = b.y; q[6] = b.z; q[7] = b.w;
+  const int sw = g & 1;
+  const uint4 a = *reinterpret_cast<const uint4*>(blk + 16 + 32 * c + 16 * sw);
+  const uint4 b = *reinterpret_cast<const uint4*>(blk + 32 + 32 * c - 16 * sw);
+  const uint4 lo = sw ? b : a, hi = sw ? a : b;
+  q[0] = lo.x; q[1] = lo.y; q[2] = lo.z; q[3] = lo.w;
+  q[4] = hi.x; q[5] = hi.y; q[6] = hi.z; q[7] = hi.w;
 }
 
 // 32 zero bytes: the B source of lanes that own no activations.
@@ -249,8 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
         const uint8_t* blk = stages + stage * kGuStageBytes + mat * kGuTileBytes + (rbase + g) * pitch + kp * kQBytes;
         uint4 h0, h8;
         uint32_t q[8], q8[8];
-        load_row_block(blk, c, h0, q);
-        load_row_block(blk + 8 * pitch, c, h8, q8);
+        load_row_block(blk, c, g, h0, q);
+        load_row_block(blk + 8 * pitch, c, g, h8, q8);
         const RowScales rs = decode_scales(h0, c), rs8 = decode_scales(h8, c);
 #pragma unroll
         for (int t = 0; t < kMaxTok; ++t) {
@@ -431,8 +437,8 @@ __global__ void __launch_bounds__(kThreads, 1) down_d1_kernel(DecodeArgs a) {
         const uint8_t* blk = stages + stage * kDnStageBytes + (rbase + g) * pitch + kp * kQBytes;
         uint4 h0, h8;
         uint32_t q[8], q8[8];
-        load_row_block(blk, c, h0, q);
-        load_row_block(blk + 8 * pitch, c, h8, q8);
+        load_row_block(blk, c, g, h0, q);
+        load_row_block(blk + 8 * pitch, c, g, h8, q8);
         const RowScales rs = decode_scales(h0, c), rs8 = decode_scales(h8, c);
 #pragma unroll
         for (int t = 0; t < kMaxTok; ++t) {

@@ -1,7 +1,9 @@
 // Host runtime of libmoe.so: the C ABI of include/moe.h.
 //
-// A layer owns its router weights, a device table of expert weight pointers
-// and per-call scratch.  Experts live either in a per-layer resident copy
+// A layer owns its router weights (fp32, and as three bf16 planes for the
+// tensor-core router), TMA tensor maps over every slot its experts can occupy,
+// a device table expert -> slot, and per-call scratch.  Experts live either in
+// a per-layer resident copy
 // (cache budget SIZE_MAX) or in the device-wide streaming cache: an arena of
 // fixed-size slots with a host-side LRU, filled from pinned host RAM by
 // cudaMemcpyAsync on an internal copy-engine stream (LayerStoRm README,
@@ -142,7 +144,6 @@ struct moe_layer {
   CUtensorMap wp_map{};                 // over d_Wp, for the tensor-core router
   std::vector<const uint8_t*> host;     // (E+S)*3 borrowed pinned pointers
   uint8_t* d_resident = nullptr;        // resident copy of all experts
-  const uint8_t** d_wptr = nullptr;     // device table (E+S)*3 of weight pointers
   CUtensorMap* d_tmaps = nullptr;       // [slots][kMapsPerSlot] TMA maps (resident: one slot per expert)
   size_t n_tmap_slots = 0;
   int* d_slot_of = nullptr;             // [E+S] expert -> slot of d_tmaps
@@ -189,7 +190,7 @@ moe_status ensure_scratch(moe_layer* L, int T) {
                o_x = take((size_t)cap * s.H * 2), o_o = take((size_t)cap * s.H * 2),
                o_xq = take((size_t)cap * s.H * 2), o_xsc = take((size_t)cap * (s.H / 32) * 8),
                o_hq = take(P * s.I_pad * 2), o_hsc = take(P * (s.I_pad / 32) * 8), o_act1 = take(ES * 4),
-               o_act2 = take(ES * 4), o_nact1 = take(4), o_nact2 = take(4), o_tcnt = take((size_t)(s.H / 64) * 4),
+               o_act2 = take(ES * 4), o_nact1 = take(4), o_nact2 = take(4),
                o_err = take(4), o_tiles = take(prefill_max_tiles((int)ES, P) * 16), o_ntiles = take(4),
                o_x16 = take(P * s.H * 2), o_rinv = take(P * 4), o_h16 = take(P * s.I_pad * 2), o_hinv = take(P * 4),
                o_rpart = take(router_part_floats(cap, s.E, s.n_sm) * 4);
@@ -231,7 +232,6 @@ moe_status ensure_scratch(moe_layer* L, int T) {
   L->wk.act2 = reinterpret_cast<int*>(b + o_act2);
   L->wk.n_act1 = reinterpret_cast<int*>(b + o_nact1);
   L->wk.n_act2 = reinterpret_cast<int*>(b + o_nact2);
-  L->wk.tile_cnt = reinterpret_cast<unsigned*>(b + o_tcnt);
   L->wk.err = reinterpret_cast<unsigned*>(b + o_err);
   L->wk.tiles = reinterpret_cast<int4*>(b + o_tiles);
   L->wk.n_tiles = reinterpret_cast<int*>(b + o_ntiles);
@@ -390,7 +390,7 @@ moe_status resolve_experts(moe_layer* L, const int32_t* ids, int n, cudaStream_t
   MOE_TRY(refresh_stream_maps(L));
   Cache* c = g_cache;
   c->epoch++;
-  PtrUpdate u{};
+  SlotUpdate u{};
   for (int e = 0; e < s.E + s.S; ++e) {
     if (!need[e]) continue;
     int slot;
@@ -399,15 +399,14 @@ moe_status resolve_experts(moe_layer* L, const int32_t* ids, int n, cudaStream_t
     used_slots->push_back(slot);
     u.expert[u.n] = e;
     u.slot[u.n] = slot;
-    u.base[u.n] = c->arena + (size_t)slot * c->slot_bytes;
-    if (++u.n == PtrUpdate::kMax) {
-      CUDA_TRY(launch_set_ptrs(L->d_wptr, L->d_slot_of, u, L->gate_bytes, st));
+    if (++u.n == SlotUpdate::kMax) {
+      CUDA_TRY(launch_set_slots(L->d_slot_of, u, st));
       g_stats.launches++;
       u.n = 0;
     }
   }
   if (u.n) {
-    CUDA_TRY(launch_set_ptrs(L->d_wptr, L->d_slot_of, u, L->gate_bytes, st));
+    CUDA_TRY(launch_set_slots(L->d_slot_of, u, st));
     g_stats.launches++;
   }
   return MOE_OK;
@@ -468,7 +467,6 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
                  wk.logits, wk.ids, wk.w, wk.counts, wk.offsets, wk.perm, wk.inv, wk.act1, wk.n_act1, wk.act2,
                  wk.n_act2, wk.n_act, wk.xq, wk.xq_plane, wk.xsc, wk.ticket};
     MOE_KERNEL(MOE_K_ROUTER, launch_route_decode(ra, st));
-    ++n_launch;  // route = logits kernel + finishing kernel (one profiled range)
   } else {
     // router on the tensor cores: split-K partial logits, summed in split order by top-k
     CUtensorMap xmap;
@@ -507,7 +505,6 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     da.slot_of = L->d_slot_of;
     da.act = wk.act1;
     da.n_act = wk.n_act1;
-    da.n_act_total = wk.n_act;
     da.counts = wk.counts;
     da.offsets = wk.offsets;
     da.perm = wk.perm;
@@ -530,7 +527,6 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     da.hsc = wk.hsc;
     da.y = wk.y;
     da.out = static_cast<__nv_bfloat16*>(out);
-    da.tile_cnt = wk.tile_cnt;
     da.err = wk.err;
     da.stage_x = stage_x ? 1 : 0;
     da.act_slot_bytes = act_slot;
@@ -627,8 +623,6 @@ moe_status moe_layer_create(int hidden, int inter, int n_experts, int top_k, int
   L->expert_bytes = 2 * L->gate_bytes + L->down_bytes;
   cudaError_t e = cudaGetDevice(&L->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&s.n_sm, cudaDevAttrMultiProcessorCount, L->device);
-  if (e == cudaSuccess) e = cudaMalloc(&L->d_wptr, sizeof(void*) * 3 * (size_t)(s.E + s.S));
-  if (e == cudaSuccess) e = cudaMemset(L->d_wptr, 0, sizeof(void*) * 3 * (size_t)(s.E + s.S));
   if (e == cudaSuccess) e = cudaMalloc(&L->d_slot_of, sizeof(int) * (size_t)(s.E + s.S));
   if (e == cudaSuccess) e = cudaMemset(L->d_slot_of, 0, sizeof(int) * (size_t)(s.E + s.S));
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->copy, cudaStreamNonBlocking);
@@ -665,7 +659,6 @@ moe_status moe_layer_destroy(moe_layer_t L) {
   if (L->d_b) cudaFree(L->d_b);
   if (L->d_Wp) cudaFree(L->d_Wp);
   if (L->d_resident) cudaFree(L->d_resident);
-  if (L->d_wptr) cudaFree(L->d_wptr);
   if (L->d_tmaps) cudaFree(L->d_tmaps);
   if (L->d_slot_of) cudaFree(L->d_slot_of);
   if (L->scratch) cudaFree(L->scratch);
@@ -732,7 +725,6 @@ moe_status moe_set_experts(moe_layer_t L, const void* const* gate, const void* c
   if (budget == SIZE_MAX) {
     // resident: one device copy of every expert, uploaded now
     if (!L->d_resident) CUDA_TRY(cudaMalloc(&L->d_resident, (size_t)n * L->expert_bytes));
-    std::vector<const uint8_t*> table(3 * (size_t)n);
     for (int e = 0; e < n; ++e) {
       uint8_t* dst = L->d_resident + (size_t)e * L->expert_bytes;
       const size_t sz[3] = {L->gate_bytes, L->gate_bytes, L->down_bytes};
@@ -740,11 +732,8 @@ moe_status moe_set_experts(moe_layer_t L, const void* const* gate, const void* c
       for (int m = 0; m < 3; ++m) {
         CUDA_TRY(cudaMemcpyAsync(dst + off[m], L->host[3 * (size_t)e + m], sz[m], cudaMemcpyHostToDevice,
                                  L->copy));
-        table[3 * (size_t)e + m] = dst + off[m];
       }
     }
-    CUDA_TRY(cudaMemcpyAsync(L->d_wptr, table.data(), sizeof(void*) * table.size(), cudaMemcpyHostToDevice,
-                             L->copy));
     CUDA_TRY(cudaStreamSynchronize(L->copy));
     MOE_TRY(build_maps(L, L->d_resident, L->expert_bytes, (size_t)n));
     std::vector<int> ident(n);

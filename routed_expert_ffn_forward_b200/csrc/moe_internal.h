@@ -47,7 +47,6 @@ struct Work {
   int* n_act1;
   int* act2;          // experts with more rows
   int* n_act2;
-  unsigned* tile_cnt; // [ceil(H/64)] finished expert units per output row tile
   unsigned* err;      // device-side error flags (timeouts)
   // prefill path (tensor-core GEMMs)
   int4* tiles;        // [max tiles] (expert, n0, count, r0): up to 256 rows of one expert
@@ -83,7 +82,6 @@ struct DecodeArgs {
   const int* slot_of;        // [E+S] expert -> slot
   const int* act;            // experts this kernel handles
   const int* n_act;
-  const int* n_act_total;    // all experts with rows (units per output row tile)
   const int *counts, *offsets, *perm, *inv;
   const float* w;
   int kS, T, k, S;
@@ -96,7 +94,6 @@ struct DecodeArgs {
   float2* hsc;
   float* y;
   __nv_bfloat16* out;
-  unsigned* tile_cnt;
   unsigned* err;
   int stage_x;            // gate/up: copy x (all T tokens) to shared memory once per CTA
   size_t act_slot_bytes;  // down: bytes of one activation slot (2 * max_tok * I_pad + scales)
@@ -179,22 +176,18 @@ cudaError_t launch_topk(float* logits, int T, int E, int k, int gating,
                         const float* part = nullptr, int nsplit = 0, size_t split_stride = 0,
                         const float* bias = nullptr);
 cudaError_t launch_permute(const int* ids, int T, const Shape& s, const Work& wk, cudaStream_t st);
-cudaError_t launch_gate_up_simt(const uint8_t* const* wptr, const __nv_bfloat16* x, const Shape& s,
-                                const Work& wk, cudaStream_t st);
-cudaError_t launch_down_simt(const uint8_t* const* wptr, const Shape& s, const Work& wk, cudaStream_t st);
 cudaError_t launch_combine(const Work& wk, int T, const Shape& s, __nv_bfloat16* out, cudaStream_t st,
                            bool pdl = false);
 
-// Streaming cache: point experts at their cache slots (device pointer table).
-struct PtrUpdate {
+// Streaming cache: point experts at their cache slots (the slot_of table the
+// kernels index tensor maps with).
+struct SlotUpdate {
   static constexpr int kMax = 64;
   int n;
   int expert[kMax];
   int slot[kMax];
-  const uint8_t* base[kMax];
 };
-cudaError_t launch_set_ptrs(const uint8_t** table, int* slot_of, const PtrUpdate& u, size_t gate_bytes,
-                            cudaStream_t st);
+cudaError_t launch_set_slots(int* slot_of, const SlotUpdate& u, cudaStream_t st);
 
 // Set / clear the thread-local message returned by moe_last_error().
 int report_error(int status, const char* msg);

@@ -120,15 +120,9 @@ permute_kernel(const int* __restrict__ ids, int T, int E, int k, int S, int* __r
   }
 }
 
-__global__ void set_ptrs_kernel(const uint8_t** table, int* slot_of, PtrUpdate u, size_t gate_bytes) {
+__global__ void set_slots_kernel(int* slot_of, SlotUpdate u) {
   const int i = threadIdx.x;
-  if (i < u.n) {
-    const int e = u.expert[i];
-    slot_of[e] = u.slot[i];
-    table[3 * e + 0] = u.base[i];
-    table[3 * e + 1] = u.base[i] + gate_bytes;
-    table[3 * e + 2] = u.base[i] + 2 * gate_bytes;
-  }
+  if (i < u.n) slot_of[u.expert[i]] = u.slot[i];
 }
 
 }  // namespace
@@ -139,9 +133,8 @@ cudaError_t launch_permute(const int* ids, int T, const Shape& s, const Work& wk
   return cudaGetLastError();
 }
 
-cudaError_t launch_set_ptrs(const uint8_t** table, int* slot_of, const PtrUpdate& u, size_t gate_bytes,
-                            cudaStream_t st) {
-  set_ptrs_kernel<<<1, PtrUpdate::kMax, 0, st>>>(table, slot_of, u, gate_bytes);
+cudaError_t launch_set_slots(int* slot_of, const SlotUpdate& u, cudaStream_t st) {
+  set_slots_kernel<<<1, SlotUpdate::kMax, 0, st>>>(slot_of, u);
   return cudaGetLastError();
 }
 

@@ -1,18 +1,18 @@
-// Decode-path routing (T <= 64): two kernels chained with programmatic
-// dependent launch.
+// Decode-path routing (T <= 4): one kernel.
 //
-// route_logits_kernel: one CTA per expert computes that expert's logits for
-// every token (256 threads share the row, four tokens at a time, partial sums
-// reduced in a fixed order).  Independently of routing, every CTA also
-// converts a slice of x: each 32-element run becomes 16-bit fixed point with
-// its own power-of-two scale (a high-byte and a low-byte plane), with the
-// run's scale and sum -- the form the expert kernels read.
+// Each of E CTAs computes one expert's logits for every token (256 threads
+// share the weight row, four tokens at a time, partial sums reduced in a
+// fixed order).  Independently of routing, every CTA also converts a slice of
+// x: each 32-element run becomes 16-bit fixed point with its own power-of-two
+// scale (a high-byte and a low-byte plane), with the run's scale and sum --
+// the form the expert kernels read.
 //
-// route_finish_kernel: one CTA does the top-k + gating of every token (a warp
-// per token) and the stable counting-sort permutation of the T*k picks.  With
-// few picks (N = T*k <= 2048) each pick's sorted position is found by counting
-// the picks before it in (expert, token, slot) order, so no pass over all E
-// expert counters is needed; only experts with rows get counts and offsets.
+// The last CTA to finish (a device-wide ticket) then does the top-k + gating
+// of every token (a warp per token) and the stable counting-sort permutation
+// of the T*k picks.  With few picks each pick's sorted position is found by
+// counting the picks before it in (expert, token, slot) order, so no pass over
+// all E expert counters is needed; only experts with rows get counts and
+// offsets.
 #include "moe_internal.h"
 #include "ptx.cuh"
 #include "topk.cuh"
@@ -21,13 +21,18 @@ namespace moe {
 namespace {
 
 constexpr int kLogitThreads = 256;
-constexpr int kFinishThreads = 256;
 
-__global__ void __launch_bounds__(kLogitThreads) route_logits_kernel(RouteArgs a) {
+template <int PL>
+__device__ void route_finish(const RouteArgs& a, int* s_ids);
+
+template <int PL>
+__global__ void __launch_bounds__(kLogitThreads) route_kernel(RouteArgs a) {
+  extern __shared__ int s_dyn[];  // the finishing CTA's pick lists
   __shared__ float s_red[kLogitThreads / 32][4];
+  __shared__ bool s_last;
   const int e = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, T = a.T, E = a.E;
-  // the first kernel of a forward: let the finishing kernel start launching now
+  // the first kernel of a forward: let the expert kernel start launching now
   ptx::pdl_launch_dependents();
 
   // (1) x prep: 16-bit fixed point per 32-element run, with the run scales
@@ -79,29 +84,39 @@ __global__ void __launch_bounds__(kLogitThreads) route_logits_kernel(RouteArgs a
     }
     __syncthreads();
   }
+  // last CTA to finish: routing of every token (one device-scope fence on each
+  // side of the ticket, cumulative over the writes the barriers order)
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    s_last = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
+    __threadfence();
+  }
+  __syncthreads();
+  if (!s_last) return;
+  route_finish<PL>(a, s_dyn);
+  if (tid == 0) *a.ticket = 0u;
 }
 
 template <int PL>
-__global__ void __launch_bounds__(kFinishThreads) route_finish_kernel(RouteArgs a) {
-  extern __shared__ int s_ids[];          // [N]
+__device__ void route_finish(const RouteArgs& a, int* s_ids) {
   __shared__ int s_cnt_small, s_cnt_big;  // distinct routed experts with <= / > kD1MaxTok rows
   const int tid = threadIdx.x, warp = tid >> 5;
   const int T = a.T, E = a.E, k = a.k, S = a.S, kS = k + S, N = T * k;
   int* s_first = s_ids + N;               // [N] 1 if pick i is its expert's first pick
   int* s_count = s_first + N;             // [N] rows of pick i's expert
-  ptx::pdl_wait();                        // the logits
-  ptx::pdl_launch_dependents();
   if (tid == 0) {
     s_cnt_small = 0;
     s_cnt_big = 0;
   }
+  __syncthreads();
   // top-k + gating, one warp per token
-  for (int t = warp; t < T; t += kFinishThreads / 32)
+  for (int t = warp; t < T; t += kLogitThreads / 32)
     warp_topk_gate<PL, true>(a.logits + (size_t)t * E, E, k, a.gating, a.forced ? a.forced + (size_t)t * k : nullptr,
                              s_ids + t * k, a.w + (size_t)t * k);
   __syncthreads();
   // per pick: rows of its expert, whether it is the expert's first pick
-  for (int i = tid; i < N; i += kFinishThreads) {
+  for (int i = tid; i < N; i += kLogitThreads) {
     const int ex = s_ids[i];
     int cnt = 0, before = 0;
     for (int j = 0; j < N; ++j) {
@@ -116,7 +131,7 @@ __global__ void __launch_bounds__(kFinishThreads) route_finish_kernel(RouteArgs 
   __syncthreads();
   // sorted positions: picks of smaller experts first, then earlier picks of
   // the same expert; first picks also place their expert in the active lists
-  for (int i = tid; i < N; i += kFinishThreads) {
+  for (int i = tid; i < N; i += kLogitThreads) {
     const int ex = s_ids[i];
     int lt = 0, eq_before = 0, d_small = 0, d_big = 0;
     for (int j = 0; j < N; ++j) {
@@ -144,7 +159,7 @@ __global__ void __launch_bounds__(kFinishThreads) route_finish_kernel(RouteArgs 
     }
   }
   // shared experts: all T tokens, after the routed rows
-  for (int i = tid; i < T * S; i += kFinishThreads) {
+  for (int i = tid; i < T * S; i += kLogitThreads) {
     const int s = i / T, t = i - s * T;
     const int r = N + s * T + t;
     a.perm[r] = t * kS + k + s;
@@ -179,21 +194,12 @@ size_t route_decode_smem(int H, int T, int E, int k, int S) {
 }
 
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st) {
-  route_logits_kernel<<<a.E, kLogitThreads, 0, st>>>(a);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(1);
-  cfg.blockDim = dim3(kFinishThreads);
-  cfg.dynamicSmemBytes = route_decode_smem(a.H, a.T, a.E, a.k, a.S);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if ((a.E + 31) / 32 <= 8) return cudaLaunchKernelEx(&cfg, route_finish_kernel<8>, a);
-  return cudaLaunchKernelEx(&cfg, route_finish_kernel<32>, a);
+  const size_t smem = route_decode_smem(a.H, a.T, a.E, a.k, a.S);
+  if ((a.E + 31) / 32 <= 8)
+    route_kernel<8><<<a.E, kLogitThreads, smem, st>>>(a);
+  else
+    route_kernel<32><<<a.E, kLogitThreads, smem, st>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace moe

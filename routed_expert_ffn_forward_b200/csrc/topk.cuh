@@ -7,26 +7,26 @@
 
 namespace moe {
 
-// (value, index) order of the top-k: larger logit first, equal logits to the
-// lower expert index.  `ok` false means "no candidate".
-struct TopkCand {
-  float v;
-  int e;
-  bool ok;
-};
-__device__ __forceinline__ bool topk_better(const TopkCand& a, const TopkCand& b) {
-  if (a.ok != b.ok) return a.ok;
-  if (!a.ok) return false;
-  return a.v > b.v || (a.v == b.v && a.e < b.e);
+// Order-preserving map of a logit to an unsigned key (larger logit, larger
+// key; -0 is taken as +0 so that equal logits get equal keys).  Key 0 is
+// reserved for "no candidate" (it would be the key of a negative NaN).
+__device__ __forceinline__ uint32_t topk_key(float v) {
+  const uint32_t b = __float_as_uint(v + 0.0f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float topk_unkey(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
 // Called by a full warp.  lt: the token's E logits.  Lane l holds logits
-// l, l+32, ... (PL per lane, E <= 32*PL); k rounds of a warp arg-max pick the
-// experts in decreasing order and lane r keeps round r's pick.  With `forced`
-// (k ids) the picks are given.  Gating over the k picks: softmax (gating 0) or
-// sigmoid renormalised to sum 1 (gating 1).  Writes ids[0..k) and w[0..k).
-// kL2 reads the logits through L2 only (they were written by other CTAs of the
-// same kernel).
+// l, l+32, ... (PL per lane, E <= 32*PL).  k rounds pick the experts in
+// decreasing order -- larger logit first, equal logits to the lower expert
+// index -- each round one warp max-reduction of the keys and one
+// min-reduction of the indices that hold the max; lane r keeps round r's pick.
+// With `forced` (k ids) the picks are given.  Gating over the k picks: softmax
+// (gating 0) or sigmoid renormalised to sum 1 (gating 1).  Writes ids[0..k)
+// and w[0..k).  kL2 reads the logits through L2 only (they were written by
+// other CTAs of the same kernel).
 template <int PL, bool kL2 = false>
 __device__ __forceinline__ void warp_topk_gate(const float* __restrict__ lt, int E, int k, int gating,
                                                const int* __restrict__ forced, int* __restrict__ ids,
@@ -40,37 +40,30 @@ __device__ __forceinline__ void warp_topk_gate(const float* __restrict__ lt, int
       my_l = kL2 ? __ldcg(lt + my_e) : lt[my_e];
     }
   } else {
-    float v[PL];
-    bool taken[PL];
+    uint32_t key[PL];
 #pragma unroll
     for (int i = 0; i < PL; ++i) {
       const int e = lane + 32 * i;
-      taken[i] = e >= E;
-      v[i] = taken[i] ? 0.f : (kL2 ? __ldcg(lt + e) : lt[e]);
+      key[i] = e < E ? topk_key(kL2 ? __ldcg(lt + e) : lt[e]) : 0u;
     }
     for (int r = 0; r < k; ++r) {
-      TopkCand c{0.f, 0, false};
+      uint32_t bk = 0u, bi = 0xFFFFFFFFu;
 #pragma unroll
-      for (int i = 0; i < PL; ++i) {
-        const TopkCand d{v[i], lane + 32 * i, !taken[i]};
-        if (topk_better(d, c)) c = d;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        TopkCand d;
-        d.v = __shfl_xor_sync(0xffffffffu, c.v, o);
-        d.e = __shfl_xor_sync(0xffffffffu, c.e, o);
-        d.ok = __shfl_xor_sync(0xffffffffu, (int)c.ok, o);
-        if (topk_better(d, c)) c = d;
-      }
+      for (int i = 0; i < PL; ++i)
+        if (key[i] > bk) {
+          bk = key[i];
+          bi = (uint32_t)(lane + 32 * i);
+        }
+      const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t win = __reduce_min_sync(0xffffffffu, bk == m ? bi : 0xFFFFFFFFu);
       if (lane == r) {
-        my_e = c.e;
-        my_l = c.v;
+        my_e = (int)win;
+        my_l = topk_unkey(m);
       }
-      if ((c.e & 31) == lane) {
+      if ((int)(win & 31u) == lane) {
 #pragma unroll
         for (int i = 0; i < PL; ++i)
-          if (i == (c.e >> 5)) taken[i] = true;
+          if (i == (int)(win >> 5)) key[i] = 0u;
       }
     }
   }
