@@ -1,8 +1,7 @@
 // Decode-path routing (T <= 4): one kernel.
 //
 // Each of E CTAs computes one expert's logits for every token (256 threads
-// share the weight row, four tokens at a time, partial sums reduced in a
-// fixed order).  Independently of routing, every CTA also converts a slice of
+// share the weight row; partial sums reduced in a fixed order).  Independently of routing, every CTA also converts a slice of
 // x: each 32-element run becomes 16-bit fixed point with its own power-of-two
 // scale (a high-byte and a low-byte plane), with the run's scale and sum --
 // the form the expert kernels read.
@@ -25,17 +24,70 @@ constexpr int kLogitThreads = 256;
 template <int PL>
 __device__ void route_finish(const RouteArgs& a, int* s_ids);
 
-template <int PL>
-__global__ void __launch_bounds__(kLogitThreads) route_kernel(RouteArgs a) {
+// kT: 1 (decode of one token) or kD1MaxTok (up to that many tokens)
+template <int PL, int kT>
+__global__ void __launch_bounds__(kLogitThreads, 2) route_kernel(RouteArgs a) {
   extern __shared__ int s_dyn[];  // the finishing CTA's pick lists
-  __shared__ float s_red[kLogitThreads / 32][4];
+  __shared__ float s_red[kLogitThreads / 32][kD1MaxTok];
   __shared__ bool s_last;
   const int e = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, T = a.T, E = a.E;
   // the first kernel of a forward: let the expert kernel start launching now
   ptx::pdl_launch_dependents();
 
-  // (1) x prep: 16-bit fixed point per 32-element run, with the run scales
+  // (1) logits of expert e for the T <= 4 tokens (first: the weight row is the
+  // long-latency load); thread takes 4-element pieces h = 4*tid + 1024*i
+  // The thread's weight and activation pieces of a pass are all loaded before
+  // any arithmetic, so the CTA waits for one memory round trip per pass.
+  constexpr int kPieces = 8;                     // per pass: H <= 8192 takes one pass
+  const float4* wrow = reinterpret_cast<const float4*>(a.W + (size_t)e * H);
+  const float bias = a.b ? a.b[e] : 0.f;
+  const int nq = H / 4;
+  float acc[kT];
+#pragma unroll
+  for (int t = 0; t < kT; ++t) acc[t] = 0.f;
+  for (int base = 0; base < nq; base += kPieces * kLogitThreads) {
+    float4 w4[kPieces];
+    uint2 xv[kT][kPieces];
+#pragma unroll
+    for (int i = 0; i < kPieces; ++i) {
+      const int q = base + tid + kLogitThreads * i;
+      if (q < nq) {
+        w4[i] = __ldg(wrow + q);
+#pragma unroll
+        for (int t = 0; t < kT; ++t)
+          if (t < T) xv[t][i] = __ldg(reinterpret_cast<const uint2*>(a.x + (size_t)t * H) + q);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kT; ++t) {
+      if (t < T) {
+#pragma unroll
+        for (int i = 0; i < kPieces; ++i) {
+          if (base + tid + kLogitThreads * i < nq) {
+            acc[t] = fmaf(w4[i].x, bf16lo(xv[t][i].x), acc[t]);
+            acc[t] = fmaf(w4[i].y, bf16hi(xv[t][i].x), acc[t]);
+            acc[t] = fmaf(w4[i].z, bf16lo(xv[t][i].y), acc[t]);
+            acc[t] = fmaf(w4[i].w, bf16hi(xv[t][i].y), acc[t]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < kT; ++t) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+    if (lane == 0) s_red[warp][t] = acc[t];
+  }
+  __syncthreads();
+  if (warp == 0 && lane < T) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kLogitThreads / 32; ++w) v += s_red[w][lane];
+    a.logits[(size_t)lane * E + e] = v + bias;
+  }
+  // (2) x prep: 16-bit fixed point per 32-element run, with the run scales
   const int runs_per_tok = H / 32;
   for (int run = e + gridDim.x * warp; run < T * runs_per_tok; run += gridDim.x * (kLogitThreads / 32)) {
     const int t = run / runs_per_tok, r = run - t * runs_per_tok;
@@ -49,41 +101,6 @@ __global__ void __launch_bounds__(kLogitThreads) route_kernel(RouteArgs a) {
     if (lane == 0) a.xsc[(size_t)t * runs_per_tok + r] = rsc;
   }
 
-  // (2) logits of expert e: thread takes 4-element pieces h = 4*tid + 1024*i
-  const float4* wrow = reinterpret_cast<const float4*>(a.W + (size_t)e * H);
-  const float bias = a.b ? a.b[e] : 0.f;
-  for (int t0 = 0; t0 < T; t0 += 4) {
-    const int nt = min(4, T - t0);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int q = tid; q < H / 4; q += kLogitThreads) {
-      const float4 w4 = __ldg(wrow + q);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (i < nt) {
-          const uint2 xv = __ldg(reinterpret_cast<const uint2*>(a.x + (size_t)(t0 + i) * H) + q);
-          acc[i] = fmaf(w4.x, bf16lo(xv.x), acc[i]);
-          acc[i] = fmaf(w4.y, bf16hi(xv.x), acc[i]);
-          acc[i] = fmaf(w4.z, bf16lo(xv.y), acc[i]);
-          acc[i] = fmaf(w4.w, bf16hi(xv.y), acc[i]);
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-      if (lane == 0) s_red[warp][i] = acc[i];
-    }
-    __syncthreads();
-    if (warp == 0 && lane < nt) {
-      float v = 0.f;
-#pragma unroll
-      for (int w = 0; w < kLogitThreads / 32; ++w) v += s_red[w][lane];
-      a.logits[(size_t)(t0 + lane) * E + e] = v + bias;
-    }
-    __syncthreads();
-  }
   // last CTA to finish: routing of every token (one device-scope fence on each
   // side of the ticket, cumulative over the writes the barriers order)
   __syncthreads();
@@ -195,10 +212,19 @@ size_t route_decode_smem(int H, int T, int E, int k, int S) {
 
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st) {
   const size_t smem = route_decode_smem(a.H, a.T, a.E, a.k, a.S);
-  if ((a.E + 31) / 32 <= 8)
-    route_kernel<8><<<a.E, kLogitThreads, smem, st>>>(a);
-  else
-    route_kernel<32><<<a.E, kLogitThreads, smem, st>>>(a);
+  if (a.T > kD1MaxTok) return cudaErrorInvalidValue;
+  const bool small_e = (a.E + 31) / 32 <= 8;
+  if (a.T == 1) {
+    if (small_e)
+      route_kernel<8, 1><<<a.E, kLogitThreads, smem, st>>>(a);
+    else
+      route_kernel<32, 1><<<a.E, kLogitThreads, smem, st>>>(a);
+  } else {
+    if (small_e)
+      route_kernel<8, kD1MaxTok><<<a.E, kLogitThreads, smem, st>>>(a);
+    else
+      route_kernel<32, kD1MaxTok><<<a.E, kLogitThreads, smem, st>>>(a);
+  }
   return cudaGetLastError();
 }
 
