@@ -102,13 +102,15 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_traffic(kernel: str) -> float | None:
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
-    kernel's source has not changed since the capture."""
+def kernel_traffic(key: str) -> float | None:
+    """DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)
+    of the kernel recorded under `key` ("config<N>:<kernel>") in
+    profiles/traffic.json, if the kernel's source has not changed since the
+    capture; None otherwise."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p)).get(kernel)
+    d = json.load(open(p)).get(key)
     if not d:
         return None
     src = os.path.join(ROOT, d["source"])
@@ -326,7 +328,7 @@ def run_ours(args, cfg, rank: int, world: int, local_rank: int) -> dict | None:
         achieved = fl / (avg_ms / 1e3) / 1e12
         peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "kernel": kern, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": kernel_traffic(kern), "peak_source": peaks["source"]}
+                "frac": achieved / peak, "traffic": kernel_traffic(f"config{args.config}:{kern}"), "peak_source": peaks["source"]}
     else:
         kern = "gate_up"
         ab = float(np.mean([algorithmic_bytes(cfg, ids, kern) for ids in ids_cycle]))
@@ -334,7 +336,7 @@ def run_ours(args, cfg, rank: int, world: int, local_rank: int) -> dict | None:
         achieved = ab / (avg_ms / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": kernel_traffic(kern), "algorithmic_bytes": ab,
+                "frac": achieved / peak, "traffic": kernel_traffic(f"config{args.config}:{kern}"), "algorithmic_bytes": ab,
                 "peak_source": peaks["source"]}
     fwd_bytes = float(np.mean([algorithmic_bytes(cfg, ids, "forward") for ids in ids_cycle]))
     fwd_ms = total_ms / args.steps

@@ -67,8 +67,8 @@ typedef enum {
 typedef struct {
   uint64_t forwards;        /* moe_forward* calls that launched work */
   uint64_t tokens;          /* sum of T over those calls */
-  uint64_t decode_calls;    /* calls that took the decode path (T <= 64) */
-  uint64_t prefill_calls;   /* calls that took the prefill path (T > 64) */
+  uint64_t decode_calls;    /* calls that took the decode path (T <= 4) */
+  uint64_t prefill_calls;   /* calls that took the prefill path (T > 4) */
   uint64_t cache_hits;      /* streamed experts found in the cache */
   uint64_t cache_misses;    /* streamed experts fetched on demand */
   uint64_t prefetches;      /* experts fetched by moe_prefetch */
@@ -144,9 +144,13 @@ moe_status moe_set_experts(moe_layer_t layer, const void* const* gate,
 moe_status moe_set_cache_bytes(size_t bytes);
 
 /* Forward: x bf16 [T, H] and out bf16 [T, H], device pointers, row-major.
- * T >= 0 (T = 0 returns at once).  T <= 64 takes the decode path, larger T the
- * prefill path.  Work is enqueued on `stream`; in resident mode the call does
- * not wait for the GPU.  In streaming mode it reads the routing back to the
+ * T >= 0 (T = 0 returns at once).  T <= 4 takes the decode path (fused router,
+ * expert kernels on the integer tensor MMA straight from the Q4_K bytes),
+ * larger T the prefill path (router and expert projections as tcgen05 grouped
+ * GEMMs; the Q4_K weights are dequantised to fp16 in shared memory, which
+ * requires every block's |d| < 0.248 and |dmin| < 3.72, i.e. weights within
+ * about +-234; moe_check reports a violation).  Work is enqueued on `stream`;
+ * in resident mode the call does not wait for the GPU.  In streaming mode it reads the routing back to the
  * host (one stream synchronisation) to resolve cache misses before the expert
  * kernels are launched.  out must not overlap x. */
 moe_status moe_forward(moe_layer_t layer, const void* x, void* out, int T, void* stream);
@@ -181,8 +185,9 @@ moe_status moe_prefetch(moe_layer_t layer, const int32_t* ids, int n);
 /* Wait for all work on the layer's GPU, then report whether one of the layer's
  * kernels gave up on a bounded wait (a shared-memory pipeline barrier that did
  * not complete within its time limit; the kernel then stops early and its
- * output is invalid).  Returns MOE_ERR_CUDA with a message in that case and
- * clears the record; MOE_OK otherwise. */
+ * output is invalid) or met a Q4_K block outside the fp16 range of the
+ * prefill path.  Returns MOE_ERR_CUDA with a message in that case and clears
+ * the record; MOE_OK otherwise. */
 moe_status moe_check(moe_layer_t layer);
 
 moe_status moe_get_stats(moe_stats* out);

@@ -575,7 +575,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     }
     g_stats.forwards++;
     g_stats.tokens += (uint64_t)T;
-    if (T <= kDecodeMaxT)
+    if (fast)
       g_stats.decode_calls++;
     else
       g_stats.prefill_calls++;

@@ -15,7 +15,6 @@ namespace moe {
 
 constexpr int kQK = 256;        // weights per Q4_K super-block
 constexpr int kQBytes = 144;    // bytes per Q4_K super-block
-constexpr int kDecodeMaxT = 64; // T <= this takes the decode path
 constexpr int kD1MaxTok = 4;    // experts with <= this many rows use the per-sub-block decode kernels
 constexpr int kTileRows = 64;   // weight rows per decode work unit
 
