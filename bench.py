@@ -121,10 +121,15 @@ def kernel_traffic(key: str) -> float | None:
 
 def algorithmic_bytes(cfg, ids: np.ndarray, which: str) -> float:
     """Bytes a kernel must move at least once per launch for this routing.
-    gate_up: gate+up weights of every active expert, x rows, h writes (fp32).
-    forward: every active expert's weights, the router weight, x and out."""
+    gate_up: gate+up weights of every expert the kernel runs, x rows, h writes.
+    forward: every active expert's weights, the router weight, x and out.
+    For T > 4 the gate/up kernel is the tensor-core GEMM, which runs the
+    experts with more than 4 rows (the others take the decode kernels)."""
     T = ids.shape[0]
     active = len(np.unique(ids)) + cfg.n_shared
+    if which == "gate_up" and T > 4:
+        counts = np.bincount(ids.ravel(), minlength=cfg.n_experts)
+        active = int(np.sum(counts > 4)) + cfg.n_shared
     nb_h, nb_i = cfg.hidden // 256, (cfg.inter + 255) // 256
     gate = cfg.inter * nb_h * 144
     down = cfg.hidden * nb_i * 144

@@ -89,8 +89,9 @@ enum {
   MOE_K_DOWN = 4,    /* down projection */
   MOE_K_COMBINE = 5, /* weighted combine */
   MOE_K_PREP = 6,    /* prefill only: activation rows and SwiGLU output to scaled fp16 */
-  MOE_K_FORWARD = 7, /* whole forward, first kernel start to last kernel end */
-  MOE_K_COUNT = 8
+  MOE_K_SMALL = 7,   /* prefill only: the decode kernels for experts with <= 4 rows */
+  MOE_K_FORWARD = 8, /* whole forward, first kernel start to last kernel end */
+  MOE_K_COUNT = 9
 };
 typedef struct {
   uint64_t forwards;             /* forwards profiled */

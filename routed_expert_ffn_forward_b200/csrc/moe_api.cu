@@ -90,7 +90,7 @@ uint64_t g_cache_gen = 0;
 
 // Profiling: events recorded around each kernel launch of a forward, in launch
 // order, each range attributed to one MOE_K_* step; resolved by moe_get_profile.
-constexpr int kProfRanges = 12;              // launches per forward at most
+constexpr int kProfRanges = 16;              // launches per forward at most
 struct ProfRec {
   int n = 0;
   int kid[kProfRanges];
@@ -499,45 +499,51 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     lk.lock();
     MOE_TRY(resolve_experts(L, hid, T * s.k, st, &used));
   }
+  // arguments of the per-sub-block decode kernels (all experts on the decode
+  // path; on the prefill path the experts with <= kD1MaxTok rows)
+  DecodeArgs da{};
+  da.tmaps = L->d_tmaps;
+  da.slot_of = L->d_slot_of;
+  da.act = wk.act1;
+  da.n_act = wk.n_act1;
+  da.counts = wk.counts;
+  da.offsets = wk.offsets;
+  da.perm = wk.perm;
+  da.inv = wk.inv;
+  da.w = wk.w;
+  da.kS = s.k + s.S;
+  da.T = T;
+  da.k = s.k;
+  da.S = s.S;
+  da.H = s.H;
+  da.I = s.I;
+  da.I_pad = s.I_pad;
+  da.nbh = s.nbh;
+  da.nbi = s.nbi;
+  da.xq = wk.xq;
+  da.xq_plane = wk.xq_plane;
+  da.xsc = wk.xsc;
+  da.hq = wk.hq;
+  da.hq_plane = wk.hq_plane;
+  da.hsc = wk.hsc;
+  da.y = wk.y;
+  da.out = static_cast<__nv_bfloat16*>(out);
+  da.err = wk.err;
+  da.stage_x = stage_x ? 1 : 0;
+  da.act_slot_bytes = act_slot;
   if (fast) {
-    DecodeArgs da{};
-    da.tmaps = L->d_tmaps;
-    da.slot_of = L->d_slot_of;
-    da.act = wk.act1;
-    da.n_act = wk.n_act1;
-    da.counts = wk.counts;
-    da.offsets = wk.offsets;
-    da.perm = wk.perm;
-    da.inv = wk.inv;
-    da.w = wk.w;
-    da.kS = s.k + s.S;
-    da.T = T;
-    da.k = s.k;
-    da.S = s.S;
-    da.H = s.H;
-    da.I = s.I;
-    da.I_pad = s.I_pad;
-    da.nbh = s.nbh;
-    da.nbi = s.nbi;
-    da.xq = wk.xq;
-    da.xq_plane = wk.xq_plane;
-    da.xsc = wk.xsc;
-    da.hq = wk.hq;
-    da.hq_plane = wk.hq_plane;
-    da.hsc = wk.hsc;
-    da.y = wk.y;
-    da.out = static_cast<__nv_bfloat16*>(out);
-    da.err = wk.err;
-    da.stage_x = stage_x ? 1 : 0;
-    da.act_slot_bytes = act_slot;
     MOE_KERNEL(MOE_K_GATE_UP, launch_gate_up_d1(da, max_tok, s.n_sm, st));
     MOE_KERNEL(MOE_K_DOWN, launch_down_d1(da, max_tok, s.n_sm, st));
     MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true));
   } else {
-    // prefill: tensor-core GEMMs over tiles of up to 256 rows of one expert
+    // prefill: tensor-core GEMMs over tiles of up to 256 rows of one expert;
+    // experts with <= kD1MaxTok rows (when their kernels fit) stream through
+    // the decode kernels instead, which do not dequantise
     const int kS = s.k + s.S, P = T * kS;
+    const bool split_small = down_d1_smem(kD1MaxTok, act_slot) <= kMaxDecodeSmem;
     MOE_KERNEL(MOE_K_PERMUTE, launch_permute(wk.ids, T, s, wk, st));
-    MOE_KERNEL(MOE_K_PERMUTE, launch_build_tiles(wk, st));
+    MOE_KERNEL(MOE_K_PERMUTE, launch_build_tiles(wk, split_small ? kD1MaxTok : 0, st));
+    if (split_small) MOE_KERNEL(MOE_K_PREP, launch_quant_x(xb, wk, T, s.H, st));
     MOE_KERNEL(MOE_K_PREP, launch_gather_rows(xb, wk, P, kS, s.H, st));
     GemmArgs ga{};
     ga.wmaps = L->d_tmaps;
@@ -552,6 +558,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     ga.out_rows = s.I;
     ga.err = wk.err;
     MOE_KERNEL(MOE_K_GATE_UP, launch_prefill_gemm(0, L->x16_map, ga, s.n_sm, st));
+    if (split_small) MOE_KERNEL(MOE_K_SMALL, launch_gate_up_d1(da, kD1MaxTok, s.n_sm, st));
     MOE_KERNEL(MOE_K_PREP, launch_convert_h(wk, P, s.I, s.I_pad, st));
     ga.ft = s.H / 256;
     ga.nkb = s.nbi;
@@ -560,6 +567,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     ga.out_ld = s.H;
     ga.out_rows = s.H;
     MOE_KERNEL(MOE_K_DOWN, launch_prefill_gemm(1, L->h16_map, ga, s.n_sm, st));
+    if (split_small) MOE_KERNEL(MOE_K_SMALL, launch_down_d1(da, kD1MaxTok, s.n_sm, st));
     MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true));
   }
 #undef MOE_KERNEL

@@ -150,7 +150,9 @@ struct GemmArgs {
 };
 size_t prefill_gemm_smem();
 size_t prefill_max_tiles(int n_experts_total, size_t pairs);
-cudaError_t launch_build_tiles(const Work& wk, cudaStream_t st);
+// Tiles for the experts with more than small_rows rows; the others are listed in act1.
+cudaError_t launch_build_tiles(const Work& wk, int small_rows, cudaStream_t st);
+cudaError_t launch_quant_x(const __nv_bfloat16* x, const Work& wk, int T, int H, cudaStream_t st);
 cudaError_t launch_gather_rows(const __nv_bfloat16* x, const Work& wk, int P, int kS, int H, cudaStream_t st);
 cudaError_t launch_convert_h(const Work& wk, int P, int I, int I_pad, cudaStream_t st);
 cudaError_t launch_prefill_gemm(int mode, const CUtensorMap& bmap, const GemmArgs& a, int n_sm, cudaStream_t st);

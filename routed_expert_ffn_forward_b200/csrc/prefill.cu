@@ -383,31 +383,63 @@ done:
 }
 
 // ---------------------------------------------------------------- helper kernels
-// Tiles: each expert with rows, in chunks of kGN rows: (expert, n0, count, r0).
-// One block; experts are taken 1024 at a time with a block scan of their tile counts.
+// Tiles: each expert with more than `small_rows` rows, in chunks of kGN rows:
+// (expert, n0, count, r0).  Experts with 1..small_rows rows go to `small`
+// (for the decode kernels, which stream their weights once without
+// dequantising them).  One block; experts are taken 1024 at a time with block
+// scans of their tile counts and of their membership of `small`.
 __global__ void __launch_bounds__(1024) build_tiles_kernel(const int* __restrict__ act, const int* __restrict__ n_act,
                                                            const int* __restrict__ counts,
                                                            const int* __restrict__ offsets, int4* __restrict__ tiles,
-                                                           int* __restrict__ n_tiles) {
+                                                           int* __restrict__ n_tiles, int small_rows,
+                                                           int* __restrict__ small, int* __restrict__ n_small) {
   __shared__ int s_warp[32];
   ptx::pdl_wait();
   const int na = __ldcg(n_act);
-  int base = 0;
+  int base = 0, sbase = 0;
   for (int c0 = 0; c0 < na; c0 += blockDim.x) {
     const int i = c0 + threadIdx.x;
-    int e = 0, c = 0, r0 = 0, nt = 0;
+    int e = 0, c = 0, r0 = 0, nt = 0, sm = 0;
     if (i < na) {
       e = __ldcg(act + i);
       c = __ldcg(counts + e);
       r0 = __ldcg(offsets + e);
-      nt = (c + kGN - 1) / kGN;
+      sm = c <= small_rows ? 1 : 0;
+      nt = sm ? 0 : (c + kGN - 1) / kGN;
     }
-    int tot;
+    int tot, stot;
     const int pos = base + block_exclusive_scan_1024(nt, &tot, s_warp);
+    __syncthreads();
+    const int spos = sbase + block_exclusive_scan_1024(sm, &stot, s_warp);
     for (int j = 0; j < nt; ++j) tiles[pos + j] = make_int4(e, j * kGN, min(kGN, c - j * kGN), r0);
+    if (sm) small[spos] = e;
     base += tot;
+    sbase += stot;
+    __syncthreads();
   }
-  if (threadIdx.x == 0) *n_tiles = base;
+  if (threadIdx.x == 0) {
+    *n_tiles = base;
+    *n_small = sbase;
+  }
+}
+
+// x (bf16 [T, H]) as 16-bit fixed point per 32-element run for the decode
+// kernels: one warp per run.
+__global__ void __launch_bounds__(256) quant_x_kernel(const __nv_bfloat16* __restrict__ x, int T, int H,
+                                                       int8_t* __restrict__ xq, size_t plane, float2* __restrict__ xsc) {
+  ptx::pdl_wait();
+  const int runs = H / 32;
+  const int run = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (run >= T * runs) return;
+  const int t = run / runs, r = run - t * runs;
+  const size_t o = (size_t)t * H + r * 32 + lane;
+  float2 rsc;
+  int8_t hi;
+  uint8_t lo;
+  quant_run16(__bfloat162float(x[o]), hi, lo, rsc);
+  xq[o] = hi;
+  reinterpret_cast<uint8_t*>(xq + plane)[o] = lo;
+  if (lane == 0) xsc[run] = rsc;
 }
 
 // Power of two p with max * p in [2^14, 2^15) (1 for max == 0 or not finite); *inv = 1/p.
@@ -532,9 +564,15 @@ size_t prefill_gemm_smem() { return kGemmSmem; }
 
 size_t prefill_max_tiles(int n_experts_total, size_t pairs) { return (size_t)n_experts_total + pairs / kGN + 1; }
 
-cudaError_t launch_build_tiles(const Work& wk, cudaStream_t st) {
+cudaError_t launch_build_tiles(const Work& wk, int small_rows, cudaStream_t st) {
   return launch_pdl(build_tiles_kernel, dim3(1), dim3(1024), 0, st, (const int*)wk.act, (const int*)wk.n_act,
-                    (const int*)wk.counts, (const int*)wk.offsets, wk.tiles, wk.n_tiles);
+                    (const int*)wk.counts, (const int*)wk.offsets, wk.tiles, wk.n_tiles, small_rows, wk.act1,
+                    wk.n_act1);
+}
+
+cudaError_t launch_quant_x(const __nv_bfloat16* x, const Work& wk, int T, int H, cudaStream_t st) {
+  const int runs = T * (H / 32);
+  return launch_pdl(quant_x_kernel, dim3((runs + 7) / 8), dim3(256), 0, st, x, T, H, wk.xq, wk.xq_plane, wk.xsc);
 }
 
 cudaError_t launch_gather_rows(const __nv_bfloat16* x, const Work& wk, int P, int kS, int H, cudaStream_t st) {

@@ -36,7 +36,7 @@ EXPORTS = ("moe_expert_bytes", "moe_layer_create", "moe_layer_destroy", "moe_set
            "moe_check", "moe_get_stats", "moe_reset_stats", "moe_set_profiling", "moe_get_profile",
            "moe_reset_profile", "moe_route_noalloc", "moe_last_error")
 
-KERNELS = ("router", "topk", "permute", "gate_up", "down", "combine", "prep", "forward")
+KERNELS = ("router", "topk", "permute", "gate_up", "down", "combine", "prep", "small", "forward")
 
 
 class moe_stats(ctypes.Structure):
