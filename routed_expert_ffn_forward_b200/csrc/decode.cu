@@ -30,6 +30,7 @@
 // and wait (griddepcontrol.wait) before reading a predecessor's outputs.
 #include "moe_internal.h"
 #include "ptx.cuh"
+#include "q4k_decode.cuh"
 
 namespace moe {
 namespace {
@@ -47,34 +48,6 @@ constexpr int kGuStageBytes = 2 * kGuTileBytes;             // 36864
 constexpr int kDnSB = 4;
 constexpr int kDnStages = 4;
 constexpr int kDnStageBytes = kTileRows * kDnSB * kQBytes;  // 36864
-
-// Decoded scales of one row for the thread's sub-blocks 2c (lo) and 2c+1 (hi):
-// weight = s * q - m.
-struct RowScales {
-  float s_lo, s_hi, m_lo, m_hi;
-};
-
-// hdr: the 16-byte block header (fp16 d, fp16 dmin, 12 packed scale bytes).
-__device__ __forceinline__ RowScales decode_scales(uint4 hdr, int c) {
-  const float d = __half2float(__ushort_as_half((unsigned short)(hdr.x & 0xFFFFu)));
-  const float dmin = __half2float(__ushort_as_half((unsigned short)(hdr.x >> 16)));
-  const uint32_t sh = 16u * (uint32_t)(c & 1);
-  const uint32_t s0 = hdr.y >> sh, s1 = hdr.z >> sh, s2 = hdr.w >> sh;
-  uint32_t vsc, vm;
-  if (c < 2) {  // sub-blocks 0..3: low 6 bits of bytes j and j+4
-    vsc = s0 & 0x3F3Fu;
-    vm = s1 & 0x3F3Fu;
-  } else {      // sub-blocks 4..7: nibbles of byte j+4, top 2 bits of bytes j-4 / j
-    vsc = (s2 & 0x0F0Fu) | ((s0 >> 2) & 0x3030u);
-    vm = ((s2 >> 4) & 0x0F0Fu) | ((s1 >> 2) & 0x3030u);
-  }
-  RowScales r;
-  r.s_lo = d * (float)(vsc & 0xFFu);
-  r.s_hi = d * (float)((vsc >> 8) & 0xFFu);
-  r.m_lo = dmin * (float)(vm & 0xFFu);
-  r.m_hi = dmin * (float)((vm >> 8) & 0xFFu);
-  return r;
-}
 
 // One row's block header and quant chunk c (32 bytes).  Rows sit 144*SB bytes
 // apart, so every 16-byte piece starts on a multiple of 8 banks: lanes of odd

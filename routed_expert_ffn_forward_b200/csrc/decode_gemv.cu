@@ -1,0 +1,404 @@
+// Single-token decode (T = 1) expert kernels: gate/up + SwiGLU, then down, as
+// GEMVs over the raw Q4_K bytes with byte dot products (dp4a).
+//
+// One thread owns one weight row of a 128-row tile and a fixed part of each
+// super-block; a stage is one 128-row x 1 (gate/up: of each matrix) or 2
+// (down) super-block tile streamed by 2-D TMA into a shared-memory ring.  For
+// a 32-bit quant word w (four quants of sub-block 2c in its low nibbles and
+// four of sub-block 2c+1 in its high nibbles) the thread forms
+//   lo = w & 0x0F0F0F0F,  hi = (w >> 4) & 0x0F0F0F0F
+// and accumulates dp4a(lo, x_hi) and dp4a(lo, x_lo) (and the same for hi),
+// where the activations are 16-bit fixed point per 32-element run,
+// x = (256*x_hi + x_lo) * 2^-s (x_hi signed, x_lo unsigned bytes), so the
+// integer sums are exact.  Per (row, sub-block) the fp32 epilogue adds
+//   d*sc * 2^-s * (256*C_hi + C_lo) - dmin*m * X
+// (X the run's sum of the represented activations): the Q4_K weight value
+// d*sc*q - dmin*m applied exactly up to fp32 rounding -- the same arithmetic as
+// the multi-token decode kernels, with fewer instructions per weight.
+//
+// gate/up: unit = (expert, 128 rows); warp w handles matrix w>>3 (gate, up),
+// rows 32*(w&3)+lane and chunks {2h, 2h+1} (h = (w>>2)&1) of every super-block;
+// at the unit's end the two halves meet in shared memory, and gate rows meet
+// up rows for SwiGLU, written as h in the same fixed-point form.
+// down: unit = (expert, 128 output rows); warp w handles rows 32*(w&3)+lane
+// and quarter w>>2 of each stage's two super-blocks; the four parts meet in
+// shared memory in a fixed order.
+#include "moe_internal.h"
+#include "ptx.cuh"
+#include "q4k_decode.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kGvRows = 128;                    // rows per unit (one TMA box)
+constexpr int kGvConsumerWarps = 16;
+constexpr int kGvThreads = (kGvConsumerWarps + 1) * 32;
+constexpr int kGvConsumers = kGvConsumerWarps * 32;
+constexpr int kGvBox = kGvRows * kQBytes;       // one 128-row x 1 super-block box: 18432
+constexpr int kGvStageBytes = 2 * kGvBox;       // gate/up: gate + up; down: two super-blocks
+constexpr int kGvStages = 4;
+
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {  // u8 x s8
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {  // u8 x u8
+  int d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint8_t* gv_aligned(uint8_t* raw) {
+  const uint32_t pad = (1024u - (ptx::smem_u32(raw) & 1023u)) & 1023u;
+  return raw + pad;
+}
+
+// Two chunks (c0, c0+1) of one row's super-block against one token's
+// activations of that super-block: xh/xl the 256 high/low activation bytes,
+// sc the eight runs' (2^-s, X).  Adds the row's partial dot product to acc.
+__device__ __forceinline__ void gv_two_chunks(const uint8_t* blk, int c0, const uint8_t* xh, const uint8_t* xl,
+                                              const float2* sc, float& acc) {
+  const uint4 hdr = *reinterpret_cast<const uint4*>(blk);
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    const int c = c0 + cc;
+    const uint4 qa = *reinterpret_cast<const uint4*>(blk + 16 + 32 * c);
+    const uint4 qb = *reinterpret_cast<const uint4*>(blk + 32 + 32 * c);
+    const uint32_t q[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+    // activations: sub-block 2c at bytes 64c..64c+31, sub-block 2c+1 at 64c+32..
+    const uint4* ph = reinterpret_cast<const uint4*>(xh + 64 * c);
+    const uint4* pl = reinterpret_cast<const uint4*>(xl + 64 * c);
+    const uint4 h0 = ph[0], h1 = ph[1], h2 = ph[2], h3 = ph[3];
+    const uint4 l0 = pl[0], l1 = pl[1], l2 = pl[2], l3 = pl[3];
+    const uint32_t xhl[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+    const uint32_t xhh[8] = {h2.x, h2.y, h2.z, h2.w, h3.x, h3.y, h3.z, h3.w};
+    const uint32_t xll[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+    const uint32_t xlh[8] = {l2.x, l2.y, l2.z, l2.w, l3.x, l3.y, l3.z, l3.w};
+    int chl = 0, cll = 0, chh = 0, clh = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t lo = q[k] & 0x0F0F0F0Fu, hi = (q[k] >> 4) & 0x0F0F0F0Fu;
+      chl = dp4a_us(lo, xhl[k], chl);
+      cll = dp4a_uu(lo, xll[k], cll);
+      chh = dp4a_us(hi, xhh[k], chh);
+      clh = dp4a_uu(hi, xlh[k], clh);
+    }
+    const RowScales rs = decode_scales(hdr, c);
+    const float2 sl = sc[2 * c], sh = sc[2 * c + 1];
+    acc += rs.s_lo * sl.x * (float)(chl * 256 + cll) + rs.s_hi * sh.x * (float)(chh * 256 + clh) -
+           (rs.m_lo * sl.y + rs.m_hi * sh.y);
+  }
+}
+
+// ============================================================================ gate/up
+__global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(DecodeArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* smem = gv_aligned(smem_raw);
+  uint8_t* stages = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGvStages * kGvStageBytes);
+  uint64_t* empty = full + kGvStages;
+  float* s_part = reinterpret_cast<float*>(empty + kGvStages);   // [2 mats][2 halves][128]
+  int& s_abort = *reinterpret_cast<int*>(s_part + 4 * kGvRows);
+  uint8_t* s_x = reinterpret_cast<uint8_t*>(&s_abort) + 16;      // x: hi plane, lo plane, run scales
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < kGvStages; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], kGvConsumerWarps);
+    }
+    ptx::fence_barrier_init();
+  }
+  __syncthreads();
+  ptx::pdl_wait();  // routing and the fixed-point x come from the route kernel
+  ptx::pdl_launch_dependents();
+
+  const int tiles = (a.I + kGvRows - 1) / kGvRows;
+  const int n_units = __ldcg(a.n_act) * tiles;
+  const int H = a.H, runs = H / 32;
+
+  if (warp == kGvConsumerWarps) {  // producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
+        const int ai = unit / tiles, rt = unit - ai * tiles;
+        const CUtensorMap* m = a.tmaps + kMapsPerSlot * __ldcg(a.slot_of + __ldcg(a.act + ai)) + 3;
+        for (int kb = 0; kb < a.nbh; ++kb) {
+          if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
+            atomicOr(a.err, 1u);
+            return;
+          }
+          ptx::mbar_arrive_expect_tx(&full[stage], kGvStageBytes);
+          uint8_t* dst = stages + stage * kGvStageBytes;
+          ptx::tma_load_2d(dst, m, kb * 18, rt * kGvRows, &full[stage]);
+          ptx::tma_load_2d(dst + kGvBox, m + 1, kb * 18, rt * kGvRows, &full[stage]);
+          if (++stage == kGvStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // x of the token, staged once: hi plane, lo plane, run scales
+  {
+    const uint4* src_h = reinterpret_cast<const uint4*>(a.xq);
+    const uint4* src_l = reinterpret_cast<const uint4*>(a.xq + a.xq_plane);
+    uint4* dh = reinterpret_cast<uint4*>(s_x);
+    uint4* dl = reinterpret_cast<uint4*>(s_x + H);
+    for (int i = threadIdx.x; i < H / 16; i += kGvConsumers) {
+      dh[i] = __ldcg(src_h + i);
+      dl[i] = __ldcg(src_l + i);
+    }
+    float2* dsc = reinterpret_cast<float2*>(s_x + 2 * H);
+    for (int i = threadIdx.x; i < runs; i += kGvConsumers) dsc[i] = __ldcg(a.xsc + i);
+    ptx::named_barrier_sync(1, kGvConsumers);
+  }
+  const uint8_t* xh = s_x;
+  const uint8_t* xl = s_x + H;
+  const float2* xsc = reinterpret_cast<const float2*>(s_x + 2 * H);
+
+  const int mat = warp >> 3, half = (warp >> 2) & 1, row = (warp & 3) * 32 + lane;
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
+    const int ai = unit / tiles, rt = unit - ai * tiles;
+    const int e = __ldcg(a.act + ai);
+    const int r0 = __ldcg(a.offsets + e);
+    float acc = 0.f;
+    bool ok = true;
+    for (int kb = 0; kb < a.nbh; ++kb) {
+      if (!ptx::mbar_wait(&full[stage], phase)) {
+        atomicOr(a.err, 2u);
+        ok = false;
+        break;
+      }
+      const uint8_t* blk = stages + stage * kGvStageBytes + mat * kGvBox + row * kQBytes;
+      gv_two_chunks(blk, 2 * half, xh + kb * kQK, xl + kb * kQK, xsc + kb * 8, acc);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[stage]);
+      if (++stage == kGvStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    // a warp that gave up on a wait sets the flag before the barrier; every
+    // consumer warp reaches it (all waits are bounded) and they stop together
+    if (!ok) s_abort = 1;
+    ptx::named_barrier_sync(1, kGvConsumers);  // also: the previous unit's SwiGLU reads are done
+    if (s_abort) return;
+    s_part[(mat * 2 + half) * kGvRows + row] = acc;
+    ptx::named_barrier_sync(1, kGvConsumers);
+    // SwiGLU (halves summed in a fixed order), 16-bit fixed point per run:
+    // warps 0-3 own features 32*w .. 32*w+31 of the tile
+    if (warp < 4) {
+      const int f = warp * 32 + lane;
+      const float g = s_part[f] + s_part[kGvRows + f];
+      const float u = s_part[2 * kGvRows + f] + s_part[3 * kGvRows + f];
+      float2 rsc;
+      int8_t hh;
+      uint8_t hl;
+      quant_run16(silu_f(g) * u, hh, hl, rsc);
+      const int feat = rt * kGvRows + f;
+      const size_t o = (size_t)r0 * a.I_pad + feat;
+      a.hq[o] = hh;
+      reinterpret_cast<uint8_t*>(a.hq + a.hq_plane)[o] = hl;
+      if (lane == 0) a.hsc[(size_t)r0 * (a.I_pad / 32) + feat / 32] = rsc;
+    }
+  }
+}
+
+// ============================================================================ down
+// The producer also copies each unit's activations (h of the expert's token:
+// both byte planes and the run scales) into one of two shared-memory slots.
+__global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* smem = gv_aligned(smem_raw);
+  uint8_t* stages = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGvStages * kGvStageBytes);
+  uint64_t* empty = full + kGvStages;
+  uint64_t* afull = empty + kGvStages;  // activation slots
+  uint64_t* aempty = afull + 2;
+  float* s_part = reinterpret_cast<float*>(aempty + 2);  // [4 parts][128]
+  int& s_abort = *reinterpret_cast<int*>(s_part + 4 * kGvRows);
+  uint8_t* s_act = reinterpret_cast<uint8_t*>(&s_abort) + 16;  // 2 slots of act_slot_bytes
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int I_pad = a.I_pad, hruns = I_pad / 32;
+  const size_t slot_bytes = a.act_slot_bytes;   // 2 * I_pad + hruns * 8
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < kGvStages; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], kGvConsumerWarps);
+    }
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&afull[s], 1);
+      ptx::mbar_init(&aempty[s], kGvConsumerWarps);
+    }
+    ptx::fence_barrier_init();
+  }
+  __syncthreads();
+  // The routing comes from two kernels back; the kernel in between waited for
+  // it before letting this one launch, so it is complete.
+  const int tiles = a.H / kGvRows;
+  const int n_units = __ldcg(a.n_act) * tiles;
+  const int n_st = (a.nbi + 1) / 2;
+
+  if (warp == kGvConsumerWarps) {
+    if (lane == 0) {
+      int stage = 0, slot = 0;
+      uint32_t phase = 0, aphase = 0;
+      bool waited = false;
+      for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
+        const int ai = unit / tiles, rt = unit - ai * tiles;
+        const int e = __ldcg(a.act + ai);
+        const CUtensorMap* md = a.tmaps + kMapsPerSlot * __ldcg(a.slot_of + e) + 5;
+        // weights first: they do not depend on the gate/up kernel
+        for (int st = 0; st < n_st; ++st) {
+          if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
+            atomicOr(a.err, 4u);
+            if (!waited) ptx::pdl_wait();
+            return;
+          }
+          ptx::mbar_arrive_expect_tx(&full[stage], kGvStageBytes);
+          uint8_t* dst = stages + stage * kGvStageBytes;
+          // a second box past the last super-block reads zeros (never used)
+          ptx::tma_load_2d(dst, md, (2 * st) * 18, rt * kGvRows, &full[stage]);
+          ptx::tma_load_2d(dst + kGvBox, md, (2 * st + 1) * 18, rt * kGvRows, &full[stage]);
+          if (++stage == kGvStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        // then the unit's activations, written by the gate/up kernel
+        if (!waited) {
+          ptx::pdl_wait();
+          waited = true;
+        }
+        if (!ptx::mbar_wait(&aempty[slot], aphase ^ 1u)) {
+          atomicOr(a.err, 4u);
+          return;
+        }
+        const int r0 = __ldcg(a.offsets + e);
+        uint8_t* dst = s_act + slot * slot_bytes;
+        ptx::mbar_arrive_expect_tx(&afull[slot], (uint32_t)(2 * I_pad + hruns * 8));
+        ptx::bulk_load(dst, a.hq + (size_t)r0 * I_pad, (uint32_t)I_pad, &afull[slot]);
+        ptx::bulk_load(dst + I_pad, a.hq + a.hq_plane + (size_t)r0 * I_pad, (uint32_t)I_pad, &afull[slot]);
+        ptx::bulk_load(dst + 2 * I_pad, a.hsc + (size_t)r0 * hruns, (uint32_t)(hruns * 8), &afull[slot]);
+        if (++slot == 2) {
+          slot = 0;
+          aphase ^= 1u;
+        }
+      }
+      if (!waited) ptx::pdl_wait();
+    } else {
+      ptx::pdl_wait();
+    }
+    return;
+  }
+  ptx::pdl_wait();  // hq / hsc come from the gate/up kernel
+  ptx::pdl_launch_dependents();
+
+  // consumers: warp w takes rows 32*(w&3)+lane and part p = w>>2 of each
+  // stage: super-block p>>1 of the stage's two, chunks {2(p&1), 2(p&1)+1}
+  const int row = (warp & 3) * 32 + lane, part = warp >> 2;
+  const int sbi = part >> 1, c0 = 2 * (part & 1);
+  int stage = 0, slot = 0;
+  uint32_t phase = 0, aphase = 0;
+  for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
+    const int ai = unit / tiles, rt = unit - ai * tiles;
+    const int e = __ldcg(a.act + ai);
+    const int r0 = __ldcg(a.offsets + e);
+    float acc = 0.f;
+    bool ok = ptx::mbar_wait(&afull[slot], aphase);
+    if (!ok) atomicOr(a.err, 8u);
+    const uint8_t* act = s_act + slot * slot_bytes;
+    const float2* asc = reinterpret_cast<const float2*>(act + 2 * I_pad);
+    for (int st = 0; st < n_st && ok; ++st) {
+      if (!ptx::mbar_wait(&full[stage], phase)) {
+        atomicOr(a.err, 8u);
+        ok = false;
+        break;
+      }
+      const int kb = 2 * st + sbi;
+      if (kb < a.nbi) {
+        const uint8_t* blk = stages + stage * kGvStageBytes + sbi * kGvBox + row * kQBytes;
+        gv_two_chunks(blk, c0, act + kb * kQK, act + I_pad + kb * kQK, asc + kb * 8, acc);
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[stage]);
+      if (++stage == kGvStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&aempty[slot]);
+    if (++slot == 2) {
+      slot = 0;
+      aphase ^= 1u;
+    }
+    if (!ok) s_abort = 1;
+    ptx::named_barrier_sync(1, kGvConsumers);  // also: the previous unit's reads of s_part are done
+    if (s_abort) return;
+    s_part[part * kGvRows + row] = acc;
+    ptx::named_barrier_sync(1, kGvConsumers);
+    // the four parts of each row, summed in a fixed order, to y
+    if (warp < 4) {
+      const int r = warp * 32 + lane;
+      a.y[(size_t)r0 * a.H + rt * kGvRows + r] =
+          ((s_part[r] + s_part[kGvRows + r]) + s_part[2 * kGvRows + r]) + s_part[3 * kGvRows + r];
+    }
+  }
+}
+
+template <typename K>
+cudaError_t gv_launch(K kernel, uint64_t* mask, size_t smem, int n_sm, cudaStream_t st, const DecodeArgs& a) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (smem > kMaxDecodeSmem) return cudaErrorInvalidValue;
+  if (!(*mask & bit)) {  // once per device, for the largest size any shape may need
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxDecodeSmem);
+    if (e != cudaSuccess) return e;
+    *mask |= bit;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_sm);
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+}  // namespace
+
+size_t gemv_gate_up_smem(int H) {
+  return 1024 + (size_t)kGvStages * kGvStageBytes + 2 * kGvStages * 8 + 4 * kGvRows * 4 + 16 + 2 * (size_t)H +
+         (size_t)(H / 32) * 8;
+}
+size_t gemv_down_smem(size_t act_slot_bytes) {
+  return 1024 + (size_t)kGvStages * kGvStageBytes + 2 * kGvStages * 8 + 4 * 8 + 4 * kGvRows * 4 + 16 +
+         2 * act_slot_bytes;
+}
+
+cudaError_t launch_gemv_gate_up(const DecodeArgs& a, int n_sm, cudaStream_t st) {
+  static uint64_t mask = 0;
+  return gv_launch(gemv_gate_up_kernel, &mask, gemv_gate_up_smem(a.H), n_sm, st, a);
+}
+
+cudaError_t launch_gemv_down(const DecodeArgs& a, int n_sm, cudaStream_t st) {
+  static uint64_t mask = 0;
+  return gv_launch(gemv_down_kernel, &mask, gemv_down_smem(a.act_slot_bytes), n_sm, st, a);
+}
+
+}  // namespace moe

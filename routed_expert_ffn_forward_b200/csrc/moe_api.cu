@@ -43,12 +43,16 @@ moe_status fail(moe_status s, const char* fmt, ...) {
   return s;
 }
 
+// On failure the runtime's last-error record is read (and so cleared), so a
+// failed launch is reported once and not again by the next call's check.
 #define CUDA_TRY(call)                                                                       \
   do {                                                                                       \
     cudaError_t e_ = (call);                                                                 \
-    if (e_ != cudaSuccess)                                                                   \
+    if (e_ != cudaSuccess) {                                                                 \
+      (void)cudaGetLastError();                                                              \
       return fail(e_ == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA, "%s: %s", #call, \
                   cudaGetErrorString(e_));                                                   \
+    }                                                                                        \
   } while (0)
 
 #define MOE_TRY(call)               \
@@ -532,8 +536,14 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
   da.stage_x = stage_x ? 1 : 0;
   da.act_slot_bytes = act_slot;
   if (fast) {
-    MOE_KERNEL(MOE_K_GATE_UP, launch_gate_up_d1(da, max_tok, s.n_sm, st));
-    MOE_KERNEL(MOE_K_DOWN, launch_down_d1(da, max_tok, s.n_sm, st));
+    const bool gemv = T == 1 && gemv_gate_up_smem(s.H) <= kMaxDecodeSmem && gemv_down_smem(act_slot) <= kMaxDecodeSmem;
+    if (gemv) {
+      MOE_KERNEL(MOE_K_GATE_UP, launch_gemv_gate_up(da, s.n_sm, st));
+      MOE_KERNEL(MOE_K_DOWN, launch_gemv_down(da, s.n_sm, st));
+    } else {
+      MOE_KERNEL(MOE_K_GATE_UP, launch_gate_up_d1(da, max_tok, s.n_sm, st));
+      MOE_KERNEL(MOE_K_DOWN, launch_down_d1(da, max_tok, s.n_sm, st));
+    }
     MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true));
   } else {
     // prefill: tensor-core GEMMs over tiles of up to 256 rows of one expert;

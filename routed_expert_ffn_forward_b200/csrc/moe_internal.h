@@ -103,6 +103,12 @@ cudaError_t launch_gate_up_d1(const DecodeArgs& a, int max_tok, int n_sm, cudaSt
 cudaError_t launch_down_d1(const DecodeArgs& a, int max_tok, int n_sm, cudaStream_t st);
 size_t gate_up_d1_smem(int max_tok, size_t x_stage_bytes);
 size_t down_d1_smem(int max_tok, size_t act_slot_bytes);
+// T = 1: GEMV kernels on byte dot products (128-row units); act_slot_bytes of
+// one token's h (2 * I_pad + I_pad / 32 * 8)
+cudaError_t launch_gemv_gate_up(const DecodeArgs& a, int n_sm, cudaStream_t st);
+cudaError_t launch_gemv_down(const DecodeArgs& a, int n_sm, cudaStream_t st);
+size_t gemv_gate_up_smem(int H);
+size_t gemv_down_smem(size_t act_slot_bytes);
 
 // Tensor maps of one expert's Q4_K matrices at `base`, kMapsPerSlot of them:
 // [0..2] gate, up, down with boxes of 64 rows x 2 (gate/up) or 4 (down)

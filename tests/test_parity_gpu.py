@@ -157,3 +157,34 @@ def test_forced_routing(torch):
         L.forward_routed(to_dev(torch, x), np.full((5, 2), 16, dtype=np.int32))
     assert ei.value.status == moe.MOE_ERR_INVALID_ARG
     L.destroy()
+
+
+def test_prefill_weight_range_is_reported(torch):
+    """The prefill GEMMs dequantise to fp16 scaled by 2^8; a Q4_K block whose d
+    could take a weight past that range is reported by moe_check (the decode
+    kernels use the weights exactly and have no such limit)."""
+    from routed_expert_ffn_forward_b200.layer import MoELayer
+    cfg = C0
+    L = MoELayer(cfg.hidden, cfg.inter, cfg.n_experts, cfg.top_k, cfg.n_shared)
+    L.set_router(synth.router_weight(cfg), synth.router_bias(cfg), cfg.gating)
+
+    def fill(e, views):
+        for m, v in enumerate(views):
+            rows, cols = (cfg.inter, cfg.hidden) if m < 2 else (cfg.hidden, cfg.inter)
+            synth.q4k_tensor(cfg.seed, 0, e, m, rows, cols, out=v)
+        views[0][0, 0:2] = np.frombuffer(np.float16(1.0).tobytes(), dtype=np.uint8)  # d = 1.0: |w| up to 945
+
+    L.fill_experts(fill)
+    L.register_experts()
+    x = synth.activations(cfg, tokens=1)
+    L.forward(to_dev(torch, x))          # decode path: exact weights, no flag
+    torch.cuda.synchronize()
+    moe.moe_check(L.handle)
+    x = synth.activations(cfg, tokens=64)
+    L.forward(to_dev(torch, x))          # prefill path: ~8 rows per expert, tensor-core GEMMs
+    torch.cuda.synchronize()
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_check(L.handle)
+    assert "fp16 range" in str(ei.value)
+    moe.moe_check(L.handle)              # the record is cleared
+    L.destroy()
