@@ -163,10 +163,12 @@ moe_status moe_forward(moe_layer_t layer, const void* x, void* out, int T, void*
 moe_status moe_forward_routed(moe_layer_t layer, const void* x, void* out, int T,
                               const int32_t* forced_ids, void* stream);
 
-/* Forward on HOST buffers: copies x (host, bf16 [T, H]) in, runs moe_forward
- * and copies out (host, bf16 [T, H]) back, all on `stream`; returns once the
- * copies are enqueued (synchronise the stream before reading out).  Pinned
- * buffers make the copies asynchronous. */
+/* Forward on HOST buffers: x (host, bf16 [T, H]) in, moe_forward, out (host,
+ * bf16 [T, H]) back, all on `stream`; returns once the work is enqueued
+ * (synchronise the stream before reading out).  With T <= 4 and pinned
+ * buffers (16-byte aligned) the kernels read x and write out in host memory
+ * in place; otherwise x and out are copied through device buffers (pinned
+ * buffers make those copies asynchronous). */
 moe_status moe_forward_host(moe_layer_t layer, const void* x_host, void* out_host,
                             int T, void* stream);
 

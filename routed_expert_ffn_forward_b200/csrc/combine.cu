@@ -14,16 +14,19 @@ __global__ void combine_kernel(const float* __restrict__ y, const float* __restr
   constexpr int kMaxKS = 40;  // top_k + n_shared at most
   __shared__ int s_row[kMaxKS];
   __shared__ float s_w[kMaxKS];
+  const int t = blockIdx.y, kS = k + S;
+  // the token's y rows and weights, once per block, so the y loads below are
+  // independent of each other.  They come from the routing kernels, at least
+  // two launches back: every kernel of a forward waits for its predecessor
+  // before it lets its dependents launch, so those are complete when this
+  // kernel starts, and the loads go ahead of the wait for the down kernel.
+  if (threadIdx.x < kS) {
+    s_row[threadIdx.x] = __ldcg(inv + t * kS + threadIdx.x);
+    s_w[threadIdx.x] = threadIdx.x < k ? __ldcg(w + (size_t)t * k + threadIdx.x) : 1.f;
+  }
   // launched as a programmatic dependent of the down kernel: wait for it (a
   // no-op when launched normally)
   ptx::pdl_wait();
-  const int t = blockIdx.y, kS = k + S;
-  // the token's y rows and weights, once per block, so the y loads below are
-  // independent of each other
-  if (threadIdx.x < kS) {
-    s_row[threadIdx.x] = inv[t * kS + threadIdx.x];
-    s_w[threadIdx.x] = threadIdx.x < k ? w[(size_t)t * k + threadIdx.x] : 1.f;
-  }
   __syncthreads();
   const int o = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (o >= H) return;

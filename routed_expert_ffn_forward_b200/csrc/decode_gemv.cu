@@ -6,23 +6,26 @@
 // (down) super-block tile streamed by 2-D TMA into a shared-memory ring.  For
 // a 32-bit quant word w (four quants of sub-block 2c in its low nibbles and
 // four of sub-block 2c+1 in its high nibbles) the thread forms
-//   lo = w & 0x0F0F0F0F,  hi = (w >> 4) & 0x0F0F0F0F
+//   lo = w & 0x0F0F0F0F,  hi = w & 0xF0F0F0F0  (16 x the high quants)
 // and accumulates dp4a(lo, x_hi) and dp4a(lo, x_lo) (and the same for hi),
 // where the activations are 16-bit fixed point per 32-element run,
 // x = (256*x_hi + x_lo) * 2^-s (x_hi signed, x_lo unsigned bytes), so the
 // integer sums are exact.  Per (row, sub-block) the fp32 epilogue adds
 //   d*sc * 2^-s * (256*C_hi + C_lo) - dmin*m * X
-// (X the run's sum of the represented activations): the Q4_K weight value
+// (X the run's sum of the represented activations; the 1/16 of the high
+// nibbles is folded into the scale, exactly): the Q4_K weight value
 // d*sc*q - dmin*m applied exactly up to fp32 rounding -- the same arithmetic as
 // the multi-token decode kernels, with fewer instructions per weight.
 //
-// gate/up: unit = (expert, 128 rows); warp w handles matrix w>>3 (gate, up),
-// rows 32*(w&3)+lane and chunks {2h, 2h+1} (h = (w>>2)&1) of every super-block;
-// at the unit's end the two halves meet in shared memory, and gate rows meet
-// up rows for SwiGLU, written as h in the same fixed-point form.
-// down: unit = (expert, 128 output rows); warp w handles rows 32*(w&3)+lane
-// and quarter w>>2 of each stage's two super-blocks; the four parts meet in
-// shared memory in a fixed order.
+// A thread takes one chunk of two rows, so each activation load serves two
+// rows and the two rows' integer chains run side by side.
+// gate/up: unit = (expert, 128 rows); warp w handles chunk w>>2 of every
+// super-block for row 32*(w&3)+lane of both matrices; at the unit's end the
+// four chunk parts meet in shared memory (fixed order), and gate rows meet up
+// rows for SwiGLU, written as h in the same fixed-point form.
+// down: unit = (expert, 128 output rows); warp w handles rows 32*(w&1)+lane
+// and +64, super-block w>>3 of each stage's two and chunk (w>>1)&3; the eight
+// parts of a row meet in shared memory in a fixed order.
 #include "moe_internal.h"
 #include "ptx.cuh"
 #include "q4k_decode.cuh"
@@ -54,40 +57,42 @@ __device__ __forceinline__ uint8_t* gv_aligned(uint8_t* raw) {
   return raw + pad;
 }
 
-// Two chunks (c0, c0+1) of one row's super-block against one token's
-// activations of that super-block: xh/xl the 256 high/low activation bytes,
-// sc the eight runs' (2^-s, X).  Adds the row's partial dot product to acc.
-__device__ __forceinline__ void gv_two_chunks(const uint8_t* blk, int c0, const uint8_t* xh, const uint8_t* xl,
-                                              const float2* sc, float& acc) {
-  const uint4 hdr = *reinterpret_cast<const uint4*>(blk);
+// Chunk c of R rows' super-blocks (blk[r]: the rows' 144-byte blocks) against
+// one token's activations of that super-block: xh/xl the 256 high/low
+// activation bytes, sc the eight runs' (2^-s, X).  The chunk's activations are
+// loaded once for the R rows.  Adds row r's partial dot product to acc[r].
+template <int R>
+__device__ __forceinline__ void gv_chunk_rows(const uint8_t* const (&blk)[R], int c, const uint8_t* xh,
+                                              const uint8_t* xl, const float2* sc, float (&acc)[R]) {
+  // activations: sub-block 2c at bytes 64c..64c+31, sub-block 2c+1 at 64c+32..
+  const uint4* ph = reinterpret_cast<const uint4*>(xh + 64 * c);
+  const uint4* pl = reinterpret_cast<const uint4*>(xl + 64 * c);
+  const uint4 h0 = ph[0], h1 = ph[1], h2 = ph[2], h3 = ph[3];
+  const uint4 l0 = pl[0], l1 = pl[1], l2 = pl[2], l3 = pl[3];
+  const uint32_t xhl[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+  const uint32_t xhh[8] = {h2.x, h2.y, h2.z, h2.w, h3.x, h3.y, h3.z, h3.w};
+  const uint32_t xll[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+  const uint32_t xlh[8] = {l2.x, l2.y, l2.z, l2.w, l3.x, l3.y, l3.z, l3.w};
+  const float2 sl = sc[2 * c], sh = sc[2 * c + 1];
 #pragma unroll
-  for (int cc = 0; cc < 2; ++cc) {
-    const int c = c0 + cc;
-    const uint4 qa = *reinterpret_cast<const uint4*>(blk + 16 + 32 * c);
-    const uint4 qb = *reinterpret_cast<const uint4*>(blk + 32 + 32 * c);
+  for (int r = 0; r < R; ++r) {
+    const uint4 hdr = *reinterpret_cast<const uint4*>(blk[r]);
+    const uint4 qa = *reinterpret_cast<const uint4*>(blk[r] + 16 + 32 * c);
+    const uint4 qb = *reinterpret_cast<const uint4*>(blk[r] + 32 + 32 * c);
     const uint32_t q[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-    // activations: sub-block 2c at bytes 64c..64c+31, sub-block 2c+1 at 64c+32..
-    const uint4* ph = reinterpret_cast<const uint4*>(xh + 64 * c);
-    const uint4* pl = reinterpret_cast<const uint4*>(xl + 64 * c);
-    const uint4 h0 = ph[0], h1 = ph[1], h2 = ph[2], h3 = ph[3];
-    const uint4 l0 = pl[0], l1 = pl[1], l2 = pl[2], l3 = pl[3];
-    const uint32_t xhl[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-    const uint32_t xhh[8] = {h2.x, h2.y, h2.z, h2.w, h3.x, h3.y, h3.z, h3.w};
-    const uint32_t xll[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-    const uint32_t xlh[8] = {l2.x, l2.y, l2.z, l2.w, l3.x, l3.y, l3.z, l3.w};
     int chl = 0, cll = 0, chh = 0, clh = 0;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const uint32_t lo = q[k] & 0x0F0F0F0Fu, hi = (q[k] >> 4) & 0x0F0F0F0Fu;
+      // high nibbles left in place: 16x the quant, so the sums are 16x too
+      const uint32_t lo = q[k] & 0x0F0F0F0Fu, hi = q[k] & 0xF0F0F0F0u;
       chl = dp4a_us(lo, xhl[k], chl);
       cll = dp4a_uu(lo, xll[k], cll);
       chh = dp4a_us(hi, xhh[k], chh);
       clh = dp4a_uu(hi, xlh[k], clh);
     }
     const RowScales rs = decode_scales(hdr, c);
-    const float2 sl = sc[2 * c], sh = sc[2 * c + 1];
-    acc += rs.s_lo * sl.x * (float)(chl * 256 + cll) + rs.s_hi * sh.x * (float)(chh * 256 + clh) -
-           (rs.m_lo * sl.y + rs.m_hi * sh.y);
+    acc[r] += rs.s_lo * sl.x * (float)(chl * 256 + cll) + (rs.s_hi * 0.0625f) * sh.x * (float)(chh * 256 + clh) -
+              (rs.m_lo * sl.y + rs.m_hi * sh.y);
   }
 }
 
@@ -98,8 +103,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(DecodeArgs 
   uint8_t* stages = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGvStages * kGvStageBytes);
   uint64_t* empty = full + kGvStages;
-  float* s_part = reinterpret_cast<float*>(empty + kGvStages);   // [2 mats][2 halves][128]
-  int& s_abort = *reinterpret_cast<int*>(s_part + 4 * kGvRows);
+  float* s_part = reinterpret_cast<float*>(empty + kGvStages);   // [2 mats][4 chunks][128]
+  int& s_abort = *reinterpret_cast<int*>(s_part + 8 * kGvRows);
   uint8_t* s_x = reinterpret_cast<uint8_t*>(&s_abort) + 16;      // x: hi plane, lo plane, run scales
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -162,14 +167,16 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(DecodeArgs 
   const uint8_t* xl = s_x + H;
   const float2* xsc = reinterpret_cast<const float2*>(s_x + 2 * H);
 
-  const int mat = warp >> 3, half = (warp >> 2) & 1, row = (warp & 3) * 32 + lane;
+  // warp w: chunk c = w >> 2 of every super-block, row 32*(w&3)+lane of both
+  // matrices (the chunk's activations serve the gate row and the up row)
+  const int c = warp >> 2, row = (warp & 3) * 32 + lane;
   int stage = 0;
   uint32_t phase = 0;
   for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
     const int ai = unit / tiles, rt = unit - ai * tiles;
     const int e = __ldcg(a.act + ai);
     const int r0 = __ldcg(a.offsets + e);
-    float acc = 0.f;
+    float acc[2] = {0.f, 0.f};  // gate, up
     bool ok = true;
     for (int kb = 0; kb < a.nbh; ++kb) {
       if (!ptx::mbar_wait(&full[stage], phase)) {
@@ -177,8 +184,9 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(DecodeArgs 
         ok = false;
         break;
       }
-      const uint8_t* blk = stages + stage * kGvStageBytes + mat * kGvBox + row * kQBytes;
-      gv_two_chunks(blk, 2 * half, xh + kb * kQK, xl + kb * kQK, xsc + kb * 8, acc);
+      const uint8_t* bg = stages + stage * kGvStageBytes + row * kQBytes;
+      const uint8_t* const blk[2] = {bg, bg + kGvBox};
+      gv_chunk_rows<2>(blk, c, xh + kb * kQK, xl + kb * kQK, xsc + kb * 8, acc);
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&empty[stage]);
       if (++stage == kGvStages) {
@@ -191,14 +199,17 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(DecodeArgs 
     if (!ok) s_abort = 1;
     ptx::named_barrier_sync(1, kGvConsumers);  // also: the previous unit's SwiGLU reads are done
     if (s_abort) return;
-    s_part[(mat * 2 + half) * kGvRows + row] = acc;
+    s_part[c * kGvRows + row] = acc[0];
+    s_part[(4 + c) * kGvRows + row] = acc[1];
     ptx::named_barrier_sync(1, kGvConsumers);
-    // SwiGLU (halves summed in a fixed order), 16-bit fixed point per run:
+    // SwiGLU (chunk parts summed in a fixed order), 16-bit fixed point per run:
     // warps 0-3 own features 32*w .. 32*w+31 of the tile
     if (warp < 4) {
       const int f = warp * 32 + lane;
-      const float g = s_part[f] + s_part[kGvRows + f];
-      const float u = s_part[2 * kGvRows + f] + s_part[3 * kGvRows + f];
+      const float* pg = s_part + f;
+      const float* pu = s_part + 4 * kGvRows + f;
+      const float g = ((pg[0] + pg[kGvRows]) + pg[2 * kGvRows]) + pg[3 * kGvRows];
+      const float u = ((pu[0] + pu[kGvRows]) + pu[2 * kGvRows]) + pu[3 * kGvRows];
       float2 rsc;
       int8_t hh;
       uint8_t hl;
@@ -215,6 +226,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(DecodeArgs 
 // ============================================================================ down
 // The producer also copies each unit's activations (h of the expert's token:
 // both byte planes and the run scales) into one of two shared-memory slots.
+// It issues the first unit's weights before waiting for the gate/up kernel.
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = gv_aligned(smem_raw);
@@ -223,8 +235,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
   uint64_t* empty = full + kGvStages;
   uint64_t* afull = empty + kGvStages;  // activation slots
   uint64_t* aempty = afull + 2;
-  float* s_part = reinterpret_cast<float*>(aempty + 2);  // [4 parts][128]
-  int& s_abort = *reinterpret_cast<int*>(s_part + 4 * kGvRows);
+  float* s_part = reinterpret_cast<float*>(aempty + 2);  // [8 parts][128]
+  int& s_abort = *reinterpret_cast<int*>(s_part + 8 * kGvRows);
   uint8_t* s_act = reinterpret_cast<uint8_t*>(&s_abort) + 16;  // 2 slots of act_slot_bytes
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int I_pad = a.I_pad, hruns = I_pad / 32;
@@ -253,11 +265,34 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
       int stage = 0, slot = 0;
       uint32_t phase = 0, aphase = 0;
       bool waited = false;
+      // The unit's activations (h of the expert's token, written by the
+      // gate/up kernel: both byte planes and the run scales) go to a slot.
+      auto load_act = [&](int e) -> bool {
+        if (!ptx::mbar_wait(&aempty[slot], aphase ^ 1u)) return false;
+        const int r0 = __ldcg(a.offsets + e);
+        uint8_t* dst = s_act + slot * slot_bytes;
+        ptx::mbar_arrive_expect_tx(&afull[slot], (uint32_t)(2 * I_pad + hruns * 8));
+        ptx::bulk_load(dst, a.hq + (size_t)r0 * I_pad, (uint32_t)I_pad, &afull[slot]);
+        ptx::bulk_load(dst + I_pad, a.hq + a.hq_plane + (size_t)r0 * I_pad, (uint32_t)I_pad, &afull[slot]);
+        ptx::bulk_load(dst + 2 * I_pad, a.hsc + (size_t)r0 * hruns, (uint32_t)(hruns * 8), &afull[slot]);
+        if (++slot == 2) {
+          slot = 0;
+          aphase ^= 1u;
+        }
+        return true;
+      };
       for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
         const int ai = unit / tiles, rt = unit - ai * tiles;
         const int e = __ldcg(a.act + ai);
         const CUtensorMap* md = a.tmaps + kMapsPerSlot * __ldcg(a.slot_of + e) + 5;
-        // weights first: they do not depend on the gate/up kernel
+        // Once the gate/up kernel is complete, a unit's activations are issued
+        // before its weights, so they never hold up the unit's first stage.
+        if (waited && !load_act(e)) {
+          atomicOr(a.err, 4u);
+          return;
+        }
+        // the first unit's weights do not depend on the gate/up kernel: they
+        // are issued before waiting for it
         for (int st = 0; st < n_st; ++st) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
             atomicOr(a.err, 4u);
@@ -274,24 +309,13 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
             phase ^= 1u;
           }
         }
-        // then the unit's activations, written by the gate/up kernel
         if (!waited) {
           ptx::pdl_wait();
           waited = true;
-        }
-        if (!ptx::mbar_wait(&aempty[slot], aphase ^ 1u)) {
-          atomicOr(a.err, 4u);
-          return;
-        }
-        const int r0 = __ldcg(a.offsets + e);
-        uint8_t* dst = s_act + slot * slot_bytes;
-        ptx::mbar_arrive_expect_tx(&afull[slot], (uint32_t)(2 * I_pad + hruns * 8));
-        ptx::bulk_load(dst, a.hq + (size_t)r0 * I_pad, (uint32_t)I_pad, &afull[slot]);
-        ptx::bulk_load(dst + I_pad, a.hq + a.hq_plane + (size_t)r0 * I_pad, (uint32_t)I_pad, &afull[slot]);
-        ptx::bulk_load(dst + 2 * I_pad, a.hsc + (size_t)r0 * hruns, (uint32_t)(hruns * 8), &afull[slot]);
-        if (++slot == 2) {
-          slot = 0;
-          aphase ^= 1u;
+          if (!load_act(e)) {
+            atomicOr(a.err, 4u);
+            return;
+          }
         }
       }
       if (!waited) ptx::pdl_wait();
@@ -303,17 +327,18 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
   ptx::pdl_wait();  // hq / hsc come from the gate/up kernel
   ptx::pdl_launch_dependents();
 
-  // consumers: warp w takes rows 32*(w&3)+lane and part p = w>>2 of each
-  // stage: super-block p>>1 of the stage's two, chunks {2(p&1), 2(p&1)+1}
-  const int row = (warp & 3) * 32 + lane, part = warp >> 2;
-  const int sbi = part >> 1, c0 = 2 * (part & 1);
+  // consumers: warp w takes part p = w >> 1 of each stage -- super-block
+  // p >> 2 of the stage's two, chunk p & 3 -- for rows 32*(w&1)+lane and
+  // 64 rows further (the chunk's activations serve both rows)
+  const int row = (warp & 1) * 32 + lane, part = warp >> 1;
+  const int sbi = part >> 2, c = part & 3;
   int stage = 0, slot = 0;
   uint32_t phase = 0, aphase = 0;
   for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
     const int ai = unit / tiles, rt = unit - ai * tiles;
     const int e = __ldcg(a.act + ai);
     const int r0 = __ldcg(a.offsets + e);
-    float acc = 0.f;
+    float acc[2] = {0.f, 0.f};  // rows row, row + 64
     bool ok = ptx::mbar_wait(&afull[slot], aphase);
     if (!ok) atomicOr(a.err, 8u);
     const uint8_t* act = s_act + slot * slot_bytes;
@@ -326,8 +351,9 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
       }
       const int kb = 2 * st + sbi;
       if (kb < a.nbi) {
-        const uint8_t* blk = stages + stage * kGvStageBytes + sbi * kGvBox + row * kQBytes;
-        gv_two_chunks(blk, c0, act + kb * kQK, act + I_pad + kb * kQK, asc + kb * 8, acc);
+        const uint8_t* b0 = stages + stage * kGvStageBytes + sbi * kGvBox + row * kQBytes;
+        const uint8_t* const blk[2] = {b0, b0 + 64 * kQBytes};
+        gv_chunk_rows<2>(blk, c, act + kb * kQK, act + I_pad + kb * kQK, asc + kb * 8, acc);
       }
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&empty[stage]);
@@ -345,13 +371,16 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
     if (!ok) s_abort = 1;
     ptx::named_barrier_sync(1, kGvConsumers);  // also: the previous unit's reads of s_part are done
     if (s_abort) return;
-    s_part[part * kGvRows + row] = acc;
+    s_part[part * kGvRows + row] = acc[0];
+    s_part[part * kGvRows + row + 64] = acc[1];
     ptx::named_barrier_sync(1, kGvConsumers);
-    // the four parts of each row, summed in a fixed order, to y
+    // the eight parts of each row, summed in a fixed order, to y
     if (warp < 4) {
       const int r = warp * 32 + lane;
-      a.y[(size_t)r0 * a.H + rt * kGvRows + r] =
-          ((s_part[r] + s_part[kGvRows + r]) + s_part[2 * kGvRows + r]) + s_part[3 * kGvRows + r];
+      float v = s_part[r];
+#pragma unroll
+      for (int p = 1; p < 8; ++p) v += s_part[p * kGvRows + r];
+      a.y[(size_t)r0 * a.H + rt * kGvRows + r] = v;
     }
   }
 }
@@ -383,11 +412,11 @@ cudaError_t gv_launch(K kernel, uint64_t* mask, size_t smem, int n_sm, cudaStrea
 }  // namespace
 
 size_t gemv_gate_up_smem(int H) {
-  return 1024 + (size_t)kGvStages * kGvStageBytes + 2 * kGvStages * 8 + 4 * kGvRows * 4 + 16 + 2 * (size_t)H +
+  return 1024 + (size_t)kGvStages * kGvStageBytes + 2 * kGvStages * 8 + 8 * kGvRows * 4 + 16 + 2 * (size_t)H +
          (size_t)(H / 32) * 8;
 }
 size_t gemv_down_smem(size_t act_slot_bytes) {
-  return 1024 + (size_t)kGvStages * kGvStageBytes + 2 * kGvStages * 8 + 4 * 8 + 4 * kGvRows * 4 + 16 +
+  return 1024 + (size_t)kGvStages * kGvStageBytes + 2 * kGvStages * 8 + 4 * 8 + 8 * kGvRows * 4 + 16 +
          2 * act_slot_bytes;
 }
 

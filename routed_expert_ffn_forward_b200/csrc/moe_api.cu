@@ -800,6 +800,17 @@ moe_status moe_forward_routed(moe_layer_t L, const void* x, void* out, int T, co
   return forward_impl(L, x, out, T, forced_ids, static_cast<cudaStream_t>(stream));
 }
 
+// Device address of a pinned host buffer that kernels may access in place,
+// or null (pageable memory, or not mapped for the current device).
+static void* mapped_device_ptr(const void* p) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
 moe_status moe_forward_host(moe_layer_t L, const void* x_host, void* out_host, int T, void* stream) {
   g_err.clear();
   if (!L) return fail(MOE_ERR_INVALID_ARG, "null layer");
@@ -810,9 +821,22 @@ moe_status moe_forward_host(moe_layer_t L, const void* x_host, void* out_host, i
   MOE_TRY(ensure_scratch(L, T));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t bytes = (size_t)T * L->s.H * 2;
-  CUDA_TRY(cudaMemcpyAsync(L->xbuf, x_host, bytes, cudaMemcpyHostToDevice, st));
-  MOE_TRY(forward_impl(L, L->xbuf, L->obuf, T, nullptr, st));
-  CUDA_TRY(cudaMemcpyAsync(out_host, L->obuf, bytes, cudaMemcpyDeviceToHost, st));
+  // Decode path with pinned (mapped) host buffers: the kernels read x from
+  // and write out to host memory in place -- x by a staging kernel that the
+  // route kernel overlaps, out by the combine kernel.  Otherwise the buffers
+  // are copied through device memory.
+  const void* x_dev = T <= kD1MaxTok ? mapped_device_ptr(x_host) : nullptr;
+  void* o_dev = T <= kD1MaxTok ? mapped_device_ptr(out_host) : nullptr;
+  if (reinterpret_cast<uintptr_t>(o_dev) & 15u) o_dev = nullptr;
+  if (x_dev && launch_stage_in(x_dev, L->xbuf, bytes, st) == cudaSuccess) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_stats.launches += 1;
+  } else {
+    cudaGetLastError();  // an unaligned buffer takes the copy
+    CUDA_TRY(cudaMemcpyAsync(L->xbuf, x_host, bytes, cudaMemcpyHostToDevice, st));
+  }
+  MOE_TRY(forward_impl(L, L->xbuf, o_dev ? o_dev : L->obuf, T, nullptr, st));
+  if (!o_dev) CUDA_TRY(cudaMemcpyAsync(out_host, L->obuf, bytes, cudaMemcpyDeviceToHost, st));
   return MOE_OK;
 }
 

@@ -74,6 +74,10 @@ struct RouteArgs {
   unsigned* ticket;
 };
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st);
+// Copy `bytes` (a multiple of 16, both addresses 16-byte aligned) from mapped
+// host memory `src` (its device address) to device memory `dst`; the next
+// kernel may be launched as its programmatic dependent.
+cudaError_t launch_stage_in(const void* src, void* dst, size_t bytes, cudaStream_t st);
 
 // Arguments of the decode expert kernels.
 struct DecodeArgs {

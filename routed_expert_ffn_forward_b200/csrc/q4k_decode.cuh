@@ -25,11 +25,14 @@ __device__ __forceinline__ RowScales decode_scales(uint4 hdr, int c) {
     vsc = (s2 & 0x0F0Fu) | ((s0 >> 2) & 0x3030u);
     vm = ((s2 >> 4) & 0x0F0Fu) | ((s1 >> 2) & 0x3030u);
   }
+  // byte b -> float exactly: the bits 0x4B0000bb are the float 2^23 + b
+  constexpr uint32_t kMagic = 0x4B000000u;
+  constexpr float kMagicF = 8388608.f;
   RowScales r;
-  r.s_lo = d * (float)(vsc & 0xFFu);
-  r.s_hi = d * (float)((vsc >> 8) & 0xFFu);
-  r.m_lo = dmin * (float)(vm & 0xFFu);
-  r.m_hi = dmin * (float)((vm >> 8) & 0xFFu);
+  r.s_lo = d * (__uint_as_float(__byte_perm(vsc, kMagic, 0x7650)) - kMagicF);
+  r.s_hi = d * (__uint_as_float(__byte_perm(vsc, kMagic, 0x7651)) - kMagicF);
+  r.m_lo = dmin * (__uint_as_float(__byte_perm(vm, kMagic, 0x7650)) - kMagicF);
+  r.m_hi = dmin * (__uint_as_float(__byte_perm(vm, kMagic, 0x7651)) - kMagicF);
   return r;
 }
 

@@ -6,7 +6,7 @@
 // scale (a high-byte and a low-byte plane), with the run's scale and sum --
 // the form the expert kernels read.
 //
-// The last CTA to finish (a device-wide ticket) then does the top-k + gating
+// The last CTA to write its logits (a device-wide ticket) then does the top-k + gating
 // of every token (a warp per token) and the stable counting-sort permutation
 // of the T*k picks.  With few picks each pick's sorted position is found by
 // counting the picks before it in (expert, token, slot) order, so no pass over
@@ -33,12 +33,17 @@ __global__ void __launch_bounds__(kLogitThreads, 2) route_kernel(RouteArgs a) {
   const int e = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, T = a.T, E = a.E;
   // the first kernel of a forward: let the expert kernel start launching now
+  // (it waits for this kernel's completion before it reads anything)
   ptx::pdl_launch_dependents();
 
   // (1) logits of expert e for the T <= 4 tokens (first: the weight row is the
   // long-latency load); thread takes 4-element pieces h = 4*tid + 1024*i
   // The thread's weight and activation pieces of a pass are all loaded before
   // any arithmetic, so the CTA waits for one memory round trip per pass.
+  // Launched as a programmatic dependent (of the kernel that stages x from
+  // host memory, or of whatever precedes the forward), the kernel issues the
+  // constant router weights before it waits for its predecessor; x and every
+  // write come after the wait.
   constexpr int kPieces = 8;                     // per pass: H <= 8192 takes one pass
   const float4* wrow = reinterpret_cast<const float4*>(a.W + (size_t)e * H);
   const float bias = a.b ? a.b[e] : 0.f;
@@ -52,11 +57,16 @@ __global__ void __launch_bounds__(kLogitThreads, 2) route_kernel(RouteArgs a) {
 #pragma unroll
     for (int i = 0; i < kPieces; ++i) {
       const int q = base + tid + kLogitThreads * i;
+      if (q < nq) w4[i] = __ldg(wrow + q);
+    }
+    ptx::pdl_wait();  // returns at once after the first pass
+#pragma unroll
+    for (int i = 0; i < kPieces; ++i) {
+      const int q = base + tid + kLogitThreads * i;
       if (q < nq) {
-        w4[i] = __ldg(wrow + q);
 #pragma unroll
         for (int t = 0; t < kT; ++t)
-          if (t < T) xv[t][i] = __ldg(reinterpret_cast<const uint2*>(a.x + (size_t)t * H) + q);
+          if (t < T) xv[t][i] = __ldcg(reinterpret_cast<const uint2*>(a.x + (size_t)t * H) + q);
       }
     }
 #pragma unroll
@@ -87,9 +97,17 @@ __global__ void __launch_bounds__(kLogitThreads, 2) route_kernel(RouteArgs a) {
     for (int w = 0; w < kLogitThreads / 32; ++w) v += s_red[w][lane];
     a.logits[(size_t)lane * E + e] = v + bias;
   }
-  // (2) x prep: 16-bit fixed point per 32-element run, with the run scales
+  // (2) the ticket, as soon as the logits are written: the last CTA to take
+  // it does the routing of every token.  One release-acquire atomic per CTA,
+  // cumulative over the writes the barrier orders before it.
+  __syncthreads();
+  if (tid == 0) s_last = ptx::atom_add_acq_rel_gpu(a.ticket, 1u) == gridDim.x - 1;
+  __syncthreads();
+  // (3) x prep: 16-bit fixed point per 32-element run, with the run scales;
+  // the highest warps take the runs (the finishing CTA's top-k runs on warp 0)
   const int runs_per_tok = H / 32;
-  for (int run = e + gridDim.x * warp; run < T * runs_per_tok; run += gridDim.x * (kLogitThreads / 32)) {
+  const int xw = kLogitThreads / 32 - 1 - warp;
+  for (int run = e + gridDim.x * xw; run < T * runs_per_tok; run += gridDim.x * (kLogitThreads / 32)) {
     const int t = run / runs_per_tok, r = run - t * runs_per_tok;
     const int h = r * 32 + lane;
     float2 rsc;
@@ -101,15 +119,6 @@ __global__ void __launch_bounds__(kLogitThreads, 2) route_kernel(RouteArgs a) {
     if (lane == 0) a.xsc[(size_t)t * runs_per_tok + r] = rsc;
   }
 
-  // last CTA to finish: routing of every token (one device-scope fence on each
-  // side of the ticket, cumulative over the writes the barriers order)
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    s_last = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
-    __threadfence();
-  }
-  __syncthreads();
   if (!s_last) return;
   route_finish<PL>(a, s_dyn);
   if (tid == 0) *a.ticket = 0u;
@@ -214,18 +223,20 @@ cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st) {
   const size_t smem = route_decode_smem(a.H, a.T, a.E, a.k, a.S);
   if (a.T > kD1MaxTok) return cudaErrorInvalidValue;
   const bool small_e = (a.E + 31) / 32 <= 8;
-  if (a.T == 1) {
-    if (small_e)
-      route_kernel<8, 1><<<a.E, kLogitThreads, smem, st>>>(a);
-    else
-      route_kernel<32, 1><<<a.E, kLogitThreads, smem, st>>>(a);
-  } else {
-    if (small_e)
-      route_kernel<8, kD1MaxTok><<<a.E, kLogitThreads, smem, st>>>(a);
-    else
-      route_kernel<32, kD1MaxTok><<<a.E, kLogitThreads, smem, st>>>(a);
-  }
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.E);
+  cfg.blockDim = dim3(kLogitThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (a.T == 1)
+    return small_e ? cudaLaunchKernelEx(&cfg, route_kernel<8, 1>, a) : cudaLaunchKernelEx(&cfg, route_kernel<32, 1>, a);
+  return small_e ? cudaLaunchKernelEx(&cfg, route_kernel<8, kD1MaxTok>, a)
+                 : cudaLaunchKernelEx(&cfg, route_kernel<32, kD1MaxTok>, a);
 }
 
 }  // namespace moe

@@ -139,6 +139,39 @@ def test_deterministic_and_host_path(torch):
     L.destroy()
 
 
+@pytest.mark.parametrize("T", [1, 3, 4, 5])
+def test_host_path_pinned_pageable_unaligned(torch, T):
+    # decode sizes read and write pinned host buffers in place; pageable or
+    # unaligned buffers, and T > 4, are copied: every route gives the device result
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    cfg = SMALL["c0_shared_sigmoid_bias"]
+    L = layer_from_config(cfg)
+    x = synth.activations(cfg, tokens=T)
+    ref = to_bits(torch, L.forward(to_dev(torch, x)))
+    n = T * cfg.hidden
+    # pinned, aligned
+    xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    oh = torch.full_like(xh, 7.0).pin_memory()
+    moe.moe_forward_host(L.handle, xh.data_ptr(), oh.data_ptr(), T, None)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(oh.view(torch.int16).numpy().view(np.uint16).reshape(ref.shape), ref)
+    # pageable
+    xp = np.ascontiguousarray(x.view(np.uint16))
+    op = np.zeros_like(xp)
+    moe.moe_forward_host(L.handle, xp.ctypes.data, op.ctypes.data, T, None)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(op.reshape(ref.shape), ref)
+    # pinned, 2 bytes off a 16-byte boundary
+    xu = torch.zeros(n + 8, dtype=torch.bfloat16).pin_memory()
+    ou = torch.zeros(n + 8, dtype=torch.bfloat16).pin_memory()
+    xu[1:n + 1] = torch.from_numpy(x.view(np.int16).reshape(-1)).view(torch.bfloat16)
+    moe.moe_forward_host(L.handle, xu.data_ptr() + 2, ou.data_ptr() + 2, T, None)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(ou[1:n + 1].view(torch.int16).numpy().view(np.uint16).reshape(ref.shape), ref)
+    moe.moe_check(L.handle)
+    L.destroy()
+
+
 def test_forced_routing(torch):
     from routed_expert_ffn_forward_b200.layer import layer_from_config
     cfg = SMALL["c0_shared_sigmoid_bias"]
