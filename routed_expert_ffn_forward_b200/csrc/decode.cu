@@ -44,6 +44,14 @@ constexpr int kGuSB = 2;
 constexpr int kGuStages = 5;
 constexpr int kGuTileBytes = kTileRows * kGuSB * kQBytes;  // 18432
 constexpr int kGuStageBytes = 2 * kGuTileBytes;             // 36864
+// Without x staged per CTA, a stage also carries the stage's slice of each of
+// the unit's tokens' activations: hi bytes, lo bytes (kGuSB x 256 each) and
+// run scales (kGuSB x 8 float2).
+constexpr int kXSliceBytes = kGuSB * (2 * kQK + 8 * 8);   // 1152
+template <int kMaxTok, bool kStageX>
+__host__ __device__ constexpr int gu_stage_stride() {
+  return kGuStageBytes + (kStageX ? 0 : kMaxTok * kXSliceBytes);
+}
 // down: stage = 64 rows x 4 super-blocks
 constexpr int kDnSB = 4;
 constexpr int kDnStages = 4;
@@ -63,12 +71,10 @@ __device__ __forceinline__ void load_row_block(const uint8_t* blk, int c, int g,
   q[4] = hi.x; q[5] = hi.y; q[6] = hi.z; q[7] = hi.w;
 }
 
-// 32 zero bytes: the B source of lanes that own no activations.
-__device__ __align__(16) const uint8_t kZeroActs[32] = {};
 
 // One super-block of one warp's 16 rows against one activation vector.
 //  ahi/alo: the super-block's 256 activations, high (s8) and low (u8) bytes
-//           (shared or global memory; zero: 32 zero bytes in the same space)
+//           (shared memory; zero: 32 zero bytes of shared memory)
 //  sc:      (2^-s, X) of runs 2c and 2c+1 of the super-block
 // Lane (g, c) supplies B only if g == 2c (low positions of its chunk) or
 // g == 2c+1 (high positions).  The same registers feed the low-nibble MMA,
@@ -122,13 +128,16 @@ __device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw) {
 
 // ============================================================================ gate/up
 // kMaxTok: the most rows (tokens) an expert may have in this launch.  With
-// kStageX, x (all tokens) is copied to shared memory once per CTA.
+// kStageX, x (all tokens) is copied to shared memory once per CTA; without,
+// the producer bulk-copies each stage's slice of the unit's tokens' x next to
+// the stage's weights.
 template <int kMaxTok, bool kStageX>
 __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
+  constexpr int kStride = gu_stage_stride<kMaxTok, kStageX>();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw);
   uint8_t* stages = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGuStages * kGuStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGuStages * kStride);
   uint64_t* empty = full + kGuStages;
   float* s_part = reinterpret_cast<float*>(empty + kGuStages);  // [kp 2][mat 2][64][kMaxTok]
   int& s_abort = *reinterpret_cast<int*>(s_part + 4 * kTileRows * kMaxTok);
@@ -159,16 +168,38 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
       uint32_t phase = 0;
       for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
         const int ai = unit / tiles, rt = unit - ai * tiles;
-        const CUtensorMap* mg = a.tmaps + kMapsPerSlot * __ldcg(a.slot_of + __ldcg(a.act + ai));
+        const int e = __ldcg(a.act + ai);
+        const CUtensorMap* mg = a.tmaps + kMapsPerSlot * __ldcg(a.slot_of + e);
+        int cnt = 0, tok[kMaxTok];
+        if (!kStageX) {
+          cnt = __ldcg(a.counts + e);
+          const int r0 = __ldcg(a.offsets + e);
+#pragma unroll
+          for (int t = 0; t < kMaxTok; ++t) tok[t] = t < cnt ? __ldcg(a.perm + r0 + t) / a.kS : 0;
+        }
         for (int st = 0; st < n_st; ++st) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
             flag_error(a.err, 1u);
             return;
           }
-          ptx::mbar_arrive_expect_tx(&full[stage], kGuStageBytes);
-          uint8_t* dst = stages + stage * kGuStageBytes;
+          const int nsb = min(kGuSB, a.nbh - st * kGuSB);  // super-blocks of x this stage needs
+          ptx::mbar_arrive_expect_tx(&full[stage], kGuStageBytes + (uint32_t)(cnt * nsb * (2 * kQK + 64)));
+          uint8_t* dst = stages + stage * kStride;
           ptx::tma_load_2d(dst, mg, st * kGuSB * 18, rt * kTileRows, &full[stage]);
           ptx::tma_load_2d(dst + kGuTileBytes, mg + 1, st * kGuSB * 18, rt * kTileRows, &full[stage]);
+          if (!kStageX) {
+#pragma unroll
+            for (int t = 0; t < kMaxTok; ++t) {
+              if (t < cnt) {
+                uint8_t* xs = dst + kGuStageBytes + t * kXSliceBytes;
+                const size_t xo = (size_t)tok[t] * a.H + (size_t)st * kGuSB * kQK;
+                ptx::bulk_load(xs, a.xq + xo, (uint32_t)(nsb * kQK), &full[stage]);
+                ptx::bulk_load(xs + kGuSB * kQK, a.xq + a.xq_plane + xo, (uint32_t)(nsb * kQK), &full[stage]);
+                ptx::bulk_load(xs + 2 * kGuSB * kQK, a.xsc + (size_t)tok[t] * runs + (size_t)st * kGuSB * 8,
+                               (uint32_t)(nsb * 64), &full[stage]);
+              }
+            }
+          }
           if (++stage == kGuStages) {
             stage = 0;
             phase ^= 1u;
@@ -194,10 +225,10 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
     for (int i = threadIdx.x; i < a.T * runs; i += kConsumerThreads) dsc[i] = __ldcg(a.xsc + i);
     ptx::named_barrier_sync(1, kConsumerThreads);
   }
-  const uint8_t* xh_base = kStageX ? s_x : reinterpret_cast<const uint8_t*>(a.xq);
-  const uint8_t* xl_base = kStageX ? s_x + xbytes : reinterpret_cast<const uint8_t*>(a.xq + a.xq_plane);
-  const float2* xsc_base = kStageX ? reinterpret_cast<const float2*>(s_x + 2 * xbytes) : a.xsc;
-  const uint8_t* zero = kStageX ? s_zero : kZeroActs;
+  const uint8_t* xh_base = s_x;
+  const uint8_t* xl_base = s_x + xbytes;
+  const float2* xsc_base = reinterpret_cast<const float2*>(s_x + 2 * xbytes);
+  const uint8_t* zero = s_zero;
 
   // consumers: warp w takes matrix (w>>2)&1 (gate, up), rows 16*(w&3).., and
   // super-block w>>3 of every stage
@@ -211,8 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
     const int e = __ldcg(a.act + ai);
     const int cnt = __ldcg(a.counts + e), r0 = __ldcg(a.offsets + e);
     int tok[kMaxTok];
+    if (kStageX) {
 #pragma unroll
-    for (int t = 0; t < kMaxTok; ++t) tok[t] = t < cnt ? __ldcg(a.perm + r0 + t) / a.kS : 0;
+      for (int t = 0; t < kMaxTok; ++t) tok[t] = t < cnt ? __ldcg(a.perm + r0 + t) / a.kS : 0;
+    }
     float acc[kMaxTok], acc8[kMaxTok];
 #pragma unroll
     for (int t = 0; t < kMaxTok; ++t) acc[t] = acc8[t] = 0.f;
@@ -225,7 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
       }
       const int kb = st * kGuSB + kp;
       if (kb < a.nbh) {
-        const uint8_t* blk = stages + stage * kGuStageBytes + mat * kGuTileBytes + (rbase + g) * pitch + kp * kQBytes;
+        const uint8_t* sbase = stages + stage * kStride;
+        const uint8_t* blk = sbase + mat * kGuTileBytes + (rbase + g) * pitch + kp * kQBytes;
         uint4 h0, h8;
         uint32_t q[8], q8[8];
         load_row_block(blk, c, g, h0, q);
@@ -234,9 +268,16 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
 #pragma unroll
         for (int t = 0; t < kMaxTok; ++t) {
           if (t < cnt) {
-            const size_t xo = (size_t)tok[t] * a.H + kb * kQK;
-            const float4 sc = reinterpret_cast<const float4*>(xsc_base + (size_t)tok[t] * runs + kb * 8)[c];
-            sb_dot(q, q8, rs, rs8, xh_base + xo, xl_base + xo, zero, sc, g, c, acc[t], acc8[t]);
+            if (kStageX) {
+              const size_t xo = (size_t)tok[t] * a.H + kb * kQK;
+              const float4 sc = reinterpret_cast<const float4*>(xsc_base + (size_t)tok[t] * runs + kb * 8)[c];
+              sb_dot(q, q8, rs, rs8, xh_base + xo, xl_base + xo, zero, sc, g, c, acc[t], acc8[t]);
+            } else {
+              // the token's slice in this stage: hi, lo, run scales
+              const uint8_t* xs = sbase + kGuStageBytes + t * kXSliceBytes;
+              const float4 sc = reinterpret_cast<const float4*>(xs + 2 * kGuSB * kQK + kp * 64)[c];
+              sb_dot(q, q8, rs, rs8, xs + kp * kQK, xs + kGuSB * kQK + kp * kQK, zero, sc, g, c, acc[t], acc8[t]);
+            }
           }
         }
       }
@@ -468,8 +509,11 @@ __global__ void __launch_bounds__(kThreads, 1) down_d1_kernel(DecodeArgs a) {
 }  // namespace
 
 // Shared memory of the decode kernels (bytes, with 1024 of alignment slack).
+// x_stage_bytes > 0: x staged once per CTA (the max_tok = 1 kernel); 0: each
+// stage carries max_tok tokens' x slices.
 size_t gate_up_d1_smem(int max_tok, size_t x_stage_bytes) {
-  return 1024 + (size_t)kGuStages * kGuStageBytes + 2 * kGuStages * 8 + 4 * kTileRows * max_tok * 4 + 16 + 32 +
+  const size_t stride = kGuStageBytes + (x_stage_bytes ? 0 : (size_t)max_tok * kXSliceBytes);
+  return 1024 + (size_t)kGuStages * stride + 2 * kGuStages * 8 + 4 * kTileRows * max_tok * 4 + 16 + 32 +
          x_stage_bytes;
 }
 size_t down_d1_smem(int max_tok, size_t act_slot_bytes) {
