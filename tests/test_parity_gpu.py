@@ -213,8 +213,8 @@ def test_prefill_weight_range_is_reported(torch):
     L.forward(to_dev(torch, x))          # decode path: exact weights, no flag
     torch.cuda.synchronize()
     moe.moe_check(L.handle)
-    x = synth.activations(cfg, tokens=64)
-    L.forward(to_dev(torch, x))          # prefill path: ~8 rows per expert, tensor-core GEMMs
+    x = synth.activations(cfg, tokens=256)
+    L.forward(to_dev(torch, x))          # prefill path: ~32 rows per expert, tensor-core GEMMs
     torch.cuda.synchronize()
     with pytest.raises(moe.MoEError) as ei:
         moe.moe_check(L.handle)
