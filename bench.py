@@ -23,6 +23,7 @@ import json
 import os
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -45,10 +46,10 @@ def log(*a):
 class ClockSampler:
     """nvidia-smi clock/throttle samples while the timed region runs."""
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, directory: str):
         self.dev = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.path = os.path.join(directory, f"clocks_rank{device_index}.csv")
 
     def __enter__(self):
         try:
@@ -283,7 +284,7 @@ def run_ours(args, cfg, rank: int, world: int, local_rank: int) -> dict | None:
     st0 = moe.moe_get_stats()
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(local_rank, args.clocks_dir) as clk:
         for i in range(args.steps):
             step(i, evs[i])
         torch.cuda.synchronize()
@@ -404,7 +405,7 @@ def run_streaming(args, cfg, rank, world, local_rank, peaks) -> dict:
     moe.moe_reset_stats()
     barrier(world)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(local_rank, args.clocks_dir) as clk:
         ev0.record(stream)
         for s in range(args.warmup, n_steps):
             run_step(s)
@@ -474,11 +475,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=1, choices=[1, 2, 3, 4])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-dir", default=tempfile.gettempdir(),
+                    help="where the raw nvidia-smi samples of the timed region are written")
     ap.add_argument("--no-prefetch", action="store_true")
     ap.add_argument("--small", action="store_true",
                     help="32 routed experts instead of 256 (same per-launch work at T=1; for ncu captures)")
     args = ap.parse_args()
-    cfg = synth.CONFIGS[args.config]
+    cfg = synth.WORKLOADS[args.config]
     if args.small:
         import dataclasses
         cfg = dataclasses.replace(cfg, n_experts=32, name=cfg.name + " [32 experts]")
@@ -500,7 +503,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config in (1, 2):
         res["cpu_baseline"] = oracle_sample_rate(cfg, n_tokens=cfg.tokens, budget_s=20.0)
     elif rank == 0 and not args.no_cpu_baseline and world == 1:
-        res["cpu_baseline"] = oracle_sample_rate(synth.CONFIGS[1], n_tokens=3, budget_s=20.0) | {
+        res["cpu_baseline"] = oracle_sample_rate(synth.DECODE, n_tokens=3, budget_s=20.0) | {
             "sample": "decode tokens of the config-1 layer (the oracle's cost per token is the same per expert)"}
     if world > 1:
         import torch.distributed as dist

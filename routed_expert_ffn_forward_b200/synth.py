@@ -77,19 +77,19 @@ class LayerConfig:
 
 
 H, I = 7168, 2048
-CONFIGS = {
-    0: LayerConfig("tiny: H=256 I=128 E=16 k=2 S=0 T=4 softmax", 256, 128, 16, 2, 0, 4,
-                   0, 0, 1.0 / 16.0),
-    1: LayerConfig("decode: H=7168 I=2048 E=256+1 k=8 T=1 sigmoid, resident", H, I, 256, 8, 1, 1,
-                   1, 1, 1.0 / math.sqrt(H)),
-    2: LayerConfig("batched decode: T=64, Zipf(1.1) router bias", H, I, 256, 8, 1, 64,
-                   1, 2, 1.0 / math.sqrt(H), zipf_s=1.1),
-    3: LayerConfig("prefill chunk: T=4096, Zipf(0.8) router bias", H, I, 256, 8, 1, 4096,
-                   1, 3, 1.0 / math.sqrt(H), zipf_s=0.8),
-    4: LayerConfig("expert streaming: 8 layers, 12e9 B cache, T=1, 512 steps", H, I, 256, 8, 1, 1,
-                   1, 4, 1.0 / math.sqrt(H), n_layers=8, cache_bytes=12_000_000_000, steps=512,
-                   zipf_s=1.1),
-}
+TINY = LayerConfig("tiny: H=256 I=128 E=16 k=2 S=0 T=4 softmax", 256, 128, 16, 2, 0, 4,
+                   0, 0, 1.0 / 16.0)
+DECODE = LayerConfig("decode: H=7168 I=2048 E=256+1 k=8 T=1 sigmoid, resident", H, I, 256, 8, 1, 1,
+                     1, 1, 1.0 / math.sqrt(H))
+BATCHED = LayerConfig("batched decode: T=64, Zipf(1.1) router bias", H, I, 256, 8, 1, 64,
+                      1, 2, 1.0 / math.sqrt(H), zipf_s=1.1)
+PREFILL = LayerConfig("prefill chunk: T=4096, Zipf(0.8) router bias", H, I, 256, 8, 1, 4096,
+                      1, 3, 1.0 / math.sqrt(H), zipf_s=0.8)
+STREAMING = LayerConfig("expert streaming: 8 layers, 12e9 B cache, T=1, 512 steps", H, I, 256, 8, 1, 1,
+                        1, 4, 1.0 / math.sqrt(H), n_layers=8, cache_bytes=12_000_000_000, steps=512,
+                        zipf_s=1.1)
+# bench.py --config N selects WORKLOADS[N]
+WORKLOADS = {0: TINY, 1: DECODE, 2: BATCHED, 3: PREFILL, 4: STREAMING}
 
 
 def _gen(seed: int, kind: int, a: int = 0, b: int = 0, c: int = 0) -> np.random.Generator:

@@ -194,7 +194,7 @@ def test_permutation_bijection_and_stable_order():
 # ------------------------------------------------------------------ whole layer
 @pytest.mark.parametrize("variant", ["c0", "c0_shared_sigmoid"])
 def test_sparse_equals_dense_bruteforce(variant):
-    cfg = synth.CONFIGS[0]
+    cfg = synth.TINY
     if variant == "c0_shared_sigmoid":
         cfg = cfg_with(cfg, n_shared=1, gating=1, top_k=3, tokens=6)
     layer = tiny_layer(cfg)
@@ -205,7 +205,7 @@ def test_sparse_equals_dense_bruteforce(variant):
 
 
 def test_zero_scale_experts_contribute_nothing():
-    cfg = cfg_with(synth.CONFIGS[0], n_shared=1)
+    cfg = cfg_with(synth.TINY, n_shared=1)
     layer = tiny_layer(cfg, zero_routed=True)
     x = synth.activations(cfg)
     out = ref.moe_forward(x, layer, cfg.top_k, cfg.gating, 1, cfg.inter)["out64"]
@@ -223,7 +223,7 @@ def test_constant_weight_closed_form():
     blocks = (make_block(0.0625, 0.75, [2] * 8, [0] * 8, [5] * 256),
               make_block(0.03125, 0.5, [3] * 8, [0] * 8, [7] * 256),
               make_block(0.015625, 0.25, [1] * 8, [0] * 8, [11] * 256))
-    cfg = synth.CONFIGS[0]
+    cfg = synth.TINY
     layer = tiny_layer(cfg, const_block=blocks)
     x = synth.activations(cfg)
     out = ref.moe_forward(x, layer, cfg.top_k, cfg.gating, 0, cfg.inter)["out64"]
@@ -233,7 +233,7 @@ def test_constant_weight_closed_form():
 
 
 def test_token_permutation_equivariance():
-    cfg = cfg_with(synth.CONFIGS[0], tokens=8, n_shared=1, gating=1)
+    cfg = cfg_with(synth.TINY, tokens=8, n_shared=1, gating=1)
     layer = tiny_layer(cfg)
     x = synth.activations(cfg)
     p = np.random.default_rng(0).permutation(cfg.tokens)
@@ -243,7 +243,7 @@ def test_token_permutation_equivariance():
 
 
 def test_expert_relabelling_invariance():
-    cfg = cfg_with(synth.CONFIGS[0], tokens=6)
+    cfg = cfg_with(synth.TINY, tokens=6)
     layer = tiny_layer(cfg)
     x = synth.activations(cfg)
     E = cfg.n_experts
@@ -258,7 +258,7 @@ def test_expert_relabelling_invariance():
 
 
 def test_forced_routing_weights():
-    cfg = cfg_with(synth.CONFIGS[0], gating=1)
+    cfg = cfg_with(synth.TINY, gating=1)
     layer = tiny_layer(cfg)
     x = synth.activations(cfg)
     forced = np.array([[0, 5], [1, 2], [15, 3], [7, 8]])

@@ -73,7 +73,7 @@ def check_against_oracle(cfg, g, sample=None, layer_index=0):
 
 
 # ------------------------------------------------------------------ small shapes, every token
-C0 = synth.CONFIGS[0]
+C0 = synth.TINY
 SMALL = {
     "c0": C0,
     "c0_shared_sigmoid_bias": dataclasses.replace(C0, n_shared=1, gating=1, zipf_s=1.1, seed=11),
@@ -103,13 +103,13 @@ def test_zero_tokens(torch):
 
 # ------------------------------------------------------------------ full-size configurations
 def test_c1_decode_every_token(torch):
-    cfg = synth.CONFIGS[1]
+    cfg = synth.DECODE
     g = run_gpu(torch, cfg, cfg.tokens)
     check_against_oracle(cfg, g)
 
 
 def test_c2_batched_decode_sampled(torch):
-    cfg = synth.CONFIGS[2]
+    cfg = synth.BATCHED
     g = run_gpu(torch, cfg, cfg.tokens)
     counts = np.bincount(g["ids"].ravel(), minlength=cfg.n_experts)
     assert (counts > 10).sum() >= 1 and (counts.max() <= cfg.tokens)
@@ -117,14 +117,14 @@ def test_c2_batched_decode_sampled(torch):
 
 
 def test_c3_prefill_sampled(torch):
-    cfg = synth.CONFIGS[3]
+    cfg = synth.PREFILL
     g = run_gpu(torch, cfg, cfg.tokens)
     check_against_oracle(cfg, g, sample=[0, 1777, 4095])
 
 
 def test_deterministic_and_host_path(torch):
     from routed_expert_ffn_forward_b200.layer import layer_from_config
-    cfg = synth.CONFIGS[2]
+    cfg = synth.BATCHED
     L = layer_from_config(cfg)
     x = synth.activations(cfg)
     xd = to_dev(torch, x)

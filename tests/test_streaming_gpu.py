@@ -96,7 +96,7 @@ def run_trace(torch, cfg, layers, trace, steps, prefetch, model=None):
     return outs
 
 
-SMALL = dataclasses.replace(synth.CONFIGS[0], name="streaming small", n_shared=1, gating=1, n_layers=3,
+SMALL = dataclasses.replace(synth.TINY, name="streaming small", n_shared=1, gating=1, n_layers=3,
                             steps=14, seed=21)
 
 
@@ -139,7 +139,7 @@ def test_streaming_c1_shapes_against_oracle(torch):
     2 layers through a 20-slot cache (2 tokens need at most 17 experts); unrouted forward (routing read back to the
     host) and a check of one streamed token against the oracle."""
     from routed_expert_ffn_forward_b200.layer import layer_from_config
-    cfg = dataclasses.replace(synth.CONFIGS[4], n_experts=32, n_layers=2, steps=6, seed=41)
+    cfg = dataclasses.replace(synth.STREAMING, n_experts=32, n_layers=2, steps=6, seed=41)
     eb = moe.moe_expert_bytes(cfg.hidden, cfg.inter)
     moe.moe_set_cache_bytes(20 * eb)
     try:

@@ -18,7 +18,7 @@ from tests import parity_util as pu
 
 pytestmark = pytest.mark.gpu
 
-CFG = dataclasses.replace(synth.CONFIGS[2], name="no-alloc routing", hidden=1024, inter=256, n_experts=64,
+CFG = dataclasses.replace(synth.BATCHED, name="no-alloc routing", hidden=1024, inter=256, n_experts=64,
                           top_k=6, tokens=40, seed=77, router_std=1 / 32)
 
 
