@@ -131,15 +131,15 @@ __device__ void route_finish(const RouteArgs& a, int* s_ids) {
   const int T = a.T, E = a.E, k = a.k, S = a.S, kS = k + S, N = T * k;
   int* s_first = s_ids + N;               // [N] 1 if pick i is its expert's first pick
   int* s_count = s_first + N;             // [N] rows of pick i's expert
+  // top-k + gating, one warp per token (no barrier before it: the CTA's last
+  // x-prep run, on the highest warp, overlaps it)
+  for (int t = warp; t < T; t += kLogitThreads / 32)
+    warp_topk_gate<PL, true>(a.logits + (size_t)t * E, E, k, a.gating, a.forced ? a.forced + (size_t)t * k : nullptr,
+                             s_ids + t * k, a.w + (size_t)t * k);
   if (tid == 0) {
     s_cnt_small = 0;
     s_cnt_big = 0;
   }
-  __syncthreads();
-  // top-k + gating, one warp per token
-  for (int t = warp; t < T; t += kLogitThreads / 32)
-    warp_topk_gate<PL, true>(a.logits + (size_t)t * E, E, k, a.gating, a.forced ? a.forced + (size_t)t * k : nullptr,
-                             s_ids + t * k, a.w + (size_t)t * k);
   __syncthreads();
   // per pick: rows of its expert, whether it is the expert's first pick
   for (int i = tid; i < N; i += kLogitThreads) {
