@@ -1,0 +1,72 @@
+"""The benchmark's roofline arithmetic, checked on the CPU against the Q4_K
+byte counts written out by hand (144 bytes per 256 weights)."""
+import dataclasses
+import hashlib
+import json
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from routed_expert_ffn_forward_b200 import synth  # noqa: E402
+
+
+def test_decode_bytes_match_hand_count():
+    cfg = synth.DECODE                      # H = 7168, I = 2048, k = 8, S = 1, T = 1
+    ids = np.arange(8, dtype=np.int32)[None, :]
+    gate = 2048 * (7168 // 256) * 144       # one gate (or up) matrix: 8,257,536 B
+    down = 7168 * (2048 // 256) * 144       # 8,257,536 B
+    assert gate == down == 8_257_536
+    experts = 9                             # 8 routed + the shared one
+    assert bench.algorithmic_bytes(cfg, ids, "gate_up") == experts * 2 * gate + 7168 * 2 + 9 * 2048 * 2
+    assert bench.algorithmic_bytes(cfg, ids, "down") == experts * down + 9 * 2048 * 2 + 2 * 7168 * 2
+    fwd = experts * (2 * gate + down) + 256 * 7168 * 4 + 2 * 7168 * 2
+    assert bench.algorithmic_bytes(cfg, ids, "forward") == fwd
+    assert abs(fwd - 230.3e6) < 0.1e6      # the per-token figure the layer is quoted on
+
+
+def test_repeated_experts_counted_once():
+    cfg = dataclasses.replace(synth.DECODE, tokens=3)
+    ids = np.array([[0, 1, 2, 3, 4, 5, 6, 7]] * 3, dtype=np.int32)   # three tokens, same experts
+    one = bench.algorithmic_bytes(cfg, ids[:1], "forward")
+    three = bench.algorithmic_bytes(cfg, ids, "forward")
+    assert three - one == 2 * 2 * 7168 * 2   # only x and out grow with the tokens
+
+
+def test_prefill_gate_up_counts_only_gemm_experts():
+    cfg = synth.BATCHED                     # T = 64: experts with <= 4 rows take the decode kernels
+    ids = np.zeros((64, 8), dtype=np.int32)
+    ids[:, 0] = 0                           # expert 0: 64 rows (GEMM)
+    ids[:, 1:] = np.arange(1, 8)[None, :] + 7 * (np.arange(64)[:, None] % 4)
+    ids[:60, 7] = 100 + np.arange(60) // 4  # 15 experts x 4 rows (decode kernels)
+    # columns 1-6: 24 experts x 16 rows (GEMM); column 7 of the last 4 tokens:
+    # 4 experts x 1 row (decode kernels)
+    gate = 2048 * 28 * 144
+    counts = np.bincount(ids.ravel(), minlength=256)
+    assert np.all(np.sort(ids, axis=1)[:, 1:] != np.sort(ids, axis=1)[:, :-1])  # distinct picks per token
+    assert int(np.sum(counts > 4)) == 25 and int(np.sum((counts > 0) & (counts <= 4))) == 19
+    gemm = 25 + 1                           # + the shared expert
+    expect = gemm * 2 * gate + 64 * 7168 * 2 + 64 * 9 * 2048 * 2
+    assert bench.algorithmic_bytes(cfg, ids, "gate_up") == expect
+
+
+def test_prefill_flops():
+    cfg = synth.PREFILL
+    assert bench.flops(cfg, cfg.tokens) == 2.0 * 4096 * 9 * 3 * 7168 * 2048
+    assert abs(bench.flops(cfg, cfg.tokens) - 3.247e12) < 0.001e12
+
+
+def test_traffic_entry_tracks_its_source():
+    """A recorded DRAM byte count is reported only while the kernel's source is
+    the one it was captured from."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    for key, d in json.load(open(p)).items():
+        src = os.path.join(ROOT, d["source"])
+        current = hashlib.sha256(open(src, "rb").read()).hexdigest() == d["sha256"]
+        got = bench.kernel_traffic(key)
+        assert (got == float(d["bytes_per_launch"])) if current else got is None
+    assert bench.kernel_traffic("config9:nothing") is None
