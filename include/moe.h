@@ -146,14 +146,18 @@ moe_status moe_set_cache_bytes(size_t bytes);
 
 /* Forward: x bf16 [T, H] and out bf16 [T, H], device pointers, row-major.
  * T >= 0 (T = 0 returns at once).  T <= 4 takes the decode path (fused router,
- * expert kernels on the integer tensor MMA straight from the Q4_K bytes),
- * larger T the prefill path (router and expert projections as tcgen05 grouped
- * GEMMs; the Q4_K weights are dequantised to fp16 in shared memory, which
- * requires every block's |d| < 0.248 and |dmin| < 3.72, i.e. weights within
- * about +-234; moe_check reports a violation).  Work is enqueued on `stream`;
- * in resident mode the call does not wait for the GPU.  In streaming mode it reads the routing back to the
- * host (one stream synchronisation) to resolve cache misses before the expert
- * kernels are launched.  out must not overlap x. */
+ * expert kernels straight from the Q4_K bytes: byte dot products for T = 1,
+ * the integer tensor MMA for 2..4), larger T the prefill path (router and the
+ * projections of experts with more than 4 rows as tcgen05 grouped GEMMs; the
+ * Q4_K weights are dequantised to fp16 in shared memory, which requires every
+ * block's |d| < 0.248 and |dmin| < 3.72, i.e. weights within about +-234;
+ * moe_check reports a violation; experts with at most 4 rows take the decode
+ * kernels).  Work is enqueued on `stream`; in resident mode the call does not
+ * wait for the GPU.  The first kernel is launched as a programmatic dependent
+ * of the stream's previous work: it waits for that work before it reads x.
+ * In streaming mode the call reads the routing back to the host (one stream
+ * synchronisation) to resolve cache misses before the expert kernels are
+ * launched.  out must not overlap x. */
 moe_status moe_forward(moe_layer_t layer, const void* x, void* out, int T, void* stream);
 
 /* Forward with the routing given: forced_ids int32 [T, top_k] on the HOST
