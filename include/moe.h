@@ -153,8 +153,9 @@ moe_status moe_set_cache_bytes(size_t bytes);
  * block's |d| < 0.248 and |dmin| < 3.72, i.e. weights within about +-234;
  * moe_check reports a violation; experts with at most 4 rows take the decode
  * kernels).  Work is enqueued on `stream`; in resident mode the call does not
- * wait for the GPU.  The first kernel is launched as a programmatic dependent
- * of the stream's previous work: it waits for that work before it reads x.
+ * wait for the GPU.  On the decode path the first kernel is launched as a
+ * programmatic dependent of the stream's previous work: it waits for that
+ * work before it reads x or writes anything.
  * In streaming mode the call reads the routing back to the host (one stream
  * synchronisation) to resolve cache misses before the expert kernels are
  * launched.  out must not overlap x. */
