@@ -134,6 +134,25 @@ def test_round_bf16_ties_and_single_rounding():
     assert ref.round_bf16(np.array([-(1.0 + 2 ** -8 + 2 ** -40)]))[0] == (one + 1) | 0x8000
 
 
+def test_bf16_to_f64_matches_torch_on_every_pattern():
+    # every 16-bit pattern that is not a NaN, against torch's own bf16 -> fp32
+    torch = pytest.importorskip("torch")
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float32).numpy()
+    keep = ~np.isnan(t)
+    assert keep.sum() == (1 << 16) - 2 * 127          # 127 NaN mantissas per sign
+    np.testing.assert_array_equal(ref.bf16_to_f64(bits[keep]), t[keep].astype(np.float64))
+
+
+# ------------------------------------------------------------------ SwiGLU activation
+def test_silu_matches_scipy_expit():
+    # silu(z) = z * sigmoid(z), against scipy's logistic function, up to |z| = 700
+    sp = pytest.importorskip("scipy.special")
+    z = np.concatenate([np.linspace(-700.0, 700.0, 20001), np.linspace(-8.0, 8.0, 4001),
+                        [0.0, -0.0, 1e-300, -1e-300, 36.7, -36.7]])
+    np.testing.assert_allclose(ref.silu(z), z * sp.expit(z), rtol=1e-14, atol=1e-300)
+
+
 # ------------------------------------------------------------------ router
 def test_router_logits_one_hot():
     rng = np.random.default_rng(2)
@@ -268,13 +287,34 @@ def test_forced_routing_weights():
     np.testing.assert_array_equal(r["ids"], forced)
 
 
+def test_token_subset_rows_equal_full_rows():
+    # computing only some output rows gives those rows of the full run, in the
+    # subset's order, with and without forced routing (the float rows up to
+    # the summation order of the BLAS kernel, which depends on the row count)
+    cfg = cfg_with(synth.TINY, tokens=9, n_shared=1, gating=1, top_k=3)
+    layer = tiny_layer(cfg)
+    x = synth.activations(cfg)
+    subset = [7, 2, 5, 0]
+    forced = np.random.default_rng(8).integers(0, cfg.n_experts, (cfg.tokens, cfg.top_k))
+    for f in (None, forced):
+        full = ref.moe_forward(x, layer, cfg.top_k, cfg.gating, 1, cfg.inter, forced_ids=f)
+        part = ref.moe_forward(x, layer, cfg.top_k, cfg.gating, 1, cfg.inter, forced_ids=f, token_subset=subset)
+        np.testing.assert_array_equal(part["tokens"], subset)
+        for key in ("out_bf16", "ids"):
+            np.testing.assert_array_equal(part[key], full[key][subset], err_msg=key)
+        for key in ("out64", "w", "logits", "gap"):
+            np.testing.assert_allclose(part[key], full[key][subset], rtol=1e-12, atol=0, err_msg=key)
+
+
 # ------------------------------------------------------------------ planted mistakes
 def _pins_pass() -> bool:
     checks = [test_q4k_hand_block, test_q4k_closed_form_constant, test_q4k_weight_order,
               test_q4k_scale_pack_round_trip, test_topk_matches_stable_argsort_and_ties,
               test_gate_weights_sum_to_one_and_softmax_dense,
               lambda: test_sparse_equals_dense_bruteforce("c0_shared_sigmoid"),
-              test_constant_weight_closed_form, test_permutation_bijection_and_stable_order]
+              test_constant_weight_closed_form, test_permutation_bijection_and_stable_order,
+              test_bf16_to_f64_matches_torch_on_every_pattern, test_silu_matches_scipy_expit,
+              test_token_subset_rows_equal_full_rows]
     for c in checks:
         try:
             c()
@@ -305,6 +345,26 @@ MUTANTS = {
     "unstable permutation": ("permutation", lambda orig: (
         lambda ids, E: (lambda c, o, p: (c, o, p[::-1].copy()))(*orig(ids, E)))),
 }
+
+
+def _subset_forced_by_position(orig):
+    # the bug: a subset run takes forced_ids row i for the subset's i-th token
+    # instead of the row of that token
+    def bad(x_bits, layer, k, gating, n_shared, inter, forced_ids=None, token_subset=None):
+        if forced_ids is not None and token_subset is not None:
+            f = np.asarray(forced_ids).copy()
+            f[np.asarray(token_subset)] = np.asarray(forced_ids)[:len(token_subset)]
+            forced_ids = f
+        return orig(x_bits, layer, k, gating, n_shared, inter, forced_ids=forced_ids, token_subset=token_subset)
+    return bad
+
+
+MUTANTS.update({
+    "bf16 shifted by 15": ("bf16_to_f64", lambda orig: (
+        lambda bits: (np.asarray(bits, np.uint16).astype(np.uint32) << 15).view(np.float32).astype(np.float64))),
+    "silu without the z factor": ("silu", lambda orig: (lambda z: 1.0 / (1.0 + np.exp(-z)))),
+    "subset ignores its forced rows": ("moe_forward", _subset_forced_by_position),
+})
 
 
 def _unmasked_ffn(xr, g, u, d):
