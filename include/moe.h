@@ -215,16 +215,22 @@ moe_status moe_reset_profile(void);
  * on a latency-critical path that cannot take cudaMalloc's implicit
  * synchronisation, so they cannot create a moe_layer.  The pages have no
  * counterpart to this call.
- * x bf16 [T, H], W fp32 [E, H], bias fp32 [E] or NULL: device pointers.
- * ids int32 [T, top_k] and weights fp32 [T, top_k]: device outputs, same
- * meaning as in moe_get_routing.  Work is enqueued on `stream`.
+ * x bf16 [T, H] (16-byte aligned), W fp32 [E, H] (16-byte aligned), bias fp32
+ * [E] or NULL: device pointers.  ids int32 [T, top_k] and weights fp32
+ * [T, top_k]: device outputs, same meaning as in moe_get_routing.  bias, ids
+ * and weights must be 4-byte aligned.  A misaligned pointer is rejected with
+ * MOE_ERR_INVALID_ARG before anything is launched.  Work is enqueued on
+ * `stream`.
  * Allocates nothing: the [T, E] logits scratch is a fixed array inside the
  * library of 65536 floats (256 KiB, held on every GPU that loads the library
  * until the process exits), so T * E must be <= 65536 (MOE_ERR_UNSUPPORTED
- * otherwise).  The first call on a GPU looks up the array's device address;
- * make that first call before any stream capture.  All calls on a GPU share
- * the array: calls whose kernels may overlap on the GPU (different streams
- * without ordering) race on it.  H: multiple of 256; E <= 1024;
+ * otherwise).  The first call on a GPU looks up the array's device address
+ * and caches it with the current context; a call in a new context (after
+ * cudaDeviceReset) looks it up again.  Make the first call on each GPU, and
+ * the first after a reset, outside stream capture: inside capture it returns
+ * MOE_ERR_NOT_READY.  All calls on a GPU share the array and it keeps the last
+ * call's contents: calls whose kernels may overlap on the GPU (different
+ * streams without ordering) race on it.  H: multiple of 256; E <= 1024;
  * top_k <= min(32, E). */
 moe_status moe_route_noalloc(const void* x, const float* W, const float* bias, int T, int H, int E,
                              int top_k, moe_gating gating, int32_t* ids, float* weights,
