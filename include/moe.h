@@ -99,7 +99,8 @@ typedef struct {
   uint64_t launches[MOE_K_COUNT];/* launches per MOE_K_* */
 } moe_profile;
 
-/* Size in bytes of one expert (gate + up + down) in Q4_K.  0 on bad args. */
+/* Size in bytes of one expert (gate + up + down) in Q4_K.  0 on bad args.
+ * Source: LayerStoRm README, "Get a model" (GGUF Q4_K weights). */
 size_t moe_expert_bytes(int hidden, int inter, moe_quant quant);
 
 /* Create a layer on the current GPU.
@@ -108,17 +109,24 @@ size_t moe_expert_bytes(int hidden, int inter, moe_quant quant);
  * top_k: 1..min(32, E).  n_shared: S, 0..8 always-on experts (weight 1).
  * quant must be MOE_Q4_K.  *out receives the handle.
  * Errors: INVALID_ARG (shape out of range, out == NULL), UNSUPPORTED (quant),
- * CUDA/OOM (small device allocations). */
+ * CUDA/OOM (small device allocations).
+ * Source: LayerStoRm README, "References" (DeepSeek-V3 MoE: routed experts,
+ * top-k routing, always-on shared experts) and "Get a model" (Q4_K). */
 moe_status moe_layer_create(int hidden, int inter, int n_experts, int top_k,
                             int n_shared, moe_quant quant, moe_layer_t* out);
 
-/* Destroy a layer: waits for its outstanding work, frees its device memory and
- * drops its experts from the shared cache.  NULL is a no-op. */
+/* Destroy a layer: waits for the layer's outstanding work (its last forward
+ * and its internal copy stream), frees its device memory (cudaFree itself may
+ * wait for the GPU) and drops its experts from the shared cache.  NULL is a
+ * no-op.  No counterpart on the pages (resource management). */
 moe_status moe_layer_destroy(moe_layer_t layer);
 
 /* Router weights: W fp32 [E, H] row-major and bias fp32 [E] (NULL = zero),
  * host or device pointers; both are copied, so the caller keeps ownership.
- * The bias is added to the logits and used for both selection and weights. */
+ * The bias is added to the logits and used for both selection and weights.
+ * Source: LayerStoRm README, "TL;DR" (the router picks each token's few
+ * experts); the gating functions are the plainest readings of the pages'
+ * DeepSeek-V3 reference ("References"). */
 moe_status moe_set_router(moe_layer_t layer, const float* W, const float* bias,
                           moe_gating gating);
 
@@ -129,8 +137,12 @@ moe_status moe_set_router(moe_layer_t layer, const float* W, const float* bias,
  * copied, and cache misses are copied from it later.  In resident mode (see
  * moe_set_cache_bytes) every expert is uploaded to device memory here, and the
  * call returns when the upload is done.
+ * The call also scans every weight row's block scales once (host threads) to
+ * choose the power-of-two scale of the prefill path's fp16 dequantisation.
  * Errors: INVALID_ARG (NULL entry or a pointer that is not pinned host memory),
- * OOM (resident copy does not fit). */
+ * OOM (resident copy does not fit).
+ * Source: LayerStoRm README, "TL;DR" and "Requirements" (the whole expert set
+ * pinned in host RAM, the GPU holding what is needed). */
 moe_status moe_set_experts(moe_layer_t layer, const void* const* gate,
                            const void* const* up, const void* const* down);
 
@@ -141,7 +153,10 @@ moe_status moe_set_experts(moe_layer_t layer, const void* const* gate,
  * floor(bytes / slot_bytes) slots form an LRU cache in front of pinned host
  * RAM; misses are copied with cudaMemcpyAsync on an internal copy-engine
  * stream and compute waits on per-slot events.  Changing the budget empties
- * the streaming cache (it waits for the GPU first). */
+ * the streaming cache (it waits for the GPU first).
+ * Source: LayerStoRm README, "TL;DR" (GPU memory as a cache of experts,
+ * streamed in and overlapped with compute); rebasdaily LayerStoRm explainer
+ * (the host link as the final bottleneck). */
 moe_status moe_set_cache_bytes(size_t bytes);
 
 /* Forward: x bf16 [T, H] and out bf16 [T, H], device pointers, row-major.
@@ -149,22 +164,28 @@ moe_status moe_set_cache_bytes(size_t bytes);
  * expert kernels straight from the Q4_K bytes: byte dot products for T = 1,
  * the integer tensor MMA for 2..4), larger T the prefill path (router and the
  * projections of experts with more than 4 rows as tcgen05 grouped GEMMs; the
- * Q4_K weights are dequantised to fp16 in shared memory, which requires every
- * block's |d| < 0.248 and |dmin| < 3.72, i.e. weights within about +-234;
- * moe_check reports a violation; experts with at most 4 rows take the decode
- * kernels).  Work is enqueued on `stream`; in resident mode the call does not
- * wait for the GPU.  On the decode path the first kernel is launched as a
+ * Q4_K weights are dequantised to fp16 in shared memory under a power-of-two
+ * scale per weight row that moe_set_experts derives from the row's blocks, so
+ * any finite Q4_K block is in range; experts with at most 4 rows take the
+ * decode kernels).  Work is enqueued on `stream`; in resident mode the call does not
+ * wait for the GPU, except that the first forward at a T larger than any
+ * before on this layer allocates its per-call scratch, waiting for the
+ * layer's previous forward first.  On the decode path the first kernel is launched as a
  * programmatic dependent of the stream's previous work: it waits for that
  * work before it reads x or writes anything.
  * In streaming mode the call reads the routing back to the host (one stream
  * synchronisation) to resolve cache misses before the expert kernels are
- * launched.  out must not overlap x. */
+ * launched.  out must not overlap x.
+ * Source: LayerStoRm README, "TL;DR" (router, activated experts, combine) and
+ * "Notes" (a deterministic expert combine). */
 moe_status moe_forward(moe_layer_t layer, const void* x, void* out, int T, void* stream);
 
 /* Forward with the routing given: forced_ids int32 [T, top_k] on the HOST
  * (validated: every id in 0..E-1).  The gate weights are the gating function
  * of the router logits at these ids.  In streaming mode no synchronisation is
- * needed: the cache is resolved from the host ids before anything launches. */
+ * needed: the cache is resolved from the host ids before anything launches.
+ * No counterpart on the pages: a test and benchmark hook that replays a
+ * routing trace. */
 moe_status moe_forward_routed(moe_layer_t layer, const void* x, void* out, int T,
                               const int32_t* forced_ids, void* stream);
 
@@ -173,38 +194,47 @@ moe_status moe_forward_routed(moe_layer_t layer, const void* x, void* out, int T
  * (synchronise the stream before reading out).  With T <= 4 and pinned
  * buffers (16-byte aligned) the kernels read x and write out in host memory
  * in place; otherwise x and out are copied through device buffers (pinned
- * buffers make those copies asynchronous). */
+ * buffers make those copies asynchronous).  No counterpart on the pages: the
+ * end-to-end entry for callers that hold activations in host memory. */
 moe_status moe_forward_host(moe_layer_t layer, const void* x_host, void* out_host,
                             int T, void* stream);
 
 /* Routing of the last forward: ids int32 [T, top_k] and weights fp32
  * [T, top_k] (either may be NULL), copied on `stream` to device or host
- * memory.  ids[t] are ordered by decreasing logit. */
+ * memory.  ids[t] are ordered by decreasing logit.  No counterpart on the
+ * pages (inspection). */
 moe_status moe_get_routing(moe_layer_t layer, int32_t* ids, float* weights, void* stream);
 
-/* Router logits of the last forward, fp32 [T, E], copied on `stream`. */
+/* Router logits of the last forward, fp32 [T, E], copied on `stream`.  No
+ * counterpart on the pages (inspection). */
 moe_status moe_get_logits(moe_layer_t layer, float* logits, void* stream);
 
 /* Streaming mode: start fetching the given experts (host array of n ids in
  * 0..E+S-1) into the cache now, on the copy stream, so a later forward finds
- * them ready.  A no-op for resident layers and for experts already cached. */
+ * them ready.  A no-op for resident layers and for experts already cached.
+ * Source: LayerStoRm README, "Status and limitations" (predictive prefetch)
+ * and "References" (PreScope, SP-MoE: prefetching the next layer's experts). */
 moe_status moe_prefetch(moe_layer_t layer, const int32_t* ids, int n);
 
-/* Wait for all work on the layer's GPU, then report whether one of the layer's
- * kernels gave up on a bounded wait (a shared-memory pipeline barrier that did
- * not complete within its time limit; the kernel then stops early and its
- * output is invalid) or met a Q4_K block outside the fp16 range of the
- * prefill path.  Returns MOE_ERR_CUDA with a message in that case and clears
- * the record; MOE_OK otherwise. */
+/* Wait for the layer's own outstanding work (its last forward, on whatever
+ * stream it ran, and its internal copy stream; other work on the GPU is not
+ * waited for), then report whether one of the layer's kernels gave up on a
+ * bounded wait (a shared-memory pipeline barrier that did not complete
+ * within its time limit; the kernel then stops early and its output is
+ * invalid).  Returns MOE_ERR_CUDA with a message in that case and clears the
+ * record; MOE_OK otherwise.  No counterpart on the pages (failure detection). */
 moe_status moe_check(moe_layer_t layer);
 
+/* Counters of all layers (moe_stats), process-wide; reset keeps the cache
+ * geometry.  No counterpart on the pages (metrics). */
 moe_status moe_get_stats(moe_stats* out);
 moe_status moe_reset_stats(void);
 
 /* Profiling (global, off by default): when on, every forward records CUDA
  * events around each of its kernels.  moe_get_profile waits for the recorded
  * events, adds their times into *out and forgets them; moe_reset_profile
- * drops recorded events without waiting. */
+ * drops recorded events without waiting.  No counterpart on the pages
+ * (tracing). */
 moe_status moe_set_profiling(int enable);
 moe_status moe_get_profile(moe_profile* out);
 moe_status moe_reset_profile(void);

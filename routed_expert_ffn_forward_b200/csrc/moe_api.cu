@@ -16,6 +16,7 @@
 // fill of that slot waits on it before overwriting.
 #include <algorithm>
 #include <cstdarg>
+#include <thread>
 #include <cstdio>
 #include <cstring>
 #include <list>
@@ -148,6 +149,7 @@ struct moe_layer {
   CUtensorMap wp_map{};                 // over d_Wp, for the tensor-core router
   std::vector<const uint8_t*> host;     // (E+S)*3 borrowed pinned pointers
   uint8_t* d_resident = nullptr;        // resident copy of all experts
+  int8_t* d_wexp = nullptr;             // [E+S][2I + H] prefill weight-scale exponents per weight row
   CUtensorMap* d_tmaps = nullptr;       // [slots][kMapsPerSlot] TMA maps (resident: one slot per expert)
   size_t n_tmap_slots = 0;
   int* d_slot_of = nullptr;             // [E+S] expert -> slot of d_tmaps
@@ -160,6 +162,9 @@ struct moe_layer {
   __nv_bfloat16* xbuf = nullptr;
   __nv_bfloat16* obuf = nullptr;
   int32_t* h_ids = nullptr;             // pinned, for reading routing back
+  unsigned* h_err = nullptr;            // pinned word for reading the error flags back
+  cudaEvent_t done = nullptr;           // recorded on the stream at the end of every forward
+  bool done_rec = false;
   int last_T = 0;
   CUtensorMap x16_map{}, h16_map{};     // B operands of the prefill GEMMs (over the scratch)
 };
@@ -176,8 +181,19 @@ moe_status check_device(const moe_layer* L) {
 
 size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
 
+// Wait for the layer's own outstanding work: its last forward (on whatever
+// stream it ran) and its copy stream.  Other work on the device is not waited for.
+moe_status wait_layer(moe_layer* L) {
+  if (L->done && L->done_rec) CUDA_TRY(cudaEventSynchronize(L->done));
+  if (L->copy) CUDA_TRY(cudaStreamSynchronize(L->copy));
+  return MOE_OK;
+}
+
 // Grow the per-call scratch to hold T tokens (power of two, at least 64).
-moe_status ensure_scratch(moe_layer* L, int T) {
+// The old scratch may still be read by the layer's last forward, so that is
+// waited for before it is freed; the new one is zeroed on `st`, ahead of the
+// forward that needs it.
+moe_status ensure_scratch(moe_layer* L, int T, cudaStream_t st) {
   if (T <= L->T_cap) return MOE_OK;
   int cap = 64;
   while (cap < T) cap <<= 1;
@@ -199,7 +215,7 @@ moe_status ensure_scratch(moe_layer* L, int T) {
                o_x16 = take(P * s.H * 2), o_rinv = take(P * 4), o_h16 = take(P * s.I_pad * 2), o_hinv = take(P * 4),
                o_rpart = take(router_part_floats(cap, s.E, s.n_sm) * 4);
   if (L->scratch) {
-    CUDA_TRY(cudaDeviceSynchronize());
+    MOE_TRY(wait_layer(L));
     cudaFree(L->scratch);
     L->scratch = nullptr;
     L->T_cap = 0;
@@ -247,9 +263,11 @@ moe_status ensure_scratch(moe_layer* L, int T) {
   if (encode_act16(&L->x16_map, L->wk.x16, P, s.H) != cudaSuccess ||
       encode_act16(&L->h16_map, L->wk.h16, P, s.I_pad) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activation maps");
-  // zero everything once: the ticket must start at 0
-  CUDA_TRY(cudaMemset(L->scratch, 0, off));
-  CUDA_TRY(cudaDeviceSynchronize());
+  // zero everything once, ahead of the forward on its stream: the ticket
+  // and the error word must start at 0
+  CUDA_TRY(cudaMemsetAsync(L->scratch, 0, off, st));
+  CUDA_TRY(cudaEventRecord(L->done, st));
+  L->done_rec = true;
   L->T_cap = cap;
   return MOE_OK;
 }
@@ -433,7 +451,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
   if (T == 0) return MOE_OK;
   if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 15)
     return fail(MOE_ERR_INVALID_ARG, "x and out must be 16-byte aligned");
-  MOE_TRY(ensure_scratch(L, T));
+  MOE_TRY(ensure_scratch(L, T, st));
   const Work& wk = L->wk;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   // one kernel launch, optionally bracketed by profiling events
@@ -566,6 +584,9 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     ga.out = wk.h;
     ga.out_ld = s.I_pad;
     ga.out_rows = s.I;
+    ga.wexp = L->d_wexp;
+    ga.wexp_stride = 2 * s.I + s.H;
+    ga.wexp_down = 2 * s.I;
     ga.err = wk.err;
     MOE_KERNEL(MOE_K_GATE_UP, launch_prefill_gemm(0, L->x16_map, ga, s.n_sm, st));
     if (split_small) MOE_KERNEL(MOE_K_SMALL, launch_gate_up_d1(da, kD1MaxTok, s.n_sm, st));
@@ -581,6 +602,8 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true));
   }
 #undef MOE_KERNEL
+  CUDA_TRY(cudaEventRecord(L->done, st));
+  L->done_rec = true;
   {
     if (!lk.owns_lock()) lk.lock();
     if (prof) g_prof_pending.push_back(pr);
@@ -644,6 +667,8 @@ moe_status moe_layer_create(int hidden, int inter, int n_experts, int top_k, int
   if (e == cudaSuccess) e = cudaMalloc(&L->d_slot_of, sizeof(int) * (size_t)(s.E + s.S));
   if (e == cudaSuccess) e = cudaMemset(L->d_slot_of, 0, sizeof(int) * (size_t)(s.E + s.S));
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->copy, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->done, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaMallocHost(&L->h_err, sizeof(unsigned));
   if (e != cudaSuccess) {
     moe_layer_destroy(L);
     return fail(e == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA, "layer setup: %s",
@@ -660,7 +685,9 @@ moe_status moe_layer_create(int hidden, int inter, int n_experts, int top_k, int
 moe_status moe_layer_destroy(moe_layer_t L) {
   g_err.clear();
   if (!L) return MOE_OK;
-  cudaDeviceSynchronize();
+  // the layer's own work only; cudaFree below may still wait for the device
+  // as the CUDA runtime requires
+  if (wait_layer(L) != MOE_OK) (void)cudaGetLastError();
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (g_cache) {
@@ -677,10 +704,13 @@ moe_status moe_layer_destroy(moe_layer_t L) {
   if (L->d_b) cudaFree(L->d_b);
   if (L->d_Wp) cudaFree(L->d_Wp);
   if (L->d_resident) cudaFree(L->d_resident);
+  if (L->d_wexp) cudaFree(L->d_wexp);
   if (L->d_tmaps) cudaFree(L->d_tmaps);
   if (L->d_slot_of) cudaFree(L->d_slot_of);
   if (L->scratch) cudaFree(L->scratch);
   if (L->h_ids) cudaFreeHost(L->h_ids);
+  if (L->h_err) cudaFreeHost(L->h_err);
+  if (L->done) cudaEventDestroy(L->done);
   if (L->copy) cudaStreamDestroy(L->copy);
   delete L;
   return MOE_OK;
@@ -704,8 +734,8 @@ moe_status moe_set_router(moe_layer_t L, const float* W, const float* bias, moe_
   }
   // bf16 planes of W for the tensor-core router (T > 4)
   if (!L->d_Wp) CUDA_TRY(cudaMalloc(&L->d_Wp, 3 * (size_t)L->s.E * L->s.H * sizeof(__nv_bfloat16)));
-  CUDA_TRY(launch_split_router(L->d_W, L->s.E, L->s.H, L->d_Wp, nullptr));
-  CUDA_TRY(cudaDeviceSynchronize());
+  CUDA_TRY(launch_split_router(L->d_W, L->s.E, L->s.H, L->d_Wp, L->copy));
+  CUDA_TRY(cudaStreamSynchronize(L->copy));
   if (encode_sw128_16(&L->wp_map, L->d_Wp, true, 3 * (size_t)L->s.E, L->s.H, 128) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the router planes");
   L->gating = gating;
@@ -733,6 +763,26 @@ moe_status moe_set_experts(moe_layer_t L, const void* const* gate, const void* c
       host[3 * (size_t)e + m] = static_cast<const uint8_t*>(p[m]);
     }
   }
+  // power-of-two scales of the prefill GEMMs' fp16 weights, one per weight
+  // row, from the host bytes (several threads: a layer is gigabytes)
+  const int stride = 2 * L->s.I + L->s.H;
+  std::vector<int8_t> wexp((size_t)n * stride);
+  {
+    const int nth = (int)std::max(1u, std::min(16u, std::thread::hardware_concurrency()));
+    std::vector<std::thread> pool;
+    for (int t = 0; t < nth; ++t)
+      pool.emplace_back([&, t] {
+        for (int e = t; e < n; e += nth) {
+          int8_t* o = wexp.data() + (size_t)e * stride;
+          q4k_row_exponents(host[3 * (size_t)e], L->s.I, L->s.nbh, o);
+          q4k_row_exponents(host[3 * (size_t)e + 1], L->s.I, L->s.nbh, o + L->s.I);
+          q4k_row_exponents(host[3 * (size_t)e + 2], L->s.H, L->s.nbi, o + 2 * L->s.I);
+        }
+      });
+    for (auto& th : pool) th.join();
+  }
+  if (!L->d_wexp) CUDA_TRY(cudaMalloc(&L->d_wexp, wexp.size()));
+  CUDA_TRY(cudaMemcpy(L->d_wexp, wexp.data(), wexp.size(), cudaMemcpyHostToDevice));
   size_t budget;
   {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -818,8 +868,8 @@ moe_status moe_forward_host(moe_layer_t L, const void* x_host, void* out_host, i
   if (T == 0) return MOE_OK;
   if (!x_host || !out_host) return fail(MOE_ERR_INVALID_ARG, "null x or out");
   MOE_TRY(check_device(L));
-  MOE_TRY(ensure_scratch(L, T));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_TRY(ensure_scratch(L, T, st));
   const size_t bytes = (size_t)T * L->s.H * 2;
   // Decode path with pinned (mapped) host buffers: the kernels read x from
   // and write out to host memory in place -- x by a staging kernel that the
@@ -882,17 +932,15 @@ moe_status moe_check(moe_layer_t L) {
   g_err.clear();
   if (!L) return fail(MOE_ERR_INVALID_ARG, "null layer");
   MOE_TRY(check_device(L));
-  CUDA_TRY(cudaDeviceSynchronize());
+  MOE_TRY(wait_layer(L));
   if (!L->scratch) return MOE_OK;
-  unsigned flags = 0;
-  CUDA_TRY(cudaMemcpy(&flags, L->wk.err, sizeof flags, cudaMemcpyDeviceToHost));
+  CUDA_TRY(cudaMemcpyAsync(L->h_err, L->wk.err, sizeof(unsigned), cudaMemcpyDeviceToHost, L->copy));
+  CUDA_TRY(cudaStreamSynchronize(L->copy));
+  const unsigned flags = *L->h_err;
   if (flags) {
-    CUDA_TRY(cudaMemset(L->wk.err, 0, sizeof flags));
-    return fail(MOE_ERR_CUDA,
-                "%s (flags 0x%x)",
-                (flags & 0xFFu) || (flags & ~0x1FFu) ? "a kernel of this layer gave up waiting"
-                                                      : "a Q4_K weight exceeds the fp16 range of the prefill GEMMs",
-                flags);
+    CUDA_TRY(cudaMemsetAsync(L->wk.err, 0, sizeof(unsigned), L->copy));
+    CUDA_TRY(cudaStreamSynchronize(L->copy));
+    return fail(MOE_ERR_CUDA, "a kernel of this layer gave up waiting (flags 0x%x)", flags);
   }
   return MOE_OK;
 }

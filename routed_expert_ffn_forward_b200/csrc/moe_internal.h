@@ -156,6 +156,11 @@ struct GemmArgs {
   const float* rinv;         // [P] inverse activation scale of each row
   float* out;                // h [P, I_pad] or y [P, H]
   int out_ld, out_rows;      // row pitch (floats); features stored (mode 0: I)
+  // per expert, per weight row: the exponent k of the 2^k scale applied to
+  // the dequantised fp16 weights (gate rows [0, I), up rows [I, 2I), down
+  // rows [2I, 2I + H)); wexp_stride = 2I + H, wexp_down = 2I
+  const int8_t* wexp;
+  int wexp_stride, wexp_down;
   unsigned* err;
 };
 size_t prefill_gemm_smem();
@@ -199,6 +204,12 @@ struct SlotUpdate {
   int slot[kMax];
 };
 cudaError_t launch_set_slots(int* slot_of, const SlotUpdate& u, cudaStream_t st);
+
+// Exponents k (<= 8) of the power-of-two weight scales of the prefill GEMMs,
+// one per weight row of one Q4_K matrix of `rows` rows x `nb` super-blocks:
+// the largest k with 2^k * max over the row's blocks of (|d|*945 + |dmin|*63)
+// below 60000, so that no fp16 intermediate of the dequantisation overflows.
+void q4k_row_exponents(const uint8_t* q4k, int rows, int nb, int8_t* out);
 
 // Set / clear the thread-local message returned by moe_last_error().
 int report_error(int status, const char* msg);

@@ -26,9 +26,10 @@
 //
 // Numerics: activations are fp16 scaled per row by a power of two (largest
 // magnitude in [2^14, 2^15), 1/scale kept in `rinv`); weights are fp16 scaled
-// by 2^8 (sub-block scale and min rounded to fp16, one rounding per weight);
-// products accumulate in fp32 and the epilogue undoes both scales.  A weight
-// that would not fit fp16 after the 2^8 scale sets error bit 256.
+// per weight row by 2^k (sub-block scale and min rounded to fp16, one rounding
+// per weight), k <= 8 chosen on the host from the row's blocks so that every
+// intermediate stays below 60000 (`wexp`); products accumulate in fp32 and the
+// epilogue undoes both scales exactly (powers of two).
 //
 // K order: within every group of four K elements both operands are stored in
 // the order (0, 2, 1, 3), so two quant nibbles of one 32-bit word become one
@@ -50,8 +51,6 @@ constexpr int kDeqWarps = 8;
 constexpr int kEpiWarps = 8;
 constexpr int kFirstDeq = 3, kFirstEpi = kFirstDeq + kDeqWarps;
 constexpr int kGemmThreads = (kFirstEpi + kEpiWarps) * 32;  // 608
-constexpr float kWScale = 256.f, kWScaleInv = 1.f / 256.f;
-constexpr float kWMax = 60000.f;               // largest |weight| * 2^8 accepted
 
 constexpr size_t kSmemRaw = (size_t)kNR * 2 * kRawBytes;
 constexpr size_t kSmemA = (size_t)kNS * 2 * kABytes;
@@ -60,12 +59,12 @@ constexpr size_t kSmemBar = 8 * (2 * kNR + 3 * kNS + 2 + 1) + 16;
 constexpr size_t kGemmSmem = 1024 + kSmemRaw + kSmemA + kSmemB + kSmemBar;
 static_assert(kGemmSmem <= 227 * 1024, "GEMM shared memory");
 
-// fp16x2 scale pair (s_lo, s_hi) = 2^8 * d * (sc_2c, sc_2c+1) and min pair
-// (nm_lo, nm_hi) = -2^8 * dmin * (m_2c, m_2c+1) of chunk c of a Q4_K block
+// fp16x2 scale pair (s_lo, s_hi) = 2^k * d * (sc_2c, sc_2c+1) and min pair
+// (nm_lo, nm_hi) = -2^k * dmin * (m_2c, m_2c+1) of chunk c of a Q4_K block
 // whose first 16 bytes are `hdr` (fp16 d, fp16 dmin, 12 scale bytes).  All
 // in fp16 arithmetic: the 6-bit fields become fp16 integers through the 1024
 // exponent trick, and d * sc rounds once, as a float product converted to
-// fp16 would.  `d2s`/`nm2s` are (2^8 d, 2^8 d) and (-2^8 dmin, -2^8 dmin).
+// fp16 would.  `d2s`/`nm2s` are (2^k d, 2^k d) and (-2^k dmin, -2^k dmin).
 __device__ __forceinline__ void chunk_scales(uint4 hdr, int c, __half2 d2s, __half2 nm2s, __half2& s2, __half2& nm2) {
   const uint32_t sh = 16u * (uint32_t)(c & 1);
   const uint32_t s0 = hdr.y >> sh, s1 = hdr.z >> sh, s2w = hdr.w >> sh;
@@ -91,6 +90,15 @@ __device__ __forceinline__ uint32_t deq2(uint32_t t, __half2 off, __half2 s, __h
   const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&t), off);
   const __half2 v = __hfma2(q, s, nm);
   return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// 2^e as a float, exactly, for -126 <= e <= 127
+__device__ __forceinline__ float pow2f(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
+// 2^e as an fp16 pair, exactly, for -14 <= e <= 15
+__device__ __forceinline__ __half2 pow2h2(int e) {
+  const uint32_t b = (uint32_t)(15 + e) << 10;
+  const uint32_t v = b | (b << 16);
+  return *reinterpret_cast<const __half2*>(&v);
 }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* raw) {
@@ -120,10 +128,22 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmArgs& a, uint32_t tmem, 
   ptx::tc_fence_after();
   const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
   const int pair0 = tl.w + tl.y;
+  // 2^-k of the weight rows this thread's accumulator lanes belong to
+  const int8_t* wx = a.wexp + (size_t)tl.x * a.wexp_stride;
+  float s0, s1;
+  if (kMode == 0) {
+    const int feat = min(f * kGM + mrow, a.out_rows - 1);
+    s0 = pow2f(-__ldg(wx + feat));
+    s1 = pow2f(-__ldg(wx + a.out_rows + feat));
+  } else {
+    const int orow = f * 2 * kGM + mrow;
+    s0 = pow2f(-__ldg(wx + a.wexp_down + orow));
+    s1 = pow2f(-__ldg(wx + a.wexp_down + orow + kGM));
+  }
   for (int c0 = 32 * sub; c0 < tl.z; c0 += 32 * (kEpiWarps / 4)) {
     const int nc = min(32, tl.z - c0);
     // lane i holds the inverse scale of column c0 + i
-    const float my_inv = __ldg(a.rinv + pair0 + c0 + min(lane, nc - 1)) * kWScaleInv;
+    const float my_inv = __ldg(a.rinv + pair0 + c0 + min(lane, nc - 1));
     uint32_t r0[32], r1[32];
     ptx::tmem_ld32x2(tq + c0, tq + kGN + c0, r0, r1);
     if (kMode == 0) {
@@ -133,7 +153,7 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmArgs& a, uint32_t tmem, 
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float inv = __shfl_sync(0xffffffffu, my_inv, i);
-        const float g = __uint_as_float(r0[i]) * inv, up = __uint_as_float(r1[i]) * inv;
+        const float g = __uint_as_float(r0[i]) * (inv * s0), up = __uint_as_float(r1[i]) * (inv * s1);
         const float hv = __fdividef(g, 1.f + __expf(-g)) * up;   // silu(g) * up
         if (i < nc && frow) outp[(size_t)i * a.out_ld] = hv;
       }
@@ -144,8 +164,8 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmArgs& a, uint32_t tmem, 
       for (int i = 0; i < 32; ++i) {
         const float inv = __shfl_sync(0xffffffffu, my_inv, i);
         if (i < nc) {
-          outp[(size_t)i * a.out_ld] = __uint_as_float(r0[i]) * inv;
-          outp[(size_t)i * a.out_ld + kGM] = __uint_as_float(r1[i]) * inv;
+          outp[(size_t)i * a.out_ld] = __uint_as_float(r0[i]) * (inv * s0);
+          outp[(size_t)i * a.out_ld + kGM] = __uint_as_float(r1[i]) * (inv * s1);
         }
       }
     }
@@ -305,11 +325,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
     const int r = ((warp - kFirstDeq) & 3) * 32 + lane;       // weight row of the half, 0..127
     const uint32_t sw = (uint32_t)((r >> 1) & 3);             // 64B swizzle of row r
     const __half2 off_lo = __float2half2_rn(1024.f), off_hi = __float2half2_rn(64.f);
-    const __half2 kWScale2 = __float2half2_rn(kWScale), kNegWScale2 = __float2half2_rn(-kWScale);
+    const __half2 kNeg2 = __float2half2_rn(-1.f);
     int rs = 0, as = 0;
     uint32_t rph = 0, aph = 0;
-    bool bad = false;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      // this thread's weight row and its power-of-two scale 2^k
+      const int ex = __ldcg(a.tiles + u / a.ft).x, f = u % a.ft;
+      const int8_t* wx = a.wexp + (size_t)ex * a.wexp_stride;
+      const int wrow = kMode == 0 ? min(f * kGM + r, a.out_rows - 1) + m * a.out_rows
+                                  : a.wexp_down + f * 2 * kGM + m * kGM + r;
+      const __half2 wsc2 = pow2h2(__ldg(wx + wrow));
+      const __half2 nwsc2 = __hmul2(wsc2, kNeg2);
       for (int kb = 0; kb < a.nkb; ++kb) {
         if (!ptx::mbar_wait(&raw_full[rs], rph)) {
           atomicOr(a.err, 64u);
@@ -317,13 +343,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
         }
         const uint8_t* row = s_rawbuf + (2 * rs + m) * kRawBytes + r * kQBytes;
         const uint4 hdr = *reinterpret_cast<const uint4*>(row);
-        // (d, d) and (dmin, dmin) scaled by 2^8 (exact); a block whose d or dmin could
-        // take a weight past kWMax (with the largest 6-bit scale) is flagged
+        // (d, d) and (dmin, dmin) scaled by the row's 2^k (exact)
         const uint32_t dd = __byte_perm(hdr.x, 0u, 0x1010u), mm = __byte_perm(hdr.x, 0u, 0x3232u);
         const __half2 d2 = *reinterpret_cast<const __half2*>(&dd), dm2 = *reinterpret_cast<const __half2*>(&mm);
-        bad |= !(__hlt(__habs(__low2half(d2)), __float2half_rn(kWMax / (kWScale * 63.f * 15.f))) &&
-                 __hlt(__habs(__low2half(dm2)), __float2half_rn(kWMax / (kWScale * 63.f))));
-        const __half2 d2s = __hmul2(d2, kWScale2), nm2s = __hmul2(dm2, kNegWScale2);
+        const __half2 d2s = __hmul2(d2, wsc2), nm2s = __hmul2(dm2, nwsc2);
         for (int c = 0; c < 4; ++c) {
           // chunk c: 32 quant bytes; low nibbles are sub-block 2c, high nibbles 2c+1
           const uint4 qa = *reinterpret_cast<const uint4*>(row + 16 + 32 * c);
@@ -365,7 +388,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
         if (++rs == kNR) { rs = 0; rph ^= 1u; }
       }
     }
-    if (bad) atomicOr(a.err, 256u);
   } else {
     // ------------------------------------------------------------ epilogue
     uint32_t fph = 0;
