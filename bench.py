@@ -147,25 +147,61 @@ def flops(cfg, T: int) -> float:
 
 
 # ----------------------------------------------------------------------------- CPU oracle baseline
-def oracle_sample_rate(cfg, n_tokens: int, budget_s: float) -> dict:
-    """Time the oracle (as it stands) on a bounded sample: whole tokens of the
-    workload, one after another, until the budget is used (at least one)."""
+def _oracle_tokens(cfg, first: int, n_tokens: int, budget_s: float):
+    """Whole tokens of the workload through the oracle (as it stands), one
+    after another from token `first`, until the budget is used (at least
+    one), BLAS limited to one thread.  Returns (tokens, seconds)."""
     from threadpoolctl import threadpool_limits
 
     from oracle import moe_ref as ref
     layer = dict(router_w=synth.router_weight(cfg), router_b=synth.router_bias(cfg),
                  experts=lambda e: synth.expert_tensors(cfg, 0, e))
-    x = synth.activations(cfg, tokens=max(n_tokens, 1))
+    x = synth.activations(cfg, tokens=first + n_tokens)
     done, t0 = 0, time.perf_counter()
     with threadpool_limits(limits=1):
         while done < n_tokens and (done == 0 or time.perf_counter() - t0 < budget_s):
-            ref.moe_forward(x[done:done + 1], layer, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter)
+            t = first + done
+            ref.moe_forward(x[t:t + 1], layer, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter)
             done += 1
-    dt = time.perf_counter() - t0
+    return done, time.perf_counter() - t0
+
+
+def _oracle_worker(job):
+    cfg_index, first, n_tokens, budget_s = job
+    return _oracle_tokens(synth.WORKLOADS[cfg_index], first, n_tokens, budget_s)
+
+
+def oracle_sample_rate(cfg_index: int, n_tokens: int, budget_s: float) -> dict:
+    """The oracle on one host core: whole tokens, one after another."""
+    cfg = synth.WORKLOADS[cfg_index]
+    done, dt = _oracle_tokens(cfg, 0, n_tokens, budget_s)
     return {"value": done / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{done} token(s) of the workload's layer through the fp64 numpy oracle "
                       f"(full routing + {cfg.top_k}+{cfg.n_shared} experts each), BLAS limited to 1 thread",
             "seconds": dt}
+
+
+def oracle_all_cores(cfg_index: int, budget_s: float, max_workers: int = 16) -> dict:
+    """The oracle on the host's cores: one spawned process per core (at most
+    `max_workers`: each holds ~1 GB of fp64 weights), each running whole
+    tokens of its own with BLAS limited to one thread, for about `budget_s`.
+    value = all workers' tokens / the longest worker's time."""
+    import multiprocessing as mp
+    cfg = synth.WORKLOADS[cfg_index]
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    workers = max(1, min(cores, max_workers))
+    jobs = [(cfg_index, 64 * w, 64, budget_s) for w in range(workers)]
+    t0 = time.perf_counter()
+    with mp.get_context("spawn").Pool(workers) as pool:
+        res = pool.map(_oracle_worker, jobs)
+    wall = time.perf_counter() - t0
+    tokens = sum(r[0] for r in res)
+    secs = max(r[1] for r in res)
+    return {"value": tokens / secs, "unit": "tokens/s", "cores": workers, "kind": "oracle",
+            "sample": f"{tokens} tokens of the workload's layer through the fp64 numpy oracle on {workers} "
+                      f"processes (one per core, {cores} cores available, BLAS 1 thread each), "
+                      f"~{budget_s:.0f} s each",
+            "seconds": secs, "wall_s": wall}
 
 
 _EXPERT_CACHE: dict = {}
@@ -240,23 +276,25 @@ def config_json(cfg, args) -> dict:
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def run_ours(args, cfg, rank: int, world: int, local_rank: int) -> dict | None:
+DTYPE_DECODE = "q4_k x fx16 -> i32"      # exact Q4_K weights, 16-bit fixed-point activations, int32 sums
+DTYPE_PREFILL = "q4_k->f16 x f16 -> f32"  # Q4_K dequantised to fp16 (power-of-two scaled), fp32 accumulate
+
+
+def measure_resident(args, cfg, rank, world, local_rank, peaks, steps, warmup, e2e=True) -> dict:
+    """Time `steps` forwards of one resident layer of `cfg` (after `warmup`),
+    L2 flushed before each, CUDA events on the forward's stream; then the same
+    steps again with per-kernel profiling events, and optionally the
+    end-to-end host-buffer path."""
     import torch
 
-    from routed_expert_ffn_forward_b200 import build, moe
+    from routed_expert_ffn_forward_b200 import moe
     from routed_expert_ffn_forward_b200.layer import layer_from_config
-
-    build.build()
-    torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
-    peaks = measured_peaks()
-    if args.config == 4:
-        return run_streaming(args, cfg, rank, world, local_rank, peaks)
     moe.moe_set_cache_bytes(moe.SIZE_MAX)
     t0 = time.time()
     L = layer_from_config(cfg)
-    log(f"[rank {rank}] layer ready in {time.time() - t0:.1f}s")
+    log(f"[rank {rank}] layer '{cfg.name}' ready in {time.time() - t0:.1f}s")
     T = cfg.tokens
     n_pool = 16 if T > 1 else 64
     xs = [synth.activations(cfg, 0, i, tokens=T) for i in range(n_pool)]
@@ -277,15 +315,15 @@ def run_ours(args, cfg, rank: int, world: int, local_rank: int) -> dict | None:
         L.forward(x_dev[i % n_pool], out, stream.cuda_stream)
         e.record(stream)
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         step(i, (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     st0 = moe.moe_get_stats()
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local_rank, args.clocks_dir) as clk:
-        for i in range(args.steps):
+        for i in range(steps):
             step(i, evs[i])
         torch.cuda.synchronize()
     barrier(world)
@@ -300,71 +338,116 @@ def run_ours(args, cfg, rank: int, world: int, local_rank: int) -> dict | None:
     # one whose time is reported as `value`.)
     moe.moe_reset_profile()
     moe.moe_set_profiling(True)
-    for i in range(args.steps):
+    for i in range(steps):
         step(i, (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
     torch.cuda.synchronize()
     moe.moe_set_profiling(False)
     prof = moe.moe_get_profile()
 
-    # e2e: the same forward through moe_forward_host, host buffers in and out
-    xh = torch.from_numpy(np.stack(xs).view(np.int16)).view(torch.bfloat16).pin_memory()
-    oh = torch.empty((T, cfg.hidden), dtype=torch.bfloat16).pin_memory()
-    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(min(args.warmup, 3)):
-        moe.moe_forward_host(L.handle, xh[i].data_ptr(), oh.data_ptr(), T, stream.cuda_stream)
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()
-        s, e = e2e_evs[i]
-        s.record(stream)
-        moe.moe_forward_host(L.handle, xh[i % n_pool].data_ptr(), oh.data_ptr(), T, stream.cuda_stream)
-        e.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(float(np.sum([s.elapsed_time(e) for s, e in e2e_evs])), world, dev)
+    e2e_res = None
+    if e2e:
+        # the same forward through moe_forward_host, host buffers in and out
+        xh = torch.from_numpy(np.stack(xs).view(np.int16)).view(torch.bfloat16).pin_memory()
+        oh = torch.empty((T, cfg.hidden), dtype=torch.bfloat16).pin_memory()
+        e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)]
+        for i in range(min(warmup, 3)):
+            moe.moe_forward_host(L.handle, xh[i].data_ptr(), oh.data_ptr(), T, stream.cuda_stream)
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.zero_()
+            s, e = e2e_evs[i]
+            s.record(stream)
+            moe.moe_forward_host(L.handle, xh[i % n_pool].data_ptr(), oh.data_ptr(), T, stream.cuda_stream)
+            e.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(float(np.sum([s.elapsed_time(e) for s, e in e2e_evs])), world, dev)
+        e2e_res = {"value": T * steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": T * cfg.hidden * 2, "d2h_bytes_per_step": T * cfg.hidden * 2,
+                   "api": "moe_forward_host (pinned host x and out)"}
     L.destroy()
+    L.host = None
+    del flush, x_dev
 
-    tokens_total = T * args.steps * world
-    value = tokens_total / (total_ms / 1e3)
-    # roofline of the dominant kernel
-    ids_cycle = [ids_pool[i % n_pool] for i in range(args.steps)]
-    if args.config == 3:
-        kern = "gate_up"
-        fl = np.mean([flops(cfg, T) * 2 / 3 for _ in ids_cycle])
-        avg_ms = prof["ms"][kern] / max(1, prof["launches"][kern])
+    ids_cycle = [ids_pool[i % n_pool] for i in range(steps)]
+    fwd_ms = total_ms / steps
+    kern = "gate_up"
+    avg_ms = prof["ms"][kern] / max(1, prof["launches"][kern])
+    if T > 4:
+        # the gate/up GEMM runs the experts with more than 4 rows (plus the shared one)
+        fl = float(np.mean([gate_up_gemm_flops(cfg, ids) for ids in ids_cycle]))
         achieved = fl / (avg_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops"]
+        peak = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
         roof = {"bound": "tensor", "kernel": kern, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": kernel_traffic(f"config{args.config}:{kern}"), "peak_source": peaks["source"]}
+                "frac": achieved / peak, "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+                "flops_per_launch": fl, "traffic": kernel_traffic(f"config{cfg_index(cfg)}:{kern}"),
+                "peak_source": peaks["source"] + " (sustained bf16; fp16 has the same nominal rate)"}
     else:
-        kern = "gate_up"
         ab = float(np.mean([algorithmic_bytes(cfg, ids, kern) for ids in ids_cycle]))
-        avg_ms = prof["ms"][kern] / max(1, prof["launches"][kern])
         achieved = ab / (avg_ms / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": kernel_traffic(f"config{args.config}:{kern}"), "algorithmic_bytes": ab,
-                "peak_source": peaks["source"]}
+                "frac": achieved / peak, "traffic": kernel_traffic(f"config{cfg_index(cfg)}:{kern}"),
+                "algorithmic_bytes": ab, "peak_source": peaks["source"]}
     fwd_bytes = float(np.mean([algorithmic_bytes(cfg, ids, "forward") for ids in ids_cycle]))
-    fwd_ms = total_ms / args.steps
     kernels = {k: {"avg_us": 1e3 * prof["ms"][k] / max(1, prof["launches"][k]),
                    "share": prof["ms"][k] / max(1e-12, sum(prof["ms"][q] for q in moe.KERNELS[:-1]))}
-               for k in moe.KERNELS[:-1]}
-    if args.config == 3:
-        metric, unit = "moe_layer_prefill_tokens_per_s", "tokens/s"
-    else:
-        metric, unit = "moe_layer_decode_tokens_per_s", "tokens/s"
-    res = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": fwd_ms, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "int8" if cfg.tokens <= 4 else "f16", "data": "synthetic",
-           "config": config_json(cfg, args), "roofline": roof,
-           "forward_hbm": {"algorithmic_bytes": fwd_bytes, "achieved_gbs": fwd_bytes / (fwd_ms / 1e3) / 1e9,
-                           "frac": fwd_bytes / (fwd_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
-           "prefill_tflops": flops(cfg, T) / (fwd_ms / 1e3) / 1e12 if args.config == 3 else None,
-           "kernels": kernels,
-           "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
-                   "h2d_bytes_per_step": T * cfg.hidden * 2, "d2h_bytes_per_step": T * cfg.hidden * 2,
-                   "api": "moe_forward_host (pinned host x and out)"},
-           "gpu_launches": launches, "clocks": clk.summary()}
+               for k in moe.KERNELS[:-1] if prof["launches"][k]}
+    return {"value": T * steps * world / (total_ms / 1e3), "ms_per_step": fwd_ms, "roofline": roof,
+            "forward_hbm": {"algorithmic_bytes": fwd_bytes, "achieved_gbs": fwd_bytes / (fwd_ms / 1e3) / 1e9,
+                            "frac": fwd_bytes / (fwd_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+            "tflops": flops(cfg, T) / (fwd_ms / 1e3) / 1e12, "kernels": kernels, "e2e": e2e_res,
+            "gpu_launches": launches, "clocks": clk.summary(),
+            "dtype": DTYPE_DECODE if T <= 4 else DTYPE_PREFILL}
+
+
+def gate_up_gemm_flops(cfg, ids: np.ndarray) -> float:
+    """FLOPs of the prefill gate/up GEMM for this routing: 2 * rows * 2I * H
+    over the experts with more than 4 rows, plus the shared experts."""
+    T = ids.shape[0]
+    counts = np.bincount(ids.ravel(), minlength=cfg.n_experts)
+    rows = int(counts[counts > 4].sum()) + T * cfg.n_shared
+    return 2.0 * rows * 2 * cfg.inter * cfg.hidden
+
+
+def cfg_index(cfg) -> int:
+    for k, v in synth.WORKLOADS.items():
+        if v.name == cfg.name:
+            return k
+    return -1
+
+
+def run_ours(args, cfg, rank: int, world: int, local_rank: int) -> dict | None:
+    import torch
+
+    from routed_expert_ffn_forward_b200 import build
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    peaks = measured_peaks()
+    if args.config == 4:
+        return run_streaming(args, cfg, rank, world, local_rank, peaks)
+    m = measure_resident(args, cfg, rank, world, local_rank, peaks, args.steps, args.warmup)
+    T = cfg.tokens
+    metric = "moe_layer_prefill_tokens_per_s" if args.config == 3 else "moe_layer_decode_tokens_per_s"
+    res = {"metric": metric, "value": m["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": m["dtype"], "data": "synthetic", "config": config_json(cfg, args),
+           "roofline": m["roofline"], "forward_hbm": m["forward_hbm"],
+           "prefill_tflops": m["tflops"] if T > 4 else None, "kernels": m["kernels"], "e2e": m["e2e"],
+           "gpu_launches": m["gpu_launches"], "clocks": m["clocks"]}
+    if args.config == 1 and not args.no_extra and not args.small:
+        # the batched-decode and prefill workloads of the same layer shape, one
+        # resident layer at a time, same steps and warm-up
+        for key, idx in (("batched", 2), ("prefill", 3)):
+            c = synth.WORKLOADS[idx]
+            x = measure_resident(args, c, rank, world, local_rank, peaks, args.steps, args.warmup, e2e=False)
+            res[key] = {"workload": c.name, "tokens": c.tokens, "tokens_per_s": x["value"],
+                        "ms_per_step": x["ms_per_step"], "tflops": x["tflops"], "forward_hbm": x["forward_hbm"],
+                        "roofline": x["roofline"], "kernels": x["kernels"], "gpu_launches": x["gpu_launches"],
+                        "clocks": x["clocks"], "dtype": x["dtype"]}
+        res["prefill_tflops"] = res["prefill"]["tflops"]
+        res["gpu_launches"] += res["batched"]["gpu_launches"] + res["prefill"]["gpu_launches"]
     return res
 
 
@@ -421,7 +504,7 @@ def run_streaming(args, cfg, rank, world, local_rank, peaks) -> dict:
     lookups = st["cache_hits"] + st["cache_misses"]
     return {"metric": "moe_streaming_decode_tokens_per_s", "value": args.steps * world / secs, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE_DECODE, "data": "synthetic",
             "config": config_json(cfg, args),
             "roofline": {"bound": "h2d", "achieved": h2d_gbs, "peak": h2d_peak, "unit": "GB/s",
                          "frac": h2d_gbs / h2d_peak, "traffic": None,
@@ -478,6 +561,8 @@ def main():
     ap.add_argument("--clocks-dir", default=tempfile.gettempdir(),
                     help="where the raw nvidia-smi samples of the timed region are written")
     ap.add_argument("--no-prefetch", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="config 1 only: skip the batched-decode and prefill lines added to the JSON")
     ap.add_argument("--small", action="store_true",
                     help="32 routed experts instead of 256 (same per-launch work at T=1; for ncu captures)")
     args = ap.parse_args()
@@ -500,11 +585,16 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
     res = run_ours(args, cfg, rank, world, local_rank)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config in (1, 2):
-        res["cpu_baseline"] = oracle_sample_rate(cfg, n_tokens=cfg.tokens, budget_s=20.0)
-    elif rank == 0 and not args.no_cpu_baseline and world == 1:
-        res["cpu_baseline"] = oracle_sample_rate(synth.DECODE, n_tokens=3, budget_s=20.0) | {
-            "sample": "decode tokens of the config-1 layer (the oracle's cost per token is the same per expert)"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the oracle on this host's cores (one process per core), with the
+        # one-core figure beside it; configs 3 and 4 take config-1 tokens (the
+        # oracle's cost per token is the same per expert)
+        idx = args.config if args.config in (1, 2) else 1
+        res["cpu_baseline"] = oracle_all_cores(idx, budget_s=15.0)
+        res["cpu_baseline_1core"] = oracle_sample_rate(idx, n_tokens=3, budget_s=10.0)
+        if idx != args.config:
+            for k in ("cpu_baseline", "cpu_baseline_1core"):
+                res[k]["sample"] += "; decode tokens of the config-1 layer (same per-expert cost)"
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

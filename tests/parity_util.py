@@ -56,3 +56,35 @@ def check_outputs(out_bits: np.ndarray, ref_bits: np.ndarray, what: str = ""):
     assert max_rel <= MAX_REL, f"{what}: max|err|/max|ref| = {max_rel:.3e}"
     assert mean_rel <= MEAN_REL, f"{what}: sum|err|/sum|ref| = {mean_rel:.3e}"
     return max_rel, mean_rel
+
+
+# ------------------------------------------------------------------ oracle rows in parallel
+def _oracle_rows_job(job):
+    cfg, layer_index, x_bits, forced, tokens = job
+    from threadpoolctl import threadpool_limits
+
+    from routed_expert_ffn_forward_b200 import synth
+    layer = dict(router_w=synth.router_weight(cfg, layer_index), router_b=synth.router_bias(cfg, layer_index),
+                 experts=lambda e: synth.expert_tensors(cfg, layer_index, e))
+    with threadpool_limits(limits=1):      # one core per process
+        r = ref.moe_forward(x_bits, layer, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter, forced_ids=forced,
+                            token_subset=tokens)
+    return r["out_bf16"]
+
+
+def oracle_rows(cfg, layer_index, x_bits, forced, tokens, workers=None):
+    """The oracle's bf16 output rows for `tokens` (forced routing), computed by
+    up to `workers` spawned processes, each over a share of the tokens (the
+    oracle itself is unchanged; this only runs several of it at once)."""
+    import multiprocessing as mp
+    import os
+    tokens = np.asarray(tokens)
+    if workers is None:
+        cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+        workers = max(1, min(16, cores, len(tokens)))
+    chunks = [c for c in np.array_split(tokens, workers) if len(c)]
+    if len(chunks) == 1:
+        return _oracle_rows_job((cfg, layer_index, x_bits, forced, chunks[0]))
+    with mp.get_context("spawn").Pool(len(chunks)) as pool:
+        parts = pool.map(_oracle_rows_job, [(cfg, layer_index, x_bits, forced, c) for c in chunks])
+    return np.concatenate(parts, axis=0)

@@ -70,3 +70,19 @@ def test_traffic_entry_tracks_its_source():
         got = bench.kernel_traffic(key)
         assert (got == float(d["bytes_per_launch"])) if current else got is None
     assert bench.kernel_traffic("config9:nothing") is None
+
+
+def test_gate_up_gemm_flops_hand_count():
+    cfg = dataclasses.replace(synth.DECODE, tokens=6)
+    # expert 0: 6 rows (GEMM), expert 1: 5 rows (GEMM), experts 2..: 1 row each (decode kernels)
+    ids = np.array([[0, 1] + [10 * j + t for j in range(1, 7)] for t in range(6)], dtype=np.int32)
+    ids[5, 1] = 99                          # expert 1 keeps 5 rows
+    rows = 6 + 5 + 6 * 1                    # the two GEMM experts, plus the shared expert's 6 rows
+    assert bench.gate_up_gemm_flops(cfg, ids) == 2.0 * rows * 2 * 2048 * 7168
+
+
+def test_oracle_all_cores_reports_its_workers():
+    r = bench.oracle_all_cores(0, budget_s=0.2, max_workers=2)
+    assert r["kind"] == "oracle" and r["unit"] == "tokens/s"
+    assert 1 <= r["cores"] <= 2 and r["value"] > 0
+    assert str(r["cores"]) in r["sample"]

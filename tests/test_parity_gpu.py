@@ -54,8 +54,9 @@ def run_gpu(torch, cfg, T, layer_index=0, layer=None):
     return res
 
 
-def check_against_oracle(cfg, g, sample=None, layer_index=0):
-    """Index rule on every token, outputs on `sample` tokens (all if None)."""
+def check_against_oracle(cfg, g, sample=None, layer_index=0, parallel=False):
+    """Index rule on every token, outputs on `sample` tokens (all if None);
+    with `parallel` the oracle rows are computed by several processes."""
     ol = oracle_layer(cfg, layer_index)
     x = g["x"]
     T = x.shape[0]
@@ -67,9 +68,12 @@ def check_against_oracle(cfg, g, sample=None, layer_index=0):
     w_or = ref.gate_weights(l64, g["ids"].astype(np.int64), cfg.gating)
     np.testing.assert_allclose(g["w"], w_or, rtol=1e-5, atol=1e-6)
     forced = np.where(near[:, None], g["ids"], ref.topk_ids(l64, cfg.top_k))
-    r = ref.moe_forward(x, ol, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter, forced_ids=forced,
-                        token_subset=toks)
-    return pu.check_outputs(g["out"][toks], r["out_bf16"], cfg.name)
+    if parallel:
+        want = pu.oracle_rows(cfg, layer_index, x, forced, toks)
+    else:
+        want = ref.moe_forward(x, ol, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter, forced_ids=forced,
+                               token_subset=toks)["out_bf16"]
+    return pu.check_outputs(g["out"][toks], want, cfg.name)
 
 
 # ------------------------------------------------------------------ small shapes, every token
@@ -85,7 +89,7 @@ SMALL = {
 
 
 @pytest.mark.parametrize("name", sorted(SMALL))
-@pytest.mark.parametrize("T", [1, 4, 17, 64, 65, 200])
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 17, 64, 65, 200])
 def test_small_every_token(torch, name, T):
     cfg = SMALL[name]
     g = run_gpu(torch, cfg, T)
@@ -108,18 +112,41 @@ def test_c1_decode_every_token(torch):
     check_against_oracle(cfg, g)
 
 
-def test_c2_batched_decode_sampled(torch):
+def test_c2_batched_decode_every_token(torch):
     cfg = synth.BATCHED
     g = run_gpu(torch, cfg, cfg.tokens)
     counts = np.bincount(g["ids"].ravel(), minlength=cfg.n_experts)
     assert (counts > 10).sum() >= 1 and (counts.max() <= cfg.tokens)
-    check_against_oracle(cfg, g, sample=[0, 1, 17, 31, 42, 63])
+    check_against_oracle(cfg, g, parallel=True)
+
+
+def prefill_sample(ids: np.ndarray, n_experts: int, tile: int = 256) -> np.ndarray:
+    """Tokens whose rows reach every kind of work unit of the prefill path:
+    the first and last row of every 256-row tile of the three experts with
+    the most rows, one token of every expert with at most 4 rows (the decode
+    kernels) and one of every expert with 5..16 rows (small GEMM tiles).
+    Rows of an expert are its (token, slot) pairs in token order."""
+    T, k = ids.shape
+    counts = np.bincount(ids.ravel(), minlength=n_experts)
+    rows_of = {e: np.nonzero((ids == e).any(axis=1))[0] for e in range(n_experts) if counts[e]}
+    pick = {0, T - 1}
+    for e in np.argsort(-counts, kind="stable")[:3]:
+        toks = rows_of[int(e)]
+        for t0 in range(0, len(toks), tile):
+            pick.add(int(toks[t0]))
+            pick.add(int(toks[min(t0 + tile, len(toks)) - 1]))
+    for e, toks in rows_of.items():
+        if counts[e] <= 16:
+            pick.add(int(toks[0]))
+    return np.array(sorted(pick))
 
 
 def test_c3_prefill_sampled(torch):
     cfg = synth.PREFILL
     g = run_gpu(torch, cfg, cfg.tokens)
-    check_against_oracle(cfg, g, sample=[0, 1777, 4095])
+    sample = prefill_sample(g["ids"], cfg.n_experts)
+    assert len(sample) >= 64
+    check_against_oracle(cfg, g, sample=sample, parallel=True)
 
 
 def test_deterministic_and_host_path(torch):

@@ -168,6 +168,52 @@ def test_streaming_c1_shapes_against_oracle(torch):
     pu.check_outputs(o, r["out_bf16"], "streamed c1 shapes")
 
 
+def test_streaming_full_shapes_sampled_against_oracle(torch):
+    """The expert-streaming workload at its own shapes: 8 layers x (256 + 1)
+    experts of hidden 7168 / inter 2048 in pinned host RAM (~51 GB), a
+    12e9-byte cache (484 slots), the routing trace replayed through
+    moe_forward_routed with next-layer prefetch for 10 steps (more fetches
+    than slots, so slots are reused); four sampled (step, layer) outputs are
+    compared with the oracle run on the same forced ids."""
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    cfg = synth.STREAMING
+    steps = 10
+    samples = [(2, 0), (5, 3), (7, 7), (9, 4)]
+    trace = synth.streaming_trace(dataclasses.replace(cfg, steps=steps))
+    eb = moe.moe_expert_bytes(cfg.hidden, cfg.inter)
+    moe.moe_set_cache_bytes(cfg.cache_bytes)
+    layers = []
+    got = {}
+    try:
+        layers = [layer_from_config(cfg, l) for l in range(cfg.n_layers)]
+        moe.moe_reset_stats()
+        for s in range(steps):
+            for l in range(cfg.n_layers):
+                nl, ns = (l + 1, s) if l + 1 < cfg.n_layers else (0, s + 1)
+                if ns < steps:
+                    layers[nl].prefetch(trace[ns, nl])
+                x = synth.activations(cfg, l, s, tokens=1)
+                out = layers[l].forward_routed(to_dev(torch, x), trace[s, l][None])
+                if (s, l) in samples:
+                    got[(s, l)] = (x, out.view(torch.int16).cpu().numpy().view(np.uint16))
+        torch.cuda.synchronize()
+        for L in layers:
+            moe.moe_check(L.handle)
+        st = moe.moe_get_stats()
+    finally:
+        for L in layers:
+            L.destroy()
+            L.host = None
+        moe.moe_set_cache_bytes(moe.SIZE_MAX)
+        if hasattr(torch._C, "_host_emptyCache"):
+            torch._C._host_emptyCache()     # give the 51 GB of pinned host memory back
+    assert st["cache_slots"] == cfg.cache_bytes // eb == 484
+    assert st["evictions"] > 0
+    for (s, l), (x, out) in got.items():
+        want = pu.oracle_rows(cfg, l, x, trace[s, l][None].astype(np.int64), [0], workers=1)
+        pu.check_outputs(out, want, f"streamed step {s} layer {l}")
+
+
 def test_cache_too_small_is_an_error(torch):
     from routed_expert_ffn_forward_b200.layer import layer_from_config
     cfg = SMALL
