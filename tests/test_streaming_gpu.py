@@ -134,10 +134,13 @@ def test_streaming_matches_resident_and_lru_model(torch, prefetch, slots):
         assert model.evictions > 0
 
 
-def test_streaming_c1_shapes_against_oracle(torch):
+@pytest.mark.parametrize("T", [1, 2])
+def test_streaming_c1_shapes_against_oracle(torch, T):
     """Full-size expert shapes (hidden 7168, inter 2048), 32 experts per layer,
-    2 layers through a 20-slot cache (2 tokens need at most 17 experts); unrouted forward (routing read back to the
-    host) and a check of one streamed token against the oracle."""
+    2 layers through a 20-slot cache (2 tokens need at most 17 experts);
+    unrouted forwards (the routing is read back to the host before the
+    experts are fetched, so one token takes the split decode kernels here)
+    and a check of the last streamed output against the oracle."""
     from routed_expert_ffn_forward_b200.layer import layer_from_config
     cfg = dataclasses.replace(synth.STREAMING, n_experts=32, n_layers=2, steps=6, seed=41)
     eb = moe.moe_expert_bytes(cfg.hidden, cfg.inter)
@@ -148,9 +151,9 @@ def test_streaming_c1_shapes_against_oracle(torch):
         outs = []
         for s in range(3):
             for l in range(cfg.n_layers):
-                x = synth.activations(cfg, l, s, tokens=2)
+                x = synth.activations(cfg, l, s, tokens=T)
                 o = layers[l].forward(to_dev(torch, x))
-                ids, _ = layers[l].routing(2)
+                ids, _ = layers[l].routing(T)
                 outs.append((l, x, o.view(torch.int16).cpu().numpy().view(np.uint16), ids.cpu().numpy()))
         st = moe.moe_get_stats()
         for L in layers:
@@ -172,13 +175,14 @@ def test_streaming_full_shapes_sampled_against_oracle(torch):
     """The expert-streaming workload at its own shapes: 8 layers x (256 + 1)
     experts of hidden 7168 / inter 2048 in pinned host RAM (~51 GB), a
     12e9-byte cache (484 slots), the routing trace replayed through
-    moe_forward_routed with next-layer prefetch for 10 steps (more fetches
-    than slots, so slots are reused); four sampled (step, layer) outputs are
-    compared with the oracle run on the same forced ids."""
+    moe_forward_routed with next-layer prefetch for 40 steps (they touch ~560
+    distinct experts, more than the slots, so slots are reused); four sampled
+    (step, layer) outputs are compared with the oracle run on the same forced
+    ids."""
     from routed_expert_ffn_forward_b200.layer import layer_from_config
     cfg = synth.STREAMING
-    steps = 10
-    samples = [(2, 0), (5, 3), (7, 7), (9, 4)]
+    steps = 40
+    samples = [(3, 0), (17, 3), (29, 7), (39, 4)]
     trace = synth.streaming_trace(dataclasses.replace(cfg, steps=steps))
     eb = moe.moe_expert_bytes(cfg.hidden, cfg.inter)
     moe.moe_set_cache_bytes(cfg.cache_bytes)
