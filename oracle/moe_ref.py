@@ -95,6 +95,108 @@ def q4k_dequant(raw: np.ndarray) -> np.ndarray:
     return w.reshape(lead + (nb * QK_K,))
 
 
+# --------------------------------------------------------------------------- other GGUF block types
+# UD-Q*_K_XL files mix block types per tensor (LayerStoRm README, "Get a
+# model"; "License and attributions": GGUF and MXFP4 decode paths).  Each
+# function below dequantises one public GGUF block type exactly, in fp64.
+# GGML type ids: Q8_0 = 8, Q4_K = 12, Q5_K = 13, Q6_K = 14, MXFP4 = 39.
+
+Q8_0, Q4_K, Q5_K, Q6_K, MXFP4 = 8, 12, 13, 14, 39
+BLOCK = {Q8_0: (32, 34), Q4_K: (256, 144), Q5_K: (256, 176), Q6_K: (256, 210), MXFP4: (32, 17)}
+
+
+def _blocks(raw, nbytes):
+    raw = np.asarray(raw, dtype=np.uint8)
+    lead = raw.shape[:-1]
+    nb = raw.shape[-1] // nbytes
+    return raw.reshape(lead + (nb, nbytes)), lead, nb
+
+
+def _f16(two_bytes):
+    return two_bytes.copy().view(np.float16)[..., 0].astype(np.float64)
+
+
+def q8_0_dequant(raw):
+    """Q8_0: blocks of 32 weights in 34 bytes: fp16 d, then 32 signed bytes q;
+    weight = d * q."""
+    b, lead, nb = _blocks(raw, 34)
+    d = _f16(b[..., 0:2])
+    q = b[..., 2:34].view(np.int8).astype(np.float64)
+    return (d[..., None] * q).reshape(lead + (nb * 32,))
+
+
+def q5_k_dequant(raw):
+    """Q5_K: 256 weights in 176 bytes: fp16 d, fp16 dmin, the 12 packed scale
+    bytes of Q4_K (eight 6-bit scales and mins), 32 bytes of fifth bits qh,
+    128 bytes of low nibbles qs.  Chunk c (64 weights) takes bytes 32c..32c+31
+    of qs: the low nibble of byte i is weight 64c+i (sub-block 2c, fifth bit =
+    bit 2c of qh[i]), the high nibble weight 64c+32+i (sub-block 2c+1, fifth
+    bit = bit 2c+1 of qh[i]).  weight = d*sc_j*q - dmin*m_j, q in 0..31."""
+    b, lead, nb = _blocks(raw, 176)
+    d, dmin = _f16(b[..., 0:2]), _f16(b[..., 2:4])
+    sc, mn = q4k_scale_min(b[..., 4:16])
+    qh = b[..., 16:48].astype(np.int64)
+    qs = b[..., 48:176].reshape(lead + (nb, 4, 32)).astype(np.int64)
+    q = np.empty(lead + (nb, 8, 32), dtype=np.int64)
+    for c in range(4):
+        q[..., 2 * c, :] = (qs[..., c, :] & 0x0F) | (((qh >> (2 * c)) & 1) << 4)
+        q[..., 2 * c + 1, :] = (qs[..., c, :] >> 4) | (((qh >> (2 * c + 1)) & 1) << 4)
+    w = d[..., None, None] * sc[..., None] * q - dmin[..., None, None] * mn[..., None]
+    return w.reshape(lead + (nb * 256,))
+
+
+def q6_k_dequant(raw):
+    """Q6_K: 256 weights in 210 bytes: 128 bytes of low nibbles ql, 64 bytes of
+    high bit pairs qh, 16 signed 8-bit scales, fp16 d.  Two halves of 128
+    weights, half h using ql[64h..], qh[32h..], scales[8h..].  Within a half,
+    for i in 0..31 and g = i // 16, the four weights
+      i      : low nibble of ql[i],      bits 0-1 of qh[i], scale g
+      i + 32 : low nibble of ql[i + 32], bits 2-3 of qh[i], scale g + 2
+      i + 64 : high nibble of ql[i],     bits 4-5 of qh[i], scale g + 4
+      i + 96 : high nibble of ql[i + 32], bits 6-7 of qh[i], scale g + 6
+    have the 6-bit value q = nibble | (pair << 4); weight = d * scale * (q - 32)."""
+    b, lead, nb = _blocks(raw, 210)
+    ql = b[..., 0:128].astype(np.int64)
+    qh = b[..., 128:192].astype(np.int64)
+    scales = b[..., 192:208].view(np.int8).astype(np.float64)
+    d = _f16(b[..., 208:210])
+    w = np.empty(lead + (nb, 256), dtype=np.float64)
+    for h in range(2):
+        L, Hh, S = ql[..., 64 * h:64 * h + 64], qh[..., 32 * h:32 * h + 32], scales[..., 8 * h:8 * h + 8]
+        for part, (lo, sh, nib_hi, off) in enumerate(((0, 0, False, 0), (32, 2, False, 2),
+                                                       (0, 4, True, 4), (32, 6, True, 6))):
+            nib = (L[..., lo:lo + 32] >> 4) if nib_hi else (L[..., lo:lo + 32] & 0x0F)
+            q = (nib | (((Hh >> sh) & 3) << 4)) - 32
+            g = np.arange(32) // 16
+            sc = S[..., off + g]
+            w[..., 128 * h + 32 * part:128 * h + 32 * part + 32] = d[..., None] * sc * q
+    return w.reshape(lead + (nb * 256,))
+
+
+# FP4 E2M1 values of the 16 codes (bit 3 = sign): 0, 0.5, 1, 1.5, 2, 3, 4, 6
+_E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0])
+
+
+def mxfp4_dequant(raw):
+    """MXFP4 (OCP microscaling FP4): blocks of 32 weights in 17 bytes: an E8M0
+    scale byte e (the power of two 2^(e-127)), then 16 bytes of FP4 E2M1 codes:
+    element i is the low nibble of byte i, element 16+i its high nibble;
+    weight = e2m1(code) * 2^(e-127)."""
+    b, lead, nb = _blocks(raw, 17)
+    e = b[..., 0].astype(np.int64)
+    qs = b[..., 1:17].astype(np.int64)
+    codes = np.concatenate([qs & 0x0F, qs >> 4], axis=-1)
+    w = _E2M1[codes] * np.ldexp(1.0, e - 127)[..., None]
+    return w.reshape(lead + (nb * 32,))
+
+
+def dequant(raw, qtype: int) -> np.ndarray:
+    """Dequantise a matrix of any supported GGUF block type ([..., row bytes])."""
+    fn = {Q4_K: q4k_dequant, Q5_K: q5_k_dequant, Q6_K: q6_k_dequant, Q8_0: q8_0_dequant,
+          MXFP4: mxfp4_dequant}[qtype]
+    return fn(raw)
+
+
 # --------------------------------------------------------------------------- router
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     """bf16 bit patterns (uint16) -> fp64, exactly."""
@@ -179,11 +281,12 @@ def silu(z):
     return z / (1.0 + np.exp(-z))
 
 
-def expert_ffn(xr: np.ndarray, gate_raw, up_raw, down_raw, inter: int) -> np.ndarray:
-    """SwiGLU expert on rows xr [n, H] (fp64): y = W_d (silu(W_g x) * (W_u x))."""
-    wg = q4k_dequant(gate_raw)                    # [I, H]
-    wu = q4k_dequant(up_raw)                      # [I, H]
-    wd = q4k_dequant(down_raw)                    # [H, I_pad]
+def expert_ffn(xr: np.ndarray, gate_raw, up_raw, down_raw, inter: int, quants=(Q4_K, Q4_K, Q4_K)) -> np.ndarray:
+    """SwiGLU expert on rows xr [n, H] (fp64): y = W_d (silu(W_g x) * (W_u x));
+    `quants` are the GGUF block types of gate, up and down."""
+    wg = dequant(gate_raw, quants[0])             # [I, H]
+    wu = dequant(up_raw, quants[1])               # [I, H]
+    wd = dequant(down_raw, quants[2])             # [H, I_pad]
     h = silu(xr @ wg.T) * (xr @ wu.T)             # [n, I]
     return h @ wd[:, :inter].T                    # padded inputs of h are zero
 
@@ -217,9 +320,11 @@ def moe_forward(x_bits: np.ndarray, layer, k: int, gating: int, n_shared: int,
                 inter: int, forced_ids=None, token_subset=None):
     """Whole layer on the CPU.
 
-    layer: dict with 'router_w' [E,H] fp32, 'router_b' [E] or None and
+    layer: dict with 'router_w' [E,H] fp32, 'router_b' [E] or None,
            'experts': callable e -> (gate_raw, up_raw, down_raw) for
-           e in 0..E+S-1 (shared experts numbered after the routed ones).
+           e in 0..E+S-1 (shared experts numbered after the routed ones) and
+           optionally 'quants': the GGUF block types of gate, up and down
+           (default Q4_K for all three).
     forced_ids: optional [T,k] expert ids to use instead of the top-k (the
            weights are then the gating function of the logits at those ids).
     token_subset: optional token indices; only those output rows are computed.
@@ -240,11 +345,11 @@ def moe_forward(x_bits: np.ndarray, layer, k: int, gating: int, n_shared: int,
     for e in needed:
         rows = [(n, j) for n in range(len(tokens)) for j in range(k) if ids[n, j] == e]
         ns = [n for n, _ in rows]
-        y = expert_ffn(xs[ns], *layer["experts"](e), inter)
+        y = expert_ffn(xs[ns], *layer["experts"](e), inter, layer.get("quants", (Q4_K,) * 3))
         for (n, j), yr in zip(rows, y):
             out[n] += w[n, j] * yr
     for s in range(n_shared):
-        out += expert_ffn(xs, *layer["experts"](E + s), inter)
+        out += expert_ffn(xs, *layer["experts"](E + s), inter, layer.get("quants", (Q4_K,) * 3))
     return dict(out64=out, out_bf16=round_bf16(out), ids=ids, w=w, logits=l,
                 gap=topk_gap(l, k), tokens=tokens)
 
@@ -268,7 +373,7 @@ def dense_moe(x_bits: np.ndarray, layer, k: int, gating: int, n_shared: int, int
             gate[t, order] = sg / sg.sum()
     out = np.zeros_like(x)
     for e in range(E):
-        out += gate[:, e:e + 1] * expert_ffn(x, *layer["experts"](e), inter)
+        out += gate[:, e:e + 1] * expert_ffn(x, *layer["experts"](e), inter, layer.get("quants", (Q4_K,) * 3))
     for s in range(n_shared):
-        out += expert_ffn(x, *layer["experts"](E + s), inter)
+        out += expert_ffn(x, *layer["experts"](E + s), inter, layer.get("quants", (Q4_K,) * 3))
     return out

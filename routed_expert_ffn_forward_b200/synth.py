@@ -29,6 +29,17 @@ import numpy as np
 QK_K = 256
 Q4K_BLOCK_BYTES = 144
 
+# GGUF block types (GGML type id -> (weights per block, bytes per block))
+Q8_0, Q4_K, Q5_K, Q6_K, MXFP4 = 8, 12, 13, 14, 39
+BLOCKS = {Q8_0: (32, 34), Q4_K: (256, 144), Q5_K: (256, 176), Q6_K: (256, 210), MXFP4: (32, 17)}
+
+
+def row_bytes(qtype: int, cols: int) -> int:
+    """Bytes of one weight row of `cols` inputs (padded to whole blocks)."""
+    n, b = BLOCKS[qtype]
+    return (cols + n - 1) // n * b
+
+
 GATE, UP, DOWN = 0, 1, 2
 
 # stream kinds (high byte of the Philox stream id)
@@ -54,6 +65,7 @@ class LayerConfig:
     cache_bytes: Optional[int] = None
     steps: int = 1
     keep_p: float = 0.6
+    quants: tuple = (Q4_K, Q4_K, Q4_K)    # GGUF block types of gate, up, down
 
     @property
     def blocks_h(self) -> int:
@@ -65,15 +77,19 @@ class LayerConfig:
 
     @property
     def gate_bytes(self) -> int:
-        return self.inter * self.blocks_h * Q4K_BLOCK_BYTES
+        return self.inter * row_bytes(self.quants[0], self.hidden)
+
+    @property
+    def up_bytes(self) -> int:
+        return self.inter * row_bytes(self.quants[1], self.hidden)
 
     @property
     def down_bytes(self) -> int:
-        return self.hidden * self.blocks_i * Q4K_BLOCK_BYTES
+        return self.hidden * row_bytes(self.quants[2], self.inter)
 
     @property
     def expert_bytes(self) -> int:
-        return 2 * self.gate_bytes + self.down_bytes
+        return self.gate_bytes + self.up_bytes + self.down_bytes
 
 
 H, I = 7168, 2048
@@ -137,12 +153,47 @@ def q4k_tensor(seed: int, layer: int, expert: int, matrix: int, rows: int, cols:
     return out
 
 
+def q_tensor(qtype: int, seed: int, layer: int, expert: int, matrix: int, rows: int, cols: int,
+             out: Optional[np.ndarray] = None) -> np.ndarray:
+    """Draw one weight matrix [rows, cols] of any supported GGUF block type as
+    raw bytes [rows, row_bytes].  Quant bytes are uniform random; the scale
+    fields are drawn so that weights are of order one, like the Q4_K ones:
+      Q4_K  d ~ U(1e-3, 1e-2), dmin ~ U(0, 5e-3)             (q4k_tensor)
+      Q5_K  d ~ U(5e-4, 5e-3), dmin ~ U(0, 5e-3)             (q up to 31)
+      Q6_K  d ~ U(5e-5, 5e-4), 16 int8 scales uniform        (|w| <= d*128*32)
+      Q8_0  d ~ U(1e-3, 1e-2)                                (|w| <= d*128)
+      MXFP4 scale exponent e uniform on 124..127             (|w| <= 6)
+    fp16 fields are drawn in fp64 and rounded to fp16."""
+    if qtype == Q4_K:
+        return q4k_tensor(seed, layer, expert, matrix, rows, cols, out)
+    n_el, nbytes = BLOCKS[qtype]
+    nb = (cols + n_el - 1) // n_el
+    n = rows * nb
+    g = _gen(seed, _K_WEIGHT, layer, expert, matrix)
+    if out is None:
+        out = np.empty((rows, nb * nbytes), dtype=np.uint8)
+    blk = out.reshape(n, nbytes)
+    blk[:] = g.integers(0, 256, size=(n, nbytes), dtype=np.uint8)
+    f16 = lambda v: v.astype(np.float16).view(np.uint8).reshape(n, 2)
+    if qtype == Q5_K:
+        blk[:, 0:2] = f16(g.uniform(5e-4, 5e-3, n))
+        blk[:, 2:4] = f16(g.uniform(0.0, 5e-3, n))
+    elif qtype == Q6_K:
+        blk[:, 208:210] = f16(g.uniform(5e-5, 5e-4, n))
+    elif qtype == Q8_0:
+        blk[:, 0:2] = f16(g.uniform(1e-3, 1e-2, n))
+    elif qtype == MXFP4:
+        blk[:, 0] = g.integers(124, 128, size=n, dtype=np.uint8)
+    return out
+
+
 def expert_tensors(cfg: LayerConfig, layer: int, expert: int):
-    """(gate, up, down) raw Q4_K bytes for routed expert ``expert`` (shared experts
-    are numbered E..E+S-1)."""
-    gate = q4k_tensor(cfg.seed, layer, expert, GATE, cfg.inter, cfg.hidden)
-    up = q4k_tensor(cfg.seed, layer, expert, UP, cfg.inter, cfg.hidden)
-    down = q4k_tensor(cfg.seed, layer, expert, DOWN, cfg.hidden, cfg.inter)
+    """(gate, up, down) raw bytes of the configured block types for routed
+    expert ``expert`` (shared experts are numbered E..E+S-1)."""
+    qg, qu, qd = cfg.quants
+    gate = q_tensor(qg, cfg.seed, layer, expert, GATE, cfg.inter, cfg.hidden)
+    up = q_tensor(qu, cfg.seed, layer, expert, UP, cfg.inter, cfg.hidden)
+    down = q_tensor(qd, cfg.seed, layer, expert, DOWN, cfg.hidden, cfg.inter)
     return gate, up, down
 
 

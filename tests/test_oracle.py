@@ -314,7 +314,9 @@ def _pins_pass() -> bool:
               lambda: test_sparse_equals_dense_bruteforce("c0_shared_sigmoid"),
               test_constant_weight_closed_form, test_permutation_bijection_and_stable_order,
               test_bf16_to_f64_matches_torch_on_every_pattern, test_silu_matches_scipy_expit,
-              test_token_subset_rows_equal_full_rows]
+              test_token_subset_rows_equal_full_rows, test_q8_0_closed_form, test_q5_k_fifth_bit_positions,
+              test_q6_k_positions_and_offset, test_mxfp4_code_table_and_scale]
+    checks += [lambda q=q: test_block_types_match_gguf_library(q) for q in (ref.Q5_K, ref.Q6_K, ref.Q8_0, ref.MXFP4)]
     for c in checks:
         try:
             c()
@@ -340,8 +342,9 @@ MUTANTS = {
         lambda l, ids, g: orig(l, ids, g) if g else
         (np.exp(np.take_along_axis(l, ids, 1)) / np.exp(l).sum(1, keepdims=True)))),
     "silu on up instead of gate": ("expert_ffn", lambda orig: (
-        lambda xr, g, u, d, inter: orig(xr, u, g, d, inter))),
-    "padding not masked": ("expert_ffn", lambda orig: (lambda xr, g, u, d, inter: _unmasked_ffn(xr, g, u, d))),
+        lambda xr, g, u, d, inter, quants=(12, 12, 12): orig(xr, u, g, d, inter, quants))),
+    "padding not masked": ("expert_ffn", lambda orig: (
+        lambda xr, g, u, d, inter, quants=(12, 12, 12): _unmasked_ffn(xr, g, u, d))),
     "unstable permutation": ("permutation", lambda orig: (
         lambda ids, E: (lambda c, o, p: (c, o, p[::-1].copy()))(*orig(ids, E)))),
 }
@@ -359,12 +362,40 @@ def _subset_forced_by_position(orig):
     return bad
 
 
+def _q6k_offset16(orig):
+    def bad(raw):
+        b = np.asarray(raw, np.uint8).reshape(-1, 210)
+        d = b[:, 208:210].copy().view(np.float16)[:, 0].astype(np.float64)
+        sc = b[:, 192:208].view(np.int8).astype(np.float64)
+        # the mistake: a zero point of 16 instead of 32
+        w = orig(raw).reshape(-1, 256)
+        scale = np.concatenate([np.concatenate([sc[:, 8 * h + 2 * p + np.arange(32) // 16] for p in range(4)], 1)
+                                for h in range(2)], 1)
+        return (w + d[:, None] * scale * 16.0).reshape(np.asarray(raw).shape[:-1] + (-1,))
+    return bad
+
+
 MUTANTS.update({
+    "Q8_0 read as unsigned": ("q8_0_dequant", lambda orig: (lambda raw: (lambda b: (
+        b[..., 0:2].copy().view(np.float16)[..., 0].astype(np.float64)[..., None] *
+        b[..., 2:34].astype(np.float64)).reshape(-1))(np.asarray(raw, np.uint8).reshape(-1, 34)))),
+    "Q5_K fifth bits swapped": ("q5_k_dequant", lambda orig: (lambda raw: orig(_swap_q5_bits(raw)))),
+    "Q6_K zero point 16": ("q6_k_dequant", _q6k_offset16),
+    "MXFP4 bias 128": ("mxfp4_dequant", lambda orig: (lambda raw: 0.5 * orig(raw))),
     "bf16 shifted by 15": ("bf16_to_f64", lambda orig: (
         lambda bits: (np.asarray(bits, np.uint16).astype(np.uint32) << 15).view(np.float32).astype(np.float64))),
     "silu without the z factor": ("silu", lambda orig: (lambda z: 1.0 / (1.0 + np.exp(-z)))),
     "subset ignores its forced rows": ("moe_forward", _subset_forced_by_position),
 })
+
+
+def _swap_q5_bits(raw):
+    # the mistake: fifth bit of the low nibble taken from bit 2c+1 and vice versa
+    b = np.asarray(raw, np.uint8).reshape(-1, 176).copy()
+    qh = b[:, 16:48].astype(np.int64)
+    even, odd = qh & 0x55, (qh >> 1) & 0x55
+    b[:, 16:48] = ((even << 1) | odd).astype(np.uint8)
+    return b.reshape(np.asarray(raw).shape)
 
 
 def _unmasked_ffn(xr, g, u, d):
@@ -385,3 +416,95 @@ def test_pins_catch_planted_mistakes(name, monkeypatch):
     attr, make = MUTANTS[name]
     monkeypatch.setattr(ref, attr, make(getattr(ref, attr)))
     assert not _pins_pass(), f"planted mistake '{name}' went unnoticed"
+
+
+# ------------------------------------------------------------------ other GGUF block types
+def _sane_blocks(qtype, n, seed):
+    """Random blocks of a GGUF type with finite scale fields."""
+    rng = np.random.default_rng(seed)
+    bs = ref.BLOCK[qtype][1]
+    raw = rng.integers(0, 256, (n, bs), dtype=np.uint8)
+    f16 = lambda v: np.asarray(v, np.float16).view(np.uint8).reshape(-1, 2)
+    if qtype in (ref.Q5_K,):
+        raw[:, 0:2] = f16(rng.uniform(-0.02, 0.02, n))
+        raw[:, 2:4] = f16(rng.uniform(0, 0.01, n))
+    elif qtype == ref.Q6_K:
+        raw[:, 208:210] = f16(rng.uniform(-0.01, 0.01, n))
+    elif qtype == ref.Q8_0:
+        raw[:, 0:2] = f16(rng.uniform(-0.02, 0.02, n))
+    elif qtype == ref.MXFP4:
+        raw[:, 0] = rng.integers(110, 140, n)
+    return raw.reshape(-1)
+
+
+@pytest.mark.parametrize("qtype", [ref.Q5_K, ref.Q6_K, ref.Q8_0, ref.MXFP4])
+def test_block_types_match_gguf_library(qtype):
+    gguf = pytest.importorskip("gguf")
+    from gguf.quants import dequantize
+    raw = _sane_blocks(qtype, 64, qtype)
+    ours = ref.dequant(raw, qtype)
+    lib = dequantize(raw, gguf.GGMLQuantizationType(qtype)).astype(np.float64).reshape(ours.shape)
+    np.testing.assert_allclose(ours, lib, rtol=1e-6, atol=1e-7 * np.abs(lib).max())
+
+
+def test_q8_0_closed_form():
+    blk = np.zeros(34, np.uint8)
+    blk[0:2] = np.frombuffer(np.float16(0.25).tobytes(), np.uint8)
+    blk[2:] = np.arange(-16, 16, dtype=np.int8).view(np.uint8)
+    np.testing.assert_array_equal(ref.q8_0_dequant(blk), 0.25 * np.arange(-16, 16))
+
+
+def test_q5_k_fifth_bit_positions():
+    # all quants zero, one fifth bit set: exactly one weight becomes d*sc*16
+    for pos in (0, 31, 32, 63, 64, 130, 255):
+        blk = np.zeros(176, np.uint8)
+        blk[0:2] = np.frombuffer(np.float16(1.0).tobytes(), np.uint8)
+        blk[4:16] = pack_scales(np.ones((1, 8), np.int64), np.zeros((1, 8), np.int64))[0]
+        c, rem = divmod(pos, 64)
+        half, i = divmod(rem, 32)
+        blk[16 + i] = 1 << (2 * c + half)
+        w = ref.q5_k_dequant(blk)
+        assert np.flatnonzero(w).tolist() == [pos] and w[pos] == 16.0
+
+
+def test_q6_k_positions_and_offset():
+    # ql = qh = 0 gives q - 32 = -32 everywhere; then one low nibble of 5 at
+    # each byte lands on its documented position
+    blk = np.zeros(210, np.uint8)
+    blk[192:208] = np.arange(1, 17, dtype=np.int8).view(np.uint8)     # scale s = 1..16
+    blk[208:210] = np.frombuffer(np.float16(0.5).tobytes(), np.uint8)
+    base = ref.q6_k_dequant(blk)
+    for h in (0, 1):
+        for part in range(4):
+            for i in (0, 17, 31):
+                w = 128 * h + 32 * part + i
+                g = i // 16 + 2 * part + 8 * h
+                assert base[w] == 0.5 * (g + 1) * -32
+    b2 = blk.copy()
+    b2[64 + 40] = 0x05            # half 1, ql[40]: low nibble -> weight 128+32+8, high nibble -> 128+96+8
+    w2 = ref.q6_k_dequant(b2)
+    diff = np.flatnonzero(w2 != base).tolist()
+    assert diff == [128 + 40]
+    assert w2[168] == 0.5 * 11 * (5 - 32)   # scale index 8 + 0 + 2 = 10 -> s = 11
+
+
+def test_mxfp4_code_table_and_scale():
+    blk = np.zeros(17, np.uint8)
+    blk[0] = 127 + 3                                       # 2^3
+    blk[1:17] = (np.arange(16) | (np.arange(16)[::-1] << 4)).astype(np.uint8)
+    w = ref.mxfp4_dequant(blk)
+    e2m1 = [0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.0, -0.5, -1, -1.5, -2, -3, -4, -6]
+    np.testing.assert_array_equal(w[:16], 8.0 * np.array(e2m1))
+    np.testing.assert_array_equal(w[16:], 8.0 * np.array(e2m1[::-1]))
+
+
+@pytest.mark.parametrize("quants", [(13, 8, 14), (39, 39, 39), (14, 12, 8)])
+def test_sparse_equals_dense_mixed_block_types(quants):
+    cfg = cfg_with(synth.TINY, n_shared=1, gating=1, top_k=3, tokens=5, inter=300, quants=quants, seed=9)
+    layer = dict(router_w=synth.router_weight(cfg), router_b=synth.router_bias(cfg),
+                 experts=lambda e: synth.expert_tensors(cfg, 0, e), quants=quants)
+    x = synth.activations(cfg)
+    sparse = ref.moe_forward(x, layer, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter)["out64"]
+    dense = ref.dense_moe(x, layer, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter)
+    np.testing.assert_allclose(sparse, dense, rtol=1e-11, atol=1e-9 * np.abs(dense).max())
+    assert np.isfinite(sparse).all() and np.abs(sparse).max() > 0
