@@ -57,7 +57,15 @@ typedef enum {
   MOE_ERR_NOT_READY = -6        /* router or experts not set yet */
 } moe_status;
 
-typedef enum { MOE_Q4_K = 12 } moe_quant; /* GGUF type id; the only one supported */
+/* GGUF block types (GGML type ids).  Q4_K runs every path; the others run
+ * each token through the single-token kernel (see moe_layer_create_mixed). */
+typedef enum {
+  MOE_Q8_0 = 8,   /* 32 weights: fp16 scale, 32 signed bytes */
+  MOE_Q4_K = 12,  /* 256 weights: fp16 d, dmin, 6-bit scales/mins, 4-bit quants */
+  MOE_Q5_K = 13,  /* as Q4_K with a fifth quant bit */
+  MOE_Q6_K = 14,  /* 256 weights: 6-bit quants, 16 signed 8-bit scales, fp16 d */
+  MOE_MXFP4 = 39  /* 32 weights: E8M0 power-of-two scale, FP4 E2M1 values */
+} moe_quant;
 
 typedef enum {
   MOE_GATE_SOFTMAX_TOPK = 0,  /* softmax over the top_k selected logits */
@@ -91,7 +99,8 @@ enum {
   MOE_K_PREP = 6,    /* prefill only: activation rows and SwiGLU output to scaled fp16 */
   MOE_K_SMALL = 7,   /* prefill only: the decode kernels for experts with <= 4 rows */
   MOE_K_FORWARD = 8, /* whole forward, first kernel start to last kernel end */
-  MOE_K_COUNT = 9
+  MOE_K_FUSED = 9,   /* decode of one token as one kernel (router through combine) */
+  MOE_K_COUNT = 10
 };
 typedef struct {
   uint64_t forwards;             /* forwards profiled */
@@ -99,8 +108,11 @@ typedef struct {
   uint64_t launches[MOE_K_COUNT];/* launches per MOE_K_* */
 } moe_profile;
 
-/* Size in bytes of one expert (gate + up + down) in Q4_K.  0 on bad args.
- * Source: LayerStoRm README, "Get a model" (GGUF Q4_K weights). */
+/* Bytes one expert (gate + up + down, all of type `quant`) occupies in device
+ * memory, i.e. one cache slot: its GGUF bytes, except that Q6_K blocks are
+ * padded from 210 to 224 bytes and MXFP4 blocks grouped eight at a time from
+ * 136 into 144 bytes (16-byte aligned groups for the copy engines).  0 on bad
+ * args.  Source: LayerStoRm README, "Get a model" (GGUF weights). */
 size_t moe_expert_bytes(int hidden, int inter, moe_quant quant);
 
 /* Create a layer on the current GPU.
@@ -114,6 +126,21 @@ size_t moe_expert_bytes(int hidden, int inter, moe_quant quant);
  * top-k routing, always-on shared experts) and "Get a model" (Q4_K). */
 moe_status moe_layer_create(int hidden, int inter, int n_experts, int top_k,
                             int n_shared, moe_quant quant, moe_layer_t* out);
+
+/* Create a layer whose gate and up weights are of one GGUF block type and
+ * down weights of another, as in UD-Q*_K_XL files that mix block types per
+ * tensor.  moe_layer_create(..., q, out) equals this with q for both.  A
+ * layer with both types Q4_K takes every path of moe_forward; any other
+ * layer runs each token through the single-token kernel (one launch per
+ * token, in order, on the forward's stream), so its throughput at T tokens is
+ * T times the single-token time.  Types Q8_0 and MXFP4 for the down weights
+ * need inter to be a multiple of 256.  The host pointers of moe_set_experts
+ * hold GGUF rows of these types (rows of ceil(cols / block) blocks).
+ * Errors: as moe_layer_create; UNSUPPORTED for another type.
+ * Source: LayerStoRm README, "Get a model" (UD-Q4_K_XL GGUF files) and
+ * "License and attributions" (GGUF and MXFP4 decode paths). */
+moe_status moe_layer_create_mixed(int hidden, int inter, int n_experts, int top_k, int n_shared,
+                                  moe_quant quant_gate_up, moe_quant quant_down, moe_layer_t* out);
 
 /* Destroy a layer: waits for the layer's outstanding work (its last forward
  * and its internal copy stream), frees its device memory (cudaFree itself may
@@ -158,6 +185,27 @@ moe_status moe_set_experts(moe_layer_t layer, const void* const* gate,
  * streamed in and overlapped with compute); rebasdaily LayerStoRm explainer
  * (the host link as the final bottleneck). */
 moe_status moe_set_cache_bytes(size_t bytes);
+
+typedef enum {
+  MOE_CACHE_LRU = 0, /* evict the least recently used expert (default) */
+  MOE_CACHE_LFU = 1  /* evict the least frequently used expert, least recent among equals */
+} moe_cache_policy;
+
+/* Replacement policy of the streaming cache (process-wide; takes effect at
+ * the next miss, keeps the cached experts).  MOE_CACHE_LFU counts, for every
+ * (layer, expert) seen, its arrivals: forwards of its layer that used it when
+ * the layer's previous forward did not (prefetches excluded), halving all
+ * counts after every 64 x slots arrivals so that popularity ages.  A miss
+ * takes an empty slot if there is one, else evicts, preferably among experts
+ * that their layer's previous forward did not use, the one with the fewest
+ * arrivals (the least recently used among equals).  An expert a layer keeps
+ * using stays; among the rest the popular ones stay where LRU would let
+ * one-off experts push them out.
+ * Errors: INVALID_ARG for an unknown policy.
+ * Source: glm-flash-lite project page, "How it works" (experts kept in tiers
+ * ranked by how often they are used); LayerStoRm README, "Status and
+ * limitations" (cache and prefetch policy as active work). */
+moe_status moe_set_cache_policy(int policy);
 
 /* Forward: x bf16 [T, H] and out bf16 [T, H], device pointers, row-major.
  * T >= 0 (T = 0 returns at once).  T <= 4 takes the decode path (fused router,
@@ -265,6 +313,17 @@ moe_status moe_reset_profile(void);
 moe_status moe_route_noalloc(const void* x, const float* W, const float* bias, int T, int H, int E,
                              int top_k, moe_gating gating, int32_t* ids, float* weights,
                              void* stream);
+
+/* Test hooks for failure detection (process-wide, off by default), read by
+ * the single-token kernel at each launch.  wait_limit_ns: limit of its bounded
+ * waits (0 = the default 2 s); the final wait for its own copies in flight
+ * keeps the default.  hold_barrier > 0: its grid barrier waits for that many
+ * arrivals more than there are CTAs, so the wait runs out and the kernel
+ * returns with an error that moe_check reports (which also resets the
+ * kernel's counters, so the next forward runs normally).  No GPU fault is
+ * involved: the kernel's CTAs give up and exit.  No counterpart on the pages
+ * (failure detection). */
+moe_status moe_set_test_hooks(uint64_t wait_limit_ns, int hold_barrier);
 
 /* Message of the last failed call on this thread ("" if none). */
 const char* moe_last_error(void);

@@ -1,9 +1,12 @@
 """Build libmoe.so in-tree with nvcc for sm_100a.
 
-    python -m routed_expert_ffn_forward_b200.build [--force] [--verbose]
+    python -m routed_expert_ffn_forward_b200.build [--force] [--verbose] [--debug-bounds]
 
 nvcc cross-compiles, so this runs without a GPU.  The library lands next to
-this file (``libmoe.so``) and is what the ctypes binding loads.
+this file (``libmoe.so``) and is what the ctypes binding loads.  The
+bounds-checking variant (``libmoe_debug.so``, built with -DMOE_DEBUG_BOUNDS:
+every index a kernel reads from memory is checked before use) sits beside it;
+the binding loads it when MOE_LIB_VARIANT=debug.
 """
 from __future__ import annotations
 
@@ -19,6 +22,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe.so")
+LIB_DEBUG = os.path.join(PKG, "libmoe_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
@@ -36,19 +40,22 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = (sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
             glob.glob(os.path.join(INCLUDE, "*.h")))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and not _stale():
-        return LIB
-    objdir = os.path.join(PKG, "_build")
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          debug_bounds: bool = False) -> str:
+    lib = LIB_DEBUG if debug_bounds else LIB
+    if not force and not _stale(lib):
+        return lib
+    extra = list(extra or []) + (["-DMOE_DEBUG_BOUNDS"] if debug_bounds else [])
+    objdir = os.path.join(PKG, "_build_debug" if debug_bounds else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     procs = []
@@ -69,21 +76,22 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
             print(f"nvcc failed on {src}", file=sys.stderr)
     if failed:
         raise RuntimeError("libmoe.so build failed")
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--debug-bounds", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, debug_bounds=a.debug_bounds))
 
 
 if __name__ == "__main__":

@@ -10,7 +10,7 @@ namespace {
 
 __global__ void combine_kernel(const float* __restrict__ y, const float* __restrict__ w,
                                const int* __restrict__ inv, int H, int k, int S,
-                               __nv_bfloat16* __restrict__ out) {
+                               __nv_bfloat16* __restrict__ out, int n_rows, unsigned* err) {
   constexpr int kMaxKS = 40;  // top_k + n_shared at most
   __shared__ int s_row[kMaxKS];
   __shared__ float s_w[kMaxKS];
@@ -21,7 +21,7 @@ __global__ void combine_kernel(const float* __restrict__ y, const float* __restr
   // before it lets its dependents launch, so those are complete when this
   // kernel starts, and the loads go ahead of the wait for the down kernel.
   if (threadIdx.x < kS) {
-    s_row[threadIdx.x] = __ldcg(inv + t * kS + threadIdx.x);
+    s_row[threadIdx.x] = in_range(__ldcg(inv + t * kS + threadIdx.x), n_rows, err);
     s_w[threadIdx.x] = threadIdx.x < k ? __ldcg(w + (size_t)t * k + threadIdx.x) : 1.f;
   }
   // launched as a programmatic dependent of the down kernel: wait for it (a
@@ -66,7 +66,7 @@ cudaError_t launch_combine(const Work& wk, int T, const Shape& s, __nv_bfloat16*
   const int threads = 64;  // more, smaller blocks: the combine is latency-bound at small T
   dim3 grid((s.H / 4 + threads - 1) / threads, T);
   if (!pdl) {
-    combine_kernel<<<grid, threads, 0, st>>>(wk.y, wk.w, wk.inv, s.H, s.k, s.S, out);
+    combine_kernel<<<grid, threads, 0, st>>>(wk.y, wk.w, wk.inv, s.H, s.k, s.S, out, T * (s.k + s.S), wk.err);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -79,7 +79,7 @@ cudaError_t launch_combine(const Work& wk, int T, const Shape& s, __nv_bfloat16*
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, combine_kernel, (const float*)wk.y, (const float*)wk.w, (const int*)wk.inv, s.H,
-                            s.k, s.S, out);
+                            s.k, s.S, out, T * (s.k + s.S), wk.err);
 }
 
 }  // namespace moe

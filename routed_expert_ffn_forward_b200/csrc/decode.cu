@@ -166,20 +166,23 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      ptx::IssueLog log;
       for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
         const int ai = unit / tiles, rt = unit - ai * tiles;
-        const int e = __ldcg(a.act + ai);
-        const CUtensorMap* mg = a.tmaps + kMapsPerSlot * __ldcg(a.slot_of + e);
+        const int e = in_range(__ldcg(a.act + ai), a.n_ex, a.err);
+        const CUtensorMap* mg = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + e), a.n_slots, a.err);
         int cnt = 0, tok[kMaxTok];
         if (!kStageX) {
           cnt = __ldcg(a.counts + e);
-          const int r0 = __ldcg(a.offsets + e);
+          const int r0 = in_range(__ldcg(a.offsets + e), a.n_rows, a.err);
 #pragma unroll
-          for (int t = 0; t < kMaxTok; ++t) tok[t] = t < cnt ? __ldcg(a.perm + r0 + t) / a.kS : 0;
+          for (int t = 0; t < kMaxTok; ++t)
+            tok[t] = t < cnt ? in_range(__ldcg(a.perm + in_range(r0 + t, a.n_rows, a.err)) / a.kS, a.T, a.err) : 0;
         }
         for (int st = 0; st < n_st; ++st) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
             flag_error(a.err, 1u);
+            log.drain(full, kGuStages);
             return;
           }
           const int nsb = min(kGuSB, a.nbh - st * kGuSB);  // super-blocks of x this stage needs
@@ -200,12 +203,14 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
               }
             }
           }
+          log.note(stage, phase);
           if (++stage == kGuStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
+      log.drain(full, kGuStages);
     }
     return;
   }
@@ -239,12 +244,13 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
   uint32_t phase = 0;
   for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
     const int ai = unit / tiles, rt = unit - ai * tiles;
-    const int e = __ldcg(a.act + ai);
-    const int cnt = __ldcg(a.counts + e), r0 = __ldcg(a.offsets + e);
+    const int e = in_range(__ldcg(a.act + ai), a.n_ex, a.err);
+    const int cnt = __ldcg(a.counts + e), r0 = in_range(__ldcg(a.offsets + e), a.n_rows, a.err);
     int tok[kMaxTok];
     if (kStageX) {
 #pragma unroll
-      for (int t = 0; t < kMaxTok; ++t) tok[t] = t < cnt ? __ldcg(a.perm + r0 + t) / a.kS : 0;
+      for (int t = 0; t < kMaxTok; ++t)
+        tok[t] = t < cnt ? in_range(__ldcg(a.perm + in_range(r0 + t, a.n_rows, a.err)) / a.kS, a.T, a.err) : 0;
     }
     float acc[kMaxTok], acc8[kMaxTok];
 #pragma unroll
@@ -373,19 +379,23 @@ __global__ void __launch_bounds__(kThreads, 1) down_d1_kernel(DecodeArgs a) {
       int stage = 0, slot = 0;
       uint32_t phase = 0, aphase = 0;
       bool waited = false;
+      ptx::IssueLog log, alog;
       for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
         const int ai = unit / tiles, rt = unit - ai * tiles;
-        const int e = __ldcg(a.act + ai);
-        const CUtensorMap* md = a.tmaps + kMapsPerSlot * __ldcg(a.slot_of + e) + 2;
+        const int e = in_range(__ldcg(a.act + ai), a.n_ex, a.err);
+        const CUtensorMap* md = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + e), a.n_slots, a.err) + 2;
         // weights first: they do not depend on the gate/up kernel
         for (int st = 0; st < n_st; ++st) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
             flag_error(a.err, 4u);
             if (!waited) ptx::pdl_wait();
+            log.drain(full, kDnStages);
+            alog.drain(afull, 2);
             return;
           }
           ptx::mbar_arrive_expect_tx(&full[stage], kDnStageBytes);
           ptx::tma_load_2d(stages + stage * kDnStageBytes, md, st * kDnSB * 18, rt * kTileRows, &full[stage]);
+          log.note(stage, phase);
           if (++stage == kDnStages) {
             stage = 0;
             phase ^= 1u;
@@ -398,9 +408,11 @@ __global__ void __launch_bounds__(kThreads, 1) down_d1_kernel(DecodeArgs a) {
         }
         if (!ptx::mbar_wait(&aempty[slot], aphase ^ 1u)) {
           flag_error(a.err, 4u);
+          log.drain(full, kDnStages);
+          alog.drain(afull, 2);
           return;
         }
-        const int cnt = __ldcg(a.counts + e), r0 = __ldcg(a.offsets + e);
+        const int cnt = __ldcg(a.counts + e), r0 = in_range(__ldcg(a.offsets + e), a.n_rows, a.err);
         const uint32_t nb = (uint32_t)(cnt * a.I_pad);
         const uint32_t sb = (uint32_t)(cnt * hruns * 8);
         uint8_t* dst = s_act + slot * a.act_slot_bytes;
@@ -409,12 +421,15 @@ __global__ void __launch_bounds__(kThreads, 1) down_d1_kernel(DecodeArgs a) {
         ptx::bulk_load(dst, a.hq + ho, nb, &afull[slot]);
         ptx::bulk_load(dst + plane_bytes, a.hq + a.hq_plane + ho, nb, &afull[slot]);
         ptx::bulk_load(dst + 2 * plane_bytes, a.hsc + (size_t)r0 * hruns, sb, &afull[slot]);
+        alog.note(slot, aphase);
         if (++slot == 2) {
           slot = 0;
           aphase ^= 1u;
         }
       }
       if (!waited) ptx::pdl_wait();
+      log.drain(full, kDnStages);
+      alog.drain(afull, 2);
     } else {
       ptx::pdl_wait();
     }
@@ -431,8 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1) down_d1_kernel(DecodeArgs a) {
   uint32_t phase = 0, aphase = 0;
   for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
     const int ai = unit / tiles, rt = unit - ai * tiles;
-    const int e = __ldcg(a.act + ai);
-    const int cnt = __ldcg(a.counts + e), r0 = __ldcg(a.offsets + e);
+    const int e = in_range(__ldcg(a.act + ai), a.n_ex, a.err);
+    const int cnt = __ldcg(a.counts + e), r0 = in_range(__ldcg(a.offsets + e), a.n_rows, a.err);
     float acc[kMaxTok], acc8[kMaxTok];
 #pragma unroll
     for (int t = 0; t < kMaxTok; ++t) acc[t] = acc8[t] = 0.f;

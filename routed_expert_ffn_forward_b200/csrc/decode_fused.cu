@@ -1,0 +1,608 @@
+// Single-token decode (T = 1) as one persistent kernel: router, top-k and
+// gating, gate/up + SwiGLU, down and the weighted combine, with no kernel
+// boundary between the steps.
+//
+// One CTA per SM (16 consumer warps + 1 TMA producer warp).  Steps meet
+// through counters in global memory instead of kernel boundaries, so the
+// weight stream never drains between them:
+//
+//  1. Router.  Each CTA computes the logits of experts blockIdx.x,
+//     blockIdx.x + grid, ... (256 threads per expert row; the constant router
+//     weights are loaded before the kernel waits for its predecessor), then
+//     arrives on a grid-wide barrier.  Every CTA needs the routing, and after
+//     the barrier each one runs the same top-k + gating over the E logits
+//     itself (identical inputs and code, so identical results), which costs
+//     one warp a few hundred cycles and saves a second barrier.
+//  2. Gate/up + SwiGLU.  Unit = (expert j of the token's k + S, 128 weight
+//     rows), the shared experts first: they need no routing, so their CTAs
+//     stream weights from the first cycle, overlapping the router.  A unit
+//     writes its 128 features of h_j (16-bit fixed point per 32-element run)
+//     and adds one to ready[j] (release).
+//  3. Down.  Unit = (expert j, 64 output rows), claimed dynamically from a
+//     counter (shared experts first), so units balance across SMs.  The
+//     producer issues the unit's weights at once and bulk-copies h_j into
+//     shared memory once ready[j] counts every gate/up unit of j (acquire).
+//     The unit writes its 64 rows of y_j (fp32) and adds one to done[tile].
+//  4. Combine.  The unit that completes a 64-row output tile (done[tile]
+//     reaches k + S) sums the tile's y rows in the fixed order j = 0..k-1
+//     (weighted), then the shared experts, rounds to bf16 and writes out:
+//     no atomics on the data, the same order every run (LayerStoRm README,
+//     "Notes": a deterministic expert combine).
+//
+// The dot products are those of the single-token GEMVs (exact integer dp4a
+// sums of the raw Q4_K nibbles against fixed-point activations, fp32
+// epilogue per sub-block; see gemv_dot.cuh).
+//
+// Every wait is bounded (2 s): an mbarrier, the grid barrier, a readiness
+// counter.  A CTA that gives up sets an error bit that moe_check reports; the
+// producer drains every copy it issued before the CTA exits.  The grid
+// barrier assumes every CTA is resident at once: the grid is one CTA per SM
+// and the shared-memory footprint admits one CTA per SM.
+#include "gemv_dot.cuh"
+#include "moe_internal.h"
+#include "ptx.cuh"
+#include "qdot.cuh"
+#include "topk.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kFzWarps = 16;                       // consumer warps
+constexpr int kFzThreads = (kFzWarps + 1) * 32;
+constexpr int kFzConsumers = kFzWarps * 32;
+constexpr int kFzGuRows = 128;                     // gate/up unit: weight rows of gate and of up
+constexpr int kFzDnRows = 64;                      // down unit: output rows
+constexpr int kFzDnSb = 4;                         // 256-weight groups per down stage
+constexpr int kFzStages = 4;                       // at most; a stage is 256 x the group size (Q4_K: 36,864 B)
+constexpr uint64_t kFzLimitNs = 2000000000ull;
+
+// error bits (moe_check): which wait gave up
+constexpr unsigned kErrFzProducer = 1u << 10, kErrFzConsumer = 1u << 11, kErrFzGrid = 1u << 12,
+                   kErrFzReady = 1u << 13;
+
+// global sync words (FusedArgs::sync)
+constexpr int kSyncBarCount = 0, kSyncBarGen = 1, kSyncNext = 2, kSyncReady = 8, kSyncTile = 64;
+
+// Shared-memory layout (offsets from the 1024-aligned base).
+struct FzLayout {
+  uint32_t bars, unit, ids, w, flags, part, xh, xl, xsc, uni, total;
+  __host__ __device__ FzLayout(int H, size_t act_slot, int ring_bytes) {
+    auto up16 = [](uint32_t v) { return (v + 15u) & ~15u; };
+    bars = (uint32_t)ring_bytes;                      // full[4] empty[4] afull[2] aempty[2] route[1]
+    unit = bars + 13 * 8;                             // int [kFzStages]
+    ids = unit + kFzStages * 4;                       // int [40]
+    w = ids + 40 * 4;                                 // float [40]
+    flags = w + 40 * 4;                               // int [4]
+    part = up16(flags + 16);                          // float [1024]
+    xh = part + 1024 * 4;                             // u8 [H]
+    xl = xh + (uint32_t)H;                            // u8 [H]
+    xsc = xl + (uint32_t)H;                           // float2 [H/32]
+    uni = up16(xsc + (uint32_t)(H / 32) * 8);         // bf16 x [H] | act slots [2][act_slot]
+    const uint32_t u1 = (uint32_t)H * 2, u2 = 2 * (uint32_t)act_slot;
+    total = up16(uni + (u1 > u2 ? u1 : u2));
+  }
+};
+
+__device__ __forceinline__ uint8_t* fz_aligned(uint8_t* raw) {
+  const uint32_t pad = (1024u - (ptx::smem_u32(raw) & 1023u)) & 1023u;
+  return raw + pad;
+}
+
+// Spin (one thread) until *p != v (acquire); false after `lim` ns.
+__device__ __forceinline__ bool spin_while_eq(const uint32_t* p, uint32_t v, uint64_t lim) {
+  if (ptx::ld_acquire_gpu(p) != v) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (ptx::ld_acquire_gpu(p) == v) {
+    __nanosleep(64);
+    if (ptx::globaltimer() - t0 > lim) return false;
+  }
+  return true;
+}
+// Spin (one thread) until *p >= v (acquire); false after `lim` ns.
+__device__ __forceinline__ bool spin_until_ge(const uint32_t* p, uint32_t v, uint64_t lim) {
+  if (ptx::ld_acquire_gpu(p) >= v) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (ptx::ld_acquire_gpu(p) < v) {
+    __nanosleep(32);
+    if (ptx::globaltimer() - t0 > lim) return false;
+  }
+  return true;
+}
+
+template <int PL>
+__global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const FusedArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* sm = fz_aligned(smem_raw);
+  const int H = a.H, E = a.E, k = a.k, S = a.S, kS = k + S;
+  const FzLayout lay(H, a.act_slot_bytes, a.stages * a.stage_bytes);
+  const int n_stages = a.stages, stage_bytes = a.stage_bytes;
+  const int gu_box = kFzGuRows * a.sbb_gu, dn_box = kFzDnRows * a.sbb_d;   // bytes of one box
+  const int gu_el = a.sbb_gu / 8, dn_el = a.sbb_d / 8;                    // 8-byte elements per group
+  uint8_t* ring = sm;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + lay.bars);
+  uint64_t* empty = full + kFzStages;
+  uint64_t* afull = empty + kFzStages;
+  uint64_t* aempty = afull + 2;
+  uint64_t* route_ready = aempty + 2;
+  int* s_unit = reinterpret_cast<int*>(sm + lay.unit);
+  int* s_ids = reinterpret_cast<int*>(sm + lay.ids);
+  float* s_w = reinterpret_cast<float*>(sm + lay.w);
+  volatile int* s_flag = reinterpret_cast<volatile int*>(sm + lay.flags);  // [0] abort [1] combine [2] gen
+  float* s_part = reinterpret_cast<float*>(sm + lay.part);
+  uint8_t* s_xh = sm + lay.xh;
+  uint8_t* s_xl = sm + lay.xl;
+  float2* s_xsc = reinterpret_cast<float2*>(sm + lay.xsc);
+  uint8_t* s_uni = sm + lay.uni;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gu_tiles = (a.I + kFzGuRows - 1) / kFzGuRows;
+  const int n_gu = kS * gu_tiles;
+  const int dn_tiles = H / kFzDnRows;
+  const int n_dn = kS * dn_tiles;
+  const int n_dst = (a.nbi + kFzDnSb - 1) / kFzDnSb;  // stages per down unit
+  uint32_t* sync = a.sync;
+  // limit of every wait but the final drain (a test hook may shorten it)
+  const uint64_t lim = a.wait_ns ? a.wait_ns : kFzLimitNs;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < n_stages; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], kFzWarps);
+    }
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&afull[s], 1);
+      ptx::mbar_init(&aempty[s], kFzWarps);
+    }
+    ptx::mbar_init(route_ready, 1);
+    s_flag[0] = 0;
+    s_flag[1] = 0;
+    ptx::fence_barrier_init();
+  }
+  __syncthreads();
+
+  // ------------------------------------------------------------------ producer
+  if (warp == kFzWarps) {
+    if (lane != 0) return;
+    int stage = 0;
+    uint32_t phase = 0, issued = 0, last_par = 0;  // per stage: a copy was issued, its phase parity
+    int aslot = 0;
+    uint32_t aphase = 0, a_issued = 0, a_last = 0;
+    bool routed = false, ok = true;
+    // in streaming mode the expert -> slot table comes from the previous kernel
+    if (!a.early) ptx::pdl_wait();
+    auto expert_of = [&](int j) { return in_range(j < k ? s_ids[j] : E + (j - k), E + S, a.err); };
+    auto next_stage = [&]() {
+      if (++stage == n_stages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    };
+    // gate/up: static units blockIdx.x, + grid, ...; the shared experts first
+    for (int u = blockIdx.x; u < n_gu && ok; u += gridDim.x) {
+      const int jj = u / gu_tiles, rt = u - jj * gu_tiles;
+      const int j = jj < S ? k + jj : jj - S;
+      if (j < k && !routed) {
+        if (!ptx::mbar_wait_sleep(route_ready, 0, 64, lim)) {
+          ok = false;
+          break;
+        }
+        routed = true;
+      }
+      const CUtensorMap* m = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + expert_of(j)), a.n_slots, a.err) + 3;
+      for (int kb = 0; kb < a.nbh; ++kb) {
+        if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, lim)) {
+          ok = false;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * gu_box));
+        uint8_t* dst = ring + stage * stage_bytes;
+        ptx::tma_load_2d(dst, m, kb * gu_el, rt * kFzGuRows, &full[stage]);
+        ptx::tma_load_2d(dst + gu_box, m + 1, kb * gu_el, rt * kFzGuRows, &full[stage]);
+        issued |= 1u << stage;
+        last_par = (last_par & ~(1u << stage)) | (phase << stage);
+        next_stage();
+      }
+    }
+    // down: units claimed from a counter that CTA 0 zeroed before the grid
+    // barrier; the routing (and so that zeroing) is known once route_ready fires
+    if (ok && !routed) {
+      ok = ptx::mbar_wait_sleep(route_ready, 0, 64, lim);
+      routed = ok;
+    }
+    while (ok) {
+      if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, lim)) {
+        ok = false;
+        break;
+      }
+      const int u = (int)atomicAdd(sync + kSyncNext, 1u);
+      if (u >= n_dn) {
+        s_unit[stage] = -1;          // end of work
+        ptx::mbar_arrive(&full[stage]);
+        break;
+      }
+      const int jj = u / dn_tiles, rt = u - jj * dn_tiles;
+      const int j = jj < S ? k + jj : jj - S;
+      const CUtensorMap* md = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + expert_of(j)), a.n_slots, a.err) + 6;
+      for (int st = 0; st < n_dst; ++st) {
+        if (st > 0 && !ptx::mbar_wait(&empty[stage], phase ^ 1u, lim)) {
+          ok = false;
+          break;
+        }
+        const int nbox = min(kFzDnSb, a.nbi - st * kFzDnSb);
+        s_unit[stage] = u;
+        ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(nbox * dn_box));
+        uint8_t* dst = ring + stage * stage_bytes;
+        for (int b = 0; b < nbox; ++b)
+          ptx::tma_load_2d(dst + b * dn_box, md, (st * kFzDnSb + b) * dn_el, rt * kFzDnRows, &full[stage]);
+        issued |= 1u << stage;
+        last_par = (last_par & ~(1u << stage)) | (phase << stage);
+        next_stage();
+      }
+      if (!ok) break;
+      // h_j, once every gate/up unit of expert j has published its features
+      if (!ptx::mbar_wait(&aempty[aslot], aphase ^ 1u, lim)) {
+        ok = false;
+        break;
+      }
+      if (!spin_until_ge(sync + kSyncReady + j, (uint32_t)gu_tiles, lim)) {
+        atomicOr(a.err, kErrFzReady);
+        ok = false;
+        break;
+      }
+      ptx::fence_proxy_async_global();  // generic-proxy writes of h, read below by the bulk copy
+      const int I_pad = a.I_pad, hruns = I_pad / 32;
+      uint8_t* adst = s_uni + aslot * a.act_slot_bytes;
+      ptx::mbar_arrive_expect_tx(&afull[aslot], (uint32_t)(2 * I_pad + hruns * 8));
+      ptx::bulk_load(adst, a.hq + (size_t)j * I_pad, (uint32_t)I_pad, &afull[aslot]);
+      ptx::bulk_load(adst + I_pad, a.hq + a.hq_plane + (size_t)j * I_pad, (uint32_t)I_pad, &afull[aslot]);
+      ptx::bulk_load(adst + 2 * I_pad, a.hsc + (size_t)j * hruns, (uint32_t)(hruns * 8), &afull[aslot]);
+      a_issued |= 1u << aslot;
+      a_last = (a_last & ~(1u << aslot)) | (aphase << aslot);
+      if (++aslot == 2) {
+        aslot = 0;
+        aphase ^= 1u;
+      }
+    }
+    if (!ok) atomicOr(a.err, kErrFzProducer);
+    // never leave with a copy into shared memory in flight
+    for (int s = 0; s < n_stages; ++s)
+      if ((issued >> s) & 1u) ptx::mbar_wait(&full[s], (last_par >> s) & 1u);
+    for (int s = 0; s < 2; ++s)
+      if ((a_issued >> s) & 1u) ptx::mbar_wait(&afull[s], (a_last >> s) & 1u);
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int tid = threadIdx.x;
+  // every consumer warp reaches every cbar() (all waits are bounded and every
+  // decision to stop is taken from s_flag right after one), so none is left
+  // waiting on a named barrier
+  auto cbar = [] {
+    __syncwarp();
+    ptx::named_barrier_sync(1, kFzConsumers);
+  };
+  auto fail = [&](unsigned bit) {
+    atomicOr(a.err, bit);
+    s_flag[0] = 1;
+  };
+
+  // (1) router logits: two expert rows at a time (warps 0-7 and 8-15); a
+  // thread takes the float4 pieces ht + 256 i of its row, 8 per pass, all
+  // loaded before any arithmetic
+  {
+    const int half = warp >> 3, ht = tid & 255;
+    const int nq = H / 4;                                 // float4 pieces per row
+    constexpr int kPieces = 8;
+    __nv_bfloat16* s_x = reinterpret_cast<__nv_bfloat16*>(s_uni);
+    const uint2* xv = reinterpret_cast<const uint2*>(s_x);
+    bool first = true;
+    for (int e0 = blockIdx.x; e0 < E; e0 += 2 * gridDim.x) {
+      const int e = e0 + half * gridDim.x;
+      const float4* wrow = reinterpret_cast<const float4*>(a.W + (size_t)min(e, E - 1) * H);
+      float acc = 0.f;
+      for (int base = 0; base < nq; base += kPieces * 256) {
+        float4 w4[kPieces];
+#pragma unroll
+        for (int i = 0; i < kPieces; ++i) {
+          const int q = base + ht + 256 * i;
+          if (e < E && q < nq) w4[i] = __ldg(wrow + q);
+        }
+        if (first) {
+          // x comes from the previous kernel (or the caller): wait, then stage
+          // it; the constant router weights above are already in flight
+          ptx::pdl_wait();
+          const uint4* src = reinterpret_cast<const uint4*>(a.x);
+          for (int i = tid; i < H / 8; i += kFzConsumers) reinterpret_cast<uint4*>(s_x)[i] = __ldcg(src + i);
+          cbar();
+          first = false;
+        }
+#pragma unroll
+        for (int i = 0; i < kPieces; ++i) {
+          const int q = base + ht + 256 * i;
+          if (e < E && q < nq) {
+            const uint2 v = xv[q];
+            acc = fmaf(w4[i].x, bf16lo(v.x), acc);
+            acc = fmaf(w4[i].y, bf16hi(v.x), acc);
+            acc = fmaf(w4[i].z, bf16lo(v.y), acc);
+            acc = fmaf(w4[i].w, bf16hi(v.y), acc);
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) s_part[warp] = acc;
+      cbar();
+      if ((warp & 7) == 0 && lane == 0 && e < E) {
+        float v = 0.f;
+#pragma unroll
+        for (int w8 = 0; w8 < 8; ++w8) v += s_part[half * 8 + w8];
+        a.logits[e] = v + (a.b ? a.b[e] : 0.f);
+      }
+      cbar();
+    }
+    if (first) {  // no expert row here: still wait for x
+      ptx::pdl_wait();
+      const uint4* src = reinterpret_cast<const uint4*>(a.x);
+      for (int i = tid; i < H / 8; i += kFzConsumers) reinterpret_cast<uint4*>(s_x)[i] = __ldcg(src + i);
+    }
+    // CTA 0 zeroes the step counters for this launch before it arrives: no
+    // CTA touches them until it has passed the barrier
+    if (blockIdx.x == 0) {
+      if (tid == 0) sync[kSyncNext] = 0u;
+      for (int i = tid; i < kS; i += kFzConsumers) sync[kSyncReady + i] = 0u;
+      for (int i = tid; i < dn_tiles; i += kFzConsumers) sync[kSyncTile + i] = 0u;
+    }
+    __threadfence();
+    cbar();
+    if (tid == 0) {
+      const uint32_t gen = ptx::ld_acquire_gpu(sync + kSyncBarGen);
+      s_flag[2] = (int)gen;
+      __threadfence();
+      const uint32_t old = atomicAdd(sync + kSyncBarCount, 1u);
+      if (old == gridDim.x - 1 + (uint32_t)a.hold) {   // hold > 0 (a test hook): never released
+        sync[kSyncBarCount] = 0u;      // ready for the next launch
+        __threadfence();
+        ptx::st_release_gpu(sync + kSyncBarGen, gen + 1u);
+      }
+    }
+  }
+
+  // (2) x as 16-bit fixed point per 32-element run (each CTA its own copy)
+  {
+    const __nv_bfloat16* s_x = reinterpret_cast<const __nv_bfloat16*>(s_uni);
+    for (int run = warp; run < H / 32; run += kFzWarps) {
+      float2 rsc;
+      int8_t xh;
+      uint8_t xl;
+      quant_run16(__bfloat162float(s_x[run * 32 + lane]), xh, xl, rsc);
+      s_xh[run * 32 + lane] = (uint8_t)xh;
+      s_xl[run * 32 + lane] = xl;
+      if (lane == 0) s_xsc[run] = rsc;
+    }
+    cbar();
+  }
+
+  // the routing: every CTA selects from the E logits itself, after the barrier
+  bool routed = false;
+  auto route = [&]() {
+    if (tid == 0) {
+      if (!spin_while_eq(sync + kSyncBarGen, (uint32_t)s_flag[2], lim)) fail(kErrFzGrid);
+    }
+    cbar();
+    if (!s_flag[0] && warp == 0) {
+      warp_topk_gate<PL, true>(a.logits, E, k, a.gating, a.forced, s_ids, s_w);
+      __syncwarp();
+      if (lane < S) {
+        s_ids[k + lane] = E + lane;
+        s_w[k + lane] = 1.f;
+      }
+      if (blockIdx.x == 0 && lane < k) {
+        a.ids[lane] = s_ids[lane];
+        a.w[lane] = s_w[lane];
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(route_ready);
+    }
+    cbar();
+    routed = true;
+  };
+
+  int stage = 0;
+  uint32_t phase = 0;
+  auto next_stage = [&]() {
+    if (++stage == n_stages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  };
+
+  // (3) gate/up + SwiGLU units
+  {
+    const int c = warp >> 2, row = (warp & 3) * 32 + lane;
+    for (int u = blockIdx.x; u < n_gu; u += gridDim.x) {
+      const int jj = u / gu_tiles, rt = u - jj * gu_tiles;
+      const int j = jj < S ? k + jj : jj - S;
+      if (j < k && !routed) {
+        route();
+        if (s_flag[0]) return;
+      }
+      float acc[2] = {0.f, 0.f};  // gate row, up row
+      bool ok = true;
+      for (int kb = 0; kb < a.nbh; ++kb) {
+        if (!ptx::mbar_wait(&full[stage], phase, lim)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* bg = ring + stage * stage_bytes + row * a.sbb_gu;
+        const uint8_t* const blk[2] = {bg, bg + gu_box};
+        const uint8_t *xh = s_xh + kb * kQK, *xl = s_xl + kb * kQK;
+        const float2* xs = s_xsc + kb * 8;
+        switch (a.qgu) {   // uniform across the CTA
+          case kQ5_K: q_chunk_rows<kQ5_K, 2>(blk, c, xh, xl, xs, acc); break;
+          case kQ6_K: q_chunk_rows<kQ6_K, 2>(blk, c, xh, xl, xs, acc); break;
+          case kQ8_0: q_chunk_rows<kQ8_0, 2>(blk, c, xh, xl, xs, acc); break;
+          case kMXFP4: q_chunk_rows<kMXFP4, 2>(blk, c, xh, xl, xs, acc); break;
+          default: q_chunk_rows<kQ4_K, 2>(blk, c, xh, xl, xs, acc); break;
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&empty[stage]);
+        next_stage();
+      }
+      if (!ok) fail(kErrFzConsumer);
+      cbar();
+      if (s_flag[0]) return;
+      s_part[c * kFzGuRows + row] = acc[0];
+      s_part[(4 + c) * kFzGuRows + row] = acc[1];
+      cbar();
+      // SwiGLU (chunk parts summed in a fixed order) -> h_j, warps 0-3
+      if (warp < 4) {
+        const int f = warp * 32 + lane;
+        const float* pg = s_part + f;
+        const float* pu = s_part + 4 * kFzGuRows + f;
+        const float g = ((pg[0] + pg[kFzGuRows]) + pg[2 * kFzGuRows]) + pg[3 * kFzGuRows];
+        const float up = ((pu[0] + pu[kFzGuRows]) + pu[2 * kFzGuRows]) + pu[3 * kFzGuRows];
+        float2 rsc;
+        int8_t hh;
+        uint8_t hl;
+        quant_run16(silu_f(g) * up, hh, hl, rsc);
+        const int feat = rt * kFzGuRows + f;
+        const size_t o = (size_t)j * a.I_pad + feat;
+        a.hq[o] = hh;
+        reinterpret_cast<uint8_t*>(a.hq + a.hq_plane)[o] = hl;
+        if (lane == 0) a.hsc[(size_t)j * (a.I_pad / 32) + feat / 32] = rsc;
+        __threadfence();
+      }
+      // publish the features (the ready counters are zeroed before the barrier)
+      if (!routed) {
+        route();
+        if (s_flag[0]) return;
+      } else {
+        cbar();
+      }
+      if (tid == 0) {
+        ptx::fence_proxy_async_global();
+        ptx::red_add_release_gpu(sync + kSyncReady + j, 1u);
+      }
+    }
+  }
+  if (!routed) {
+    route();
+    if (s_flag[0]) return;
+  }
+
+  // (4) down units, then the combine of each completed output tile
+  {
+    const int r0 = lane, sb = warp >> 2, c = warp & 3;   // rows lane and lane + 32; part = warp
+    const int I_pad = a.I_pad;
+    int aslot = 0;
+    uint32_t aphase = 0;
+    while (true) {
+      bool ok = ptx::mbar_wait(&full[stage], phase, lim);
+      const int u = ok ? s_unit[stage] : -1;   // -1 from the producer: end of work
+      const int jj = u / dn_tiles, rt = u - jj * dn_tiles;
+      const int j = jj < S ? k + jj : jj - S;
+      float acc[2] = {0.f, 0.f};
+      if (ok && u >= 0) {
+        ok = ptx::mbar_wait(&afull[aslot], aphase, lim);
+        const uint8_t* act = s_uni + aslot * a.act_slot_bytes;
+        const float2* asc = reinterpret_cast<const float2*>(act + 2 * I_pad);
+        for (int st = 0; st < n_dst && ok; ++st) {
+          if (st > 0 && !ptx::mbar_wait(&full[stage], phase, lim)) {
+            ok = false;
+            break;
+          }
+          const int kb = st * kFzDnSb + sb;
+          if (kb < a.nbi) {
+            const uint8_t* b0 = ring + stage * stage_bytes + sb * dn_box + r0 * a.sbb_d;
+            const uint8_t* const blk[2] = {b0, b0 + 32 * a.sbb_d};
+            const uint8_t *xh = act + kb * kQK, *xl = act + I_pad + kb * kQK;
+            const float2* xs = asc + kb * 8;
+            switch (a.qd) {   // uniform across the CTA
+              case kQ5_K: q_chunk_rows<kQ5_K, 2>(blk, c, xh, xl, xs, acc); break;
+              case kQ6_K: q_chunk_rows<kQ6_K, 2>(blk, c, xh, xl, xs, acc); break;
+              case kQ8_0: q_chunk_rows<kQ8_0, 2>(blk, c, xh, xl, xs, acc); break;
+              case kMXFP4: q_chunk_rows<kMXFP4, 2>(blk, c, xh, xl, xs, acc); break;
+              default: q_chunk_rows<kQ4_K, 2>(blk, c, xh, xl, xs, acc); break;
+            }
+          }
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&empty[stage]);
+          next_stage();
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&aempty[aslot]);
+        if (++aslot == 2) {
+          aslot = 0;
+          aphase ^= 1u;
+        }
+      }
+      if (!ok) fail(kErrFzConsumer);
+      cbar();                          // also: the previous unit's reads of s_part are done
+      if (s_flag[0]) return;
+      if (u < 0) break;                // every warp read the same end marker
+      s_part[warp * kFzDnRows + r0] = acc[0];
+      s_part[warp * kFzDnRows + r0 + 32] = acc[1];
+      cbar();
+      // the 16 parts of each row, in a fixed order, to y_j
+      const int o0 = rt * kFzDnRows;
+      if (warp < 2) {
+        const int r = warp * 32 + lane;
+        float v = s_part[r];
+#pragma unroll
+        for (int p = 1; p < kFzWarps; ++p) v += s_part[p * kFzDnRows + r];
+        a.y[(size_t)j * H + o0 + r] = v;
+        __threadfence();
+      }
+      cbar();
+      if (tid == 0) s_flag[1] = ptx::atom_add_acq_rel_gpu(sync + kSyncTile + rt, 1u) == (uint32_t)(kS - 1);
+      cbar();
+      if (s_flag[1] && warp < 2) {
+        // last contribution to this tile: out = sum_j w_j y_j (+ shared), fixed order
+        const int o = o0 + warp * 32 + lane;
+        float acc2 = 0.f;
+        for (int q = 0; q < k; ++q) acc2 = fmaf(s_w[q], __ldcg(a.y + (size_t)q * H + o), acc2);
+        for (int q = k; q < kS; ++q) acc2 += __ldcg(a.y + (size_t)q * H + o);
+        a.out[o] = __float2bfloat16_rn(acc2);
+      }
+    }
+  }
+  ptx::pdl_launch_dependents();
+}
+
+}  // namespace
+
+size_t decode1_fused_smem(int H, size_t act_slot_bytes, int ring_bytes) {
+  return 1024 + FzLayout(H, act_slot_bytes, ring_bytes).total;
+}
+
+cudaError_t launch_decode1_fused(const FusedArgs& a, int n_sm, cudaStream_t st) {
+  static uint64_t attr_done[2] = {0, 0};
+  const size_t smem = decode1_fused_smem(a.H, a.act_slot_bytes, a.stages * a.stage_bytes);
+  if (smem > kMaxDecodeSmem || a.T != 1 || a.k + a.S > 40 || a.H % kFzDnRows || a.H > 16384 || a.E > 1024 ||
+      a.stages < 2 || a.stages > kFzStages || a.stage_bytes < 256 * std::max(a.sbb_gu, a.sbb_d))
+    return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  const bool small_e = a.E <= 256;
+  auto kern = small_e ? decode1_fused_kernel<8> : decode1_fused_kernel<32>;
+  uint64_t& done = attr_done[small_e ? 0 : 1];
+  if (!(done & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxDecodeSmem);
+    if (e != cudaSuccess) return e;
+    done |= bit;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_sm);
+  cfg.blockDim = dim3(kFzThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+}  // namespace moe

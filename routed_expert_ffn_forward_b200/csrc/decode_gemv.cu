@@ -28,6 +28,7 @@
 // parts of a row meet in shared memory in a fixed order.
 #include "moe_internal.h"
 #include "ptx.cuh"
+#include "gemv_dot.cuh"
 #include "q4k_decode.cuh"
 
 namespace moe {
@@ -41,59 +42,9 @@ constexpr int kGvBox = kGvRows * kQBytes;       // one 128-row x 1 super-block b
 constexpr int kGvStageBytes = 2 * kGvBox;       // gate/up: gate + up; down: two super-blocks
 constexpr int kGvStages = 4;
 
-__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {  // u8 x s8
-  int d;
-  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {  // u8 x u8
-  int d;
-  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
 __device__ __forceinline__ uint8_t* gv_aligned(uint8_t* raw) {
   const uint32_t pad = (1024u - (ptx::smem_u32(raw) & 1023u)) & 1023u;
   return raw + pad;
-}
-
-// Chunk c of R rows' super-blocks (blk[r]: the rows' 144-byte blocks) against
-// one token's activations of that super-block: xh/xl the 256 high/low
-// activation bytes, sc the eight runs' (2^-s, X).  The chunk's activations are
-// loaded once for the R rows.  Adds row r's partial dot product to acc[r].
-template <int R>
-__device__ __forceinline__ void gv_chunk_rows(const uint8_t* const (&blk)[R], int c, const uint8_t* xh,
-                                              const uint8_t* xl, const float2* sc, float (&acc)[R]) {
-  // activations: sub-block 2c at bytes 64c..64c+31, sub-block 2c+1 at 64c+32..
-  const uint4* ph = reinterpret_cast<const uint4*>(xh + 64 * c);
-  const uint4* pl = reinterpret_cast<const uint4*>(xl + 64 * c);
-  const uint4 h0 = ph[0], h1 = ph[1], h2 = ph[2], h3 = ph[3];
-  const uint4 l0 = pl[0], l1 = pl[1], l2 = pl[2], l3 = pl[3];
-  const uint32_t xhl[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-  const uint32_t xhh[8] = {h2.x, h2.y, h2.z, h2.w, h3.x, h3.y, h3.z, h3.w};
-  const uint32_t xll[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-  const uint32_t xlh[8] = {l2.x, l2.y, l2.z, l2.w, l3.x, l3.y, l3.z, l3.w};
-  const float2 sl = sc[2 * c], sh = sc[2 * c + 1];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const uint4 hdr = *reinterpret_cast<const uint4*>(blk[r]);
-    const uint4 qa = *reinterpret_cast<const uint4*>(blk[r] + 16 + 32 * c);
-    const uint4 qb = *reinterpret_cast<const uint4*>(blk[r] + 32 + 32 * c);
-    const uint32_t q[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-    int chl = 0, cll = 0, chh = 0, clh = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      // high nibbles left in place: 16x the quant, so the sums are 16x too
-      const uint32_t lo = q[k] & 0x0F0F0F0Fu, hi = q[k] & 0xF0F0F0F0u;
-      chl = dp4a_us(lo, xhl[k], chl);
-      cll = dp4a_uu(lo, xll[k], cll);
-      chh = dp4a_us(hi, xhh[k], chh);
-      clh = dp4a_uu(hi, xlh[k], clh);
-    }
-    const RowScales rs = decode_scales(hdr, c);
-    acc[r] += rs.s_lo * sl.x * (float)(chl * 256 + cll) + (rs.s_hi * 0.0625f) * sh.x * (float)(chh * 256 + clh) -
-              (rs.m_lo * sl.y + rs.m_hi * sh.y);
-  }
 }
 
 // ============================================================================ gate/up
@@ -127,24 +78,29 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(DecodeArgs 
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      ptx::IssueLog log;
       for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
         const int ai = unit / tiles, rt = unit - ai * tiles;
-        const CUtensorMap* m = a.tmaps + kMapsPerSlot * __ldcg(a.slot_of + __ldcg(a.act + ai)) + 3;
+        const int e = in_range(__ldcg(a.act + ai), a.n_ex, a.err);
+        const CUtensorMap* m = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + e), a.n_slots, a.err) + 3;
         for (int kb = 0; kb < a.nbh; ++kb) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
             atomicOr(a.err, 1u);
+            log.drain(full, kGvStages);
             return;
           }
           ptx::mbar_arrive_expect_tx(&full[stage], kGvStageBytes);
           uint8_t* dst = stages + stage * kGvStageBytes;
           ptx::tma_load_2d(dst, m, kb * 18, rt * kGvRows, &full[stage]);
           ptx::tma_load_2d(dst + kGvBox, m + 1, kb * 18, rt * kGvRows, &full[stage]);
+          log.note(stage, phase);
           if (++stage == kGvStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
+      log.drain(full, kGvStages);
     }
     return;
   }
@@ -174,8 +130,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(DecodeArgs 
   uint32_t phase = 0;
   for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
     const int ai = unit / tiles, rt = unit - ai * tiles;
-    const int e = __ldcg(a.act + ai);
-    const int r0 = __ldcg(a.offsets + e);
+    const int e = in_range(__ldcg(a.act + ai), a.n_ex, a.err);
+    const int r0 = in_range(__ldcg(a.offsets + e), a.n_rows, a.err);
     float acc[2] = {0.f, 0.f};  // gate, up
     bool ok = true;
     for (int kb = 0; kb < a.nbh; ++kb) {
@@ -265,16 +221,18 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
       int stage = 0, slot = 0;
       uint32_t phase = 0, aphase = 0;
       bool waited = false;
+      ptx::IssueLog log, alog;
       // The unit's activations (h of the expert's token, written by the
       // gate/up kernel: both byte planes and the run scales) go to a slot.
       auto load_act = [&](int e) -> bool {
         if (!ptx::mbar_wait(&aempty[slot], aphase ^ 1u)) return false;
-        const int r0 = __ldcg(a.offsets + e);
+        const int r0 = in_range(__ldcg(a.offsets + e), a.n_rows, a.err);
         uint8_t* dst = s_act + slot * slot_bytes;
         ptx::mbar_arrive_expect_tx(&afull[slot], (uint32_t)(2 * I_pad + hruns * 8));
         ptx::bulk_load(dst, a.hq + (size_t)r0 * I_pad, (uint32_t)I_pad, &afull[slot]);
         ptx::bulk_load(dst + I_pad, a.hq + a.hq_plane + (size_t)r0 * I_pad, (uint32_t)I_pad, &afull[slot]);
         ptx::bulk_load(dst + 2 * I_pad, a.hsc + (size_t)r0 * hruns, (uint32_t)(hruns * 8), &afull[slot]);
+        alog.note(slot, aphase);
         if (++slot == 2) {
           slot = 0;
           aphase ^= 1u;
@@ -283,12 +241,14 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
       };
       for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
         const int ai = unit / tiles, rt = unit - ai * tiles;
-        const int e = __ldcg(a.act + ai);
-        const CUtensorMap* md = a.tmaps + kMapsPerSlot * __ldcg(a.slot_of + e) + 5;
+        const int e = in_range(__ldcg(a.act + ai), a.n_ex, a.err);
+        const CUtensorMap* md = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + e), a.n_slots, a.err) + 5;
         // Once the gate/up kernel is complete, a unit's activations are issued
         // before its weights, so they never hold up the unit's first stage.
         if (waited && !load_act(e)) {
           atomicOr(a.err, 4u);
+          log.drain(full, kGvStages);
+          alog.drain(afull, 2);
           return;
         }
         // the first unit's weights do not depend on the gate/up kernel: they
@@ -297,6 +257,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
             atomicOr(a.err, 4u);
             if (!waited) ptx::pdl_wait();
+            log.drain(full, kGvStages);
+            alog.drain(afull, 2);
             return;
           }
           ptx::mbar_arrive_expect_tx(&full[stage], kGvStageBytes);
@@ -304,6 +266,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
           // a second box past the last super-block reads zeros (never used)
           ptx::tma_load_2d(dst, md, (2 * st) * 18, rt * kGvRows, &full[stage]);
           ptx::tma_load_2d(dst + kGvBox, md, (2 * st + 1) * 18, rt * kGvRows, &full[stage]);
+          log.note(stage, phase);
           if (++stage == kGvStages) {
             stage = 0;
             phase ^= 1u;
@@ -314,11 +277,15 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
           waited = true;
           if (!load_act(e)) {
             atomicOr(a.err, 4u);
+            log.drain(full, kGvStages);
+            alog.drain(afull, 2);
             return;
           }
         }
       }
       if (!waited) ptx::pdl_wait();
+      log.drain(full, kGvStages);
+      alog.drain(afull, 2);
     } else {
       ptx::pdl_wait();
     }
@@ -336,8 +303,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
   uint32_t phase = 0, aphase = 0;
   for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
     const int ai = unit / tiles, rt = unit - ai * tiles;
-    const int e = __ldcg(a.act + ai);
-    const int r0 = __ldcg(a.offsets + e);
+    const int e = in_range(__ldcg(a.act + ai), a.n_ex, a.err);
+    const int r0 = in_range(__ldcg(a.offsets + e), a.n_rows, a.err);
     float acc[2] = {0.f, 0.f};  // rows row, row + 64
     bool ok = ptx::mbar_wait(&afull[slot], aphase);
     if (!ok) atomicOr(a.err, 8u);

@@ -25,6 +25,8 @@
 #include <unordered_map>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/moe.h"
 #include "moe_internal.h"
 
@@ -33,6 +35,16 @@ using namespace moe;
 namespace {
 
 thread_local std::string g_err;
+
+// NVTX range for the duration of a scope: the host-side steps of a forward
+// (routing read-back, cache resolution, launches) show up on a timeline
+// under a profiler; without one a push/pop costs a few nanoseconds.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 moe_status fail(moe_status s, const char* fmt, ...) {
   char buf[512];
@@ -67,6 +79,9 @@ constexpr int kMaxTokens = 32768;
 std::mutex g_mu;            // guards the cache, the stats and the budget
 moe_stats g_stats{};
 size_t g_cache_bytes = SIZE_MAX;
+int g_cache_policy = MOE_CACHE_LRU;
+uint64_t g_hook_wait_ns = 0;  // moe_set_test_hooks
+int g_hook_hold = 0;
 uint32_t g_next_layer_id = 1;
 
 struct Slot {
@@ -89,7 +104,20 @@ struct Cache {
   cudaStream_t copy = nullptr;
   uint64_t epoch = 0;
   uint64_t gen = 0;  // changes whenever the arena is (re)allocated
+  // MOE_CACHE_LFU bookkeeping for every (layer, expert) key seen, cached or
+  // not: how often it entered use (used by a forward of its layer after not
+  // being used by that layer's previous forward), and the layer's forward
+  // index at its last use.  Arrival counts halve every kAgeEvery * n_slots
+  // arrivals, so that old popularity fades.
+  struct Use {
+    uint32_t arrivals = 0;
+    uint64_t last_fwd = 0;
+  };
+  std::unordered_map<uint64_t, Use> use;
+  std::unordered_map<uint32_t, uint64_t> layer_fwds;  // layer id -> forwards resolved so far
+  uint64_t arrivals = 0;
 };
+constexpr uint64_t kAgeEvery = 64;
 Cache* g_cache = nullptr;
 uint64_t g_cache_gen = 0;
 
@@ -140,7 +168,8 @@ struct moe_layer {
   uint32_t id = 0;
   int device = 0;
   Shape s{};
-  size_t gate_bytes = 0, down_bytes = 0, expert_bytes = 0;
+  size_t gate_bytes = 0, down_bytes = 0, expert_bytes = 0;  // device bytes (a cache slot: expert_bytes)
+  size_t host_expert_bytes = 0;                              // GGUF bytes of one expert in host memory
   moe_gating gating = MOE_GATE_SIGMOID_RENORM;
   bool router_set = false, experts_set = false, resident = false;
   float* d_W = nullptr;
@@ -213,7 +242,7 @@ moe_status ensure_scratch(moe_layer* L, int T, cudaStream_t st) {
                o_act2 = take(ES * 4), o_nact1 = take(4), o_nact2 = take(4),
                o_err = take(4), o_tiles = take(prefill_max_tiles((int)ES, P) * 16), o_ntiles = take(4),
                o_x16 = take(P * s.H * 2), o_rinv = take(P * 4), o_h16 = take(P * s.I_pad * 2), o_hinv = take(P * 4),
-               o_rpart = take(router_part_floats(cap, s.E, s.n_sm) * 4);
+               o_rpart = take(router_part_floats(cap, s.E, s.n_sm) * 4), o_sync = take(kSyncWords * 4);
   if (L->scratch) {
     MOE_TRY(wait_layer(L));
     cudaFree(L->scratch);
@@ -260,6 +289,7 @@ moe_status ensure_scratch(moe_layer* L, int T, cudaStream_t st) {
   L->wk.h16 = reinterpret_cast<__half*>(b + o_h16);
   L->wk.hinv = reinterpret_cast<float*>(b + o_hinv);
   L->wk.rpart = reinterpret_cast<float*>(b + o_rpart);
+  L->wk.sync = reinterpret_cast<unsigned*>(b + o_sync);
   if (encode_act16(&L->x16_map, L->wk.x16, P, s.H) != cudaSuccess ||
       encode_act16(&L->h16_map, L->wk.h16, P, s.I_pad) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activation maps");
@@ -325,21 +355,47 @@ moe_status cache_fetch(moe_layer* L, int e, uint64_t pin_epoch, bool prefetch, i
   const uint64_t key = slot_key(L, e);
   auto it = c->where.find(key);
   int s;
+  if (!prefetch && g_cache_policy == MOE_CACHE_LFU) {
+    const uint64_t f = c->layer_fwds[L->id];
+    Cache::Use& u = c->use[key];
+    if (u.last_fwd == 0 || f - u.last_fwd > 1) {
+      u.arrivals++;
+      if (++c->arrivals % (kAgeEvery * (uint64_t)c->n_slots) == 0)
+        for (auto& kv : c->use) kv.second.arrivals >>= 1;
+    }
+    u.last_fwd = f;
+  }
   if (it != c->where.end()) {
     s = it->second;
     if (!prefetch) g_stats.cache_hits++;
   } else {
-    // victim: least recently used slot not needed by the current forward
+    // victim, among the slots not needed by the current forward: LRU takes
+    // the least recently used.  LFU takes an empty slot if there is one, else
+    // prefers experts not used by their layer's previous forward and among
+    // those the one that entered use least often; the least recently used
+    // among equals
     int victim = -1;
+    uint64_t best = UINT64_MAX;
     for (auto r = c->lru.rbegin(); r != c->lru.rend(); ++r) {
       if (c->slots[*r].epoch != c->epoch || c->epoch == 0) {
-        victim = *r;
-        break;
+        const uint64_t k2 = c->slots[*r].key;
+        if (g_cache_policy != MOE_CACHE_LFU || k2 == UINT64_MAX) {
+          victim = *r;
+          break;
+        }
+        const Cache::Use& u = c->use[k2];
+        const bool recent = u.last_fwd != 0 && c->layer_fwds[(uint32_t)(k2 >> 32)] - u.last_fwd < 2;
+        const uint64_t score = ((uint64_t)recent << 32) | u.arrivals;
+        if (score < best) {
+          best = score;
+          victim = *r;
+        }
       }
     }
     if (victim < 0)
       return fail(MOE_ERR_CACHE_TOO_SMALL, "one forward needs more than the %d cache slots", c->n_slots);
     s = victim;
+    NvtxRange nv(prefetch ? "moe.prefetch_copy" : "moe.miss_copy");
     Slot& sl = c->slots[s];
     if (sl.key != UINT64_MAX) {
       c->where.erase(sl.key);
@@ -348,14 +404,15 @@ moe_status cache_fetch(moe_layer* L, int e, uint64_t pin_epoch, bool prefetch, i
     if (sl.used_rec) CUDA_TRY(cudaStreamWaitEvent(c->copy, sl.used, 0));
     uint8_t* dst = c->arena + (size_t)s * c->slot_bytes;
     const uint8_t* const* hp = &L->host[3 * (size_t)e];
-    CUDA_TRY(cudaMemcpyAsync(dst, hp[0], L->gate_bytes, cudaMemcpyHostToDevice, c->copy));
-    CUDA_TRY(cudaMemcpyAsync(dst + L->gate_bytes, hp[1], L->gate_bytes, cudaMemcpyHostToDevice, c->copy));
-    CUDA_TRY(cudaMemcpyAsync(dst + 2 * L->gate_bytes, hp[2], L->down_bytes, cudaMemcpyHostToDevice, c->copy));
+    const Shape& sh = L->s;
+    CUDA_TRY(copy_matrix_h2d(dst, hp[0], sh.I, sh.qgu, sh.hrow_gu, sh.drow_gu, c->copy));
+    CUDA_TRY(copy_matrix_h2d(dst + L->gate_bytes, hp[1], sh.I, sh.qgu, sh.hrow_gu, sh.drow_gu, c->copy));
+    CUDA_TRY(copy_matrix_h2d(dst + 2 * L->gate_bytes, hp[2], sh.H, sh.qd, sh.hrow_d, sh.drow_d, c->copy));
     CUDA_TRY(cudaEventRecord(sl.ready, c->copy));
     sl.ready_rec = true;
     sl.key = key;
     c->where[key] = s;
-    g_stats.h2d_bytes += L->expert_bytes;
+    g_stats.h2d_bytes += L->host_expert_bytes;
     if (prefetch)
       g_stats.prefetches++;
     else
@@ -374,7 +431,7 @@ moe_status cache_fetch(moe_layer* L, int e, uint64_t pin_epoch, bool prefetch, i
 moe_status build_maps(moe_layer* L, const uint8_t* arena, size_t stride, size_t n_slots) {
   std::vector<CUtensorMap> maps(kMapsPerSlot * n_slots);
   for (size_t i = 0; i < n_slots; ++i) {
-    if (encode_expert_maps(&maps[kMapsPerSlot * i], arena + i * stride, L->s.H, L->s.I) != cudaSuccess)
+    if (encode_expert_maps(&maps[kMapsPerSlot * i], arena + i * stride, L->s) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for slot %zu", i);
   }
   if (L->n_tmap_slots < n_slots) {
@@ -404,6 +461,7 @@ moe_status refresh_stream_maps(moe_layer* L) {
 // Caller holds g_mu until the `used` events of these slots are recorded.
 moe_status resolve_experts(moe_layer* L, const int32_t* ids, int n, cudaStream_t st,
                            std::vector<int>* used_slots) {
+  NvtxRange nv("moe.resolve_experts");
   const Shape& s = L->s;
   std::vector<char> need(s.E + s.S, 0);
   for (int i = 0; i < n; ++i) need[ids[i]] = 1;
@@ -412,6 +470,7 @@ moe_status resolve_experts(moe_layer* L, const int32_t* ids, int n, cudaStream_t
   MOE_TRY(refresh_stream_maps(L));
   Cache* c = g_cache;
   c->epoch++;
+  c->layer_fwds[L->id]++;
   SlotUpdate u{};
   for (int e = 0; e < s.E + s.S; ++e) {
     if (!need[e]) continue;
@@ -436,6 +495,7 @@ moe_status resolve_experts(moe_layer* L, const int32_t* ids, int n, cudaStream_t
 
 moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int32_t* forced,
                         cudaStream_t st) {
+  NvtxRange nv(T == 1 ? "moe.forward T=1" : T <= kD1MaxTok ? "moe.forward decode" : "moe.forward prefill");
   if (!L) return fail(MOE_ERR_INVALID_ARG, "null layer");
   if (T < 0 || T > kMaxTokens) return fail(MOE_ERR_INVALID_ARG, "T=%d outside 0..%d", T, kMaxTokens);
   if (T > 0 && (!x || !out)) return fail(MOE_ERR_INVALID_ARG, "null x or out");
@@ -457,9 +517,13 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
   // one kernel launch, optionally bracketed by profiling events
   ProfRec pr{};
   bool prof;
+  uint64_t hook_wait_ns;
+  int hook_hold;
   {
     std::lock_guard<std::mutex> lk0(g_mu);
     prof = g_profiling;
+    hook_wait_ns = g_hook_wait_ns;
+    hook_hold = g_hook_hold;
     if (prof)
       for (int i = 0; i < 2 * kProfRanges; ++i) pr.ev[i] = prof_event();
   }
@@ -484,6 +548,115 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
   const bool fast = T <= kD1MaxTok && down_d1_smem(max_tok, act_slot) <= kMaxDecodeSmem;
   if (forced)
     CUDA_TRY(cudaMemcpyAsync(wk.forced, forced, (size_t)T * s.k * 4, cudaMemcpyHostToDevice, st));
+  // One token: the whole forward as one persistent kernel, when the experts
+  // are resident or the routing is given (a streamed forward that routes on
+  // the GPU must read the routing back before its experts can be fetched).
+  // Layers with other block types than Q4_K run every token this way.
+  const size_t act1 = 2 * (size_t)s.I_pad + (size_t)(s.I_pad / 32) * 8;
+  int ring_stages = 0, ring_stage_bytes = 0;
+  decode1_ring(s.sbb_gu, s.sbb_d, &ring_stages, &ring_stage_bytes);
+  const bool fused_ok = s.k + s.S <= 40 && s.H % 64 == 0 &&
+                        decode1_fused_smem(s.H, act1, ring_stages * ring_stage_bytes) <= kMaxDecodeSmem;
+  const bool q4k = s.qgu == kQ4_K && s.qd == kQ4_K;
+  if (!q4k && !fused_ok)
+    return fail(MOE_ERR_UNSUPPORTED, "block types %d/%d need the single-token kernel, which this shape does not fit",
+                s.qgu, s.qd);
+  if ((T == 1 && (L->resident || forced) && fused_ok) || !q4k) {
+    std::unique_lock<std::mutex> lk(g_mu, std::defer_lock);
+    std::vector<int> used;
+    const int* dev_forced = forced ? wk.forced : nullptr;
+    if (!L->resident) {
+      const int32_t* hid = forced;
+      if (!hid) {
+        // route on the GPU first, read the picks back, then run the tokens
+        // with those picks as their routing
+        if (T <= kD1MaxTok) {
+          RouteArgs ra{xb, L->d_W, L->d_b, nullptr, T, s.H, s.E, s.k, s.S, (int)L->gating, wk.logits, wk.ids, wk.w,
+                       wk.counts, wk.offsets, wk.perm, wk.inv, wk.act1, wk.n_act1, wk.act2, wk.n_act2, wk.n_act,
+                       wk.xq, wk.xq_plane, wk.xsc, wk.ticket};
+          MOE_KERNEL(MOE_K_ROUTER, launch_route_decode(ra, st));
+        } else {
+          CUtensorMap xmap;
+          if (encode_sw128_16(&xmap, xb, true, (size_t)T, s.H, 128) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
+          RouterGemmArgs rg{};
+          rg.T = T;
+          rg.E = s.E;
+          rg.nsplit = router_gemm_splits(T, s.E, s.H, s.n_sm);
+          rg.nk_split = s.H / 64 / rg.nsplit;
+          rg.part = wk.rpart;
+          rg.split_stride = (size_t)T * s.E;
+          rg.err = wk.err;
+          MOE_KERNEL(MOE_K_ROUTER, launch_router_gemm(xmap, L->wp_map, rg, st));
+          MOE_KERNEL(MOE_K_TOPK, launch_topk(wk.logits, T, s.E, s.k, (int)L->gating, nullptr, wk.ids, wk.w, st,
+                                             wk.rpart, rg.nsplit, rg.split_stride, L->d_b));
+        }
+        CUDA_TRY(cudaMemcpyAsync(L->h_ids, wk.ids, (size_t)T * s.k * 4, cudaMemcpyDeviceToHost, st));
+        CUDA_TRY(cudaStreamSynchronize(st));
+        hid = L->h_ids;
+        CUDA_TRY(cudaMemcpyAsync(wk.forced, wk.ids, (size_t)T * s.k * 4, cudaMemcpyDeviceToDevice, st));
+        dev_forced = wk.forced;
+      }
+      lk.lock();
+      MOE_TRY(resolve_experts(L, hid, T * s.k, st, &used));
+    }
+    FusedArgs fa{};
+    fa.tmaps = L->d_tmaps;
+    fa.slot_of = L->d_slot_of;
+    fa.W = L->d_W;
+    fa.b = L->d_b;
+    fa.T = 1;
+    fa.H = s.H;
+    fa.I = s.I;
+    fa.I_pad = s.I_pad;
+    fa.E = s.E;
+    fa.k = s.k;
+    fa.S = s.S;
+    fa.nbh = s.nbh;
+    fa.nbi = s.nbi;
+    fa.gating = (int)L->gating;
+    fa.hq = wk.hq;
+    fa.hq_plane = wk.hq_plane;
+    fa.hsc = wk.hsc;
+    fa.y = wk.y;
+    fa.sync = wk.sync;
+    fa.err = wk.err;
+    fa.act_slot_bytes = act1;
+    fa.early = L->resident ? 1 : 0;
+    fa.n_slots = (int)L->n_tmap_slots;
+    fa.wait_ns = hook_wait_ns;
+    fa.hold = hook_hold;
+    fa.qgu = s.qgu;
+    fa.qd = s.qd;
+    fa.sbb_gu = s.sbb_gu;
+    fa.sbb_d = s.sbb_d;
+    fa.stages = ring_stages;
+    fa.stage_bytes = ring_stage_bytes;
+    // one launch per token, in order (each reuses the kernel's scratch rows)
+    for (int t = 0; t < T; ++t) {
+      fa.x = xb + (size_t)t * s.H;
+      fa.out = static_cast<__nv_bfloat16*>(out) + (size_t)t * s.H;
+      fa.forced = dev_forced ? dev_forced + (size_t)t * s.k : nullptr;
+      fa.logits = wk.logits + (size_t)t * s.E;
+      fa.ids = wk.ids + (size_t)t * s.k;
+      fa.w = wk.w + (size_t)t * s.k;
+      MOE_KERNEL(MOE_K_FUSED, launch_decode1_fused(fa, s.n_sm, st));
+    }
+    CUDA_TRY(cudaEventRecord(L->done, st));
+    L->done_rec = true;
+    if (!lk.owns_lock()) lk.lock();
+    if (prof) g_prof_pending.push_back(pr);
+    g_stats.launches += (uint64_t)n_launch;
+    for (int slot : used) {
+      CUDA_TRY(cudaEventRecord(g_cache->slots[slot].used, st));
+      g_cache->slots[slot].used_rec = true;
+    }
+    g_stats.forwards++;
+    g_stats.tokens += (uint64_t)T;
+    g_stats.decode_calls++;
+    L->last_T = T;
+    return MOE_OK;
+  }
   if (fast) {
     RouteArgs ra{xb, L->d_W, L->d_b, forced ? wk.forced : nullptr, T, s.H, s.E, s.k, s.S, (int)L->gating,
                  wk.logits, wk.ids, wk.w, wk.counts, wk.offsets, wk.perm, wk.inv, wk.act1, wk.n_act1, wk.act2,
@@ -553,6 +726,9 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
   da.err = wk.err;
   da.stage_x = stage_x ? 1 : 0;
   da.act_slot_bytes = act_slot;
+  da.n_ex = s.E + s.S;
+  da.n_slots = (int)L->n_tmap_slots;
+  da.n_rows = T * (s.k + s.S);
   if (fast) {
     const bool gemv = T == 1 && gemv_gate_up_smem(s.H) <= kMaxDecodeSmem && gemv_down_smem(act_slot) <= kMaxDecodeSmem;
     if (gemv) {
@@ -588,6 +764,8 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     ga.wexp_stride = 2 * s.I + s.H;
     ga.wexp_down = 2 * s.I;
     ga.err = wk.err;
+    ga.n_ex = s.E + s.S;
+    ga.n_slots = (int)L->n_tmap_slots;
     MOE_KERNEL(MOE_K_GATE_UP, launch_prefill_gemm(0, L->x16_map, ga, s.n_sm, st));
     if (split_small) MOE_KERNEL(MOE_K_SMALL, launch_gate_up_d1(da, kD1MaxTok, s.n_sm, st));
     MOE_KERNEL(MOE_K_PREP, launch_convert_h(wk, P, s.I, s.I_pad, st));
@@ -630,17 +808,29 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
 extern "C" {
 
 size_t moe_expert_bytes(int hidden, int inter, moe_quant quant) {
-  if (quant != MOE_Q4_K || hidden <= 0 || inter <= 0 || hidden % kQK) return 0;
+  const int q = (int)quant;
+  if (!dev_sb_bytes(q) || hidden <= 0 || inter <= 0 || hidden % kQK) return 0;
+  if (host_block_elems(q) != kQK && inter % kQK) return 0;
   const size_t nbh = hidden / kQK, nbi = (inter + kQK - 1) / kQK;
-  return 2 * (size_t)inter * nbh * kQBytes + (size_t)hidden * nbi * kQBytes;
+  return 2 * (size_t)inter * nbh * dev_sb_bytes(q) + (size_t)hidden * nbi * dev_sb_bytes(q);
 }
 
 moe_status moe_layer_create(int hidden, int inter, int n_experts, int top_k, int n_shared,
                             moe_quant quant, moe_layer_t* out) {
+  return moe_layer_create_mixed(hidden, inter, n_experts, top_k, n_shared, quant, quant, out);
+}
+
+moe_status moe_layer_create_mixed(int hidden, int inter, int n_experts, int top_k, int n_shared,
+                                  moe_quant quant_gate_up, moe_quant quant_down, moe_layer_t* out) {
   g_err.clear();
   if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
-  if (quant != MOE_Q4_K) return fail(MOE_ERR_UNSUPPORTED, "quant type %d (only Q4_K=12)", (int)quant);
+  const int qgu = (int)quant_gate_up, qd = (int)quant_down;
+  if (!dev_sb_bytes(qgu) || !dev_sb_bytes(qd))
+    return fail(MOE_ERR_UNSUPPORTED, "quant types %d, %d (supported: Q8_0=8, Q4_K=12, Q5_K=13, Q6_K=14, MXFP4=39)",
+                qgu, qd);
+  if (host_block_elems(qd) != kQK && inter % kQK)
+    return fail(MOE_ERR_UNSUPPORTED, "inter=%d must be a multiple of 256 for down weights of type %d", inter, qd);
   if (hidden <= 0 || hidden > 16384 || hidden % kQK)
     return fail(MOE_ERR_INVALID_ARG, "hidden=%d must be a multiple of 256 in 256..16384", hidden);
   if (inter <= 0 || inter > 16384) return fail(MOE_ERR_INVALID_ARG, "inter=%d outside 1..16384", inter);
@@ -659,9 +849,18 @@ moe_status moe_layer_create(int hidden, int inter, int n_experts, int top_k, int
   s.nbh = hidden / kQK;
   s.nbi = (inter + kQK - 1) / kQK;
   s.I_pad = s.nbi * kQK;
-  L->gate_bytes = (size_t)inter * s.nbh * kQBytes;
-  L->down_bytes = (size_t)hidden * s.nbi * kQBytes;
+  s.qgu = qgu;
+  s.qd = qd;
+  s.sbb_gu = dev_sb_bytes(qgu);
+  s.sbb_d = dev_sb_bytes(qd);
+  s.hrow_gu = (size_t)((hidden + host_block_elems(qgu) - 1) / host_block_elems(qgu)) * host_block_bytes(qgu);
+  s.hrow_d = (size_t)((inter + host_block_elems(qd) - 1) / host_block_elems(qd)) * host_block_bytes(qd);
+  s.drow_gu = (size_t)s.nbh * s.sbb_gu;
+  s.drow_d = (size_t)s.nbi * s.sbb_d;
+  L->gate_bytes = (size_t)inter * s.drow_gu;
+  L->down_bytes = (size_t)hidden * s.drow_d;
   L->expert_bytes = 2 * L->gate_bytes + L->down_bytes;
+  L->host_expert_bytes = 2 * (size_t)inter * s.hrow_gu + (size_t)hidden * s.hrow_d;
   cudaError_t e = cudaGetDevice(&L->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&s.n_sm, cudaDevAttrMultiProcessorCount, L->device);
   if (e == cudaSuccess) e = cudaMalloc(&L->d_slot_of, sizeof(int) * (size_t)(s.E + s.S));
@@ -748,6 +947,7 @@ moe_status moe_set_experts(moe_layer_t L, const void* const* gate, const void* c
   g_err.clear();
   if (!L || !gate || !up || !down) return fail(MOE_ERR_INVALID_ARG, "null argument");
   MOE_TRY(check_device(L));
+  NvtxRange nv("moe.set_experts");
   const int n = L->s.E + L->s.S;
   std::vector<const uint8_t*> host(3 * (size_t)n);
   for (int e = 0; e < n; ++e) {
@@ -774,9 +974,11 @@ moe_status moe_set_experts(moe_layer_t L, const void* const* gate, const void* c
       pool.emplace_back([&, t] {
         for (int e = t; e < n; e += nth) {
           int8_t* o = wexp.data() + (size_t)e * stride;
-          q4k_row_exponents(host[3 * (size_t)e], L->s.I, L->s.nbh, o);
-          q4k_row_exponents(host[3 * (size_t)e + 1], L->s.I, L->s.nbh, o + L->s.I);
-          q4k_row_exponents(host[3 * (size_t)e + 2], L->s.H, L->s.nbi, o + 2 * L->s.I);
+          if (L->s.qgu == kQ4_K) {
+            q4k_row_exponents(host[3 * (size_t)e], L->s.I, L->s.nbh, o);
+            q4k_row_exponents(host[3 * (size_t)e + 1], L->s.I, L->s.nbh, o + L->s.I);
+          }
+          if (L->s.qd == kQ4_K) q4k_row_exponents(host[3 * (size_t)e + 2], L->s.H, L->s.nbi, o + 2 * L->s.I);
         }
       });
     for (auto& th : pool) th.join();
@@ -795,12 +997,11 @@ moe_status moe_set_experts(moe_layer_t L, const void* const* gate, const void* c
     if (!L->d_resident) CUDA_TRY(cudaMalloc(&L->d_resident, (size_t)n * L->expert_bytes));
     for (int e = 0; e < n; ++e) {
       uint8_t* dst = L->d_resident + (size_t)e * L->expert_bytes;
-      const size_t sz[3] = {L->gate_bytes, L->gate_bytes, L->down_bytes};
       const size_t off[3] = {0, L->gate_bytes, 2 * L->gate_bytes};
-      for (int m = 0; m < 3; ++m) {
-        CUDA_TRY(cudaMemcpyAsync(dst + off[m], L->host[3 * (size_t)e + m], sz[m], cudaMemcpyHostToDevice,
-                                 L->copy));
-      }
+      const int rows[3] = {L->s.I, L->s.I, L->s.H}, q[3] = {L->s.qgu, L->s.qgu, L->s.qd};
+      const size_t hrow[3] = {L->s.hrow_gu, L->s.hrow_gu, L->s.hrow_d}, drow[3] = {L->s.drow_gu, L->s.drow_gu, L->s.drow_d};
+      for (int m = 0; m < 3; ++m)
+        CUDA_TRY(copy_matrix_h2d(dst + off[m], L->host[3 * (size_t)e + m], rows[m], q[m], hrow[m], drow[m], L->copy));
     }
     CUDA_TRY(cudaStreamSynchronize(L->copy));
     MOE_TRY(build_maps(L, L->d_resident, L->expert_bytes, (size_t)n));
@@ -835,6 +1036,23 @@ moe_status moe_set_cache_bytes(size_t bytes) {
     g_stats.slot_bytes = 0;
   }
   g_cache_bytes = bytes;
+  return MOE_OK;
+}
+
+moe_status moe_set_test_hooks(uint64_t wait_limit_ns, int hold_barrier) {
+  g_err.clear();
+  if (hold_barrier < 0) return fail(MOE_ERR_INVALID_ARG, "hold_barrier=%d", hold_barrier);
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_hook_wait_ns = wait_limit_ns;
+  g_hook_hold = hold_barrier;
+  return MOE_OK;
+}
+
+moe_status moe_set_cache_policy(int policy) {
+  g_err.clear();
+  if (policy != MOE_CACHE_LRU && policy != MOE_CACHE_LFU) return fail(MOE_ERR_INVALID_ARG, "policy=%d", policy);
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_cache_policy = policy;
   return MOE_OK;
 }
 
@@ -938,8 +1156,13 @@ moe_status moe_check(moe_layer_t L) {
   CUDA_TRY(cudaStreamSynchronize(L->copy));
   const unsigned flags = *L->h_err;
   if (flags) {
+    // a kernel that gave up may have left its barrier and step counters
+    // half-way: start them from zero again
+    CUDA_TRY(cudaMemsetAsync(L->wk.sync, 0, kSyncWords * sizeof(unsigned), L->copy));
     CUDA_TRY(cudaMemsetAsync(L->wk.err, 0, sizeof(unsigned), L->copy));
     CUDA_TRY(cudaStreamSynchronize(L->copy));
+    if (flags & kErrBoundsBit)
+      return fail(MOE_ERR_CUDA, "an index a kernel read from memory was out of range (flags 0x%x)", flags);
     return fail(MOE_ERR_CUDA, "a kernel of this layer gave up waiting (flags 0x%x)", flags);
   }
   return MOE_OK;

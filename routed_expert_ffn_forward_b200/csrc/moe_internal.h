@@ -13,6 +13,21 @@
 
 namespace moe {
 
+// GGUF block types (GGML type ids)
+constexpr int kQ8_0 = 8, kQ4_K = 12, kQ5_K = 13, kQ6_K = 14, kMXFP4 = 39;
+// Device bytes of one group of 256 weights of type q, as the kernels read
+// them: the GGUF bytes, except that Q6_K blocks (210 bytes) are padded to 224
+// and MXFP4 blocks (17 bytes, 32 weights) are grouped eight at a time into
+// 144, so that every group starts on a 16-byte boundary.  0: not supported.
+__host__ __device__ constexpr int dev_sb_bytes(int q) {
+  return q == kQ4_K ? 144 : q == kQ5_K ? 176 : q == kQ6_K ? 224 : q == kQ8_0 ? 272 : q == kMXFP4 ? 144 : 0;
+}
+// Host (GGUF) block geometry: weights and bytes per block.
+constexpr int host_block_elems(int q) { return q == kQ8_0 || q == kMXFP4 ? 32 : 256; }
+constexpr int host_block_bytes(int q) {
+  return q == kQ4_K ? 144 : q == kQ5_K ? 176 : q == kQ6_K ? 210 : q == kQ8_0 ? 34 : q == kMXFP4 ? 17 : 0;
+}
+
 constexpr int kQK = 256;        // weights per Q4_K super-block
 constexpr int kQBytes = 144;    // bytes per Q4_K super-block
 constexpr int kD1MaxTok = 4;    // experts with <= this many rows use the per-sub-block decode kernels
@@ -55,7 +70,9 @@ struct Work {
   __half* h16;        // [P_cap, I_pad] SwiGLU output, fp16 scaled by 1/hinv, same K order
   float* hinv;        // [P]
   float* rpart;       // router partial logits [splits][T][E]
+  unsigned* sync;     // [kSyncWords] grid barrier and step counters of the fused single-token kernel
 };
+constexpr int kSyncWords = 512;
 
 struct RouteArgs {
   const __nv_bfloat16* x;
@@ -100,6 +117,7 @@ struct DecodeArgs {
   unsigned* err;
   int stage_x;            // gate/up: copy x (all T tokens) to shared memory once per CTA
   size_t act_slot_bytes;  // down: bytes of one activation slot (2 * max_tok * I_pad + scales)
+  int n_ex, n_slots, n_rows;  // bounds of expert ids (E+S), cache slots, rows (T(k+S)); debug builds
 };
 constexpr size_t kMaxDecodeSmem = 227 * 1024;
 // max_tok: 1 (every expert has one row, T == 1) or kD1MaxTok
@@ -114,12 +132,55 @@ cudaError_t launch_gemv_down(const DecodeArgs& a, int n_sm, cudaStream_t st);
 size_t gemv_gate_up_smem(int H);
 size_t gemv_down_smem(size_t act_slot_bytes);
 
+// T = 1 as one persistent kernel: router, top-k, gate/up + SwiGLU, down and
+// combine (one CTA per SM; steps meet through counters in `sync`).
+struct FusedArgs {
+  const CUtensorMap* tmaps;  // [slots][kMapsPerSlot]
+  const int* slot_of;        // [E+S] expert -> slot
+  const __nv_bfloat16* x;    // [H]
+  const float* W;            // router [E, H]
+  const float* b;            // router bias [E] or null
+  const int* forced;         // device [k] or null
+  int T, H, I, I_pad, E, k, S, nbh, nbi, gating;
+  float* logits;             // [E]
+  int* ids;                  // [k]
+  float* w;                  // [k]
+  int8_t* hq;                // h of expert j (j = 0..k+S-1) at row j: [2][rows][I_pad]
+  size_t hq_plane;
+  float2* hsc;               // [rows][I_pad / 32]
+  float* y;                  // [k+S, H]
+  __nv_bfloat16* out;        // [H]
+  unsigned* sync;            // kSyncWords, zero before the first launch
+  unsigned* err;
+  size_t act_slot_bytes;     // 2 * I_pad + I_pad / 32 * 8
+  int early;                 // weights and slot table constant: stream them before the predecessor ends
+  uint64_t wait_ns;          // limit of the bounded waits (0: the default 2 s); test hook
+  int hold;                  // > 0: the grid barrier waits for that many arrivals more (test hook)
+  int n_slots;               // bound of cache slots (debug builds)
+  int qgu, qd;               // GGUF block types of gate/up and of down
+  int sbb_gu, sbb_d;         // their device bytes per 256-weight group
+  int stages, stage_bytes;   // weight ring: stages x (256 x the larger group size)
+};
+// Weight-ring geometry of the single-token kernel for these group sizes.
+inline void decode1_ring(int sbb_gu, int sbb_d, int* stages, int* stage_bytes) {
+  *stage_bytes = 256 * std::max(sbb_gu, sbb_d);
+  *stages = std::min(4, 147456 / *stage_bytes);
+}
+size_t decode1_fused_smem(int H, size_t act_slot_bytes, int ring_bytes);
+cudaError_t launch_decode1_fused(const FusedArgs& a, int n_sm, cudaStream_t st);
+
 // Tensor maps of one expert's Q4_K matrices at `base`, kMapsPerSlot of them:
 // [0..2] gate, up, down with boxes of 64 rows x 2 (gate/up) or 4 (down)
 // super-blocks (decode kernels); [3..5] gate, up, down with boxes of 128 rows x
-// 1 super-block (prefill GEMMs).
-constexpr int kMapsPerSlot = 6;
-cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, int H, int I);
+// 1 super-block (single-token GEMVs and prefill GEMMs); [6] down with boxes of
+// 64 rows x 1 super-block (the fused single-token kernel).
+constexpr int kMapsPerSlot = 7;
+struct Shape;
+cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, const Shape& s);
+// Copy one weight matrix of `rows` rows from its GGUF host bytes into the
+// device layout of its type (dev_sb_bytes), asynchronously on `st`.
+cudaError_t copy_matrix_h2d(uint8_t* dst, const uint8_t* src, int rows, int q, size_t hrow, size_t drow,
+                            cudaStream_t st);
 // 2-D map over a row-major 16-bit matrix [rows, cols] (fp16 or bf16) with
 // 128B-swizzled boxes of box_rows rows x 64 columns (cols a multiple of 64).
 cudaError_t encode_sw128_16(CUtensorMap* map, const void* base, bool bf16, size_t rows, int cols, int box_rows);
@@ -162,6 +223,7 @@ struct GemmArgs {
   const int8_t* wexp;
   int wexp_stride, wexp_down;
   unsigned* err;
+  int n_ex, n_slots;         // bounds of expert ids and cache slots (debug builds)
 };
 size_t prefill_gemm_smem();
 size_t prefill_max_tiles(int n_experts_total, size_t pairs);
@@ -179,6 +241,10 @@ struct Shape {
   int nbi;    // super-blocks per down row     = ceil(I / 256)
   int I_pad;  // nbi * 256
   int n_sm;   // streaming multiprocessors of the device
+  int qgu, qd;            // GGUF block types of gate and up (shared), and of down
+  int sbb_gu, sbb_d;      // device bytes per 256-weight group (dev_sb_bytes)
+  size_t hrow_gu, hrow_d; // host (GGUF) bytes per row
+  size_t drow_gu, drow_d; // device bytes per row: nbh * sbb_gu, nbi * sbb_d
 };
 
 // ---- kernels (one launch helper per kernel; all enqueue on `st`) ----------
@@ -216,6 +282,24 @@ int report_error(int status, const char* msg);
 void clear_error();
 
 // ---- device helpers -------------------------------------------------------
+// Debug builds (-DMOE_DEBUG_BOUNDS, libmoe_debug.so) check every index that a
+// kernel reads from memory before it addresses memory with it: an expert id,
+// a cache slot, a row offset or a permutation entry.  A bad one sets
+// kErrBoundsBit in the layer's error word (moe_check reports it) and is
+// replaced by 0, so the access stays in bounds.  Release builds skip the check.
+constexpr unsigned kErrBoundsBit = 1u << 20;
+#ifdef __CUDACC__
+#ifdef MOE_DEBUG_BOUNDS
+__device__ __forceinline__ int in_range(int v, int n, unsigned* err) {
+  if ((unsigned)v < (unsigned)n) return v;
+  atomicOr(err, kErrBoundsBit);
+  return 0;
+}
+#else
+__device__ __forceinline__ int in_range(int v, int, unsigned*) { return v; }
+#endif
+#endif
+
 #ifdef __CUDACC__
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }

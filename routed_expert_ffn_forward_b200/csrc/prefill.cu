@@ -129,7 +129,7 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmArgs& a, uint32_t tmem, 
   const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
   const int pair0 = tl.w + tl.y;
   // 2^-k of the weight rows this thread's accumulator lanes belong to
-  const int8_t* wx = a.wexp + (size_t)tl.x * a.wexp_stride;
+  const int8_t* wx = a.wexp + (size_t)in_range(tl.x, a.n_ex, a.err) * a.wexp_stride;
   float s0, s1;
   if (kMode == 0) {
     const int feat = min(f * kGM + mrow, a.out_rows - 1);
@@ -231,7 +231,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
       for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
         const int4 tl = __ldcg(a.tiles + u / ft);  // (expert, n0, count, r0)
         const int f = u % ft;
-        const CUtensorMap* wm = a.wmaps + kMapsPerSlot * __ldcg(a.slot_of + tl.x) + 3;
+        const int ex = in_range(tl.x, a.n_ex, a.err);
+        const CUtensorMap* wm = a.wmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + ex), a.n_slots, a.err) + 3;
         const CUtensorMap* m0 = kMode == 0 ? wm : wm + 2;
         const CUtensorMap* m1 = kMode == 0 ? wm + 1 : wm + 2;
         const int y0 = kMode == 0 ? f * kGM : f * 2 * kGM;
@@ -330,7 +331,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
     uint32_t rph = 0, aph = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       // this thread's weight row and its power-of-two scale 2^k
-      const int ex = __ldcg(a.tiles + u / a.ft).x, f = u % a.ft;
+      const int ex = in_range(__ldcg(a.tiles + u / a.ft).x, a.n_ex, a.err), f = u % a.ft;
       const int8_t* wx = a.wexp + (size_t)ex * a.wexp_stride;
       const int wrow = kMode == 0 ? min(f * kGM + r, a.out_rows - 1) + m * a.out_rows
                                   : a.wexp_down + f * 2 * kGM + m * kGM + r;

@@ -25,6 +25,24 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v
   return old;
 }
 
+// Device-scope acquire load / release store / release add of one 32-bit word.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Order this thread's generic-proxy global accesses with its async-proxy
+// (TMA / bulk copy) global accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -76,6 +94,22 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, 
     if (globaltimer() - t0 > limit_ns) return false;
   }
 }
+
+// Which stages of a ring a producer thread filled last, and in which phase,
+// so that it can wait for its copies in flight before it leaves (a CTA must
+// not exit while a copy into its shared memory is still landing).
+struct IssueLog {
+  uint32_t issued = 0, par = 0;
+  __device__ __forceinline__ void note(int s, uint32_t phase) {
+    issued |= 1u << s;
+    par = (par & ~(1u << s)) | (phase << s);
+  }
+  // bounded by the default limit, whatever limit the aborted wait had
+  __device__ __forceinline__ void drain(uint64_t* full, int n) const {
+    for (int s = 0; s < n; ++s)
+      if ((issued >> s) & 1u) mbar_wait(&full[s], (par >> s) & 1u);
+  }
+};
 
 // ---- TMA --------------------------------------------------------------------
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {

@@ -1,10 +1,10 @@
-// Tensor maps (TMA descriptors) over Q4_K expert matrices.
+// Tensor maps (TMA descriptors) over the expert weight matrices.
 //
-// A matrix of R rows and nb super-blocks per row is viewed as a 2-D array of
-// 8-byte elements, nb*18 wide and R high (row pitch nb*144 bytes, a multiple
-// of 16).  A box is 64 or 128 rows by SB super-blocks (SB*18 elements, SB*144
-// bytes); boxes past the last row or block read zeros, which decode to zero
-// weights.  16-bit operand matrices of the tensor-core GEMMs (activations,
+// A matrix of R rows and nb groups of 256 weights per row (sbb device bytes
+// per group: 144 for Q4_K, see dev_sb_bytes) is viewed as a 2-D array of
+// 8-byte elements, nb*sbb/8 wide and R high (row pitch nb*sbb bytes, a
+// multiple of 16).  A box is 64 or 128 rows by a few groups; boxes past the
+// last row or group read zeros, which decode to zero weights.  16-bit operand matrices of the tensor-core GEMMs (activations,
 // router planes) use 128-byte-swizzled boxes of 64 columns.
 #include <mutex>
 
@@ -30,12 +30,16 @@ EncodeFn encode_fn() {
   return fn;
 }
 
-cudaError_t encode_q4k(CUtensorMap* m, const uint8_t* base, int rows, int nb, int box_blocks, int box_rows) {
+// Matrix of `rows` rows of nb groups of `sbb` bytes (a multiple of 16), boxes
+// of box_rows rows x box_blocks groups.
+cudaError_t encode_q4k(CUtensorMap* m, const uint8_t* base, int rows, int nb, int box_blocks, int box_rows,
+                       int sbb = kQBytes) {
   EncodeFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
-  const cuuint64_t dims[2] = {(cuuint64_t)nb * 18, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)nb * kQBytes};
-  const cuuint32_t box[2] = {(cuuint32_t)box_blocks * 18, (cuuint32_t)box_rows};
+  const int el = sbb / 8;   // 8-byte elements per group
+  const cuuint64_t dims[2] = {(cuuint64_t)nb * el, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)nb * sbb};
+  const cuuint32_t box[2] = {(cuuint32_t)(box_blocks * el), (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -45,15 +49,28 @@ cudaError_t encode_q4k(CUtensorMap* m, const uint8_t* base, int rows, int nb, in
 
 }  // namespace
 
-cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, int H, int I) {
-  const int nbh = H / kQK, nbi = (I + kQK - 1) / kQK;
-  const size_t gate_bytes = (size_t)I * nbh * kQBytes;
+cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, const Shape& s) {
+  const int H = s.H, I = s.I, nbh = s.nbh, nbi = s.nbi;
+  const size_t gate_bytes = (size_t)I * s.drow_gu;
   const uint8_t* mats[3] = {base, base + gate_bytes, base + 2 * gate_bytes};
-  const int rows[3] = {I, I, H}, nb[3] = {nbh, nbh, nbi};
+  const int rows[3] = {I, I, H}, nb[3] = {nbh, nbh, nbi}, sbb[3] = {s.sbb_gu, s.sbb_gu, s.sbb_d};
   cudaError_t e = cudaSuccess;
-  for (int m = 0; m < 3 && e == cudaSuccess; ++m) e = encode_q4k(&maps[m], mats[m], rows[m], nb[m], m < 2 ? 2 : 4, kTileRows);
-  for (int m = 0; m < 3 && e == cudaSuccess; ++m) e = encode_q4k(&maps[3 + m], mats[m], rows[m], nb[m], 1, 128);
+  for (int m = 0; m < 3 && e == cudaSuccess; ++m)
+    e = encode_q4k(&maps[m], mats[m], rows[m], nb[m], m < 2 ? 2 : 4, kTileRows, sbb[m]);
+  for (int m = 0; m < 3 && e == cudaSuccess; ++m) e = encode_q4k(&maps[3 + m], mats[m], rows[m], nb[m], 1, 128, sbb[m]);
+  if (e == cudaSuccess) e = encode_q4k(&maps[6], mats[2], rows[2], nb[2], 1, 64, sbb[2]);
   return e;
+}
+
+cudaError_t copy_matrix_h2d(uint8_t* dst, const uint8_t* src, int rows, int q, size_t hrow, size_t drow,
+                            cudaStream_t st) {
+  if (hrow == drow) return cudaMemcpyAsync(dst, src, (size_t)rows * hrow, cudaMemcpyHostToDevice, st);
+  // each GGUF block (Q6_K, 210 bytes) or group of eight (MXFP4, 136 bytes)
+  // into its 16-byte-aligned device slot
+  const size_t hb = q == kQ6_K ? 210 : q == kMXFP4 ? 136 : 0;
+  const size_t db = (size_t)dev_sb_bytes(q);
+  if (!hb || hrow % hb || drow % db || hrow / hb != drow / db) return cudaErrorInvalidValue;
+  return cudaMemcpy2DAsync(dst, db, src, hb, hb, (size_t)rows * (hrow / hb), cudaMemcpyHostToDevice, st);
 }
 
 cudaError_t encode_sw128_16(CUtensorMap* map, const void* base, bool bf16, size_t rows, int cols, int box_rows) {

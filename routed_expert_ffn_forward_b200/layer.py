@@ -17,13 +17,17 @@ from . import moe, synth
 
 
 class MoELayer:
-    def __init__(self, hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int):
+    def __init__(self, hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int,
+                 quants=(moe.MOE_Q4_K, moe.MOE_Q4_K, moe.MOE_Q4_K)):
+        """quants: GGUF block types of gate, up and down (gate and up share one)."""
         self.H, self.I, self.E, self.k, self.S = hidden, inter, n_experts, top_k, n_shared
-        self.handle = moe.moe_layer_create(hidden, inter, n_experts, top_k, n_shared, moe.MOE_Q4_K)
-        self.expert_bytes = moe.moe_expert_bytes(hidden, inter)
-        nbh, nbi = hidden // 256, (inter + 255) // 256
-        self.gate_bytes = inter * nbh * 144
-        self.down_bytes = hidden * nbi * 144
+        if quants[0] != quants[1]:
+            raise ValueError("gate and up weights share one block type")
+        self.quants = tuple(quants)
+        self.handle = moe.moe_layer_create_mixed(hidden, inter, n_experts, top_k, n_shared, quants[0], quants[2])
+        self.gate_bytes = inter * synth.row_bytes(quants[0], hidden)
+        self.down_bytes = hidden * synth.row_bytes(quants[2], inter)
+        self.expert_bytes = 2 * self.gate_bytes + self.down_bytes   # host (GGUF) bytes
         self.host: Optional[torch.Tensor] = None
 
     # ------------------------------------------------------------ setup
@@ -104,13 +108,13 @@ class MoELayer:
 def layer_from_config(cfg: synth.LayerConfig, layer_index: int = 0, threads: int = 8) -> MoELayer:
     """Create a layer, fill its pinned store from the seeded generators and
     register router + experts."""
-    L = MoELayer(cfg.hidden, cfg.inter, cfg.n_experts, cfg.top_k, cfg.n_shared)
+    L = MoELayer(cfg.hidden, cfg.inter, cfg.n_experts, cfg.top_k, cfg.n_shared, cfg.quants)
     L.set_router(synth.router_weight(cfg, layer_index), synth.router_bias(cfg, layer_index), cfg.gating)
 
     def fill(e, views):
         for m, v in enumerate(views):
             rows, cols = (cfg.inter, cfg.hidden) if m < 2 else (cfg.hidden, cfg.inter)
-            synth.q4k_tensor(cfg.seed, layer_index, e, m, rows, cols, out=v)
+            synth.q_tensor(cfg.quants[m], cfg.seed, layer_index, e, m, rows, cols, out=v)
 
     L.fill_experts(fill, threads)
     L.register_experts()

@@ -12,7 +12,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe.so")
+# MOE_LIB_VARIANT=debug loads the bounds-checking build (libmoe_debug.so)
+LIB_PATH = os.path.join(_HERE, "libmoe_debug.so" if os.environ.get("MOE_LIB_VARIANT") == "debug" else "libmoe.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = -1
@@ -24,19 +25,25 @@ MOE_ERR_NOT_READY = -6
 STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_OOM",
                 -4: "MOE_ERR_CUDA", -5: "MOE_ERR_CACHE_TOO_SMALL", -6: "MOE_ERR_NOT_READY"}
 
+MOE_Q8_0 = 8
 MOE_Q4_K = 12
+MOE_Q5_K = 13
+MOE_Q6_K = 14
+MOE_MXFP4 = 39
+MOE_CACHE_LRU = 0
+MOE_CACHE_LFU = 1
 MOE_GATE_SOFTMAX_TOPK = 0
 MOE_GATE_SIGMOID_RENORM = 1
 SIZE_MAX = (1 << 64) - 1
 
 # every entry point declared in include/moe.h
-EXPORTS = ("moe_expert_bytes", "moe_layer_create", "moe_layer_destroy", "moe_set_router",
-           "moe_set_experts", "moe_set_cache_bytes", "moe_forward", "moe_forward_routed",
+EXPORTS = ("moe_expert_bytes", "moe_layer_create", "moe_layer_create_mixed", "moe_layer_destroy", "moe_set_router",
+           "moe_set_experts", "moe_set_cache_bytes", "moe_set_cache_policy", "moe_forward", "moe_forward_routed",
            "moe_forward_host", "moe_get_routing", "moe_get_logits", "moe_prefetch",
            "moe_check", "moe_get_stats", "moe_reset_stats", "moe_set_profiling", "moe_get_profile",
-           "moe_reset_profile", "moe_route_noalloc", "moe_last_error")
+           "moe_reset_profile", "moe_route_noalloc", "moe_set_test_hooks", "moe_last_error")
 
-KERNELS = ("router", "topk", "permute", "gate_up", "down", "combine", "prep", "small", "forward")
+KERNELS = ("router", "topk", "permute", "gate_up", "down", "combine", "prep", "small", "forward", "fused")
 
 
 class moe_stats(ctypes.Structure):
@@ -74,15 +81,18 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is not built: run `python -m routed_expert_ffn_forward_b200.build`")
+            raise ImportError(f"{LIB_PATH} is not built: run `python -m routed_expert_ffn_forward_b200.build`"
+                              + (" --debug-bounds" if LIB_PATH.endswith("_debug.so") else ""))
         L = ctypes.CDLL(LIB_PATH)
         sig = {
             "moe_expert_bytes": (ctypes.c_size_t, [_I, _I, _I]),
             "moe_layer_create": (_I, [_I, _I, _I, _I, _I, _I, ctypes.POINTER(_P)]),
+            "moe_layer_create_mixed": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_P)]),
             "moe_layer_destroy": (_I, [_P]),
             "moe_set_router": (_I, [_P, _P, _P, _I]),
             "moe_set_experts": (_I, [_P, _P, _P, _P]),
             "moe_set_cache_bytes": (_I, [ctypes.c_size_t]),
+            "moe_set_cache_policy": (_I, [_I]),
             "moe_forward": (_I, [_P, _P, _P, _I, _P]),
             "moe_forward_routed": (_I, [_P, _P, _P, _I, _P, _P]),
             "moe_forward_host": (_I, [_P, _P, _P, _I, _P]),
@@ -96,6 +106,7 @@ def lib() -> ctypes.CDLL:
             "moe_get_profile": (_I, [ctypes.POINTER(moe_profile)]),
             "moe_reset_profile": (_I, []),
             "moe_route_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+            "moe_set_test_hooks": (_I, [ctypes.c_uint64, _I]),
             "moe_last_error": (ctypes.c_char_p, []),
         }
         for name, (res, args) in sig.items():
@@ -127,6 +138,14 @@ def moe_layer_create(hidden: int, inter: int, n_experts: int, top_k: int, n_shar
     return int(h.value)
 
 
+def moe_layer_create_mixed(hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int,
+                           quant_gate_up: int, quant_down: int) -> int:
+    h = _P()
+    _check(lib().moe_layer_create_mixed(hidden, inter, n_experts, top_k, n_shared, quant_gate_up, quant_down,
+                                        ctypes.byref(h)))
+    return int(h.value)
+
+
 def moe_layer_destroy(layer: int) -> None:
     _check(lib().moe_layer_destroy(layer))
 
@@ -141,6 +160,10 @@ def moe_set_experts(layer: int, gate_ptrs, up_ptrs, down_ptrs) -> None:
 
 def moe_set_cache_bytes(nbytes: int) -> None:
     _check(lib().moe_set_cache_bytes(nbytes))
+
+
+def moe_set_cache_policy(policy: int) -> None:
+    _check(lib().moe_set_cache_policy(policy))
 
 
 def moe_forward(layer: int, x: int, out: int, T: int, stream: int | None = None) -> None:
@@ -199,6 +222,10 @@ def moe_reset_profile() -> None:
 def moe_route_noalloc(x: int, W: int, bias: int | None, T: int, H: int, E: int, top_k: int, gating: int,
                       ids: int, weights: int, stream: int | None = None) -> None:
     _check(lib().moe_route_noalloc(x, W, bias or None, T, H, E, top_k, gating, ids, weights, stream or None))
+
+
+def moe_set_test_hooks(wait_limit_ns: int, hold_barrier: int) -> None:
+    _check(lib().moe_set_test_hooks(wait_limit_ns, hold_barrier))
 
 
 def moe_last_error() -> str:

@@ -149,6 +149,23 @@ def test_c3_prefill_sampled(torch):
     check_against_oracle(cfg, g, sample=sample, parallel=True)
 
 
+def test_single_token_deterministic(torch):
+    """One token runs as one persistent kernel whose down units are claimed
+    dynamically: the sums still run in a fixed order, so repeated forwards
+    give identical bits; the routing read back matches the oracle."""
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    cfg = SMALL["ragged_inter"]
+    L = layer_from_config(cfg)
+    outs = []
+    for rep in range(3):
+        x = synth.activations(cfg, 0, rep % 2, tokens=1)
+        outs.append(to_bits(torch, L.forward(to_dev(torch, x))))
+    torch.cuda.synchronize()
+    moe.moe_check(L.handle)
+    np.testing.assert_array_equal(outs[0], outs[2])
+    L.destroy()
+
+
 def test_deterministic_and_host_path(torch):
     from routed_expert_ffn_forward_b200.layer import layer_from_config
     cfg = synth.BATCHED
@@ -263,3 +280,62 @@ def test_large_weight_scales_are_exact(torch):
         assert np.abs(r["out64"]).max() > 1e3          # the large rows dominate the output
         pu.check_outputs(out, r["out_bf16"], f"large scales, T={T}")
     L.destroy()
+
+
+# ------------------------------------------------------------------ other GGUF block types
+MIXED = {
+    "q5k_q6k": dataclasses.replace(C0, n_shared=1, gating=1, quants=(13, 13, 14), seed=41),
+    "q8_0_q8_0": dataclasses.replace(C0, hidden=512, inter=256, n_experts=24, top_k=3, n_shared=1, gating=1,
+                                      quants=(8, 8, 8), seed=42, router_std=1 / 512 ** 0.5),
+    "mxfp4_q4k": dataclasses.replace(C0, n_shared=2, gating=0, quants=(39, 39, 12), seed=43),
+    "q4k_mxfp4": dataclasses.replace(C0, inter=256, quants=(12, 12, 39), seed=44),
+    "q6k_q5k_ragged": dataclasses.replace(C0, hidden=512, inter=300, n_experts=40, top_k=5, n_shared=2, gating=1,
+                                           quants=(14, 14, 13), seed=45, router_std=1 / 512 ** 0.5),
+}
+
+
+def mixed_oracle_layer(cfg, layer_index=0):
+    d = oracle_layer(cfg, layer_index)
+    d["quants"] = cfg.quants
+    return d
+
+
+@pytest.mark.parametrize("name", sorted(MIXED))
+@pytest.mark.parametrize("T", [1, 3, 17])
+def test_block_types_every_token(torch, name, T):
+    """Layers whose weights are Q5_K, Q6_K, Q8_0 or MXFP4 (gate/up sharing a
+    type, down another): every token runs the single-token kernel."""
+    cfg = MIXED[name]
+    g = run_gpu(torch, cfg, T)
+    ol = mixed_oracle_layer(cfg)
+    x = g["x"]
+    l64 = ref.router_logits(ref.bf16_to_f64(x), ol["router_w"], ol["router_b"])
+    np.testing.assert_allclose(g["logits"], l64, rtol=0, atol=1e-4 * max(1.0, np.abs(l64).max()))
+    near = pu.check_ids(g["ids"], l64, cfg.top_k)
+    np.testing.assert_allclose(g["w"], ref.gate_weights(l64, g["ids"].astype(np.int64), cfg.gating),
+                               rtol=1e-5, atol=1e-6)
+    forced = np.where(near[:, None], g["ids"], ref.topk_ids(l64, cfg.top_k))
+    r = ref.moe_forward(x, ol, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter, forced_ids=forced)
+    pu.check_outputs(g["out"], r["out_bf16"], cfg.name + f" {cfg.quants}")
+
+
+def test_block_types_c1_shapes(torch):
+    """Full-size shapes (hidden 7168, inter 2048, 64 experts + 1 shared) with
+    Q5_K gate/up and Q6_K down, one token, against the oracle."""
+    cfg = dataclasses.replace(synth.DECODE, n_experts=64, quants=(13, 13, 14), seed=46)
+    g = run_gpu(torch, cfg, 1)
+    ol = mixed_oracle_layer(cfg)
+    l64 = ref.router_logits(ref.bf16_to_f64(g["x"]), ol["router_w"], ol["router_b"])
+    near = pu.check_ids(g["ids"], l64, cfg.top_k)
+    forced = np.where(near[:, None], g["ids"], ref.topk_ids(l64, cfg.top_k))
+    r = ref.moe_forward(g["x"], ol, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter, forced_ids=forced)
+    pu.check_outputs(g["out"], r["out_bf16"], "c1 shapes Q5_K/Q6_K")
+
+
+def test_block_type_rejections(torch):
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_layer_create_mixed(256, 128, 16, 2, 0, 12, 3)          # Q4_1 is not supported
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_layer_create_mixed(256, 300, 16, 2, 0, 12, 8)          # Q8_0 down needs inter % 256 == 0
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED

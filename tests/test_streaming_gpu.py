@@ -13,6 +13,7 @@ import pytest
 from oracle import moe_ref as ref
 from routed_expert_ffn_forward_b200 import build, moe, synth
 from tests import parity_util as pu
+from tests.cache_model import CacheModel
 
 pytestmark = pytest.mark.gpu
 
@@ -26,51 +27,6 @@ def torch():
     moe.moe_set_cache_bytes(moe.SIZE_MAX)
     yield _t
     moe.moe_set_cache_bytes(moe.SIZE_MAX)
-
-
-class LRUModel:
-    """Host model of the cache policy: slots start in order 0..n-1 (front =
-    most recent); a miss takes the least recently used slot not needed by the
-    current forward; a forward touches its experts in ascending order, shared
-    experts last; prefetch misses avoid the last forward's slots."""
-
-    def __init__(self, n_slots):
-        self.order = list(range(n_slots))          # front = MRU
-        self.key = [None] * n_slots
-        self.epoch_of = [0] * n_slots
-        self.epoch = 0
-        self.hits = self.misses = self.prefetches = self.evictions = 0
-
-    def _touch(self, s):
-        self.order.remove(s)
-        self.order.insert(0, s)
-
-    def _fetch(self, key, pin, prefetch):
-        if key in self.key:
-            s = self.key.index(key)
-            if not prefetch:
-                self.hits += 1
-        else:
-            s = next(s for s in reversed(self.order) if self.epoch == 0 or self.epoch_of[s] != self.epoch)
-            if self.key[s] is not None:
-                self.evictions += 1
-            self.key[s] = key
-            if prefetch:
-                self.prefetches += 1
-            else:
-                self.misses += 1
-        self._touch(s)
-        if pin:
-            self.epoch_of[s] = self.epoch
-
-    def forward(self, layer, experts):
-        self.epoch += 1
-        for e in sorted(set(experts)):
-            self._fetch((layer, e), True, False)
-
-    def prefetch(self, layer, experts):
-        for e in experts:
-            self._fetch((layer, e), False, True)
 
 
 def to_dev(torch, bits):
@@ -100,9 +56,10 @@ SMALL = dataclasses.replace(synth.TINY, name="streaming small", n_shared=1, gati
                             steps=14, seed=21)
 
 
+@pytest.mark.parametrize("policy", ["lru", "lfu"])
 @pytest.mark.parametrize("prefetch", [False, True])
 @pytest.mark.parametrize("slots", [4, 7, 40])
-def test_streaming_matches_resident_and_lru_model(torch, prefetch, slots):
+def test_streaming_matches_resident_and_cache_model(torch, prefetch, slots, policy):
     from routed_expert_ffn_forward_b200.layer import layer_from_config
     cfg = SMALL
     trace = synth.streaming_trace(cfg)
@@ -113,16 +70,18 @@ def test_streaming_matches_resident_and_lru_model(torch, prefetch, slots):
         L.destroy()
     eb = moe.moe_expert_bytes(cfg.hidden, cfg.inter)
     moe.moe_set_cache_bytes(slots * eb + 7)
+    moe.moe_set_cache_policy(moe.MOE_CACHE_LFU if policy == "lfu" else moe.MOE_CACHE_LRU)
     try:
         layers = [layer_from_config(cfg, l) for l in range(cfg.n_layers)]
         moe.moe_reset_stats()
-        model = LRUModel(slots)
+        model = CacheModel(slots, policy)
         got = run_trace(torch, cfg, layers, trace, cfg.steps, prefetch=prefetch, model=model)
         st = moe.moe_get_stats()
         for L in layers:
             L.destroy()
     finally:
         moe.moe_set_cache_bytes(moe.SIZE_MAX)
+        moe.moe_set_cache_policy(moe.MOE_CACHE_LRU)
     for a, b in zip(got, want):
         np.testing.assert_array_equal(a, b)
     assert st["cache_slots"] == slots and st["slot_bytes"] == eb
@@ -250,3 +209,38 @@ def test_unpinned_host_memory_is_rejected(torch):
         moe.moe_forward(h, 16, 16, 1, None)
     assert ei.value.status == moe.MOE_ERR_NOT_READY
     moe.moe_layer_destroy(h)
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_streaming_block_types_against_oracle(torch, T):
+    """Q6_K gate/up (210-byte blocks, copied into 224-byte device slots) and
+    MXFP4 down (17-byte blocks grouped into 144 bytes) streamed through a small
+    cache, routed on the GPU (read back before the experts are fetched)."""
+    from routed_expert_ffn_forward_b200.layer import layer_from_config
+    cfg = dataclasses.replace(SMALL, quants=(14, 14, 39), inter=256, n_layers=2, seed=47)
+    eb = moe.moe_expert_bytes(cfg.hidden, cfg.inter, 14)
+    assert eb > 0
+    moe.moe_set_cache_bytes(8 * max(eb, moe.moe_expert_bytes(cfg.hidden, cfg.inter, 39)))
+    try:
+        layers = [layer_from_config(cfg, l) for l in range(cfg.n_layers)]
+        outs = []
+        for s in range(4):
+            for l in range(cfg.n_layers):
+                x = synth.activations(cfg, l, s, tokens=T)
+                o = layers[l].forward(to_dev(torch, x))
+                ids, _ = layers[l].routing(T)
+                outs.append((l, x, o.view(torch.int16).cpu().numpy().view(np.uint16), ids.cpu().numpy()))
+        torch.cuda.synchronize()
+        for L in layers:
+            moe.moe_check(L.handle)
+            L.destroy()
+    finally:
+        moe.moe_set_cache_bytes(moe.SIZE_MAX)
+    for l, x, o, ids in outs[-2:]:
+        layer = dict(router_w=synth.router_weight(cfg, l), router_b=synth.router_bias(cfg, l),
+                     experts=lambda e, l=l: synth.expert_tensors(cfg, l, e), quants=cfg.quants)
+        l64 = ref.router_logits(ref.bf16_to_f64(x), layer["router_w"], layer["router_b"])
+        near = pu.check_ids(ids, l64, cfg.top_k)
+        forced = np.where(near[:, None], ids, ref.topk_ids(l64, cfg.top_k))
+        r = ref.moe_forward(x, layer, cfg.top_k, cfg.gating, cfg.n_shared, cfg.inter, forced_ids=forced)
+        pu.check_outputs(o, r["out_bf16"], f"streamed {cfg.quants}")
