@@ -314,6 +314,27 @@ moe_status moe_route_noalloc(const void* x, const float* W, const float* bias, i
                              int top_k, moe_gating gating, int32_t* ids, float* weights,
                              void* stream);
 
+/* Expert parallelism (LayerStoRm README, "Notes": experts split across GPUs,
+ * with a deterministic expert-parallel combine).  Expert e of the layer
+ * (shared experts numbered E..E+S-1) belongs to rank e % world; after this
+ * call the layer fetches, caches and computes only its own experts.  Every
+ * rank runs the whole router.  world = 1 (the default) owns everything.
+ * Errors: INVALID_ARG unless 0 <= rank < world <= 1024. */
+moe_status moe_set_expert_parallel(moe_layer_t layer, int rank, int world);
+
+/* The layer's share of a forward: partial fp32 [T, H] (device, 16-byte
+ * aligned) = for every token, the sum over the token's experts that this rank
+ * owns, in the fixed combine order (weighted routed experts j = 0..k-1, then
+ * the shared ones), not rounded.  A token with none of this rank's experts
+ * gets zeros.  Otherwise as moe_forward. */
+moe_status moe_forward_partial(moe_layer_t layer, const void* x, float* partial, int T, void* stream);
+
+/* out bf16 [T, H] = bf16_rne(sum over r = 0..world-1, in rank order, of
+ * partials[r]), with partials fp32 [world][T][H] (device): the ranks'
+ * moe_forward_partial results gathered in rank order (an all-gather of T*H*4
+ * bytes per rank).  The same bits on every rank and every run. */
+moe_status moe_combine_partials(const float* partials, void* out, int T, int H, int world, void* stream);
+
 /* Test hooks for failure detection (process-wide, off by default), read by
  * the single-token kernel at each launch.  wait_limit_ns: limit of its bounded
  * waits (0 = the default 2 s); the final wait for its own copies in flight

@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         }
         routed = true;
       }
+      if (!ep_owned(expert_of(j), a.ep_rank, a.ep_world)) continue;   // another rank's expert
       const CUtensorMap* m = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + expert_of(j)), a.n_slots, a.err) + 3;
       for (int kb = 0; kb < a.nbh; ++kb) {
         if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, lim)) {
@@ -221,6 +222,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
       }
       const int jj = u / dn_tiles, rt = u - jj * dn_tiles;
       const int j = jj < S ? k + jj : jj - S;
+      if (!ep_owned(expert_of(j), a.ep_rank, a.ep_world)) continue;   // the slot stays free for the next claim
       const CUtensorMap* md = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + expert_of(j)), a.n_slots, a.err) + 6;
       for (int st = 0; st < n_dst; ++st) {
         if (st > 0 && !ptx::mbar_wait(&empty[stage], phase ^ 1u, lim)) {
@@ -400,10 +402,23 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         a.w[lane] = s_w[lane];
       }
       __syncwarp();
+      // contributions each output tile waits for: the experts this rank owns
+      int own = 0;
+      for (int q = 0; q < kS; ++q) own += ep_owned(s_ids[q], a.ep_rank, a.ep_world);
+      if (lane == 0) s_flag[3] = own;
       if (lane == 0) ptx::mbar_arrive(route_ready);
     }
     cbar();
     routed = true;
+    // a token none of whose experts this rank owns contributes zeros
+    if (!s_flag[0] && s_flag[3] == 0 && blockIdx.x == 0) {
+      for (int i = tid; i < H; i += kFzConsumers) {
+        if (a.partial)
+          a.partial[i] = 0.f;
+        else
+          a.out[i] = __float2bfloat16_rn(0.f);
+      }
+    }
   };
 
   int stage = 0;
@@ -425,6 +440,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         route();
         if (s_flag[0]) return;
       }
+      if (!ep_owned(j < k ? s_ids[j] : E + (j - k), a.ep_rank, a.ep_world)) continue;   // another rank's expert
       float acc[2] = {0.f, 0.f};  // gate row, up row
       bool ok = true;
       for (int kb = 0; kb < a.nbh; ++kb) {
@@ -553,15 +569,22 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         __threadfence();
       }
       cbar();
-      if (tid == 0) s_flag[1] = ptx::atom_add_acq_rel_gpu(sync + kSyncTile + rt, 1u) == (uint32_t)(kS - 1);
+      if (tid == 0)
+        s_flag[1] = ptx::atom_add_acq_rel_gpu(sync + kSyncTile + rt, 1u) == (uint32_t)(s_flag[3] - 1);
       cbar();
       if (s_flag[1] && warp < 2) {
-        // last contribution to this tile: out = sum_j w_j y_j (+ shared), fixed order
+        // last contribution to this tile: out = sum_j w_j y_j (+ shared), fixed
+        // order, over the experts this rank owns (all of them without EP)
         const int o = o0 + warp * 32 + lane;
         float acc2 = 0.f;
-        for (int q = 0; q < k; ++q) acc2 = fmaf(s_w[q], __ldcg(a.y + (size_t)q * H + o), acc2);
-        for (int q = k; q < kS; ++q) acc2 += __ldcg(a.y + (size_t)q * H + o);
-        a.out[o] = __float2bfloat16_rn(acc2);
+        for (int q = 0; q < k; ++q)
+          if (ep_owned(s_ids[q], a.ep_rank, a.ep_world)) acc2 = fmaf(s_w[q], __ldcg(a.y + (size_t)q * H + o), acc2);
+        for (int q = k; q < kS; ++q)
+          if (ep_owned(E + (q - k), a.ep_rank, a.ep_world)) acc2 += __ldcg(a.y + (size_t)q * H + o);
+        if (a.partial)
+          a.partial[o] = acc2;
+        else
+          a.out[o] = __float2bfloat16_rn(acc2);
       }
     }
   }

@@ -184,6 +184,7 @@ struct moe_layer {
   int* d_slot_of = nullptr;             // [E+S] expert -> slot of d_tmaps
   uint64_t cache_gen = 0;               // streaming: cache arena the maps point into
   cudaStream_t copy = nullptr;          // resident uploads
+  int ep_rank = 0, ep_world = 1;        // expert parallelism: the experts e % ep_world == ep_rank
   // scratch
   int T_cap = 0;
   void* scratch = nullptr;
@@ -466,6 +467,8 @@ moe_status resolve_experts(moe_layer* L, const int32_t* ids, int n, cudaStream_t
   std::vector<char> need(s.E + s.S, 0);
   for (int i = 0; i < n; ++i) need[ids[i]] = 1;
   for (int j = 0; j < s.S; ++j) need[s.E + j] = 1;
+  for (int e = 0; e < s.E + s.S; ++e)
+    if (!ep_owned(e, L->ep_rank, L->ep_world)) need[e] = 0;   // another rank's expert
   MOE_TRY(ensure_cache(L->device, L->expert_bytes));
   MOE_TRY(refresh_stream_maps(L));
   Cache* c = g_cache;
@@ -493,8 +496,10 @@ moe_status resolve_experts(moe_layer* L, const int32_t* ids, int n, cudaStream_t
   return MOE_OK;
 }
 
+// `partial` (fp32 [T, H]): write the unrounded sum over the experts this
+// layer owns there instead of the bf16 output (expert parallelism).
 moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int32_t* forced,
-                        cudaStream_t st) {
+                        cudaStream_t st, float* partial = nullptr) {
   NvtxRange nv(T == 1 ? "moe.forward T=1" : T <= kD1MaxTok ? "moe.forward decode" : "moe.forward prefill");
   if (!L) return fail(MOE_ERR_INVALID_ARG, "null layer");
   if (T < 0 || T > kMaxTokens) return fail(MOE_ERR_INVALID_ARG, "T=%d outside 0..%d", T, kMaxTokens);
@@ -573,7 +578,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
         if (T <= kD1MaxTok) {
           RouteArgs ra{xb, L->d_W, L->d_b, nullptr, T, s.H, s.E, s.k, s.S, (int)L->gating, wk.logits, wk.ids, wk.w,
                        wk.counts, wk.offsets, wk.perm, wk.inv, wk.act1, wk.n_act1, wk.act2, wk.n_act2, wk.n_act,
-                       wk.xq, wk.xq_plane, wk.xsc, wk.ticket};
+                       wk.xq, wk.xq_plane, wk.xsc, wk.ticket, L->ep_rank, L->ep_world};
           MOE_KERNEL(MOE_K_ROUTER, launch_route_decode(ra, st));
         } else {
           CUtensorMap xmap;
@@ -632,10 +637,13 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     fa.sbb_d = s.sbb_d;
     fa.stages = ring_stages;
     fa.stage_bytes = ring_stage_bytes;
+    fa.ep_rank = L->ep_rank;
+    fa.ep_world = L->ep_world;
     // one launch per token, in order (each reuses the kernel's scratch rows)
     for (int t = 0; t < T; ++t) {
       fa.x = xb + (size_t)t * s.H;
       fa.out = static_cast<__nv_bfloat16*>(out) + (size_t)t * s.H;
+      fa.partial = partial ? partial + (size_t)t * s.H : nullptr;
       fa.forced = dev_forced ? dev_forced + (size_t)t * s.k : nullptr;
       fa.logits = wk.logits + (size_t)t * s.E;
       fa.ids = wk.ids + (size_t)t * s.k;
@@ -660,7 +668,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
   if (fast) {
     RouteArgs ra{xb, L->d_W, L->d_b, forced ? wk.forced : nullptr, T, s.H, s.E, s.k, s.S, (int)L->gating,
                  wk.logits, wk.ids, wk.w, wk.counts, wk.offsets, wk.perm, wk.inv, wk.act1, wk.n_act1, wk.act2,
-                 wk.n_act2, wk.n_act, wk.xq, wk.xq_plane, wk.xsc, wk.ticket};
+                 wk.n_act2, wk.n_act, wk.xq, wk.xq_plane, wk.xsc, wk.ticket, L->ep_rank, L->ep_world};
     MOE_KERNEL(MOE_K_ROUTER, launch_route_decode(ra, st));
   } else {
     // router on the tensor cores: split-K partial logits, summed in split order by top-k
@@ -738,7 +746,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
       MOE_KERNEL(MOE_K_GATE_UP, launch_gate_up_d1(da, max_tok, s.n_sm, st));
       MOE_KERNEL(MOE_K_DOWN, launch_down_d1(da, max_tok, s.n_sm, st));
     }
-    MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true));
+    MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true, partial, L->ep_rank, L->ep_world));
   } else {
     // prefill: tensor-core GEMMs over tiles of up to 256 rows of one expert;
     // experts with <= kD1MaxTok rows (when their kernels fit) stream through
@@ -746,7 +754,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     const int kS = s.k + s.S, P = T * kS;
     const bool split_small = down_d1_smem(kD1MaxTok, act_slot) <= kMaxDecodeSmem;
     MOE_KERNEL(MOE_K_PERMUTE, launch_permute(wk.ids, T, s, wk, st));
-    MOE_KERNEL(MOE_K_PERMUTE, launch_build_tiles(wk, split_small ? kD1MaxTok : 0, st));
+    MOE_KERNEL(MOE_K_PERMUTE, launch_build_tiles(wk, split_small ? kD1MaxTok : 0, st, L->ep_rank, L->ep_world));
     if (split_small) MOE_KERNEL(MOE_K_PREP, launch_quant_x(xb, wk, T, s.H, st));
     MOE_KERNEL(MOE_K_PREP, launch_gather_rows(xb, wk, P, kS, s.H, st));
     GemmArgs ga{};
@@ -777,7 +785,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     ga.out_rows = s.H;
     MOE_KERNEL(MOE_K_DOWN, launch_prefill_gemm(1, L->h16_map, ga, s.n_sm, st));
     if (split_small) MOE_KERNEL(MOE_K_SMALL, launch_down_d1(da, kD1MaxTok, s.n_sm, st));
-    MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true));
+    MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true, partial, L->ep_rank, L->ep_world));
   }
 #undef MOE_KERNEL
   CUDA_TRY(cudaEventRecord(L->done, st));
@@ -1079,6 +1087,38 @@ static void* mapped_device_ptr(const void* p) {
   return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
 }
 
+moe_status moe_set_expert_parallel(moe_layer_t L, int rank, int world) {
+  g_err.clear();
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "null layer");
+  if (world < 1 || world > 1024 || rank < 0 || rank >= world)
+    return fail(MOE_ERR_INVALID_ARG, "rank=%d world=%d", rank, world);
+  L->ep_rank = rank;
+  L->ep_world = world;
+  return MOE_OK;
+}
+
+moe_status moe_forward_partial(moe_layer_t L, const void* x, float* partial, int T, void* stream) {
+  g_err.clear();
+  if (T > 0 && !partial) return fail(MOE_ERR_INVALID_ARG, "null partial");
+  if (reinterpret_cast<uintptr_t>(partial) & 15) return fail(MOE_ERR_INVALID_ARG, "partial must be 16-byte aligned");
+  // out is not written in this mode; pass the partial buffer for the checks
+  return forward_impl(L, x, partial, T, nullptr, static_cast<cudaStream_t>(stream), partial);
+}
+
+moe_status moe_combine_partials(const float* partials, void* out, int T, int H, int world, void* stream) {
+  g_err.clear();
+  if (T < 0 || H <= 0 || H % 4 || world < 1) return fail(MOE_ERR_INVALID_ARG, "T=%d H=%d world=%d", T, H, world);
+  if (T == 0) return MOE_OK;
+  if (!partials || !out) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+  if ((reinterpret_cast<uintptr_t>(partials) & 15) || (reinterpret_cast<uintptr_t>(out) & 7))
+    return fail(MOE_ERR_INVALID_ARG, "partials must be 16-byte and out 8-byte aligned");
+  CUDA_TRY(launch_combine_partials(partials, static_cast<__nv_bfloat16*>(out), T, H, world,
+                                   static_cast<cudaStream_t>(stream)));
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_stats.launches++;
+  return MOE_OK;
+}
+
 moe_status moe_forward_host(moe_layer_t L, const void* x_host, void* out_host, int T, void* stream) {
   g_err.clear();
   if (!L) return fail(MOE_ERR_INVALID_ARG, "null layer");
@@ -1140,6 +1180,7 @@ moe_status moe_prefetch(moe_layer_t L, const int32_t* ids, int n) {
   std::lock_guard<std::mutex> lk(g_mu);
   MOE_TRY(ensure_cache(L->device, L->expert_bytes));
   for (int i = 0; i < n; ++i) {
+    if (!ep_owned(ids[i], L->ep_rank, L->ep_world)) continue;   // another rank's expert
     int slot;
     MOE_TRY(cache_fetch(L, ids[i], 0, true, &slot));
   }

@@ -89,8 +89,13 @@ struct RouteArgs {
   size_t xq_plane;
   float2* xsc;
   unsigned* ticket;
+  int ep_rank, ep_world;  // expert parallelism: only experts e % ep_world == ep_rank get work
 };
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st);
+
+// Expert parallelism: expert e (shared experts numbered E..E+S-1) belongs to
+// rank e % world.  With world <= 1 every expert is owned.
+__host__ __device__ inline bool ep_owned(int e, int rank, int world) { return world <= 1 || e % world == rank; }
 // Copy `bytes` (a multiple of 16, both addresses 16-byte aligned) from mapped
 // host memory `src` (its device address) to device memory `dst`; the next
 // kernel may be launched as its programmatic dependent.
@@ -160,6 +165,8 @@ struct FusedArgs {
   int qgu, qd;               // GGUF block types of gate/up and of down
   int sbb_gu, sbb_d;         // their device bytes per 256-weight group
   int stages, stage_bytes;   // weight ring: stages x (256 x the larger group size)
+  int ep_rank, ep_world;     // expert parallelism: work only for owned experts
+  float* partial;            // non-null: write the owned experts' unrounded sum here instead of out
 };
 // Weight-ring geometry of the single-token kernel for these group sizes.
 inline void decode1_ring(int sbb_gu, int sbb_d, int* stages, int* stage_bytes) {
@@ -228,7 +235,7 @@ struct GemmArgs {
 size_t prefill_gemm_smem();
 size_t prefill_max_tiles(int n_experts_total, size_t pairs);
 // Tiles for the experts with more than small_rows rows; the others are listed in act1.
-cudaError_t launch_build_tiles(const Work& wk, int small_rows, cudaStream_t st);
+cudaError_t launch_build_tiles(const Work& wk, int small_rows, cudaStream_t st, int ep_rank = 0, int ep_world = 1);
 cudaError_t launch_quant_x(const __nv_bfloat16* x, const Work& wk, int T, int H, cudaStream_t st);
 cudaError_t launch_gather_rows(const __nv_bfloat16* x, const Work& wk, int P, int kS, int H, cudaStream_t st);
 cudaError_t launch_convert_h(const Work& wk, int P, int I, int I_pad, cudaStream_t st);
@@ -258,8 +265,14 @@ cudaError_t launch_topk(float* logits, int T, int E, int k, int gating,
                         const float* part = nullptr, int nsplit = 0, size_t split_stride = 0,
                         const float* bias = nullptr);
 cudaError_t launch_permute(const int* ids, int T, const Shape& s, const Work& wk, cudaStream_t st);
+// Weighted combine of each token's pairs in the fixed order.  With
+// `partial` (fp32 [T, H]) only the pairs whose expert this rank owns are
+// summed and the sum is written unrounded there instead of to `out`.
 cudaError_t launch_combine(const Work& wk, int T, const Shape& s, __nv_bfloat16* out, cudaStream_t st,
-                           bool pdl = false);
+                           bool pdl = false, float* partial = nullptr, int ep_rank = 0, int ep_world = 1);
+// out[t, h] = bf16_rne(sum over r = 0..world-1, in that order, of partials[r][t][h])
+cudaError_t launch_combine_partials(const float* partials, __nv_bfloat16* out, int T, int H, int world,
+                                    cudaStream_t st);
 
 // Streaming cache: point experts at their cache slots (the slot_of table the
 // kernels index tensor maps with).

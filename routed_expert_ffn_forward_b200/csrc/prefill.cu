@@ -415,7 +415,8 @@ __global__ void __launch_bounds__(1024) build_tiles_kernel(const int* __restrict
                                                            const int* __restrict__ counts,
                                                            const int* __restrict__ offsets, int4* __restrict__ tiles,
                                                            int* __restrict__ n_tiles, int small_rows,
-                                                           int* __restrict__ small, int* __restrict__ n_small) {
+                                                           int* __restrict__ small, int* __restrict__ n_small,
+                                                           int ep_rank, int ep_world) {
   __shared__ int s_warp[32];
   ptx::pdl_wait();
   const int na = __ldcg(n_act);
@@ -429,6 +430,7 @@ __global__ void __launch_bounds__(1024) build_tiles_kernel(const int* __restrict
       r0 = __ldcg(offsets + e);
       sm = c <= small_rows ? 1 : 0;
       nt = sm ? 0 : (c + kGN - 1) / kGN;
+      if (!ep_owned(e, ep_rank, ep_world)) sm = nt = 0;   // another rank's expert
     }
     int tot, stot;
     const int pos = base + block_exclusive_scan_1024(nt, &tot, s_warp);
@@ -587,10 +589,10 @@ size_t prefill_gemm_smem() { return kGemmSmem; }
 
 size_t prefill_max_tiles(int n_experts_total, size_t pairs) { return (size_t)n_experts_total + pairs / kGN + 1; }
 
-cudaError_t launch_build_tiles(const Work& wk, int small_rows, cudaStream_t st) {
+cudaError_t launch_build_tiles(const Work& wk, int small_rows, cudaStream_t st, int ep_rank, int ep_world) {
   return launch_pdl(build_tiles_kernel, dim3(1), dim3(1024), 0, st, (const int*)wk.act, (const int*)wk.n_act,
                     (const int*)wk.counts, (const int*)wk.offsets, wk.tiles, wk.n_tiles, small_rows, wk.act1,
-                    wk.n_act1);
+                    wk.n_act1, ep_rank, ep_world);
 }
 
 cudaError_t launch_quant_x(const __nv_bfloat16* x, const Work& wk, int T, int H, cudaStream_t st) {

@@ -164,7 +164,7 @@ __device__ void route_finish(const RouteArgs& a, int* s_ids) {
       const int kj = s_ids[j];
       lt += kj < ex;
       eq_before += (kj == ex) & (j < i);
-      const bool distinct_lt = (kj < ex) & (s_first[j] != 0);
+      const bool distinct_lt = (kj < ex) & (s_first[j] != 0) & ep_owned(kj, a.ep_rank, a.ep_world);
       d_small += distinct_lt & (s_count[j] <= kD1MaxTok);
       d_big += distinct_lt & (s_count[j] > kD1MaxTok);
     }
@@ -175,7 +175,9 @@ __device__ void route_finish(const RouteArgs& a, int* s_ids) {
     if (s_first[i]) {
       a.counts[ex] = s_count[i];
       a.offsets[ex] = lt;
-      if (s_count[i] <= kD1MaxTok) {
+      if (!ep_owned(ex, a.ep_rank, a.ep_world)) {
+        // another rank's expert: no work here
+      } else if (s_count[i] <= kD1MaxTok) {
         a.act1[d_small] = ex;
         atomicAdd(&s_cnt_small, 1);
       } else {
@@ -192,17 +194,24 @@ __device__ void route_finish(const RouteArgs& a, int* s_ids) {
     a.inv[t * kS + k + s] = r;
   }
   __syncthreads();
+  int own_shared = 0;  // owned shared experts (uniform across the block)
+  for (int q = 0; q < S; ++q) own_shared += ep_owned(E + q, a.ep_rank, a.ep_world);
   if (tid < S) {
     const int ex = E + tid;
     a.counts[ex] = T;
     a.offsets[ex] = N + tid * T;
-    if (T <= kD1MaxTok)
-      a.act1[s_cnt_small + tid] = ex;
-    else
-      a.act2[s_cnt_big + tid] = ex;
+    if (ep_owned(ex, a.ep_rank, a.ep_world)) {
+      int pos = 0;
+      for (int q = 0; q < tid; ++q) pos += ep_owned(E + q, a.ep_rank, a.ep_world);
+      if (T <= kD1MaxTok)
+        a.act1[s_cnt_small + pos] = ex;
+      else
+        a.act2[s_cnt_big + pos] = ex;
+    }
   }
   if (tid == 0) {
-    const int n1 = s_cnt_small + (T <= kD1MaxTok ? S : 0), n2 = s_cnt_big + (T <= kD1MaxTok ? 0 : S);
+    const int n1 = s_cnt_small + (T <= kD1MaxTok ? own_shared : 0),
+              n2 = s_cnt_big + (T <= kD1MaxTok ? 0 : own_shared);
     *a.n_act1 = n1;
     *a.n_act2 = n2;
     *a.n_act = n1 + n2;

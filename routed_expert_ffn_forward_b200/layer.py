@@ -95,6 +95,18 @@ class MoELayer:
         moe.moe_get_logits(self.handle, l.data_ptr(), torch.cuda.current_stream().cuda_stream)
         return l
 
+    def set_expert_parallel(self, rank: int, world: int) -> None:
+        moe.moe_set_expert_parallel(self.handle, rank, world)
+
+    def forward_partial(self, x: torch.Tensor, partial: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """This rank's unrounded fp32 share of the output (expert parallelism)."""
+        T = x.shape[0]
+        if partial is None:
+            partial = torch.empty((T, self.H), dtype=torch.float32, device=x.device)
+        s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+        moe.moe_forward_partial(self.handle, x.data_ptr(), partial.data_ptr(), T, s)
+        return partial
+
     def prefetch(self, ids) -> None:
         ids = np.ascontiguousarray(ids, dtype=np.int32)
         moe.moe_prefetch(self.handle, ids.ctypes.data, len(ids))

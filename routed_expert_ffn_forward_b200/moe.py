@@ -41,7 +41,8 @@ EXPORTS = ("moe_expert_bytes", "moe_layer_create", "moe_layer_create_mixed", "mo
            "moe_set_experts", "moe_set_cache_bytes", "moe_set_cache_policy", "moe_forward", "moe_forward_routed",
            "moe_forward_host", "moe_get_routing", "moe_get_logits", "moe_prefetch",
            "moe_check", "moe_get_stats", "moe_reset_stats", "moe_set_profiling", "moe_get_profile",
-           "moe_reset_profile", "moe_route_noalloc", "moe_set_test_hooks", "moe_last_error")
+           "moe_reset_profile", "moe_route_noalloc", "moe_set_test_hooks", "moe_set_expert_parallel",
+           "moe_forward_partial", "moe_combine_partials", "moe_last_error")
 
 KERNELS = ("router", "topk", "permute", "gate_up", "down", "combine", "prep", "small", "forward", "fused")
 
@@ -107,6 +108,9 @@ def lib() -> ctypes.CDLL:
             "moe_reset_profile": (_I, []),
             "moe_route_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
             "moe_set_test_hooks": (_I, [ctypes.c_uint64, _I]),
+            "moe_set_expert_parallel": (_I, [_P, _I, _I]),
+            "moe_forward_partial": (_I, [_P, _P, _P, _I, _P]),
+            "moe_combine_partials": (_I, [_P, _P, _I, _I, _I, _P]),
             "moe_last_error": (ctypes.c_char_p, []),
         }
         for name, (res, args) in sig.items():
@@ -222,6 +226,18 @@ def moe_reset_profile() -> None:
 def moe_route_noalloc(x: int, W: int, bias: int | None, T: int, H: int, E: int, top_k: int, gating: int,
                       ids: int, weights: int, stream: int | None = None) -> None:
     _check(lib().moe_route_noalloc(x, W, bias or None, T, H, E, top_k, gating, ids, weights, stream or None))
+
+
+def moe_set_expert_parallel(layer: int, rank: int, world: int) -> None:
+    _check(lib().moe_set_expert_parallel(layer, rank, world))
+
+
+def moe_forward_partial(layer: int, x: int, partial: int, T: int, stream: int | None = None) -> None:
+    _check(lib().moe_forward_partial(layer, x, partial, T, stream or None))
+
+
+def moe_combine_partials(partials: int, out: int, T: int, H: int, world: int, stream: int | None = None) -> None:
+    _check(lib().moe_combine_partials(partials, out, T, H, world, stream or None))
 
 
 def moe_set_test_hooks(wait_limit_ns: int, hold_barrier: int) -> None:
