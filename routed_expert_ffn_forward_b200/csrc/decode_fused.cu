@@ -216,7 +216,12 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
       }
       const int u = (int)atomicAdd(sync + kSyncNext, 1u);
       if (u >= n_dn) {
-        s_unit[stage] = -1;          // end of work
+        // end of work.  The stage is empty, so its last copy has landed and
+        // been read; its arrival below completes one more phase of full[stage],
+        // so the final drain must not wait for that copy's phase again (the
+        // parity would match the phase after next and never complete).
+        s_unit[stage] = -1;
+        issued &= ~(1u << stage);
         ptx::mbar_arrive(&full[stage]);
         break;
       }

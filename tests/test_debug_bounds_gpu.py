@@ -26,7 +26,9 @@ build.build(debug_bounds=True)
 cfgs = [synth.TINY, dataclasses.replace(synth.TINY, hidden=512, inter=300, n_experts=40, top_k=5, n_shared=2,
                                         gating=1, seed=13, router_std=1 / 512 ** 0.5)]
 for cfg in cfgs:
-    for stream_slots in (None, 12):
+    # resident, then streamed through a cache with room for every expert of
+    # the layer (T = 17 may route to all of them)
+    for stream_slots in (None, cfg.n_experts + cfg.n_shared + 2):
         moe.moe_set_cache_bytes(moe.SIZE_MAX if stream_slots is None
                                 else stream_slots * moe.moe_expert_bytes(cfg.hidden, cfg.inter))
         L = layer_from_config(cfg)
