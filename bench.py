@@ -465,12 +465,14 @@ def run_streaming(args, cfg, rank, world, local_rank, peaks) -> dict:
     token per layer with the trace's routing.  Each mode empties the cache,
     runs the warm-up steps, then times the steps:
       <policy>+demand     misses are fetched when a forward needs them
-      <policy>+lookahead  before layer l runs, layer l+1's router (through
-                          moe_route_noalloc) is applied to layer l's input and
-                          the experts it picks are prefetched: a predictor that
-                          reads nothing of the future
-      <policy>+trace      the next layer's experts are read from the trace and
-                          prefetched: an oracle predictor, an upper bound
+      <policy>+lookahead  layer l+1's router (moe_route_noalloc, on a
+                          high-priority side stream) is applied to layer l's
+                          input, and while layer l runs the experts it picks
+                          are prefetched: a predictor that reads nothing of
+                          the future
+      <policy>+trace      while layer l runs, layer l+1's experts are read from
+                          the trace and prefetched: an oracle predictor, an
+                          upper bound
     with policy lru or lfu (moe_set_cache_policy).  `value` is the fastest
     mode that does not read the trace."""
     import torch
@@ -495,19 +497,29 @@ def run_streaming(args, cfg, rank, world, local_rank, peaks) -> dict:
     bs = [torch.from_numpy(synth.router_bias(cfg, l)).to(dev) for l in range(cfg.n_layers)]
     p_ids = torch.empty((1, cfg.top_k), dtype=torch.int32, device=dev)
     p_w = torch.empty((1, cfg.top_k), dtype=torch.float32, device=dev)
+    p_host = torch.empty((1, cfg.top_k), dtype=torch.int32).pin_memory()
+    side = torch.cuda.Stream(dev, priority=-1)   # the predictor's router, beside the layer's forward
+    p_done = torch.cuda.Event()
     modes = args.stream_modes.split(",") if args.stream_modes else list(STREAM_MODES)
 
     def run_step(s, how):
         for l in range(cfg.n_layers):
             nl, ns = (l + 1, s) if l + 1 < cfg.n_layers else (0, s + 1)
+            if how == "lookahead":
+                # route layer l's input with layer l+1's router on the side
+                # stream, queue layer l, then prefetch while layer l runs
+                moe.moe_route_noalloc(x_dev[s, l].data_ptr(), Ws[nl].data_ptr(), bs[nl].data_ptr(), 1, cfg.hidden,
+                                      cfg.n_experts, cfg.top_k, cfg.gating, p_ids.data_ptr(), p_w.data_ptr(),
+                                      side.cuda_stream)
+                with torch.cuda.stream(side):
+                    p_host.copy_(p_ids, non_blocking=True)
+                    p_done.record(side)
+            layers[l].forward_routed(x_dev[s, l], trace[s, l][None], out, stream.cuda_stream)
             if how == "trace" and ns < n_steps:
                 layers[nl].prefetch(trace[ns, nl])
             elif how == "lookahead":
-                moe.moe_route_noalloc(x_dev[s, l].data_ptr(), Ws[nl].data_ptr(), bs[nl].data_ptr(), 1, cfg.hidden,
-                                      cfg.n_experts, cfg.top_k, cfg.gating, p_ids.data_ptr(), p_w.data_ptr(),
-                                      stream.cuda_stream)
-                layers[nl].prefetch(p_ids.cpu().numpy()[0])
-            layers[l].forward_routed(x_dev[s, l], trace[s, l][None], out, stream.cuda_stream)
+                p_done.synchronize()
+                layers[nl].prefetch(p_host.numpy()[0])
 
     res = {}
     clocks = None

@@ -197,8 +197,9 @@ typedef enum {
  * the layer's previous forward did not (prefetches excluded), halving all
  * counts after every 64 x slots arrivals so that popularity ages.  A miss
  * takes an empty slot if there is one, else evicts, preferably among experts
- * that their layer's previous forward did not use, the one with the fewest
- * arrivals (the least recently used among equals).  An expert a layer keeps
+ * neither prefetched (moe_prefetch) for their layer's next forward nor used by
+ * their layer's previous forward, the one with the fewest arrivals (the least
+ * recently used among equals).  An expert a layer keeps
  * using stays; among the rest the popular ones stay where LRU would let
  * one-off experts push them out.
  * Errors: INVALID_ARG for an unknown policy.

@@ -61,7 +61,7 @@ constexpr unsigned kErrFzProducer = 1u << 10, kErrFzConsumer = 1u << 11, kErrFzG
                    kErrFzReady = 1u << 13;
 
 // global sync words (FusedArgs::sync)
-constexpr int kSyncBarCount = 0, kSyncBarGen = 1, kSyncNext = 2, kSyncReady = 8, kSyncTile = 64;
+constexpr int kSyncBarCount = 0, kSyncBarGen = 1, kSyncNext = 2, kSyncDone = 3, kSyncReady = 8;
 
 // Shared-memory layout (offsets from the 1024-aligned base).
 struct FzLayout {
@@ -73,8 +73,8 @@ struct FzLayout {
     ids = unit + kFzStages * 4;                       // int [40]
     w = ids + 40 * 4;                                 // float [40]
     flags = w + 40 * 4;                               // int [4]
-    part = up16(flags + 16);                          // float [1024]
-    xh = part + 1024 * 4;                             // u8 [H]
+    part = up16(flags + 16);                          // float [2][1024]
+    xh = part + 2048 * 4;                             // u8 [H]
     xl = xh + (uint32_t)H;                            // u8 [H]
     xsc = xl + (uint32_t)H;                           // float2 [H/32]
     uni = up16(xsc + (uint32_t)(H / 32) * 8);         // bf16 x [H] | act slots [2][act_slot]
@@ -354,12 +354,13 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
     // CTA 0 zeroes the step counters for this launch before it arrives: no
     // CTA touches them until it has passed the barrier
     if (blockIdx.x == 0) {
-      if (tid == 0) sync[kSyncNext] = 0u;
+      if (tid == 0) {
+        sync[kSyncNext] = 0u;
+        sync[kSyncDone] = 0u;
+      }
       for (int i = tid; i < kS; i += kFzConsumers) sync[kSyncReady + i] = 0u;
-      for (int i = tid; i < dn_tiles; i += kFzConsumers) sync[kSyncTile + i] = 0u;
     }
-    __threadfence();
-    cbar();
+    cbar();   // thread 0's fence below is cumulative over these writes and the logits
     if (tid == 0) {
       const uint32_t gen = ptx::ld_acquire_gpu(sync + kSyncBarGen);
       s_flag[2] = (int)gen;
@@ -415,15 +416,6 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
     }
     cbar();
     routed = true;
-    // a token none of whose experts this rank owns contributes zeros
-    if (!s_flag[0] && s_flag[3] == 0 && blockIdx.x == 0) {
-      for (int i = tid; i < H; i += kFzConsumers) {
-        if (a.partial)
-          a.partial[i] = 0.f;
-        else
-          a.out[i] = __float2bfloat16_rn(0.f);
-      }
-    }
   };
 
   int stage = 0;
@@ -490,7 +482,6 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         a.hq[o] = hh;
         reinterpret_cast<uint8_t*>(a.hq + a.hq_plane)[o] = hl;
         if (lane == 0) a.hsc[(size_t)j * (a.I_pad / 32) + feat / 32] = rsc;
-        __threadfence();
       }
       // publish the features (the ready counters are zeroed before the barrier)
       if (!routed) {
@@ -510,11 +501,15 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
     if (s_flag[0]) return;
   }
 
-  // (4) down units, then the combine of each completed output tile
+  // (4) down units.  A unit's 64 rows of y_j are published with one release
+  // add to the count of finished units, which no thread waits on; (5) once
+  // every unit of the forward is counted, the CTAs combine slices of the
+  // output.  The unit partials are double-buffered, so the two warps that
+  // reduce them may lag the others by a unit.
   {
     const int r0 = lane, sb = warp >> 2, c = warp & 3;   // rows lane and lane + 32; part = warp
     const int I_pad = a.I_pad;
-    int aslot = 0;
+    int aslot = 0, buf = 0;
     uint32_t aphase = 0;
     while (true) {
       bool ok = ptx::mbar_wait(&full[stage], phase, lim);
@@ -557,40 +552,47 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         }
       }
       if (!ok) fail(kErrFzConsumer);
-      cbar();                          // also: the previous unit's reads of s_part are done
+      float* sp = s_part + buf * (kFzWarps * kFzDnRows);
+      if (u >= 0) {
+        sp[warp * kFzDnRows + r0] = acc[0];
+        sp[warp * kFzDnRows + r0 + 32] = acc[1];
+      }
+      cbar();                          // every warp, every unit: the partials are complete
       if (s_flag[0]) return;
       if (u < 0) break;                // every warp read the same end marker
-      s_part[warp * kFzDnRows + r0] = acc[0];
-      s_part[warp * kFzDnRows + r0 + 32] = acc[1];
-      cbar();
-      // the 16 parts of each row, in a fixed order, to y_j
-      const int o0 = rt * kFzDnRows;
       if (warp < 2) {
+        // the 16 parts of each row, in a fixed order, to y_j; then one thread
+        // publishes the unit (release: cumulative over the two warps' stores)
         const int r = warp * 32 + lane;
-        float v = s_part[r];
+        float v = sp[r];
 #pragma unroll
-        for (int p = 1; p < kFzWarps; ++p) v += s_part[p * kFzDnRows + r];
-        a.y[(size_t)j * H + o0 + r] = v;
-        __threadfence();
+        for (int p = 1; p < kFzWarps; ++p) v += sp[p * kFzDnRows + r];
+        a.y[(size_t)j * H + rt * kFzDnRows + r] = v;
+        ptx::named_barrier_sync(2, 64);
+        if (tid == 0) ptx::red_add_release_gpu(sync + kSyncDone, 1u);
       }
-      cbar();
-      if (tid == 0)
-        s_flag[1] = ptx::atom_add_acq_rel_gpu(sync + kSyncTile + rt, 1u) == (uint32_t)(s_flag[3] - 1);
-      cbar();
-      if (s_flag[1] && warp < 2) {
-        // last contribution to this tile: out = sum_j w_j y_j (+ shared), fixed
-        // order, over the experts this rank owns (all of them without EP)
-        const int o = o0 + warp * 32 + lane;
-        float acc2 = 0.f;
-        for (int q = 0; q < k; ++q)
-          if (ep_owned(s_ids[q], a.ep_rank, a.ep_world)) acc2 = fmaf(s_w[q], __ldcg(a.y + (size_t)q * H + o), acc2);
-        for (int q = k; q < kS; ++q)
-          if (ep_owned(E + (q - k), a.ep_rank, a.ep_world)) acc2 += __ldcg(a.y + (size_t)q * H + o);
-        if (a.partial)
-          a.partial[o] = acc2;
-        else
-          a.out[o] = __float2bfloat16_rn(acc2);
-      }
+      buf ^= 1;
+    }
+
+    // (5) combine: out = sum over the picks this rank owns (all of them
+    // without expert parallelism) of w_j y_j, then the shared experts, in
+    // that fixed order; CTA c takes outputs c*512 .. c*512+511, + grid*512, ...
+    if (tid == 0) {
+      const uint32_t want = (uint32_t)(s_flag[3] * dn_tiles);
+      if (!spin_until_ge(sync + kSyncDone, want, lim)) fail(kErrFzReady);
+    }
+    cbar();
+    if (s_flag[0]) return;
+    for (int o = blockIdx.x * kFzConsumers + tid; o < H; o += gridDim.x * kFzConsumers) {
+      float acc2 = 0.f;
+      for (int q = 0; q < k; ++q)
+        if (ep_owned(s_ids[q], a.ep_rank, a.ep_world)) acc2 = fmaf(s_w[q], __ldcg(a.y + (size_t)q * H + o), acc2);
+      for (int q = k; q < kS; ++q)
+        if (ep_owned(E + (q - k), a.ep_rank, a.ep_world)) acc2 += __ldcg(a.y + (size_t)q * H + o);
+      if (a.partial)
+        a.partial[o] = acc2;
+      else
+        a.out[o] = __float2bfloat16_rn(acc2);
     }
   }
   ptx::pdl_launch_dependents();

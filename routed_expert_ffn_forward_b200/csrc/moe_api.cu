@@ -107,11 +107,13 @@ struct Cache {
   // MOE_CACHE_LFU bookkeeping for every (layer, expert) key seen, cached or
   // not: how often it entered use (used by a forward of its layer after not
   // being used by that layer's previous forward), and the layer's forward
-  // index at its last use.  Arrival counts halve every kAgeEvery * n_slots
-  // arrivals, so that old popularity fades.
+  // index at its last use, and the forward a prefetch fetched it for.  Arrival
+  // counts halve every kAgeEvery * n_slots arrivals, so that old popularity
+  // fades.
   struct Use {
     uint32_t arrivals = 0;
     uint64_t last_fwd = 0;
+    uint64_t prefetched_for = 0;
   };
   std::unordered_map<uint64_t, Use> use;
   std::unordered_map<uint32_t, uint64_t> layer_fwds;  // layer id -> forwards resolved so far
@@ -366,15 +368,16 @@ moe_status cache_fetch(moe_layer* L, int e, uint64_t pin_epoch, bool prefetch, i
     }
     u.last_fwd = f;
   }
+  if (prefetch && g_cache_policy == MOE_CACHE_LFU) c->use[key].prefetched_for = c->layer_fwds[L->id] + 1;
   if (it != c->where.end()) {
     s = it->second;
     if (!prefetch) g_stats.cache_hits++;
   } else {
     // victim, among the slots not needed by the current forward: LRU takes
     // the least recently used.  LFU takes an empty slot if there is one, else
-    // prefers experts not used by their layer's previous forward and among
-    // those the one that entered use least often; the least recently used
-    // among equals
+    // keeps experts prefetched for their layer's next forward, then those used
+    // by their layer's previous forward, and among the rest takes the one that
+    // entered use least often; the least recently used among equals
     int victim = -1;
     uint64_t best = UINT64_MAX;
     for (auto r = c->lru.rbegin(); r != c->lru.rend(); ++r) {
@@ -385,8 +388,10 @@ moe_status cache_fetch(moe_layer* L, int e, uint64_t pin_epoch, bool prefetch, i
           break;
         }
         const Cache::Use& u = c->use[k2];
-        const bool recent = u.last_fwd != 0 && c->layer_fwds[(uint32_t)(k2 >> 32)] - u.last_fwd < 2;
-        const uint64_t score = ((uint64_t)recent << 32) | u.arrivals;
+        const uint64_t lf = c->layer_fwds[(uint32_t)(k2 >> 32)];
+        const bool recent = u.last_fwd != 0 && lf - u.last_fwd < 2;
+        const bool pending = u.prefetched_for > lf;   // that forward has not run yet
+        const uint64_t score = ((uint64_t)pending << 33) | ((uint64_t)recent << 32) | u.arrivals;
         if (score < best) {
           best = score;
           victim = *r;

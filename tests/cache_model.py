@@ -8,8 +8,9 @@ class CacheModel:
     its experts in ascending order, shared experts last, and a miss takes a
     slot not needed by the current forward (prefetch misses avoid the last
     forward's slots).  LRU takes the least recently used one.  LFU takes an
-    empty slot if there is one, else prefers experts that their layer's
-    previous forward did not use and among those the one with the fewest
+    empty slot if there is one, else keeps experts prefetched for their layer's
+    next forward (until that forward has run), then prefers experts that their
+    layer's previous forward did not use and among those the one with the fewest
     arrivals (forwards of its layer that used it when the layer's previous
     forward did not; all counts halve after every 64 x slots arrivals), the
     least recently used among equals."""
@@ -24,7 +25,7 @@ class CacheModel:
         self.epoch_of = [0] * n_slots
         self.epoch = 0
         self.layer_fwds = {}
-        self.use = {}                              # key -> [arrivals, last forward of its layer]
+        self.use = {}           # key -> [arrivals, last forward of its layer, forward prefetched for]
         self.arrivals = 0
         self.hits = self.misses = self.prefetches = self.evictions = 0
 
@@ -40,9 +41,10 @@ class CacheModel:
             k = self.key[s]
             if self.policy == "lru" or k is None:
                 return s
-            arrivals, last = self.use.get(k, (0, 0))
-            recent = last != 0 and self.layer_fwds[k[0]] - last < 2
-            score = (recent, arrivals)
+            arrivals, last, pf = self.use.get(k, (0, 0, 0))
+            lf = self.layer_fwds.get(k[0], 0)
+            recent = last != 0 and lf - last < 2
+            score = (pf > lf, recent, arrivals)
             if best is None or score < best:
                 best, victim = score, s
         return victim
@@ -50,7 +52,7 @@ class CacheModel:
     def _fetch(self, key, pin, prefetch):
         if not prefetch and self.policy == "lfu":
             f = self.layer_fwds[key[0]]
-            u = self.use.setdefault(key, [0, 0])
+            u = self.use.setdefault(key, [0, 0, 0])
             if u[1] == 0 or f - u[1] > 1:
                 u[0] += 1
                 self.arrivals += 1
@@ -58,6 +60,8 @@ class CacheModel:
                     for v in self.use.values():
                         v[0] >>= 1
             u[1] = f
+        if prefetch and self.policy == "lfu":
+            self.use.setdefault(key, [0, 0, 0])[2] = self.layer_fwds.get(key[0], 0) + 1
         if key in self.key:
             s = self.key.index(key)
             if not prefetch:
