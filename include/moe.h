@@ -97,7 +97,7 @@ enum {
   MOE_K_DOWN = 4,    /* down projection */
   MOE_K_COMBINE = 5, /* weighted combine */
   MOE_K_PREP = 6,    /* prefill only: activation rows and SwiGLU output to scaled fp16 */
-  MOE_K_SMALL = 7,   /* prefill only: the decode kernels for experts with <= 4 rows */
+  MOE_K_SMALL = 7,   /* prefill only: the few-row tiles (moe_set_few_row_tiles) */
   MOE_K_FORWARD = 8, /* whole forward, first kernel start to last kernel end */
   MOE_K_FUSED = 9,   /* decode of one token as one kernel (router through combine) */
   MOE_K_COUNT = 10
@@ -207,6 +207,20 @@ typedef enum {
  * ranked by how often they are used); LayerStoRm README, "Status and
  * limitations" (cache and prefetch policy as active work). */
 moe_status moe_set_cache_policy(int policy);
+
+/* Prefill path (T > 4), process-wide, read at each forward: an expert with at
+ * most max_rows rows, and the last partial 256-row tile of a larger expert
+ * when it has at most max_rows rows, runs on the few-row kernel (warp-level
+ * fp16 MMAs, Q4_K dequantised in registers: one pass over the weights at the
+ * HBM rate, whatever the row count) instead of the tensor-memory GEMM, whose
+ * cost per tile is its dequantisation of all 256 weight rows of every feature
+ * block, whatever the row count.  Both compute the same fp16 products with
+ * fp32 accumulation; the rounding order differs.  0 = off: all tiles on the
+ * GEMM and experts with <= 4 rows on the decode kernels.
+ * Default 64; errors: INVALID_ARG outside 0..64.
+ * Source: LayerStoRm README, "Notes" (decode and prefill throughput measured
+ * on the boot-verified configuration: both paths are the product). */
+moe_status moe_set_few_row_tiles(int max_rows);
 
 /* Forward: x bf16 [T, H] and out bf16 [T, H], device pointers, row-major.
  * T >= 0 (T = 0 returns at once).  T <= 4 takes the decode path (fused router,

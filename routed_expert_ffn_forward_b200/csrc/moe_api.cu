@@ -82,6 +82,7 @@ size_t g_cache_bytes = SIZE_MAX;
 int g_cache_policy = MOE_CACHE_LRU;
 uint64_t g_hook_wait_ns = 0;  // moe_set_test_hooks
 int g_hook_hold = 0;
+int g_mt_rows = kMtMaxRows;    // moe_set_few_row_tiles
 uint32_t g_next_layer_id = 1;
 
 struct Slot {
@@ -244,6 +245,7 @@ moe_status ensure_scratch(moe_layer* L, int T, cudaStream_t st) {
                o_hq = take(P * s.I_pad * 2), o_hsc = take(P * (s.I_pad / 32) * 8), o_act1 = take(ES * 4),
                o_act2 = take(ES * 4), o_nact1 = take(4), o_nact2 = take(4),
                o_err = take(4), o_tiles = take(prefill_max_tiles((int)ES, P) * 16), o_ntiles = take(4),
+               o_mtiles = take(ES * 16), o_nmtiles = take(4), o_mtnext = take(8),
                o_x16 = take(P * s.H * 2), o_rinv = take(P * 4), o_h16 = take(P * s.I_pad * 2), o_hinv = take(P * 4),
                o_rpart = take(router_part_floats(cap, s.E, s.n_sm) * 4), o_sync = take(kSyncWords * 4);
   if (L->scratch) {
@@ -287,6 +289,9 @@ moe_status ensure_scratch(moe_layer* L, int T, cudaStream_t st) {
   L->wk.err = reinterpret_cast<unsigned*>(b + o_err);
   L->wk.tiles = reinterpret_cast<int4*>(b + o_tiles);
   L->wk.n_tiles = reinterpret_cast<int*>(b + o_ntiles);
+  L->wk.mtiles = reinterpret_cast<int4*>(b + o_mtiles);
+  L->wk.n_mtiles = reinterpret_cast<int*>(b + o_nmtiles);
+  L->wk.mt_next = reinterpret_cast<unsigned*>(b + o_mtnext);
   L->wk.x16 = reinterpret_cast<__half*>(b + o_x16);
   L->wk.rinv = reinterpret_cast<float*>(b + o_rinv);
   L->wk.h16 = reinterpret_cast<__half*>(b + o_h16);
@@ -528,12 +533,13 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
   ProfRec pr{};
   bool prof;
   uint64_t hook_wait_ns;
-  int hook_hold;
+  int hook_hold, mt_rows;
   {
     std::lock_guard<std::mutex> lk0(g_mu);
     prof = g_profiling;
     hook_wait_ns = g_hook_wait_ns;
     hook_hold = g_hook_hold;
+    mt_rows = g_mt_rows;
     if (prof)
       for (int i = 0; i < 2 * kProfRanges; ++i) pr.ev[i] = prof_event();
   }
@@ -754,12 +760,16 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true, partial, L->ep_rank, L->ep_world));
   } else {
     // prefill: tensor-core GEMMs over tiles of up to 256 rows of one expert;
-    // experts with <= kD1MaxTok rows (when their kernels fit) stream through
-    // the decode kernels instead, which do not dequantise
+    // experts with <= mt_rows rows, and last partial tiles that small, run on
+    // the few-row warp-MMA kernel instead (dequantisation in registers, one
+    // weight pass at the HBM rate); with mt_rows == 0, experts with <=
+    // kD1MaxTok rows (when their kernels fit) stream through the decode
+    // kernels instead, which do not dequantise
     const int kS = s.k + s.S, P = T * kS;
-    const bool split_small = down_d1_smem(kD1MaxTok, act_slot) <= kMaxDecodeSmem;
+    const bool split_small = mt_rows == 0 && down_d1_smem(kD1MaxTok, act_slot) <= kMaxDecodeSmem;
     MOE_KERNEL(MOE_K_PERMUTE, launch_permute(wk.ids, T, s, wk, st));
-    MOE_KERNEL(MOE_K_PERMUTE, launch_build_tiles(wk, split_small ? kD1MaxTok : 0, st, L->ep_rank, L->ep_world));
+    MOE_KERNEL(MOE_K_PERMUTE,
+               launch_build_tiles(wk, split_small ? kD1MaxTok : 0, mt_rows, st, L->ep_rank, L->ep_world));
     if (split_small) MOE_KERNEL(MOE_K_PREP, launch_quant_x(xb, wk, T, s.H, st));
     MOE_KERNEL(MOE_K_PREP, launch_gather_rows(xb, wk, P, kS, s.H, st));
     GemmArgs ga{};
@@ -779,7 +789,15 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     ga.err = wk.err;
     ga.n_ex = s.E + s.S;
     ga.n_slots = (int)L->n_tmap_slots;
+    ga.n_rows = P;
     MOE_KERNEL(MOE_K_GATE_UP, launch_prefill_gemm(0, L->x16_map, ga, s.n_sm, st));
+    GemmArgs gm = ga;   // the few-row tiles
+    gm.tiles = wk.mtiles;
+    gm.n_tiles = wk.n_mtiles;
+    gm.bsrc = wk.x16;
+    gm.b_ld = s.H;
+    gm.next = wk.mt_next;
+    if (mt_rows) MOE_KERNEL(MOE_K_SMALL, launch_prefill_mt(0, gm, s.n_sm, st));
     if (split_small) MOE_KERNEL(MOE_K_SMALL, launch_gate_up_d1(da, kD1MaxTok, s.n_sm, st));
     MOE_KERNEL(MOE_K_PREP, launch_convert_h(wk, P, s.I, s.I_pad, st));
     ga.ft = s.H / 256;
@@ -789,6 +807,16 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     ga.out_ld = s.H;
     ga.out_rows = s.H;
     MOE_KERNEL(MOE_K_DOWN, launch_prefill_gemm(1, L->h16_map, ga, s.n_sm, st));
+    gm.ft = ga.ft;
+    gm.nkb = ga.nkb;
+    gm.rinv = ga.rinv;
+    gm.out = ga.out;
+    gm.out_ld = ga.out_ld;
+    gm.out_rows = ga.out_rows;
+    gm.bsrc = wk.h16;
+    gm.b_ld = s.I_pad;
+    gm.next = wk.mt_next + 1;
+    if (mt_rows) MOE_KERNEL(MOE_K_SMALL, launch_prefill_mt(1, gm, s.n_sm, st));
     if (split_small) MOE_KERNEL(MOE_K_SMALL, launch_down_d1(da, kD1MaxTok, s.n_sm, st));
     MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true, partial, L->ep_rank, L->ep_world));
   }
@@ -1058,6 +1086,15 @@ moe_status moe_set_test_hooks(uint64_t wait_limit_ns, int hold_barrier) {
   std::lock_guard<std::mutex> lk(g_mu);
   g_hook_wait_ns = wait_limit_ns;
   g_hook_hold = hold_barrier;
+  return MOE_OK;
+}
+
+moe_status moe_set_few_row_tiles(int max_rows) {
+  g_err.clear();
+  if (max_rows < 0 || max_rows > kMtMaxRows)
+    return fail(MOE_ERR_INVALID_ARG, "max_rows=%d outside 0..%d", max_rows, kMtMaxRows);
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_mt_rows = max_rows;
   return MOE_OK;
 }
 

@@ -65,6 +65,9 @@ struct Work {
   // prefill path (tensor-core GEMMs)
   int4* tiles;        // [max tiles] (expert, n0, count, r0): up to 256 rows of one expert
   int* n_tiles;
+  int4* mtiles;       // [E+S] few-row tiles (expert, n0, count <= kMtMaxRows, r0)
+  int* n_mtiles;
+  unsigned* mt_next;  // [2] unit counters of the few-row kernels (gate/up, down)
   __half* x16;        // [P_cap, H] activations of each row, fp16 scaled by 1/rinv, K order (0,2,1,3)
   float* rinv;        // [P]
   __half* h16;        // [P_cap, I_pad] SwiGLU output, fp16 scaled by 1/hinv, same K order
@@ -231,15 +234,29 @@ struct GemmArgs {
   int wexp_stride, wexp_down;
   unsigned* err;
   int n_ex, n_slots;         // bounds of expert ids and cache slots (debug builds)
+  // few-row kernel (launch_prefill_mt): its activation rows, fp16 [P, b_ld]
+  // in the GEMM's K order, and its unit counter (zeroed by build_tiles)
+  const __half* bsrc;
+  int b_ld;
+  unsigned* next;
+  int n_rows;                // activation rows P (debug builds)
 };
+constexpr int kMtMaxRows = 64;   // most activation rows of a few-row tile
 size_t prefill_gemm_smem();
 size_t prefill_max_tiles(int n_experts_total, size_t pairs);
-// Tiles for the experts with more than small_rows rows; the others are listed in act1.
-cudaError_t launch_build_tiles(const Work& wk, int small_rows, cudaStream_t st, int ep_rank = 0, int ep_world = 1);
+// GEMM tiles of up to 256 rows for the experts with more than small_rows rows
+// (the others are listed in act1); with mt_rows > 0, an expert with at most
+// mt_rows rows, and the last partial tile of a larger one when it has at most
+// mt_rows rows, become few-row tiles (mtiles) instead.
+cudaError_t launch_build_tiles(const Work& wk, int small_rows, int mt_rows, cudaStream_t st, int ep_rank = 0,
+                               int ep_world = 1);
 cudaError_t launch_quant_x(const __nv_bfloat16* x, const Work& wk, int T, int H, cudaStream_t st);
 cudaError_t launch_gather_rows(const __nv_bfloat16* x, const Work& wk, int P, int kS, int H, cudaStream_t st);
 cudaError_t launch_convert_h(const Work& wk, int P, int I, int I_pad, cudaStream_t st);
 cudaError_t launch_prefill_gemm(int mode, const CUtensorMap& bmap, const GemmArgs& a, int n_sm, cudaStream_t st);
+// The few-row tiles (a.tiles / a.n_tiles = the mtiles list) of mode 0 (gate/up)
+// or 1 (down), same outputs as the GEMM.
+cudaError_t launch_prefill_mt(int mode, const GemmArgs& a, int n_sm, cudaStream_t st);
 size_t route_decode_smem(int H, int T, int E, int k, int S);
 
 struct Shape {

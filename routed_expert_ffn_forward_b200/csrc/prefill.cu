@@ -405,46 +405,314 @@ done:
   }
 }
 
+// ============================================================================ few-row tiles
+// Tiles of at most kMtMaxRows activation rows (experts with few rows, and the
+// last partial tile of the others) stream their weights through warp-level
+// fp16 MMAs (mma.sync m16n8k16, fp32 accumulate) instead of the tensor-memory
+// GEMM above.  The weights are dequantised in registers straight into MMA
+// fragments -- the same fp16 values as the dequantisers above, 2^k row scale
+// included -- so a weight tile costs its HBM read and about 1.6 instructions
+// per weight whatever its row count, with no shared-memory round trip.
+//
+// Work unit: (tile, feature block), claimed from a counter -- gate/up 128
+// features (128 gate rows + the same 128 up rows), down 256 output rows.  A
+// stage is one super-block along K: the unit's 256 weight rows (two 2-D TMA
+// boxes of 128 rows) and the tile's activation rows (a bulk copy of 256 fp16
+// per row; rows kMtXPitch bytes apart so that the fragment loads of eight rows
+// fall on distinct banks).
+//
+// Warp w owns 16 weight rows as one MMA M tile and all of K -- gate/up: rows
+// 0-7 are the gate rows of features 8w..8w+7 and rows 8-15 their up rows, so a
+// thread holds g and u of the same (feature, token) and applies SwiGLU in
+// registers; down: output rows 16w..16w+15 -- against every activation row of
+// the tile as up to kMtMaxRows / 8 MMA N tiles.
+//
+// K order: the thread at quad position c takes, from each 16-weight half of a
+// 32-weight run, the weights 4c..4c+3: nibbles (0, 2) of its quant word form
+// one fp16 pair and (1, 3) the other, which is the order (0, 2, 1, 3) in which
+// the activations are stored within every group of four.
+constexpr int kMtWarps = 16;
+constexpr int kMtThreads = (kMtWarps + 1) * 32;          // + one producer warp
+constexpr int kMtNT = kMtMaxRows / 8;                    // MMA N tiles
+constexpr int kMtStages = 3;
+constexpr int kMtWBytes = 2 * kRawBytes;                 // 256 weight rows x 1 super-block
+constexpr int kMtXPitch = 2 * kQK + 32;                  // one activation row's 256 fp16, padded
+constexpr int kMtStageBytes = kMtWBytes + kMtMaxRows * kMtXPitch;
+constexpr size_t kMtSmem = 1024 + (size_t)kMtStages * kMtStageBytes + 16 * kMtStages + 16 * kMtStages;
+static_assert(kMtSmem <= 227 * 1024, "few-row kernel shared memory");
+static_assert(kMtStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
+
+template <int kMode>
+__global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kMtStages * kMtStageBytes);
+  uint64_t* empty = full + kMtStages;
+  int* s_unit = reinterpret_cast<int*>(empty + kMtStages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMtStages; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], kMtWarps);
+    }
+    ptx::fence_barrier_init();
+  }
+  __syncthreads();
+  ptx::pdl_wait();  // tiles, counters and activation rows of the previous kernels
+  ptx::pdl_launch_dependents();
+  const int ft = a.ft, nkb = a.nkb;
+  const int n_units = __ldcg(a.n_tiles) * ft;
+
+  if (warp == kMtWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      ptx::IssueLog log;
+      bool ok = true;
+      while (ok) {
+        const int u = (int)atomicAdd(a.next, 1u);
+        if (u >= n_units) break;
+        const int4 tl = __ldcg(a.tiles + u / ft);   // (expert, n0, count, r0)
+        const int f = u % ft;
+        const int ex = in_range(tl.x, a.n_ex, a.err);
+        const CUtensorMap* wm = a.wmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + ex), a.n_slots, a.err) + 3;
+        const CUtensorMap* m0 = kMode == 0 ? wm : wm + 2;
+        const CUtensorMap* m1 = kMode == 0 ? wm + 1 : wm + 2;
+        const int y0 = kMode == 0 ? f * kGM : f * 2 * kGM;
+        const int y1 = kMode == 0 ? f * kGM : f * 2 * kGM + kGM;
+        const int cnt = min(tl.z, kMtMaxRows);
+        const __half* xr = a.bsrc + (size_t)in_range(tl.w + tl.y, a.n_rows, a.err) * a.b_ld;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
+            atomicOr(a.err, 16u);
+            ok = false;
+            break;
+          }
+          s_unit[stage] = u;
+          ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(kMtWBytes + cnt * 2 * kQK));
+          uint8_t* dst = sm + stage * kMtStageBytes;
+          ptx::tma_load_2d(dst, m0, kb * 18, y0, &full[stage]);
+          ptx::tma_load_2d(dst + kRawBytes, m1, kb * 18, y1, &full[stage]);
+          for (int n = 0; n < cnt; ++n)
+            ptx::bulk_load(dst + kMtWBytes + n * kMtXPitch, xr + (size_t)n * a.b_ld + kb * kQK, 2 * kQK,
+                           &full[stage]);
+          log.note(stage, phase);
+          if (++stage == kMtStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (ok) {
+        // end of work: a stage with unit -1 and no bytes (its earlier issue
+        // was consumed, so it leaves the drain list)
+        if (ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
+          s_unit[stage] = -1;
+          log.issued &= ~(1u << stage);
+          ptx::mbar_arrive(&full[stage]);
+        } else {
+          atomicOr(a.err, 16u);
+        }
+      }
+      // never leave with a copy into shared memory in flight
+      log.drain(full, kMtStages);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int g = lane >> 2, c4 = lane & 3;
+  // this warp's rows: (box, row in box) of M-tile rows g and g + 8
+  const int boxA = kMode == 0 ? 0 : warp >> 3, boxB = kMode == 0 ? 1 : warp >> 3;
+  const int rowA = kMode == 0 ? 8 * warp + g : 16 * (warp & 7) + g, rowB = kMode == 0 ? rowA : rowA + 8;
+  const uint32_t offA = (uint32_t)(boxA * kRawBytes + rowA * kQBytes), offB = (uint32_t)(boxB * kRawBytes + rowB * kQBytes);
+  const __half2 off_lo = __float2half2_rn(1024.f), off_hi = __float2half2_rn(64.f);
+  const __half2 kNeg2 = __float2half2_rn(-1.f);
+  int stage = 0;
+  uint32_t phase = 0;
+  while (true) {
+    bool ok = ptx::mbar_wait(&full[stage], phase);
+    const int u = ok ? s_unit[stage] : -1;
+    if (!ok) {
+      atomicOr(a.err, 64u);
+      break;
+    }
+    if (u < 0) break;
+    const int4 tl = __ldcg(a.tiles + u / ft);
+    const int f = u % ft;
+    const int ex = in_range(tl.x, a.n_ex, a.err);
+    const int cnt = min(tl.z, kMtMaxRows), nt = (cnt + 7) >> 3;
+    // weight rows of this thread and their 2^k scales
+    const int8_t* wx = a.wexp + (size_t)ex * a.wexp_stride;
+    int wrA, wrB, oA, oB;   // wexp rows; output columns
+    if (kMode == 0) {
+      oA = oB = f * kGM + 8 * warp + g;
+      const int fr = min(oA, a.out_rows - 1);
+      wrA = fr;
+      wrB = a.out_rows + fr;
+    } else {
+      oA = f * 2 * kGM + boxA * kGM + rowA;
+      oB = f * 2 * kGM + boxB * kGM + rowB;
+      wrA = a.wexp_down + oA;
+      wrB = a.wexp_down + oB;
+    }
+    const int kA = __ldg(wx + wrA), kB = __ldg(wx + wrB);
+    const __half2 wsA = pow2h2(kA), wsB = pow2h2(kB);
+    const __half2 nwsA = __hmul2(wsA, kNeg2), nwsB = __hmul2(wsB, kNeg2);
+    float acc[kMtNT][4];
+#pragma unroll
+    for (int j = 0; j < kMtNT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (kb > 0 && !ptx::mbar_wait(&full[stage], phase)) {
+        atomicOr(a.err, 64u);
+        ok = false;
+        break;
+      }
+      const uint8_t* st = sm + stage * kMtStageBytes;
+      const uint8_t* rA = st + offA;
+      const uint8_t* rB = st + offB;
+      const uint8_t* xs = st + kMtWBytes + g * kMtXPitch + 8 * c4;   // token row g of N tile 0
+      const uint4 hA = *reinterpret_cast<const uint4*>(rA), hB = *reinterpret_cast<const uint4*>(rB);
+      __half2 d2sA, nm2sA, d2sB, nm2sB;
+      {
+        const uint32_t dA = __byte_perm(hA.x, 0u, 0x1010u), mA = __byte_perm(hA.x, 0u, 0x3232u);
+        const uint32_t dB = __byte_perm(hB.x, 0u, 0x1010u), mB = __byte_perm(hB.x, 0u, 0x3232u);
+        d2sA = __hmul2(*reinterpret_cast<const __half2*>(&dA), wsA);
+        nm2sA = __hmul2(*reinterpret_cast<const __half2*>(&mA), nwsA);
+        d2sB = __hmul2(*reinterpret_cast<const __half2*>(&dB), wsB);
+        nm2sB = __hmul2(*reinterpret_cast<const __half2*>(&mB), nwsB);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        __half2 sA2, nmA2, sB2, nmB2;
+        chunk_scales(hA, c, d2sA, nm2sA, sA2, nmA2);
+        chunk_scales(hB, c, d2sB, nm2sB, sB2, nmB2);
+        const uint32_t* qA = reinterpret_cast<const uint32_t*>(rA + 16 + 32 * c);
+        const uint32_t* qB = reinterpret_cast<const uint32_t*>(rB + 16 + 32 * c);
+        const uint32_t wA[2] = {qA[c4], qA[4 + c4]}, wB[2] = {qB[c4], qB[4 + c4]};
+#pragma unroll
+        for (int nib = 0; nib < 2; ++nib) {   // run 2c (low nibbles), run 2c + 1 (high nibbles)
+          const __half2 sa = nib ? __high2half2(sA2) : __low2half2(sA2);
+          const __half2 na = nib ? __high2half2(nmA2) : __low2half2(nmA2);
+          const __half2 sb = nib ? __high2half2(sB2) : __low2half2(sB2);
+          const __half2 nb = nib ? __high2half2(nmB2) : __low2half2(nmB2);
+          const __half2 off = nib ? off_hi : off_lo;
+          const uint32_t mask = nib ? 0x00F000F0u : 0x000F000Fu;
+          const uint32_t magic = nib ? 0x54005400u : 0x64006400u;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {   // weights 16h + 4c4 .. +3 of the run
+            const uint32_t wa = wA[h], wb = wB[h];
+            uint32_t af[4];
+            af[0] = deq2((wa & mask) | magic, off, sa, na);          // row g,     nibbles 0, 2
+            af[1] = deq2((wb & mask) | magic, off, sb, nb);          // row g + 8
+            af[2] = deq2(((wa >> 8) & mask) | magic, off, sa, na);   // row g,     nibbles 1, 3
+            af[3] = deq2(((wb >> 8) & mask) | magic, off, sb, nb);
+            const int kx = 64 * c + 32 * nib + 16 * h;
+#pragma unroll
+            for (int j = 0; j < kMtNT; ++j) {
+              if (j < nt) {
+                const uint2 bv = *reinterpret_cast<const uint2*>(xs + j * 8 * kMtXPitch + 2 * kx);
+                ptx::mma_f16(acc[j], af, bv.x, bv.y);
+              }
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[stage]);
+      if (++stage == kMtStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    if (!ok) break;
+    // epilogue: undo the row's 2^k and the activation row's scale
+    const int prow0 = tl.w + tl.y;
+    const float sA = pow2f(-kA), sB = pow2f(-kB);
+#pragma unroll
+    for (int j = 0; j < kMtNT; ++j) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int n = 8 * j + 2 * c4 + e;
+        if (j < nt && n < cnt) {
+          const int prow = prow0 + n;
+          const float inv = __ldg(a.rinv + prow);
+          float* orow = a.out + (size_t)prow * a.out_ld;
+          if (kMode == 0) {
+            if (oA < a.out_rows) {
+              const float gv = acc[j][e] * (inv * sA), up = acc[j][2 + e] * (inv * sB);
+              orow[oA] = __fdividef(gv, 1.f + __expf(-gv)) * up;   // silu(g) * u
+            }
+          } else {
+            orow[oA] = acc[j][e] * (inv * sA);
+            orow[oB] = acc[j][2 + e] * (inv * sB);
+          }
+        }
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- helper kernels
 // Tiles: each expert with more than `small_rows` rows, in chunks of kGN rows:
 // (expert, n0, count, r0).  Experts with 1..small_rows rows go to `small`
 // (for the decode kernels, which stream their weights once without
-// dequantising them).  One block; experts are taken 1024 at a time with block
-// scans of their tile counts and of their membership of `small`.
+// dequantising them).  With mt_rows > 0, an expert with at most mt_rows rows
+// becomes one few-row tile, and so does the last partial chunk of a larger
+// expert when it has at most mt_rows rows; the unit counters of the few-row
+// kernels are zeroed here.  One block; experts are taken 1024 at a time with
+// block scans of their tile counts and of their membership of the lists.
 __global__ void __launch_bounds__(1024) build_tiles_kernel(const int* __restrict__ act, const int* __restrict__ n_act,
                                                            const int* __restrict__ counts,
                                                            const int* __restrict__ offsets, int4* __restrict__ tiles,
                                                            int* __restrict__ n_tiles, int small_rows,
                                                            int* __restrict__ small, int* __restrict__ n_small,
+                                                           int mt_rows, int4* __restrict__ mtiles,
+                                                           int* __restrict__ n_mtiles, unsigned* __restrict__ mt_next,
                                                            int ep_rank, int ep_world) {
   __shared__ int s_warp[32];
   ptx::pdl_wait();
   const int na = __ldcg(n_act);
-  int base = 0, sbase = 0;
+  int base = 0, sbase = 0, mbase = 0;
   for (int c0 = 0; c0 < na; c0 += blockDim.x) {
     const int i = c0 + threadIdx.x;
-    int e = 0, c = 0, r0 = 0, nt = 0, sm = 0;
+    int e = 0, c = 0, r0 = 0, nt = 0, sm = 0, mt = 0;
     if (i < na) {
       e = __ldcg(act + i);
       c = __ldcg(counts + e);
       r0 = __ldcg(offsets + e);
       sm = c <= small_rows ? 1 : 0;
-      nt = sm ? 0 : (c + kGN - 1) / kGN;
-      if (!ep_owned(e, ep_rank, ep_world)) sm = nt = 0;   // another rank's expert
+      if (!sm) {
+        nt = (c + kGN - 1) / kGN;
+        const int last = c - (nt - 1) * kGN;   // rows of the last chunk
+        if (last <= mt_rows) {
+          mt = 1;
+          --nt;
+        }
+      }
+      if (!ep_owned(e, ep_rank, ep_world)) sm = nt = mt = 0;   // another rank's expert
     }
-    int tot, stot;
+    int tot, stot, mtot;
     const int pos = base + block_exclusive_scan_1024(nt, &tot, s_warp);
     __syncthreads();
     const int spos = sbase + block_exclusive_scan_1024(sm, &stot, s_warp);
+    __syncthreads();
+    const int mpos = mbase + block_exclusive_scan_1024(mt, &mtot, s_warp);
     for (int j = 0; j < nt; ++j) tiles[pos + j] = make_int4(e, j * kGN, min(kGN, c - j * kGN), r0);
     if (sm) small[spos] = e;
+    if (mt) mtiles[mpos] = make_int4(e, nt * kGN, c - nt * kGN, r0);
     base += tot;
     sbase += stot;
+    mbase += mtot;
     __syncthreads();
   }
   if (threadIdx.x == 0) {
     *n_tiles = base;
     *n_small = sbase;
+    *n_mtiles = mbase;
+    mt_next[0] = 0u;
+    mt_next[1] = 0u;
   }
 }
 
@@ -589,10 +857,12 @@ size_t prefill_gemm_smem() { return kGemmSmem; }
 
 size_t prefill_max_tiles(int n_experts_total, size_t pairs) { return (size_t)n_experts_total + pairs / kGN + 1; }
 
-cudaError_t launch_build_tiles(const Work& wk, int small_rows, cudaStream_t st, int ep_rank, int ep_world) {
+cudaError_t launch_build_tiles(const Work& wk, int small_rows, int mt_rows, cudaStream_t st, int ep_rank,
+                               int ep_world) {
+  if (mt_rows < 0 || mt_rows > kMtMaxRows) return cudaErrorInvalidValue;
   return launch_pdl(build_tiles_kernel, dim3(1), dim3(1024), 0, st, (const int*)wk.act, (const int*)wk.n_act,
                     (const int*)wk.counts, (const int*)wk.offsets, wk.tiles, wk.n_tiles, small_rows, wk.act1,
-                    wk.n_act1, ep_rank, ep_world);
+                    wk.n_act1, mt_rows, wk.mtiles, wk.n_mtiles, wk.mt_next, ep_rank, ep_world);
 }
 
 cudaError_t launch_quant_x(const __nv_bfloat16* x, const Work& wk, int T, int H, cudaStream_t st) {
@@ -610,6 +880,21 @@ cudaError_t launch_convert_h(const Work& wk, int P, int I, int I_pad, cudaStream
   if (I_pad / 4 > kRowThreads * kRowMaxVec) return cudaErrorInvalidValue;
   return launch_pdl(convert_h_kernel, dim3(P), dim3(kRowThreads), 0, st, (const float*)wk.h, I, I_pad, wk.h16,
                     wk.hinv);
+}
+
+cudaError_t launch_prefill_mt(int mode, const GemmArgs& a, int n_sm, cudaStream_t st) {
+  static uint64_t attr_done[2] = {0, 0};  // per mode, one bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  auto kern = mode == 0 ? q4k_mt_kernel<0> : q4k_mt_kernel<1>;
+  if (!(attr_done[mode & 1] & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMtSmem);
+    if (e != cudaSuccess) return e;
+    attr_done[mode & 1] |= bit;
+  }
+  return launch_pdl(kern, dim3(n_sm), dim3(kMtThreads), kMtSmem, st, a);
 }
 
 cudaError_t launch_prefill_gemm(int mode, const CUtensorMap& bmap, const GemmArgs& a, int n_sm, cudaStream_t st) {

@@ -38,7 +38,7 @@ SIZE_MAX = (1 << 64) - 1
 
 # every entry point declared in include/moe.h
 EXPORTS = ("moe_expert_bytes", "moe_layer_create", "moe_layer_create_mixed", "moe_layer_destroy", "moe_set_router",
-           "moe_set_experts", "moe_set_cache_bytes", "moe_set_cache_policy", "moe_forward", "moe_forward_routed",
+           "moe_set_experts", "moe_set_cache_bytes", "moe_set_cache_policy", "moe_set_few_row_tiles", "moe_forward", "moe_forward_routed",
            "moe_forward_host", "moe_get_routing", "moe_get_logits", "moe_prefetch",
            "moe_check", "moe_get_stats", "moe_reset_stats", "moe_set_profiling", "moe_get_profile",
            "moe_reset_profile", "moe_route_noalloc", "moe_set_test_hooks", "moe_set_expert_parallel",
@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
             "moe_set_experts": (_I, [_P, _P, _P, _P]),
             "moe_set_cache_bytes": (_I, [ctypes.c_size_t]),
             "moe_set_cache_policy": (_I, [_I]),
+            "moe_set_few_row_tiles": (_I, [_I]),
             "moe_forward": (_I, [_P, _P, _P, _I, _P]),
             "moe_forward_routed": (_I, [_P, _P, _P, _I, _P, _P]),
             "moe_forward_host": (_I, [_P, _P, _P, _I, _P]),
@@ -168,6 +169,10 @@ def moe_set_cache_bytes(nbytes: int) -> None:
 
 def moe_set_cache_policy(policy: int) -> None:
     _check(lib().moe_set_cache_policy(policy))
+
+
+def moe_set_few_row_tiles(max_rows: int) -> None:
+    _check(lib().moe_set_few_row_tiles(max_rows))
 
 
 def moe_forward(layer: int, x: int, out: int, T: int, stream: int | None = None) -> None:

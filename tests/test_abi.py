@@ -65,6 +65,14 @@ def test_null_arguments(lib):
     assert lib.moe_layer_destroy(None) == moe.MOE_OK
 
 
+def test_process_wide_settings_validate_on_the_host(lib):
+    for bad in (-1, 65):
+        assert lib.moe_set_few_row_tiles(bad) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_cache_policy(7) == moe.MOE_ERR_INVALID_ARG
+    for ok in (0, 64):
+        assert lib.moe_set_few_row_tiles(ok) == moe.MOE_OK
+
+
 def test_stats_without_gpu():
     moe.moe_reset_stats()
     s = moe.moe_get_stats()

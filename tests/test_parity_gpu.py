@@ -96,6 +96,21 @@ def test_small_every_token(torch, name, T):
     check_against_oracle(cfg, g)
 
 
+@pytest.mark.parametrize("max_rows", [0, 1, 8, 64])
+def test_few_row_tile_thresholds(torch, max_rows):
+    """The prefill path with the few-row kernel off (GEMM + decode kernels),
+    taking only single-row experts, the experts up to 8 rows and the last
+    partial tiles up to 8 rows, or everything up to 64 rows: every token
+    matches the oracle each way (rows per expert 1..~60 here)."""
+    cfg = SMALL["ragged_inter"]
+    try:
+        moe.moe_set_few_row_tiles(max_rows)
+        g = run_gpu(torch, cfg, 200)
+    finally:
+        moe.moe_set_few_row_tiles(64)
+    check_against_oracle(cfg, g)
+
+
 def test_zero_tokens(torch):
     from routed_expert_ffn_forward_b200.layer import layer_from_config
     L = layer_from_config(C0)
@@ -123,9 +138,11 @@ def test_c2_batched_decode_every_token(torch):
 def prefill_sample(ids: np.ndarray, n_experts: int, tile: int = 256) -> np.ndarray:
     """Tokens whose rows reach every kind of work unit of the prefill path:
     the first and last row of every 256-row tile of the three experts with
-    the most rows, one token of every expert with at most 4 rows (the decode
-    kernels) and one of every expert with 5..16 rows (small GEMM tiles).
-    Rows of an expert are its (token, slot) pairs in token order."""
+    the most rows (full GEMM tiles and their last partial tile), one token of
+    every expert with at most 64 rows (few-row tiles), and the last row of
+    every expert whose last partial tile has at most 64 rows (a few-row tile
+    after GEMM tiles).  Rows of an expert are its (token, slot) pairs in
+    token order."""
     T, k = ids.shape
     counts = np.bincount(ids.ravel(), minlength=n_experts)
     rows_of = {e: np.nonzero((ids == e).any(axis=1))[0] for e in range(n_experts) if counts[e]}
@@ -136,8 +153,10 @@ def prefill_sample(ids: np.ndarray, n_experts: int, tile: int = 256) -> np.ndarr
             pick.add(int(toks[t0]))
             pick.add(int(toks[min(t0 + tile, len(toks)) - 1]))
     for e, toks in rows_of.items():
-        if counts[e] <= 16:
+        if counts[e] <= 64:
             pick.add(int(toks[0]))
+        elif 0 < counts[e] % tile <= 64:
+            pick.add(int(toks[-1]))
     return np.array(sorted(pick))
 
 
