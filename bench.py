@@ -124,13 +124,9 @@ def algorithmic_bytes(cfg, ids: np.ndarray, which: str) -> float:
     """Bytes a kernel must move at least once per launch for this routing.
     gate_up: gate+up weights of every expert the kernel runs, x rows, h writes.
     forward: every active expert's weights, the router weight, x and out.
-    For T > 4 the gate/up kernel is the tensor-core GEMM, which runs the
-    experts with more than 4 rows (the others take the decode kernels)."""
+    (The decode path, T <= 4, where every expert runs on one kernel.)"""
     T = ids.shape[0]
     active = len(np.unique(ids)) + cfg.n_shared
-    if which == "gate_up" and T > 4:
-        counts = np.bincount(ids.ravel(), minlength=cfg.n_experts)
-        active = int(np.sum(counts > 4)) + cfg.n_shared
     nb_h, nb_i = cfg.hidden // 256, (cfg.inter + 255) // 256
     gate = cfg.inter * nb_h * 144
     down = cfg.hidden * nb_i * 144
@@ -373,7 +369,18 @@ def measure_resident(args, cfg, rank, world, local_rank, peaks, steps, warmup, e
     fwd_ms = total_ms / steps
     kern = "gate_up"
     avg_ms = prof["ms"][kern] / max(1, prof["launches"][kern])
-    if T > 4:
+    gemm_dominant = prof["ms"]["gate_up"] >= prof["ms"].get("few_gate_up", 0.0)
+    if T > 4 and not gemm_dominant:
+        # the few-row kernel carries the step: bound by HBM
+        kern = "few_gate_up"
+        avg_ms = prof["ms"][kern] / max(1, prof["launches"][kern])
+        ab = float(np.mean([few_gate_up_bytes(cfg, ids) for ids in ids_cycle]))
+        achieved = ab / (avg_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": kernel_traffic(f"config{cfg_index(cfg)}:{kern}"),
+                "algorithmic_bytes": ab, "peak_source": peaks["source"]}
+    elif T > 4:
         # the gate/up GEMM runs the experts with more than 4 rows (plus the shared one)
         fl = float(np.mean([gate_up_gemm_flops(cfg, ids) for ids in ids_cycle]))
         achieved = fl / (avg_ms / 1e3) / 1e12
@@ -407,13 +414,48 @@ def measure_resident(args, cfg, rank, world, local_rank, peaks, steps, warmup, e
             "dtype": DTYPE_DECODE if T <= 4 else DTYPE_PREFILL}
 
 
-def gate_up_gemm_flops(cfg, ids: np.ndarray) -> float:
-    """FLOPs of the prefill gate/up GEMM for this routing: 2 * rows * 2I * H
-    over the experts with more than 4 rows, plus the shared experts."""
+FEW_ROWS = 64   # the library's default moe_set_few_row_tiles
+
+
+def tile_split(cfg, ids: np.ndarray, few_rows: int = FEW_ROWS):
+    """How the prefill path splits this routing (as the library's tile
+    builder does): (rows on the tensor-memory GEMM, rows on few-row tiles,
+    number of few-row tiles).  An expert with at most few_rows rows is one
+    few-row tile; a larger one goes to the GEMM in 256-row tiles, except a
+    last partial tile of at most few_rows rows, which becomes a few-row tile."""
     T = ids.shape[0]
     counts = np.bincount(ids.ravel(), minlength=cfg.n_experts)
-    rows = int(counts[counts > 4].sum()) + T * cfg.n_shared
-    return 2.0 * rows * 2 * cfg.inter * cfg.hidden
+    return split_rows([int(c) for c in counts if c > 0] + [T] * cfg.n_shared, few_rows)
+
+
+def split_rows(rows, few_rows: int = FEW_ROWS):
+    """tile_split on a list of rows per active expert."""
+    gemm = few = n_few = 0
+    for c in rows:
+        if c <= few_rows:
+            few, n_few = few + c, n_few + 1
+            continue
+        last = c - (c - 1) // 256 * 256
+        if last <= few_rows:
+            gemm, few, n_few = gemm + c - last, few + last, n_few + 1
+        else:
+            gemm += c
+    return gemm, few, n_few
+
+
+def gate_up_gemm_flops(cfg, ids: np.ndarray) -> float:
+    """FLOPs of the prefill gate/up GEMM for this routing: 2 * rows * 2I * H
+    over the rows in its tiles (tile_split)."""
+    return 2.0 * tile_split(cfg, ids)[0] * 2 * cfg.inter * cfg.hidden
+
+
+def few_gate_up_bytes(cfg, ids: np.ndarray) -> float:
+    """Bytes the few-row gate/up kernel moves at least once: the gate and up
+    weights of every few-row tile, its x rows (fp16) and its h rows (fp32)."""
+    _, few, n_few = tile_split(cfg, ids)
+    gate = cfg.inter * (cfg.hidden // 256) * 144
+    i_pad = (cfg.inter + 255) // 256 * 256
+    return n_few * 2 * gate + few * cfg.hidden * 2 + few * i_pad * 4
 
 
 def cfg_index(cfg) -> int:

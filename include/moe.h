@@ -97,10 +97,12 @@ enum {
   MOE_K_DOWN = 4,    /* down projection */
   MOE_K_COMBINE = 5, /* weighted combine */
   MOE_K_PREP = 6,    /* prefill only: activation rows and SwiGLU output to scaled fp16 */
-  MOE_K_SMALL = 7,   /* prefill only: the few-row tiles (moe_set_few_row_tiles) */
+  MOE_K_SMALL = 7,   /* prefill only: decode kernels for experts with <= 4 rows (few-row tiles off) */
   MOE_K_FORWARD = 8, /* whole forward, first kernel start to last kernel end */
   MOE_K_FUSED = 9,   /* decode of one token as one kernel (router through combine) */
-  MOE_K_COUNT = 10
+  MOE_K_FEW_GATE_UP = 10, /* prefill only: gate/up + SwiGLU of the few-row tiles (moe_set_few_row_tiles) */
+  MOE_K_FEW_DOWN = 11,    /* prefill only: down projection of the few-row tiles */
+  MOE_K_COUNT = 12
 };
 typedef struct {
   uint64_t forwards;             /* forwards profiled */

@@ -44,7 +44,8 @@ EXPORTS = ("moe_expert_bytes", "moe_layer_create", "moe_layer_create_mixed", "mo
            "moe_reset_profile", "moe_route_noalloc", "moe_set_test_hooks", "moe_set_expert_parallel",
            "moe_forward_partial", "moe_combine_partials", "moe_last_error")
 
-KERNELS = ("router", "topk", "permute", "gate_up", "down", "combine", "prep", "small", "forward", "fused")
+KERNELS = ("router", "topk", "permute", "gate_up", "down", "combine", "prep", "small", "forward", "fused",
+           "few_gate_up", "few_down")
 
 
 class moe_stats(ctypes.Structure):

@@ -28,6 +28,14 @@ def test_header_and_binding_agree():
     assert declared_entry_points() == sorted(moe.EXPORTS)
 
 
+def test_kernel_kinds_match_the_header():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    kinds = {int(v): n.lower() for n, v in re.findall(r"\bMOE_K_([A-Z_]+)\s*=\s*(\d+)", text)}
+    count = kinds.pop(max(kinds))
+    assert count == "count" and len(moe.KERNELS) == max(kinds) + 1
+    assert all(moe.KERNELS[v] == n for v, n in kinds.items())
+
+
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_entry_points():
         assert hasattr(lib, name), name

@@ -72,13 +72,28 @@ def test_traffic_entry_tracks_its_source():
     assert bench.kernel_traffic("config9:nothing") is None
 
 
+def test_tile_split_hand_count():
+    # 600 = 256+256+88 (GEMM), 300 = 256 | 44, 64 (few), 65 (GEMM), 1 (few),
+    # 513 = 512 | 1, 320 = 256 | 64
+    assert bench.split_rows([600, 300, 64, 65, 1, 513, 320]) == (600 + 256 + 65 + 512 + 256,
+                                                                 44 + 64 + 1 + 1 + 64, 5)
+    assert bench.split_rows([600, 300, 64, 65, 1, 513, 320], few_rows=0) == (1863, 0, 0)
+    assert bench.split_rows([256, 257], few_rows=1) == (256 + 256, 1, 1)
+
+
 def test_gate_up_gemm_flops_hand_count():
-    cfg = dataclasses.replace(synth.DECODE, tokens=6)
-    # expert 0: 6 rows (GEMM), expert 1: 5 rows (GEMM), experts 2..: 1 row each (decode kernels)
-    ids = np.array([[0, 1] + [10 * j + t for j in range(1, 7)] for t in range(6)], dtype=np.int32)
-    ids[5, 1] = 99                          # expert 1 keeps 5 rows
-    rows = 6 + 5 + 6 * 1                    # the two GEMM experts, plus the shared expert's 6 rows
+    cfg = dataclasses.replace(synth.DECODE, tokens=70)
+    # expert 0 on all 70 tokens (GEMM), experts 1..7 and the rest on few rows
+    ids = np.array([[0] + [1 + (7 * t + j) % 200 for j in range(7)] for t in range(70)], dtype=np.int32)
+    rows = 70 + 70                          # expert 0 and the shared expert
     assert bench.gate_up_gemm_flops(cfg, ids) == 2.0 * rows * 2 * 2048 * 7168
+
+
+def test_tile_split_off_sends_everything_to_the_gemm():
+    cfg = dataclasses.replace(synth.DECODE, tokens=6)
+    ids = np.array([[0, 1] + [10 * j + t for j in range(1, 7)] for t in range(6)], dtype=np.int32)
+    gemm, few, n_few = bench.tile_split(cfg, ids, few_rows=0)
+    assert (gemm, few, n_few) == (6 * 8 + 6, 0, 0)
 
 
 def test_oracle_all_cores_reports_its_workers():
