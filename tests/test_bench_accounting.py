@@ -37,21 +37,22 @@ def test_repeated_experts_counted_once():
     assert three - one == 2 * 2 * 7168 * 2   # only x and out grow with the tokens
 
 
-def test_prefill_gate_up_counts_only_gemm_experts():
-    cfg = synth.BATCHED                     # T = 64: experts with <= 4 rows take the decode kernels
+def test_few_row_gate_up_bytes():
+    cfg = synth.BATCHED                     # T = 64: every expert has <= 64 rows (few-row tiles)
     ids = np.zeros((64, 8), dtype=np.int32)
-    ids[:, 0] = 0                           # expert 0: 64 rows (GEMM)
+    ids[:, 0] = 0                           # expert 0: 64 rows
     ids[:, 1:] = np.arange(1, 8)[None, :] + 7 * (np.arange(64)[:, None] % 4)
-    ids[:60, 7] = 100 + np.arange(60) // 4  # 15 experts x 4 rows (decode kernels)
-    # columns 1-6: 24 experts x 16 rows (GEMM); column 7 of the last 4 tokens:
-    # 4 experts x 1 row (decode kernels)
+    ids[:60, 7] = 100 + np.arange(60) // 4  # 15 experts x 4 rows
+    # columns 1-6: 24 experts x 16 rows; column 7 of the last 4 tokens: 4 experts x 1 row
     gate = 2048 * 28 * 144
     counts = np.bincount(ids.ravel(), minlength=256)
     assert np.all(np.sort(ids, axis=1)[:, 1:] != np.sort(ids, axis=1)[:, :-1])  # distinct picks per token
-    assert int(np.sum(counts > 4)) == 25 and int(np.sum((counts > 0) & (counts <= 4))) == 19
-    gemm = 25 + 1                           # + the shared expert
-    expect = gemm * 2 * gate + 64 * 7168 * 2 + 64 * 9 * 2048 * 2
-    assert bench.algorithmic_bytes(cfg, ids, "gate_up") == expect
+    assert int(np.sum(counts > 0)) == 44 and counts.max() == 64
+    tiles, rows = 44 + 1, 64 * 9            # + the shared expert's 64 rows
+    assert bench.tile_split(cfg, ids) == (0, rows, tiles)
+    expect = tiles * 2 * gate + rows * 7168 * 2 + rows * 2048 * 4
+    assert bench.few_gate_up_bytes(cfg, ids) == expect
+    assert bench.gate_up_gemm_flops(cfg, ids) == 0.0
 
 
 def test_prefill_flops():
