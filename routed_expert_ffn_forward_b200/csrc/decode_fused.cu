@@ -61,7 +61,10 @@ constexpr unsigned kErrFzProducer = 1u << 10, kErrFzConsumer = 1u << 11, kErrFzG
                    kErrFzReady = 1u << 13;
 
 // global sync words (FusedArgs::sync)
-constexpr int kSyncBarCount = 0, kSyncBarGen = 1, kSyncNext = 2, kSyncDone = 3, kSyncReady = 8;
+// sync words: [2] down-unit claims, [3] finished down units, [4..5] grid
+// barrier arrivals (64-bit, only ever grows: launch L waits for (L+1)·grid),
+// [8..] per-pick gate/up units done
+constexpr int kSyncNext = 2, kSyncDone = 3, kSyncBar64 = 4, kSyncReady = 8;
 
 // Shared-memory layout (offsets from the 1024-aligned base).
 struct FzLayout {
@@ -88,12 +91,12 @@ __device__ __forceinline__ uint8_t* fz_aligned(uint8_t* raw) {
   return raw + pad;
 }
 
-// Spin (one thread) until *p != v (acquire); false after `lim` ns.
-__device__ __forceinline__ bool spin_while_eq(const uint32_t* p, uint32_t v, uint64_t lim) {
-  if (ptx::ld_acquire_gpu(p) != v) return true;
+// Spin (one thread) until *p >= v (acquire, 64-bit); false after `lim` ns.
+__device__ __forceinline__ bool spin_until_ge64(const uint64_t* p, uint64_t v, uint64_t lim) {
+  if (ptx::ld_acquire_gpu_u64(p) >= v) return true;
   const uint64_t t0 = ptx::globaltimer();
-  while (ptx::ld_acquire_gpu(p) == v) {
-    __nanosleep(64);
+  while (ptx::ld_acquire_gpu_u64(p) < v) {
+    __nanosleep(32);
     if (ptx::globaltimer() - t0 > lim) return false;
   }
   return true;
@@ -112,6 +115,7 @@ __device__ __forceinline__ bool spin_until_ge(const uint32_t* p, uint32_t v, uin
 template <int PL>
 __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const FusedArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
+  __shared__ unsigned long long s_bar_target;   // grid-barrier arrivals this launch waits for
   uint8_t* sm = fz_aligned(smem_raw);
   const int H = a.H, E = a.E, k = a.k, S = a.S, kS = k + S;
   const FzLayout lay(H, a.act_slot_bytes, a.stages * a.stage_bytes);
@@ -127,7 +131,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
   int* s_unit = reinterpret_cast<int*>(sm + lay.unit);
   int* s_ids = reinterpret_cast<int*>(sm + lay.ids);
   float* s_w = reinterpret_cast<float*>(sm + lay.w);
-  volatile int* s_flag = reinterpret_cast<volatile int*>(sm + lay.flags);  // [0] abort [1] combine [2] gen
+  volatile int* s_flag = reinterpret_cast<volatile int*>(sm + lay.flags);  // [0] abort [3] owned picks
   float* s_part = reinterpret_cast<float*>(sm + lay.part);
   uint8_t* s_xh = sm + lay.xh;
   uint8_t* s_xl = sm + lay.xl;
@@ -169,6 +173,23 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
     bool routed = false, ok = true;
     // in streaming mode the expert -> slot table comes from the previous kernel
     if (!a.early) ptx::pdl_wait();
+    // While the router runs, every CTA brings a share of the shared experts'
+    // weights into L2 (they need no routing): the gate/up boxes in K order,
+    // then the down boxes.  The CTAs that run those units read them from L2.
+    for (int s = 0; s < S; ++s) {
+      if (!ep_owned(E + s, a.ep_rank, a.ep_world)) continue;
+      const CUtensorMap* m = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + E + s), a.n_slots, a.err);
+      const int n_gub = 2 * a.nbh * gu_tiles, n_items = n_gub + a.nbi * dn_tiles;
+      for (int q = blockIdx.x; q < n_items; q += gridDim.x) {
+        if (q < n_gub) {
+          const int kb = q / (2 * gu_tiles), r = q - kb * 2 * gu_tiles;
+          ptx::tma_prefetch_l2_2d(m + 3 + (r & 1), kb * gu_el, (r >> 1) * kFzGuRows);
+        } else {
+          const int q2 = q - n_gub, kb = q2 / dn_tiles, rt = q2 - kb * dn_tiles;
+          ptx::tma_prefetch_l2_2d(m + 6, kb * dn_el, rt * kFzDnRows);
+        }
+      }
+    }
     auto expert_of = [&](int j) { return in_range(j < k ? s_ids[j] : E + (j - k), E + S, a.err); };
     auto next_stage = [&]() {
       if (++stage == n_stages) {
@@ -362,15 +383,15 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
     }
     cbar();   // thread 0's fence below is cumulative over these writes and the logits
     if (tid == 0) {
-      const uint32_t gen = ptx::ld_acquire_gpu(sync + kSyncBarGen);
-      s_flag[2] = (int)gen;
-      __threadfence();
-      const uint32_t old = atomicAdd(sync + kSyncBarCount, 1u);
-      if (old == gridDim.x - 1 + (uint32_t)a.hold) {   // hold > 0 (a test hook): never released
-        sync[kSyncBarCount] = 0u;      // ready for the next launch
-        __threadfence();
-        ptx::st_release_gpu(sync + kSyncBarGen, gen + 1u);
-      }
+      // arrivals before this CTA's own are within this launch's band
+      // [L·grid, (L+1)·grid), so it waits for (L+1)·grid (+ hold, a test hook
+      // that makes the wait run out); the release add publishes the CTA's
+      // logits and CTA 0's zeroed counters (ordered before it by the barrier
+      // above)
+      uint64_t* bar = reinterpret_cast<uint64_t*>(sync + kSyncBar64);
+      const uint64_t G = gridDim.x;
+      s_bar_target = (ptx::ld_relaxed_gpu_u64(bar) / G + 1) * G + (uint64_t)a.hold;
+      ptx::red_add_release_gpu_u64(bar, 1ull);
     }
   }
 
@@ -393,7 +414,8 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
   bool routed = false;
   auto route = [&]() {
     if (tid == 0) {
-      if (!spin_while_eq(sync + kSyncBarGen, (uint32_t)s_flag[2], lim)) fail(kErrFzGrid);
+      if (!spin_until_ge64(reinterpret_cast<const uint64_t*>(sync + kSyncBar64), s_bar_target, lim))
+        fail(kErrFzGrid);
     }
     cbar();
     if (!s_flag[0] && warp == 0) {

@@ -433,7 +433,6 @@ done:
 // the activations are stored within every group of four.
 constexpr int kMtWarps = 16;
 constexpr int kMtThreads = (kMtWarps + 1) * 32;          // + one producer warp
-constexpr int kMtNT = kMtMaxRows / 8;                    // MMA N tiles
 constexpr int kMtStages = 3;
 constexpr int kMtWBytes = 2 * kRawBytes;                 // 256 weight rows x 1 super-block
 constexpr int kMtXPitch = 2 * kQK + 32;                  // one activation row's 256 fp16, padded
@@ -441,6 +440,131 @@ constexpr int kMtStageBytes = kMtWBytes + kMtMaxRows * kMtXPitch;
 constexpr size_t kMtSmem = 1024 + (size_t)kMtStages * kMtStageBytes + 16 * kMtStages + 16 * kMtStages;
 static_assert(kMtSmem <= 227 * 1024, "few-row kernel shared memory");
 static_assert(kMtStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
+
+struct MtRows {
+  int boxA, boxB, rowA, rowB;   // the 128-row box and row in it of M-tile rows g and g + 8
+};
+
+// One work unit of the few-row kernel for one consumer warp: nkb stages of
+// MMAs into NT N tiles, then the epilogue.  Returns false if a stage never
+// arrived (error flag set).
+template <int kMode, int NT>
+__device__ __forceinline__ bool mt_unit(const GemmArgs& a, const uint8_t* sm, uint64_t* full, uint64_t* empty,
+                                        int& stage, uint32_t& phase, const int4 tl, int f, int warp, int lane,
+                                        const MtRows& rw) {
+  const int g = lane >> 2, c4 = lane & 3;
+  const uint32_t offA = (uint32_t)(rw.boxA * kRawBytes + rw.rowA * kQBytes);
+  const uint32_t offB = (uint32_t)(rw.boxB * kRawBytes + rw.rowB * kQBytes);
+  const __half2 off_lo = __float2half2_rn(1024.f), off_hi = __float2half2_rn(64.f);
+  const __half2 kNeg2 = __float2half2_rn(-1.f);
+  const int ex = in_range(tl.x, a.n_ex, a.err);
+  const int cnt = min(tl.z, kMtMaxRows);
+  // weight rows of this thread and their 2^k scales
+  const int8_t* wx = a.wexp + (size_t)ex * a.wexp_stride;
+  int wrA, wrB, oA, oB;   // wexp rows; output columns
+  if (kMode == 0) {
+    oA = oB = f * kGM + 8 * warp + g;
+    const int fr = min(oA, a.out_rows - 1);
+    wrA = fr;
+    wrB = a.out_rows + fr;
+  } else {
+    oA = f * 2 * kGM + rw.boxA * kGM + rw.rowA;
+    oB = f * 2 * kGM + rw.boxB * kGM + rw.rowB;
+    wrA = a.wexp_down + oA;
+    wrB = a.wexp_down + oB;
+  }
+  const int kA = __ldg(wx + wrA), kB = __ldg(wx + wrB);
+  const __half2 wsA = pow2h2(kA), wsB = pow2h2(kB);
+  const __half2 nwsA = __hmul2(wsA, kNeg2), nwsB = __hmul2(wsB, kNeg2);
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  for (int kb = 0; kb < a.nkb; ++kb) {
+    if (kb > 0 && !ptx::mbar_wait(&full[stage], phase)) {
+      atomicOr(a.err, 64u);
+      return false;
+    }
+    const uint8_t* st = sm + stage * kMtStageBytes;
+    const uint8_t* rA = st + offA;
+    const uint8_t* rB = st + offB;
+    const uint8_t* xs = st + kMtWBytes + g * kMtXPitch + 8 * c4;   // token row g of N tile 0
+    const uint4 hA = *reinterpret_cast<const uint4*>(rA), hB = *reinterpret_cast<const uint4*>(rB);
+    __half2 d2sA, nm2sA, d2sB, nm2sB;
+    {
+      const uint32_t dA = __byte_perm(hA.x, 0u, 0x1010u), mA = __byte_perm(hA.x, 0u, 0x3232u);
+      const uint32_t dB = __byte_perm(hB.x, 0u, 0x1010u), mB = __byte_perm(hB.x, 0u, 0x3232u);
+      d2sA = __hmul2(*reinterpret_cast<const __half2*>(&dA), wsA);
+      nm2sA = __hmul2(*reinterpret_cast<const __half2*>(&mA), nwsA);
+      d2sB = __hmul2(*reinterpret_cast<const __half2*>(&dB), wsB);
+      nm2sB = __hmul2(*reinterpret_cast<const __half2*>(&mB), nwsB);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      __half2 sA2, nmA2, sB2, nmB2;
+      chunk_scales(hA, c, d2sA, nm2sA, sA2, nmA2);
+      chunk_scales(hB, c, d2sB, nm2sB, sB2, nmB2);
+      const uint32_t* qA = reinterpret_cast<const uint32_t*>(rA + 16 + 32 * c);
+      const uint32_t* qB = reinterpret_cast<const uint32_t*>(rB + 16 + 32 * c);
+      const uint32_t wA[2] = {qA[c4], qA[4 + c4]}, wB[2] = {qB[c4], qB[4 + c4]};
+#pragma unroll
+      for (int nib = 0; nib < 2; ++nib) {   // run 2c (low nibbles), run 2c + 1 (high nibbles)
+        const __half2 sa = nib ? __high2half2(sA2) : __low2half2(sA2);
+        const __half2 na = nib ? __high2half2(nmA2) : __low2half2(nmA2);
+        const __half2 sb = nib ? __high2half2(sB2) : __low2half2(sB2);
+        const __half2 nb = nib ? __high2half2(nmB2) : __low2half2(nmB2);
+        const __half2 off = nib ? off_hi : off_lo;
+        const uint32_t mask = nib ? 0x00F000F0u : 0x000F000Fu;
+        const uint32_t magic = nib ? 0x54005400u : 0x64006400u;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {   // weights 16h + 4c4 .. +3 of the run
+          const uint32_t wa = wA[h], wb = wB[h];
+          uint32_t af[4];
+          af[0] = deq2((wa & mask) | magic, off, sa, na);          // row g,     nibbles 0, 2
+          af[1] = deq2((wb & mask) | magic, off, sb, nb);          // row g + 8
+          af[2] = deq2(((wa >> 8) & mask) | magic, off, sa, na);   // row g,     nibbles 1, 3
+          af[3] = deq2(((wb >> 8) & mask) | magic, off, sb, nb);
+          const uint8_t* xk = xs + 2 * (64 * c + 32 * nib + 16 * h);
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            const uint2 bv = *reinterpret_cast<const uint2*>(xk + j * 8 * kMtXPitch);
+            ptx::mma_f16(acc[j], af, bv.x, bv.y);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&empty[stage]);
+    if (++stage == kMtStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+  // epilogue: undo the row's 2^k and the activation row's scale
+  const int prow0 = tl.w + tl.y;
+  const float sA = pow2f(-kA), sB = pow2f(-kB);
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int n = 8 * j + 2 * c4 + e;
+      if (n < cnt) {
+        const int prow = prow0 + n;
+        const float inv = __ldg(a.rinv + prow);
+        float* orow = a.out + (size_t)prow * a.out_ld;
+        if (kMode == 0) {
+          if (oA < a.out_rows) {
+            const float gv = acc[j][e] * (inv * sA), up = acc[j][2 + e] * (inv * sB);
+            orow[oA] = __fdividef(gv, 1.f + __expf(-gv)) * up;   // silu(g) * u
+          }
+        } else {
+          orow[oA] = acc[j][e] * (inv * sA);
+          orow[oB] = acc[j][2 + e] * (inv * sB);
+        }
+      }
+    }
+  }
+  return true;
+}
 
 template <int kMode>
 __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a) {
@@ -522,13 +646,13 @@ __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a)
   }
 
   // -------------------------------------------------------------- consumers
-  const int g = lane >> 2, c4 = lane & 3;
+  const int g = lane >> 2;
   // this warp's rows: (box, row in box) of M-tile rows g and g + 8
-  const int boxA = kMode == 0 ? 0 : warp >> 3, boxB = kMode == 0 ? 1 : warp >> 3;
-  const int rowA = kMode == 0 ? 8 * warp + g : 16 * (warp & 7) + g, rowB = kMode == 0 ? rowA : rowA + 8;
-  const uint32_t offA = (uint32_t)(boxA * kRawBytes + rowA * kQBytes), offB = (uint32_t)(boxB * kRawBytes + rowB * kQBytes);
-  const __half2 off_lo = __float2half2_rn(1024.f), off_hi = __float2half2_rn(64.f);
-  const __half2 kNeg2 = __float2half2_rn(-1.f);
+  MtRows rw;
+  rw.boxA = kMode == 0 ? 0 : warp >> 3;
+  rw.boxB = kMode == 0 ? 1 : warp >> 3;
+  rw.rowA = kMode == 0 ? 8 * warp + g : 16 * (warp & 7) + g;
+  rw.rowB = kMode == 0 ? rw.rowA : rw.rowA + 8;
   int stage = 0;
   uint32_t phase = 0;
   while (true) {
@@ -541,116 +665,19 @@ __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a)
     if (u < 0) break;
     const int4 tl = __ldcg(a.tiles + u / ft);
     const int f = u % ft;
-    const int ex = in_range(tl.x, a.n_ex, a.err);
-    const int cnt = min(tl.z, kMtMaxRows), nt = (cnt + 7) >> 3;
-    // weight rows of this thread and their 2^k scales
-    const int8_t* wx = a.wexp + (size_t)ex * a.wexp_stride;
-    int wrA, wrB, oA, oB;   // wexp rows; output columns
-    if (kMode == 0) {
-      oA = oB = f * kGM + 8 * warp + g;
-      const int fr = min(oA, a.out_rows - 1);
-      wrA = fr;
-      wrB = a.out_rows + fr;
-    } else {
-      oA = f * 2 * kGM + boxA * kGM + rowA;
-      oB = f * 2 * kGM + boxB * kGM + rowB;
-      wrA = a.wexp_down + oA;
-      wrB = a.wexp_down + oB;
-    }
-    const int kA = __ldg(wx + wrA), kB = __ldg(wx + wrB);
-    const __half2 wsA = pow2h2(kA), wsB = pow2h2(kB);
-    const __half2 nwsA = __hmul2(wsA, kNeg2), nwsB = __hmul2(wsB, kNeg2);
-    float acc[kMtNT][4];
-#pragma unroll
-    for (int j = 0; j < kMtNT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-    for (int kb = 0; kb < nkb; ++kb) {
-      if (kb > 0 && !ptx::mbar_wait(&full[stage], phase)) {
-        atomicOr(a.err, 64u);
-        ok = false;
-        break;
-      }
-      const uint8_t* st = sm + stage * kMtStageBytes;
-      const uint8_t* rA = st + offA;
-      const uint8_t* rB = st + offB;
-      const uint8_t* xs = st + kMtWBytes + g * kMtXPitch + 8 * c4;   // token row g of N tile 0
-      const uint4 hA = *reinterpret_cast<const uint4*>(rA), hB = *reinterpret_cast<const uint4*>(rB);
-      __half2 d2sA, nm2sA, d2sB, nm2sB;
-      {
-        const uint32_t dA = __byte_perm(hA.x, 0u, 0x1010u), mA = __byte_perm(hA.x, 0u, 0x3232u);
-        const uint32_t dB = __byte_perm(hB.x, 0u, 0x1010u), mB = __byte_perm(hB.x, 0u, 0x3232u);
-        d2sA = __hmul2(*reinterpret_cast<const __half2*>(&dA), wsA);
-        nm2sA = __hmul2(*reinterpret_cast<const __half2*>(&mA), nwsA);
-        d2sB = __hmul2(*reinterpret_cast<const __half2*>(&dB), wsB);
-        nm2sB = __hmul2(*reinterpret_cast<const __half2*>(&mB), nwsB);
-      }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        __half2 sA2, nmA2, sB2, nmB2;
-        chunk_scales(hA, c, d2sA, nm2sA, sA2, nmA2);
-        chunk_scales(hB, c, d2sB, nm2sB, sB2, nmB2);
-        const uint32_t* qA = reinterpret_cast<const uint32_t*>(rA + 16 + 32 * c);
-        const uint32_t* qB = reinterpret_cast<const uint32_t*>(rB + 16 + 32 * c);
-        const uint32_t wA[2] = {qA[c4], qA[4 + c4]}, wB[2] = {qB[c4], qB[4 + c4]};
-#pragma unroll
-        for (int nib = 0; nib < 2; ++nib) {   // run 2c (low nibbles), run 2c + 1 (high nibbles)
-          const __half2 sa = nib ? __high2half2(sA2) : __low2half2(sA2);
-          const __half2 na = nib ? __high2half2(nmA2) : __low2half2(nmA2);
-          const __half2 sb = nib ? __high2half2(sB2) : __low2half2(sB2);
-          const __half2 nb = nib ? __high2half2(nmB2) : __low2half2(nmB2);
-          const __half2 off = nib ? off_hi : off_lo;
-          const uint32_t mask = nib ? 0x00F000F0u : 0x000F000Fu;
-          const uint32_t magic = nib ? 0x54005400u : 0x64006400u;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {   // weights 16h + 4c4 .. +3 of the run
-            const uint32_t wa = wA[h], wb = wB[h];
-            uint32_t af[4];
-            af[0] = deq2((wa & mask) | magic, off, sa, na);          // row g,     nibbles 0, 2
-            af[1] = deq2((wb & mask) | magic, off, sb, nb);          // row g + 8
-            af[2] = deq2(((wa >> 8) & mask) | magic, off, sa, na);   // row g,     nibbles 1, 3
-            af[3] = deq2(((wb >> 8) & mask) | magic, off, sb, nb);
-            const int kx = 64 * c + 32 * nib + 16 * h;
-#pragma unroll
-            for (int j = 0; j < kMtNT; ++j) {
-              if (j < nt) {
-                const uint2 bv = *reinterpret_cast<const uint2*>(xs + j * 8 * kMtXPitch + 2 * kx);
-                ptx::mma_f16(acc[j], af, bv.x, bv.y);
-              }
-            }
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&empty[stage]);
-      if (++stage == kMtStages) {
-        stage = 0;
-        phase ^= 1u;
-      }
+    const int nt = (min(tl.z, kMtMaxRows) + 7) >> 3;
+    // one instantiation per N-tile count: no MMA is issued for an empty N tile
+    switch (nt) {
+      case 1: ok = mt_unit<kMode, 1>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 2: ok = mt_unit<kMode, 2>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 3: ok = mt_unit<kMode, 3>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 4: ok = mt_unit<kMode, 4>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 5: ok = mt_unit<kMode, 5>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 6: ok = mt_unit<kMode, 6>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 7: ok = mt_unit<kMode, 7>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      default: ok = mt_unit<kMode, 8>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
     }
     if (!ok) break;
-    // epilogue: undo the row's 2^k and the activation row's scale
-    const int prow0 = tl.w + tl.y;
-    const float sA = pow2f(-kA), sB = pow2f(-kB);
-#pragma unroll
-    for (int j = 0; j < kMtNT; ++j) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int n = 8 * j + 2 * c4 + e;
-        if (j < nt && n < cnt) {
-          const int prow = prow0 + n;
-          const float inv = __ldg(a.rinv + prow);
-          float* orow = a.out + (size_t)prow * a.out_ld;
-          if (kMode == 0) {
-            if (oA < a.out_rows) {
-              const float gv = acc[j][e] * (inv * sA), up = acc[j][2 + e] * (inv * sB);
-              orow[oA] = __fdividef(gv, 1.f + __expf(-gv)) * up;   // silu(g) * u
-            }
-          } else {
-            orow[oA] = acc[j][e] * (inv * sA);
-            orow[oB] = acc[j][2 + e] * (inv * sB);
-          }
-        }
-      }
-    }
   }
 }
 
@@ -660,9 +687,36 @@ __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a)
 // (for the decode kernels, which stream their weights once without
 // dequantising them).  With mt_rows > 0, an expert with at most mt_rows rows
 // becomes one few-row tile, and so does the last partial chunk of a larger
-// expert when it has at most mt_rows rows; the unit counters of the few-row
-// kernels are zeroed here.  One block; experts are taken 1024 at a time with
-// block scans of their tile counts and of their membership of the lists.
+// expert when it has at most mt_rows rows.  The few-row tiles are listed by
+// their MMA N-tile count (rows / 8, rounded up), largest first, in expert
+// order within a count: their units are claimed in list order, so the
+// longest run first.  The unit counters of the few-row kernels are zeroed
+// here.  One block of 1024 threads; experts are taken 1024 at a time with
+// block scans (GEMM tiles, small experts) and warp ballots (few-row tiles).
+struct TileCls {
+  int e, c, r0, nt, sm, mt, nb;   // expert, rows, first row, GEMM tiles, small, few-row tile, its N tiles
+};
+__device__ __forceinline__ TileCls classify(int i, int na, const int* act, const int* counts, const int* offsets,
+                                            int small_rows, int mt_rows, int ep_rank, int ep_world) {
+  TileCls t{0, 0, 0, 0, 0, 0, 0};
+  if (i >= na) return t;
+  t.e = __ldcg(act + i);
+  t.c = __ldcg(counts + t.e);
+  t.r0 = __ldcg(offsets + t.e);
+  t.sm = t.c <= small_rows ? 1 : 0;
+  if (!t.sm) {
+    t.nt = (t.c + kGN - 1) / kGN;
+    const int last = t.c - (t.nt - 1) * kGN;   // rows of the last chunk
+    if (last <= mt_rows) {
+      t.mt = 1;
+      t.nb = (last + 7) >> 3;
+      --t.nt;
+    }
+  }
+  if (!ep_owned(t.e, ep_rank, ep_world)) t.sm = t.nt = t.mt = t.nb = 0;   // another rank's expert
+  return t;
+}
+
 __global__ void __launch_bounds__(1024) build_tiles_kernel(const int* __restrict__ act, const int* __restrict__ n_act,
                                                            const int* __restrict__ counts,
                                                            const int* __restrict__ offsets, int4* __restrict__ tiles,
@@ -671,48 +725,75 @@ __global__ void __launch_bounds__(1024) build_tiles_kernel(const int* __restrict
                                                            int mt_rows, int4* __restrict__ mtiles,
                                                            int* __restrict__ n_mtiles, unsigned* __restrict__ mt_next,
                                                            int ep_rank, int ep_world) {
+  constexpr int kNB = kMtMaxRows / 8 + 1;   // N-tile counts 0..8 (0: not a few-row tile)
   __shared__ int s_warp[32];
+  __shared__ int s_bw[kNB][32];             // per count, per warp: tiles, then their first position
+  __shared__ int s_base[kNB];               // per count: first position in the list (all chunks)
   ptx::pdl_wait();
   const int na = __ldcg(n_act);
-  int base = 0, sbase = 0, mbase = 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  if (threadIdx.x < kNB) s_base[threadIdx.x] = 0;
+  __syncthreads();
+  // pass 1: GEMM tiles, small experts, and the number of few-row tiles per N-tile count
+  int base = 0, sbase = 0;
   for (int c0 = 0; c0 < na; c0 += blockDim.x) {
-    const int i = c0 + threadIdx.x;
-    int e = 0, c = 0, r0 = 0, nt = 0, sm = 0, mt = 0;
-    if (i < na) {
-      e = __ldcg(act + i);
-      c = __ldcg(counts + e);
-      r0 = __ldcg(offsets + e);
-      sm = c <= small_rows ? 1 : 0;
-      if (!sm) {
-        nt = (c + kGN - 1) / kGN;
-        const int last = c - (nt - 1) * kGN;   // rows of the last chunk
-        if (last <= mt_rows) {
-          mt = 1;
-          --nt;
-        }
-      }
-      if (!ep_owned(e, ep_rank, ep_world)) sm = nt = mt = 0;   // another rank's expert
-    }
-    int tot, stot, mtot;
-    const int pos = base + block_exclusive_scan_1024(nt, &tot, s_warp);
+    const TileCls t = classify(c0 + threadIdx.x, na, act, counts, offsets, small_rows, mt_rows, ep_rank, ep_world);
+    int tot, stot;
+    const int pos = base + block_exclusive_scan_1024(t.nt, &tot, s_warp);
     __syncthreads();
-    const int spos = sbase + block_exclusive_scan_1024(sm, &stot, s_warp);
-    __syncthreads();
-    const int mpos = mbase + block_exclusive_scan_1024(mt, &mtot, s_warp);
-    for (int j = 0; j < nt; ++j) tiles[pos + j] = make_int4(e, j * kGN, min(kGN, c - j * kGN), r0);
-    if (sm) small[spos] = e;
-    if (mt) mtiles[mpos] = make_int4(e, nt * kGN, c - nt * kGN, r0);
+    const int spos = sbase + block_exclusive_scan_1024(t.sm, &stot, s_warp);
+    for (int j = 0; j < t.nt; ++j) tiles[pos + j] = make_int4(t.e, j * kGN, min(kGN, t.c - j * kGN), t.r0);
+    if (t.sm) small[spos] = t.e;
+    if (t.mt) atomicAdd(&s_base[t.nb], 1);   // counts: the order of the adds does not matter
     base += tot;
     sbase += stot;
-    mbase += mtot;
     __syncthreads();
   }
+  // first position of each count, largest count first
   if (threadIdx.x == 0) {
+    int run = 0;
+    for (int b = kNB - 1; b >= 1; --b) {
+      const int n = s_base[b];
+      s_base[b] = run;
+      run += n;
+    }
     *n_tiles = base;
     *n_small = sbase;
-    *n_mtiles = mbase;
+    *n_mtiles = run;
     mt_next[0] = 0u;
     mt_next[1] = 0u;
+  }
+  __syncthreads();
+  if (mt_rows == 0) return;
+  // pass 2: positions of the few-row tiles (rank within their count: warp
+  // ballots, then a prefix over the warps of the chunk)
+  for (int c0 = 0; c0 < na; c0 += blockDim.x) {
+    const TileCls t = classify(c0 + threadIdx.x, na, act, counts, offsets, small_rows, mt_rows, ep_rank, ep_world);
+    int rank = 0;
+#pragma unroll
+    for (int b = 1; b < kNB; ++b) {
+      const uint32_t m = __ballot_sync(0xffffffffu, t.mt && t.nb == b);
+      if (t.mt && t.nb == b) rank = __popc(m & lt);
+      if (lane == 0) s_bw[b][warp] = __popc(m);
+    }
+    __syncthreads();
+    if (warp >= 1 && warp < kNB) {   // warp b: exclusive prefix of count b over the chunk's warps
+      const int b = warp;
+      const int v = lane < (int)(blockDim.x >> 5) ? s_bw[b][lane] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      s_bw[b][lane] = s_base[b] + incl - v;
+      __syncwarp();
+      if (lane == 31) s_base[b] += incl;   // the next chunk continues after this one
+    }
+    __syncthreads();
+    if (t.mt) mtiles[s_bw[t.nb][warp] + rank] = make_int4(t.e, t.nt * kGN, t.c - t.nt * kGN, t.r0);
+    __syncthreads();
   }
 }
 
