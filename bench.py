@@ -500,6 +500,7 @@ def run_ours(args, cfg, rank: int, world: int, local_rank: int) -> dict | None:
 
 
 STREAM_MODES = ("lru+demand", "lfu+demand", "lru+trace", "lfu+trace")
+EXTRA_STREAM_MODES = ("lfu+lookahead",)   # run only when named in --stream-modes
 
 
 def run_streaming(args, cfg, rank, world, local_rank, peaks) -> dict:
@@ -510,12 +511,18 @@ def run_streaming(args, cfg, rank, world, local_rank, peaks) -> dict:
       <policy>+trace      while layer l runs, layer l+1's experts are read from
                           the trace and prefetched: an oracle predictor, an
                           upper bound
+      lfu+lookahead       (only when named) layer l+1's router
+                          (moe_route_noalloc, on a high-priority side stream)
+                          is applied to layer l's input, and while layer l
+                          runs the experts it picks are prefetched: a
+                          predictor that reads nothing of the future
     with policy lru or lfu (moe_set_cache_policy).  `value` is the fastest
     mode that does not read the trace.  (The workload's routing is a trace
     with its own temporal correlation, not the output of the layers'
-    routers, so a predictor that applies the next layer's router to the
-    current input guesses at random here; the cache's recency and frequency
-    are the causal predictors this trace rewards.)"""
+    routers, and each (step, layer) input is a fresh draw, so the lookahead
+    predictor sees nothing that the trace follows: it guesses at random here,
+    and the cache's recency and frequency are the causal predictors this
+    trace rewards.)"""
     import torch
 
     from routed_expert_ffn_forward_b200 import moe
@@ -536,15 +543,36 @@ def run_streaming(args, cfg, rank, world, local_rank, peaks) -> dict:
     out = torch.empty((1, cfg.hidden), dtype=torch.bfloat16, device=dev)
     modes = args.stream_modes.split(",") if args.stream_modes else list(STREAM_MODES)
     for m in modes:
-        if m not in STREAM_MODES:
-            raise SystemExit(f"unknown streaming mode {m!r}; choose from {','.join(STREAM_MODES)}")
+        if m not in STREAM_MODES + EXTRA_STREAM_MODES:
+            raise SystemExit(f"unknown streaming mode {m!r}; choose from "
+                             f"{','.join(STREAM_MODES + EXTRA_STREAM_MODES)}")
+    if "lfu+lookahead" in modes:
+        Ws = [torch.from_numpy(synth.router_weight(cfg, l)).to(dev) for l in range(cfg.n_layers)]
+        bs = [torch.from_numpy(synth.router_bias(cfg, l)).to(dev) for l in range(cfg.n_layers)]
+        p_ids = torch.empty((1, cfg.top_k), dtype=torch.int32, device=dev)
+        p_w = torch.empty((1, cfg.top_k), dtype=torch.float32, device=dev)
+        p_host = torch.empty((1, cfg.top_k), dtype=torch.int32).pin_memory()
+        side = torch.cuda.Stream(dev, priority=-1)   # the predictor's router, beside the layer's forward
+        p_done = torch.cuda.Event()
 
     def run_step(s, how):
         for l in range(cfg.n_layers):
             nl, ns = (l + 1, s) if l + 1 < cfg.n_layers else (0, s + 1)
+            if how == "lookahead":
+                # route layer l's input with layer l+1's router on the side
+                # stream, queue layer l, then prefetch while layer l runs
+                moe.moe_route_noalloc(x_dev[s, l].data_ptr(), Ws[nl].data_ptr(), bs[nl].data_ptr(), 1, cfg.hidden,
+                                      cfg.n_experts, cfg.top_k, cfg.gating, p_ids.data_ptr(), p_w.data_ptr(),
+                                      side.cuda_stream)
+                with torch.cuda.stream(side):
+                    p_host.copy_(p_ids, non_blocking=True)
+                    p_done.record(side)
             layers[l].forward_routed(x_dev[s, l], trace[s, l][None], out, stream.cuda_stream)
             if how == "trace" and ns < n_steps:
                 layers[nl].prefetch(trace[ns, nl])
+            elif how == "lookahead":
+                p_done.synchronize()
+                layers[nl].prefetch(p_host.numpy()[0])
 
     res = {}
     clocks = None
@@ -640,7 +668,8 @@ def main():
     ap.add_argument("--clocks-dir", default=tempfile.gettempdir(),
                     help="where the raw nvidia-smi samples of the timed region are written")
     ap.add_argument("--stream-modes", default="",
-                    help="config 4: comma-separated modes out of " + ",".join(STREAM_MODES) + " (default: all)")
+                    help="config 4: comma-separated modes out of " + ",".join(STREAM_MODES + EXTRA_STREAM_MODES) +
+                         " (default: " + ",".join(STREAM_MODES) + ")")
     ap.add_argument("--no-extra", action="store_true",
                     help="config 1 only: skip the batched-decode and prefill lines added to the JSON")
     ap.add_argument("--small", action="store_true",
