@@ -75,8 +75,8 @@ struct FzLayout {
     unit = bars + 13 * 8;                             // int [kFzStages]
     ids = unit + kFzStages * 4;                       // int [40]
     w = ids + 40 * 4;                                 // float [40]
-    flags = w + 40 * 4;                               // int [4]
-    part = up16(flags + 16);                          // float [2][1024]
+    flags = w + 40 * 4;                               // int [4], then u64 barrier target
+    part = up16(flags + 24);                          // float [2][1024]
     xh = part + 2048 * 4;                             // u8 [H]
     xl = xh + (uint32_t)H;                            // u8 [H]
     xsc = xl + (uint32_t)H;                           // float2 [H/32]
@@ -115,7 +115,6 @@ __device__ __forceinline__ bool spin_until_ge(const uint32_t* p, uint32_t v, uin
 template <int PL>
 __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const FusedArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ unsigned long long s_bar_target;   // grid-barrier arrivals this launch waits for
   uint8_t* sm = fz_aligned(smem_raw);
   const int H = a.H, E = a.E, k = a.k, S = a.S, kS = k + S;
   const FzLayout lay(H, a.act_slot_bytes, a.stages * a.stage_bytes);
@@ -132,6 +131,8 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
   int* s_ids = reinterpret_cast<int*>(sm + lay.ids);
   float* s_w = reinterpret_cast<float*>(sm + lay.w);
   volatile int* s_flag = reinterpret_cast<volatile int*>(sm + lay.flags);  // [0] abort [3] owned picks
+  // grid-barrier arrivals this launch waits for
+  uint64_t& s_bar_target = *reinterpret_cast<uint64_t*>(sm + lay.flags + 16);
   float* s_part = reinterpret_cast<float*>(sm + lay.part);
   uint8_t* s_xh = sm + lay.xh;
   uint8_t* s_xl = sm + lay.xl;
