@@ -50,7 +50,7 @@ namespace {
 constexpr int kFzWarps = 16;                       // consumer warps
 constexpr int kFzThreads = (kFzWarps + 1) * 32;
 constexpr int kFzConsumers = kFzWarps * 32;
-constexpr int kFzGuRows = 128;                     // gate/up unit: weight rows of gate and of up
+constexpr int kFzGuRows = 64;                      // gate/up unit: weight rows of gate and of up
 constexpr int kFzDnRows = 64;                      // down unit: output rows
 constexpr int kFzDnSb = 4;                         // 256-weight groups per down stage
 constexpr int kFzStages = 4;                       // at most; a stage is 256 x the group size (Q4_K: 36,864 B)
@@ -61,10 +61,10 @@ constexpr unsigned kErrFzProducer = 1u << 10, kErrFzConsumer = 1u << 11, kErrFzG
                    kErrFzReady = 1u << 13;
 
 // global sync words (FusedArgs::sync)
-// sync words: [2] down-unit claims, [3] finished down units, [4..5] grid
+// sync words: [1] routed gate/up-unit claims, [2] down-unit claims, [3] finished down units, [4..5] grid
 // barrier arrivals (64-bit, only ever grows: launch L waits for (L+1)·grid),
 // [8..] per-pick gate/up units done
-constexpr int kSyncNext = 2, kSyncDone = 3, kSyncBar64 = 4, kSyncReady = 8;
+constexpr int kSyncGu = 1, kSyncNext = 2, kSyncDone = 3, kSyncBar64 = 4, kSyncReady = 8;
 
 // Shared-memory layout (offsets from the 1024-aligned base).
 struct FzLayout {
@@ -140,7 +140,8 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
   uint8_t* s_uni = sm + lay.uni;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gu_tiles = (a.I + kFzGuRows - 1) / kFzGuRows;
-  const int n_gu = kS * gu_tiles;
+  const int n_gu = kS * gu_tiles, n_gu_sh = S * gu_tiles;   // units: the shared experts' first
+  const int n_gst = (a.nbh + 1) / 2;                        // stages per gate/up unit
   const int dn_tiles = H / kFzDnRows;
   const int n_dn = kS * dn_tiles;
   const int n_dst = (a.nbi + kFzDnSb - 1) / kFzDnSb;  // stages per down unit
@@ -174,23 +175,6 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
     bool routed = false, ok = true;
     // in streaming mode the expert -> slot table comes from the previous kernel
     if (!a.early) ptx::pdl_wait();
-    // While the router runs, every CTA brings a share of the shared experts'
-    // weights into L2 (they need no routing): the gate/up boxes in K order,
-    // then the down boxes.  The CTAs that run those units read them from L2.
-    for (int s = 0; s < S; ++s) {
-      if (!ep_owned(E + s, a.ep_rank, a.ep_world)) continue;
-      const CUtensorMap* m = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + E + s), a.n_slots, a.err);
-      const int n_gub = 2 * a.nbh * gu_tiles, n_items = n_gub + a.nbi * dn_tiles;
-      for (int q = blockIdx.x; q < n_items; q += gridDim.x) {
-        if (q < n_gub) {
-          const int kb = q / (2 * gu_tiles), r = q - kb * 2 * gu_tiles;
-          ptx::tma_prefetch_l2_2d(m + 3 + (r & 1), kb * gu_el, (r >> 1) * kFzGuRows);
-        } else {
-          const int q2 = q - n_gub, kb = q2 / dn_tiles, rt = q2 - kb * dn_tiles;
-          ptx::tma_prefetch_l2_2d(m + 6, kb * dn_el, rt * kFzDnRows);
-        }
-      }
-    }
     auto expert_of = [&](int j) { return in_range(j < k ? s_ids[j] : E + (j - k), E + S, a.err); };
     auto next_stage = [&]() {
       if (++stage == n_stages) {
@@ -198,39 +182,48 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         phase ^= 1u;
       }
     };
-    // gate/up: static units blockIdx.x, + grid, ...; the shared experts first
-    for (int u = blockIdx.x; u < n_gu && ok; u += gridDim.x) {
+    // the stages of gate/up unit u: per stage two super-blocks (columns) of the
+    // unit's 64 gate rows and 64 up rows, one box each
+    auto issue_gu = [&](int u) -> bool {
       const int jj = u / gu_tiles, rt = u - jj * gu_tiles;
       const int j = jj < S ? k + jj : jj - S;
-      if (j < k && !routed) {
-        if (!ptx::mbar_wait_sleep(route_ready, 0, 64, lim)) {
-          ok = false;
-          break;
-        }
-        routed = true;
-      }
-      if (!ep_owned(expert_of(j), a.ep_rank, a.ep_world)) continue;   // another rank's expert
-      const CUtensorMap* m = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + expert_of(j)), a.n_slots, a.err) + 3;
-      for (int kb = 0; kb < a.nbh; ++kb) {
-        if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, lim)) {
-          ok = false;
-          break;
-        }
-        ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * gu_box));
+      const CUtensorMap* m = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + expert_of(j)), a.n_slots, a.err) + 7;
+      for (int st = 0; st < n_gst; ++st) {
+        if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, lim)) return false;
+        const int nbox = min(2, a.nbh - 2 * st);
+        s_unit[stage] = u;
+        ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * nbox * gu_box));
         uint8_t* dst = ring + stage * stage_bytes;
-        ptx::tma_load_2d(dst, m, kb * gu_el, rt * kFzGuRows, &full[stage]);
-        ptx::tma_load_2d(dst + gu_box, m + 1, kb * gu_el, rt * kFzGuRows, &full[stage]);
+        for (int b = 0; b < nbox; ++b) {
+          ptx::tma_load_2d(dst + b * gu_box, m, (2 * st + b) * gu_el, rt * kFzGuRows, &full[stage]);
+          ptx::tma_load_2d(dst + (2 + b) * gu_box, m + 1, (2 * st + b) * gu_el, rt * kFzGuRows, &full[stage]);
+        }
         issued |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (phase << stage);
         next_stage();
       }
+      return true;
+    };
+    // gate/up: the shared experts' units statically (blockIdx.x, + grid, ...:
+    // they need no routing), then the routed ones claimed from a counter that
+    // CTA 0 zeroed before the grid barrier, once route_ready fires
+    for (int u = blockIdx.x; u < n_gu_sh && ok; u += gridDim.x) {
+      if (!ep_owned(E + u / gu_tiles, a.ep_rank, a.ep_world)) continue;   // another rank's expert
+      ok = issue_gu(u);
     }
-    // down: units claimed from a counter that CTA 0 zeroed before the grid
-    // barrier; the routing (and so that zeroing) is known once route_ready fires
-    if (ok && !routed) {
+    if (ok) {
       ok = ptx::mbar_wait_sleep(route_ready, 0, 64, lim);
       routed = ok;
     }
+    while (ok) {
+      const int u = n_gu_sh + (int)atomicAdd(sync + kSyncGu, 1u);
+      if (u >= n_gu) break;
+      const int j = u / gu_tiles - S;
+      if (!ep_owned(expert_of(j), a.ep_rank, a.ep_world)) continue;
+      ok = issue_gu(u);
+    }
+    // down: units claimed from a counter that CTA 0 zeroed before the grid
+    // barrier; a down unit's code in s_unit is n_gu + its index
     while (ok) {
       if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, lim)) {
         ok = false;
@@ -257,7 +250,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
           break;
         }
         const int nbox = min(kFzDnSb, a.nbi - st * kFzDnSb);
-        s_unit[stage] = u;
+        s_unit[stage] = n_gu + u;
         ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(nbox * dn_box));
         uint8_t* dst = ring + stage * stage_bytes;
         for (int b = 0; b < nbox; ++b)
@@ -377,6 +370,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
     // CTA touches them until it has passed the barrier
     if (blockIdx.x == 0) {
       if (tid == 0) {
+        sync[kSyncGu] = 0u;
         sync[kSyncNext] = 0u;
         sync[kSyncDone] = 0u;
       }
@@ -450,147 +444,146 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
     }
   };
 
-  // (3) gate/up + SwiGLU units
+  // (3) gate/up + SwiGLU units and (4) down units, in the order the producer
+  // issues them: this CTA's shared-expert gate/up units, then routed gate/up
+  // units and down units as claimed.  The routing is needed from the first
+  // unit after the shared ones on.
   {
-    const int c = warp >> 2, row = (warp & 3) * 32 + lane;
-    for (int u = blockIdx.x; u < n_gu; u += gridDim.x) {
-      const int jj = u / gu_tiles, rt = u - jj * gu_tiles;
-      const int j = jj < S ? k + jj : jj - S;
-      if (j < k && !routed) {
-        route();
-        if (s_flag[0]) return;
-      }
-      if (!ep_owned(j < k ? s_ids[j] : E + (j - k), a.ep_rank, a.ep_world)) continue;   // another rank's expert
-      float acc[2] = {0.f, 0.f};  // gate row, up row
-      bool ok = true;
-      for (int kb = 0; kb < a.nbh; ++kb) {
-        if (!ptx::mbar_wait(&full[stage], phase, lim)) {
-          ok = false;
-          break;
-        }
-        const uint8_t* bg = ring + stage * stage_bytes + row * a.sbb_gu;
-        const uint8_t* const blk[2] = {bg, bg + gu_box};
-        const uint8_t *xh = s_xh + kb * kQK, *xl = s_xl + kb * kQK;
-        const float2* xs = s_xsc + kb * 8;
-        switch (a.qgu) {   // uniform across the CTA
-          case kQ5_K: q_chunk_rows<kQ5_K, 2>(blk, c, xh, xl, xs, acc); break;
-          case kQ6_K: q_chunk_rows<kQ6_K, 2>(blk, c, xh, xl, xs, acc); break;
-          case kQ8_0: q_chunk_rows<kQ8_0, 2>(blk, c, xh, xl, xs, acc); break;
-          case kMXFP4: q_chunk_rows<kMXFP4, 2>(blk, c, xh, xl, xs, acc); break;
-          default: q_chunk_rows<kQ4_K, 2>(blk, c, xh, xl, xs, acc); break;
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&empty[stage]);
-        next_stage();
-      }
-      if (!ok) fail(kErrFzConsumer);
-      cbar();
-      if (s_flag[0]) return;
-      s_part[c * kFzGuRows + row] = acc[0];
-      s_part[(4 + c) * kFzGuRows + row] = acc[1];
-      cbar();
-      // SwiGLU (chunk parts summed in a fixed order) -> h_j, warps 0-3
-      if (warp < 4) {
-        const int f = warp * 32 + lane;
-        const float* pg = s_part + f;
-        const float* pu = s_part + 4 * kFzGuRows + f;
-        const float g = ((pg[0] + pg[kFzGuRows]) + pg[2 * kFzGuRows]) + pg[3 * kFzGuRows];
-        const float up = ((pu[0] + pu[kFzGuRows]) + pu[2 * kFzGuRows]) + pu[3 * kFzGuRows];
-        float2 rsc;
-        int8_t hh;
-        uint8_t hl;
-        quant_run16(silu_f(g) * up, hh, hl, rsc);
-        const int feat = rt * kFzGuRows + f;
-        const size_t o = (size_t)j * a.I_pad + feat;
-        a.hq[o] = hh;
-        reinterpret_cast<uint8_t*>(a.hq + a.hq_plane)[o] = hl;
-        if (lane == 0) a.hsc[(size_t)j * (a.I_pad / 32) + feat / 32] = rsc;
-      }
-      // publish the features (the ready counters are zeroed before the barrier)
-      if (!routed) {
-        route();
-        if (s_flag[0]) return;
-      } else {
-        cbar();
-      }
-      if (tid == 0) {
-        ptx::fence_proxy_async_global();
-        ptx::red_add_release_gpu(sync + kSyncReady + j, 1u);
-      }
-    }
-  }
-  if (!routed) {
-    route();
-    if (s_flag[0]) return;
-  }
-
-  // (4) down units.  A unit's 64 rows of y_j are published with one release
-  // add to the count of finished units, which no thread waits on; (5) once
-  // every unit of the forward is counted, the CTAs combine slices of the
-  // output.  The unit partials are double-buffered, so the two warps that
-  // reduce them may lag the others by a unit.
-  {
-    const int r0 = lane, sb = warp >> 2, c = warp & 3;   // rows lane and lane + 32; part = warp
+    int n_sh = 0;   // this CTA's shared gate/up units (the producer skips the same ones)
+    for (int u = blockIdx.x; u < n_gu_sh; u += gridDim.x) n_sh += ep_owned(E + u / gu_tiles, a.ep_rank, a.ep_world);
+    const int g_row = (warp & 1) * 32 + lane, g_sb = (warp >> 1) & 1, g_c = warp >> 2;   // gate/up: row, column, chunk
+    const int r0 = lane, sb = warp >> 2, c = warp & 3;                                    // down: rows r0, r0 + 32
     const int I_pad = a.I_pad;
-    int aslot = 0, buf = 0;
+    int aslot = 0, buf = 0, seen = 0;
     uint32_t aphase = 0;
     while (true) {
+      if (seen++ == n_sh && !routed) {
+        route();
+        if (s_flag[0]) return;
+      }
       bool ok = ptx::mbar_wait(&full[stage], phase, lim);
       const int u = ok ? s_unit[stage] : -1;   // -1 from the producer: end of work
-      const int jj = u / dn_tiles, rt = u - jj * dn_tiles;
-      const int j = jj < S ? k + jj : jj - S;
-      float acc[2] = {0.f, 0.f};
-      if (ok && u >= 0) {
-        ok = ptx::mbar_wait(&afull[aslot], aphase, lim);
-        const uint8_t* act = s_uni + aslot * a.act_slot_bytes;
-        const float2* asc = reinterpret_cast<const float2*>(act + 2 * I_pad);
-        for (int st = 0; st < n_dst && ok; ++st) {
+      if (!ok) fail(kErrFzConsumer);
+      if (u < 0) {
+        cbar();
+        if (s_flag[0]) return;
+        break;
+      }
+      if (u < n_gu) {
+        // ---- gate/up unit: 64 features of pick j
+        const int jj = u / gu_tiles, rt = u - jj * gu_tiles;
+        const int j = jj < S ? k + jj : jj - S;
+        float acc[2] = {0.f, 0.f};   // gate row, up row
+        for (int st = 0; st < n_gst; ++st) {
           if (st > 0 && !ptx::mbar_wait(&full[stage], phase, lim)) {
             ok = false;
             break;
           }
-          const int kb = st * kFzDnSb + sb;
-          if (kb < a.nbi) {
-            const uint8_t* b0 = ring + stage * stage_bytes + sb * dn_box + r0 * a.sbb_d;
-            const uint8_t* const blk[2] = {b0, b0 + 32 * a.sbb_d};
-            const uint8_t *xh = act + kb * kQK, *xl = act + I_pad + kb * kQK;
-            const float2* xs = asc + kb * 8;
-            switch (a.qd) {   // uniform across the CTA
-              case kQ5_K: q_chunk_rows<kQ5_K, 2>(blk, c, xh, xl, xs, acc); break;
-              case kQ6_K: q_chunk_rows<kQ6_K, 2>(blk, c, xh, xl, xs, acc); break;
-              case kQ8_0: q_chunk_rows<kQ8_0, 2>(blk, c, xh, xl, xs, acc); break;
-              case kMXFP4: q_chunk_rows<kMXFP4, 2>(blk, c, xh, xl, xs, acc); break;
-              default: q_chunk_rows<kQ4_K, 2>(blk, c, xh, xl, xs, acc); break;
+          const int kb = 2 * st + g_sb;
+          if (kb < a.nbh) {
+            const uint8_t* bg = ring + stage * stage_bytes + g_sb * gu_box + g_row * a.sbb_gu;
+            const uint8_t* const blk[2] = {bg, bg + 2 * gu_box};
+            const uint8_t *xh = s_xh + kb * kQK, *xl = s_xl + kb * kQK;
+            const float2* xs = s_xsc + kb * 8;
+            switch (a.qgu) {   // uniform across the CTA
+              case kQ5_K: q_chunk_rows<kQ5_K, 2>(blk, g_c, xh, xl, xs, acc); break;
+              case kQ6_K: q_chunk_rows<kQ6_K, 2>(blk, g_c, xh, xl, xs, acc); break;
+              case kQ8_0: q_chunk_rows<kQ8_0, 2>(blk, g_c, xh, xl, xs, acc); break;
+              case kMXFP4: q_chunk_rows<kMXFP4, 2>(blk, g_c, xh, xl, xs, acc); break;
+              default: q_chunk_rows<kQ4_K, 2>(blk, g_c, xh, xl, xs, acc); break;
             }
           }
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&empty[stage]);
           next_stage();
         }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&aempty[aslot]);
-        if (++aslot == 2) {
-          aslot = 0;
-          aphase ^= 1u;
+        if (!ok) fail(kErrFzConsumer);
+        cbar();
+        if (s_flag[0]) return;
+        s_part[(g_sb * 4 + g_c) * kFzGuRows + g_row] = acc[0];
+        s_part[(8 + g_sb * 4 + g_c) * kFzGuRows + g_row] = acc[1];
+        cbar();
+        // SwiGLU (the 8 parts of each row summed in a fixed order) -> h_j, warps 0-1
+        if (warp < 2) {
+          const int f = warp * 32 + lane;
+          float g = s_part[f], up = s_part[8 * kFzGuRows + f];
+#pragma unroll
+          for (int p = 1; p < 8; ++p) {
+            g += s_part[p * kFzGuRows + f];
+            up += s_part[(8 + p) * kFzGuRows + f];
+          }
+          float2 rsc;
+          int8_t hh;
+          uint8_t hl;
+          quant_run16(silu_f(g) * up, hh, hl, rsc);
+          const int feat = rt * kFzGuRows + f;
+          const size_t o = (size_t)j * I_pad + feat;
+          a.hq[o] = hh;
+          reinterpret_cast<uint8_t*>(a.hq + a.hq_plane)[o] = hl;
+          if (lane == 0) a.hsc[(size_t)j * (I_pad / 32) + feat / 32] = rsc;
         }
+        cbar();
+        // publish the features (the ready counters are zeroed before the barrier)
+        if (tid == 0) {
+          ptx::fence_proxy_async_global();
+          ptx::red_add_release_gpu(sync + kSyncReady + j, 1u);
+        }
+        continue;
+      }
+      // ---- down unit: 64 output rows of pick j.  Its 64 rows of y_j are
+      // published with one release add to the count of finished units, which
+      // no thread waits on; the unit partials are double-buffered, so the two
+      // warps that reduce them may lag the others by a unit.
+      const int v = u - n_gu;
+      const int jj = v / dn_tiles, rt = v - jj * dn_tiles;
+      const int j = jj < S ? k + jj : jj - S;
+      float acc[2] = {0.f, 0.f};
+      ok = ptx::mbar_wait(&afull[aslot], aphase, lim);
+      const uint8_t* act = s_uni + aslot * a.act_slot_bytes;
+      const float2* asc = reinterpret_cast<const float2*>(act + 2 * I_pad);
+      for (int st = 0; st < n_dst && ok; ++st) {
+        if (st > 0 && !ptx::mbar_wait(&full[stage], phase, lim)) {
+          ok = false;
+          break;
+        }
+        const int kb = st * kFzDnSb + sb;
+        if (kb < a.nbi) {
+          const uint8_t* b0 = ring + stage * stage_bytes + sb * dn_box + r0 * a.sbb_d;
+          const uint8_t* const blk[2] = {b0, b0 + 32 * a.sbb_d};
+          const uint8_t *xh = act + kb * kQK, *xl = act + I_pad + kb * kQK;
+          const float2* xs = asc + kb * 8;
+          switch (a.qd) {   // uniform across the CTA
+            case kQ5_K: q_chunk_rows<kQ5_K, 2>(blk, c, xh, xl, xs, acc); break;
+            case kQ6_K: q_chunk_rows<kQ6_K, 2>(blk, c, xh, xl, xs, acc); break;
+            case kQ8_0: q_chunk_rows<kQ8_0, 2>(blk, c, xh, xl, xs, acc); break;
+            case kMXFP4: q_chunk_rows<kMXFP4, 2>(blk, c, xh, xl, xs, acc); break;
+            default: q_chunk_rows<kQ4_K, 2>(blk, c, xh, xl, xs, acc); break;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&empty[stage]);
+        next_stage();
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&aempty[aslot]);
+      if (++aslot == 2) {
+        aslot = 0;
+        aphase ^= 1u;
       }
       if (!ok) fail(kErrFzConsumer);
       float* sp = s_part + buf * (kFzWarps * kFzDnRows);
-      if (u >= 0) {
-        sp[warp * kFzDnRows + r0] = acc[0];
-        sp[warp * kFzDnRows + r0 + 32] = acc[1];
-      }
+      sp[warp * kFzDnRows + r0] = acc[0];
+      sp[warp * kFzDnRows + r0 + 32] = acc[1];
       cbar();                          // every warp, every unit: the partials are complete
       if (s_flag[0]) return;
-      if (u < 0) break;                // every warp read the same end marker
       if (warp < 2) {
         // the 16 parts of each row, in a fixed order, to y_j; then one thread
         // publishes the unit (release: cumulative over the two warps' stores)
         const int r = warp * 32 + lane;
-        float v = sp[r];
+        float yv = sp[r];
 #pragma unroll
-        for (int p = 1; p < kFzWarps; ++p) v += sp[p * kFzDnRows + r];
-        a.y[(size_t)j * H + rt * kFzDnRows + r] = v;
+        for (int p = 1; p < kFzWarps; ++p) yv += sp[p * kFzDnRows + r];
+        a.y[(size_t)j * H + rt * kFzDnRows + r] = yv;
         ptx::named_barrier_sync(2, 64);
         if (tid == 0) ptx::red_add_release_gpu(sync + kSyncDone, 1u);
       }

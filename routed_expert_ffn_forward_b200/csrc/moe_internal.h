@@ -182,9 +182,9 @@ cudaError_t launch_decode1_fused(const FusedArgs& a, int n_sm, cudaStream_t st);
 // Tensor maps of one expert's Q4_K matrices at `base`, kMapsPerSlot of them:
 // [0..2] gate, up, down with boxes of 64 rows x 2 (gate/up) or 4 (down)
 // super-blocks (decode kernels); [3..5] gate, up, down with boxes of 128 rows x
-// 1 super-block (single-token GEMVs and prefill GEMMs); [6] down with boxes of
-// 64 rows x 1 super-block (the fused single-token kernel).
-constexpr int kMapsPerSlot = 7;
+// 1 super-block (single-token GEMVs and prefill GEMMs); [6..8] down, gate, up
+// with boxes of 64 rows x 1 super-block (the fused single-token kernel).
+constexpr int kMapsPerSlot = 9;
 struct Shape;
 cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, const Shape& s);
 // Copy one weight matrix of `rows` rows from its GGUF host bytes into the

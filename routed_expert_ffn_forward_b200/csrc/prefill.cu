@@ -484,11 +484,10 @@ __device__ __forceinline__ bool mt_unit(const GemmArgs& a, const uint8_t* sm, ui
       atomicOr(a.err, 64u);
       return false;
     }
-    const uint8_t* st = sm + stage * kMtStageBytes;
-    const uint8_t* rA = st + offA;
-    const uint8_t* rB = st + offB;
-    const uint8_t* xs = st + kMtWBytes + g * kMtXPitch + 8 * c4;   // token row g of N tile 0
-    const uint4 hA = *reinterpret_cast<const uint4*>(rA), hB = *reinterpret_cast<const uint4*>(rB);
+    const uint32_t st = ptx::smem_u32(sm) + (uint32_t)(stage * kMtStageBytes);
+    const uint32_t rA = st + offA, rB = st + offB;
+    const uint32_t xs = st + kMtWBytes + g * kMtXPitch + 8 * c4;   // token row g of N tile 0
+    const uint4 hA = ptx::lds_v4(rA), hB = ptx::lds_v4(rB);
     __half2 d2sA, nm2sA, d2sB, nm2sB;
     {
       const uint32_t dA = __byte_perm(hA.x, 0u, 0x1010u), mA = __byte_perm(hA.x, 0u, 0x3232u);
@@ -503,9 +502,9 @@ __device__ __forceinline__ bool mt_unit(const GemmArgs& a, const uint8_t* sm, ui
       __half2 sA2, nmA2, sB2, nmB2;
       chunk_scales(hA, c, d2sA, nm2sA, sA2, nmA2);
       chunk_scales(hB, c, d2sB, nm2sB, sB2, nmB2);
-      const uint32_t* qA = reinterpret_cast<const uint32_t*>(rA + 16 + 32 * c);
-      const uint32_t* qB = reinterpret_cast<const uint32_t*>(rB + 16 + 32 * c);
-      const uint32_t wA[2] = {qA[c4], qA[4 + c4]}, wB[2] = {qB[c4], qB[4 + c4]};
+      const uint32_t qA = rA + 16 + 32 * c + 4 * c4, qB = rB + 16 + 32 * c + 4 * c4;
+      const uint32_t wA[2] = {ptx::lds_u32(qA), ptx::lds_u32(qA + 16)};
+      const uint32_t wB[2] = {ptx::lds_u32(qB), ptx::lds_u32(qB + 16)};
 #pragma unroll
       for (int nib = 0; nib < 2; ++nib) {   // run 2c (low nibbles), run 2c + 1 (high nibbles)
         const __half2 sa = nib ? __high2half2(sA2) : __low2half2(sA2);
@@ -523,10 +522,10 @@ __device__ __forceinline__ bool mt_unit(const GemmArgs& a, const uint8_t* sm, ui
           af[1] = deq2((wb & mask) | magic, off, sb, nb);          // row g + 8
           af[2] = deq2(((wa >> 8) & mask) | magic, off, sa, na);   // row g,     nibbles 1, 3
           af[3] = deq2(((wb >> 8) & mask) | magic, off, sb, nb);
-          const uint8_t* xk = xs + 2 * (64 * c + 32 * nib + 16 * h);
+          const uint32_t xk = xs + 2 * (64 * c + 32 * nib + 16 * h);
 #pragma unroll
           for (int j = 0; j < NT; ++j) {
-            const uint2 bv = *reinterpret_cast<const uint2*>(xk + j * 8 * kMtXPitch);
+            const uint2 bv = ptx::lds_v2(xk + j * 8 * kMtXPitch);
             ptx::mma_f16(acc[j], af, bv.x, bv.y);
           }
         }
