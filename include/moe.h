@@ -355,10 +355,11 @@ moe_status moe_combine_partials(const float* partials, void* out, int T, int H, 
 /* Test hooks for failure detection (process-wide, off by default), read by
  * the single-token kernel at each launch.  wait_limit_ns: limit of its bounded
  * waits (0 = the default 2 s); the final wait for its own copies in flight
- * keeps the default.  hold_barrier > 0: its grid barrier waits for that many
- * arrivals more than there are CTAs, so the wait runs out and the kernel
- * returns with an error that moe_check reports (which also resets the
- * kernel's counters, so the next forward runs normally).  No GPU fault is
+ * keeps the default.  hold_barrier > 0: its wait for the router's logits
+ * (the one point where every CTA waits for all the others) looks for the
+ * logits of a launch that many launches ahead, so the wait runs out and the
+ * kernel returns with an error that moe_check reports (which also resets the
+ * kernel's step counters, so the next forward runs normally).  No GPU fault is
  * involved: the kernel's CTAs give up and exit.  No counterpart on the pages
  * (failure detection). */
 moe_status moe_set_test_hooks(uint64_t wait_limit_ns, int hold_barrier);

@@ -61,10 +61,16 @@ constexpr unsigned kErrFzProducer = 1u << 10, kErrFzConsumer = 1u << 11, kErrFzG
                    kErrFzReady = 1u << 13;
 
 // global sync words (FusedArgs::sync)
-// sync words: [1] routed gate/up-unit claims, [2] down-unit claims, [3] finished down units, [4..5] grid
-// barrier arrivals (64-bit, only ever grows: launch L waits for (L+1)·grid),
-// [8..] per-pick gate/up units done
-constexpr int kSyncGu = 1, kSyncNext = 2, kSyncDone = 3, kSyncBar64 = 4, kSyncReady = 8;
+// sync words: [4..5] launch counter (64-bit; every CTA adds 1 at its start
+// and it is never reset, so a CTA of launch L reads a value in
+// [L·grid, (L+1)·grid)).  Per launch parity s = L & 1: [8+s] routed gate/up
+// unit claims, [10+s] down-unit claims, [12+s] finished down units,
+// [16+64s+j] finished gate/up units of pick j; launch L zeroes parity
+// s ^ 1 for launch L + 1 (launch L - 1, its last user, has completed).
+// [kSyncLogits..] the logits, each a 64-bit word (L + 1, fp32 bits): a
+// reader knows a logit is this launch's without any barrier or fence.
+constexpr int kSyncEpoch = 4, kSyncGu = 8, kSyncNext = 10, kSyncDone = 12, kSyncReady = 16, kSyncLogits = 256;
+static_assert(kSyncLogits + 2 * 1024 <= kSyncWords, "sync words hold 1024 tagged logits");
 
 // Shared-memory layout (offsets from the 1024-aligned base).
 struct FzLayout {
@@ -131,8 +137,8 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
   int* s_ids = reinterpret_cast<int*>(sm + lay.ids);
   float* s_w = reinterpret_cast<float*>(sm + lay.w);
   volatile int* s_flag = reinterpret_cast<volatile int*>(sm + lay.flags);  // [0] abort [3] owned picks
-  // grid-barrier arrivals this launch waits for
-  uint64_t& s_bar_target = *reinterpret_cast<uint64_t*>(sm + lay.flags + 16);
+  // this launch's index L (launch counter / grid)
+  uint64_t& s_epoch = *reinterpret_cast<uint64_t*>(sm + lay.flags + 16);
   float* s_part = reinterpret_cast<float*>(sm + lay.part);
   uint8_t* s_xh = sm + lay.xh;
   uint8_t* s_xl = sm + lay.xl;
@@ -215,8 +221,13 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
       ok = ptx::mbar_wait_sleep(route_ready, 0, 64, lim);
       routed = ok;
     }
+    // this launch's counters (s_epoch was set before route_ready fired)
+    const int par = (int)(s_epoch & 1u);
+    uint32_t* const ctr_gu = sync + kSyncGu + par;
+    uint32_t* const ctr_next = sync + kSyncNext + par;
+    const uint32_t* const ready = sync + kSyncReady + 64 * par;
     while (ok) {
-      const int u = n_gu_sh + (int)atomicAdd(sync + kSyncGu, 1u);
+      const int u = n_gu_sh + (int)atomicAdd(ctr_gu, 1u);
       if (u >= n_gu) break;
       const int j = u / gu_tiles - S;
       if (!ep_owned(expert_of(j), a.ep_rank, a.ep_world)) continue;
@@ -229,7 +240,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         ok = false;
         break;
       }
-      const int u = (int)atomicAdd(sync + kSyncNext, 1u);
+      const int u = (int)atomicAdd(ctr_next, 1u);
       if (u >= n_dn) {
         // end of work.  The stage is empty, so its last copy has landed and
         // been read; its arrival below completes one more phase of full[stage],
@@ -265,7 +276,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         ok = false;
         break;
       }
-      if (!spin_until_ge(sync + kSyncReady + j, (uint32_t)gu_tiles, lim)) {
+      if (!spin_until_ge(ready + j, (uint32_t)gu_tiles, lim)) {
         atomicOr(a.err, kErrFzReady);
         ok = false;
         break;
@@ -316,6 +327,10 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
     constexpr int kPieces = 8;
     __nv_bfloat16* s_x = reinterpret_cast<__nv_bfloat16*>(s_uni);
     const uint2* xv = reinterpret_cast<const uint2*>(s_x);
+    // this CTA's count on the launch counter, taken first so that its round
+    // trip overlaps the router's loads
+    unsigned long long launch_ctr = 0;
+    if (tid == 0) launch_ctr = atomicAdd(reinterpret_cast<unsigned long long*>(sync + kSyncEpoch), 1ull);
     bool first = true;
     for (int e0 = blockIdx.x; e0 < E; e0 += 2 * gridDim.x) {
       const int e = e0 + half * gridDim.x;
@@ -334,6 +349,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
           ptx::pdl_wait();
           const uint4* src = reinterpret_cast<const uint4*>(a.x);
           for (int i = tid; i < H / 8; i += kFzConsumers) reinterpret_cast<uint4*>(s_x)[i] = __ldcg(src + i);
+          if (tid == 0) s_epoch = launch_ctr / gridDim.x;
           cbar();
           first = false;
         }
@@ -357,7 +373,10 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         float v = 0.f;
 #pragma unroll
         for (int w8 = 0; w8 < 8; ++w8) v += s_part[half * 8 + w8];
-        a.logits[e] = v + (a.b ? a.b[e] : 0.f);
+        const float lv = v + (a.b ? a.b[e] : 0.f);
+        a.logits[e] = lv;
+        ptx::st_relaxed_gpu_u64(reinterpret_cast<uint64_t*>(sync + kSyncLogits) + e,
+                                ((uint64_t)(uint32_t)(s_epoch + 1u) << 32) | __float_as_uint(lv));
       }
       cbar();
     }
@@ -365,28 +384,20 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
       ptx::pdl_wait();
       const uint4* src = reinterpret_cast<const uint4*>(a.x);
       for (int i = tid; i < H / 8; i += kFzConsumers) reinterpret_cast<uint4*>(s_x)[i] = __ldcg(src + i);
+      if (tid == 0) s_epoch = launch_ctr / gridDim.x;
+      cbar();
     }
-    // CTA 0 zeroes the step counters for this launch before it arrives: no
-    // CTA touches them until it has passed the barrier
+    // CTA 0 zeroes the other parity's counters for the next launch (the
+    // previous launch, their last user, is complete: this is after the wait
+    // for the previous kernel)
     if (blockIdx.x == 0) {
+      const int nx = (int)((s_epoch & 1u) ^ 1u);
       if (tid == 0) {
-        sync[kSyncGu] = 0u;
-        sync[kSyncNext] = 0u;
-        sync[kSyncDone] = 0u;
+        sync[kSyncGu + nx] = 0u;
+        sync[kSyncNext + nx] = 0u;
+        sync[kSyncDone + nx] = 0u;
       }
-      for (int i = tid; i < kS; i += kFzConsumers) sync[kSyncReady + i] = 0u;
-    }
-    cbar();   // thread 0's fence below is cumulative over these writes and the logits
-    if (tid == 0) {
-      // arrivals before this CTA's own are within this launch's band
-      // [L·grid, (L+1)·grid), so it waits for (L+1)·grid (+ hold, a test hook
-      // that makes the wait run out); the release add publishes the CTA's
-      // logits and CTA 0's zeroed counters (ordered before it by the barrier
-      // above)
-      uint64_t* bar = reinterpret_cast<uint64_t*>(sync + kSyncBar64);
-      const uint64_t G = gridDim.x;
-      s_bar_target = (ptx::ld_relaxed_gpu_u64(bar) / G + 1) * G + (uint64_t)a.hold;
-      ptx::red_add_release_gpu_u64(bar, 1ull);
+      for (int i = tid; i < kS; i += kFzConsumers) sync[kSyncReady + 64 * nx + i] = 0u;
     }
   }
 
@@ -408,13 +419,33 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
   // the routing: every CTA selects from the E logits itself, after the barrier
   bool routed = false;
   auto route = [&]() {
-    if (tid == 0) {
-      if (!spin_until_ge64(reinterpret_cast<const uint64_t*>(sync + kSyncBar64), s_bar_target, lim))
-        fail(kErrFzGrid);
+    bool got = false;
+    if (warp == 0) {
+      // every logit of this launch, polled until all carry its tag (+ hold,
+      // a test hook that makes the wait run out), copied to shared memory
+      const uint32_t want = (uint32_t)(s_epoch + 1u + (uint64_t)a.hold);
+      const uint64_t* lg = reinterpret_cast<const uint64_t*>(sync + kSyncLogits);
+      float* s_lg = reinterpret_cast<float*>(s_uni);   // x (bf16) is no longer needed there
+      const uint64_t t0 = ptx::globaltimer();
+      while (true) {
+        bool mine = true;
+        for (int e = lane; e < E; e += 32) {
+          const uint64_t v = ptx::ld_relaxed_gpu_u64(lg + e);
+          mine &= (uint32_t)(v >> 32) == want;
+          s_lg[e] = __uint_as_float((uint32_t)v);
+        }
+        if (__all_sync(0xffffffffu, mine)) {
+          got = true;
+          break;
+        }
+        if (ptx::globaltimer() - t0 > lim) break;
+        __nanosleep(32);
+      }
+      if (!got && lane == 0) fail(kErrFzGrid);
+      __syncwarp();
     }
-    cbar();
-    if (!s_flag[0] && warp == 0) {
-      warp_topk_gate<PL, true>(a.logits, E, k, a.gating, a.forced, s_ids, s_w);
+    if (got) {
+      warp_topk_gate<PL, false>(reinterpret_cast<const float*>(s_uni), E, k, a.gating, a.forced, s_ids, s_w);
       __syncwarp();
       if (lane < S) {
         s_ids[k + lane] = E + lane;
@@ -526,7 +557,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         // publish the features (the ready counters are zeroed before the barrier)
         if (tid == 0) {
           ptx::fence_proxy_async_global();
-          ptx::red_add_release_gpu(sync + kSyncReady + j, 1u);
+          ptx::red_add_release_gpu(sync + kSyncReady + 64 * (int)(s_epoch & 1u) + j, 1u);
         }
         continue;
       }
@@ -585,7 +616,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         for (int p = 1; p < kFzWarps; ++p) yv += sp[p * kFzDnRows + r];
         a.y[(size_t)j * H + rt * kFzDnRows + r] = yv;
         ptx::named_barrier_sync(2, 64);
-        if (tid == 0) ptx::red_add_release_gpu(sync + kSyncDone, 1u);
+        if (tid == 0) ptx::red_add_release_gpu(sync + kSyncDone + (int)(s_epoch & 1u), 1u);
       }
       buf ^= 1;
     }
@@ -595,7 +626,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
     // that fixed order; CTA c takes outputs c*512 .. c*512+511, + grid*512, ...
     if (tid == 0) {
       const uint32_t want = (uint32_t)(s_flag[3] * dn_tiles);
-      if (!spin_until_ge(sync + kSyncDone, want, lim)) fail(kErrFzReady);
+      if (!spin_until_ge(sync + kSyncDone + (int)(s_epoch & 1u), want, lim)) fail(kErrFzReady);
     }
     cbar();
     if (s_flag[0]) return;

@@ -1239,9 +1239,10 @@ moe_status moe_check(moe_layer_t L) {
   CUDA_TRY(cudaStreamSynchronize(L->copy));
   const unsigned flags = *L->h_err;
   if (flags) {
-    // a kernel that gave up may have left its barrier and step counters
-    // half-way: start them from zero again
-    CUDA_TRY(cudaMemsetAsync(L->wk.sync, 0, kSyncWords * sizeof(unsigned), L->copy));
+    // a kernel that gave up may have left its step counters half-way: start
+    // them from zero again (not the launch counter, words 4-5, which stays a
+    // multiple of the grid: every CTA of every launch adds 1 at its start)
+    CUDA_TRY(cudaMemsetAsync(L->wk.sync + 8, 0, (kSyncWords - 8) * sizeof(unsigned), L->copy));
     CUDA_TRY(cudaMemsetAsync(L->wk.err, 0, sizeof(unsigned), L->copy));
     CUDA_TRY(cudaStreamSynchronize(L->copy));
     if (flags & kErrBoundsBit)

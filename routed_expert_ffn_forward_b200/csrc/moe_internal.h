@@ -73,9 +73,9 @@ struct Work {
   __half* h16;        // [P_cap, I_pad] SwiGLU output, fp16 scaled by 1/hinv, same K order
   float* hinv;        // [P]
   float* rpart;       // router partial logits [splits][T][E]
-  unsigned* sync;     // [kSyncWords] grid barrier and step counters of the fused single-token kernel
+  unsigned* sync;     // [kSyncWords] launch counter, step counters and tagged logits of the one-token kernel
 };
-constexpr int kSyncWords = 512;
+constexpr int kSyncWords = 2304;   // counters, then 1024 tagged 64-bit logits
 
 struct RouteArgs {
   const __nv_bfloat16* x;

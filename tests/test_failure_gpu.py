@@ -1,6 +1,7 @@
 """Failure detection on the GPU without a GPU fault: the single-token kernel's
-grid barrier is told (a test hook) to wait for one arrival more than there
-are CTAs, so no CTA ever releases it -- a flag that nothing sets.  Every CTA
+wait for the router's logits (where every CTA waits for all the others) is
+told (a test hook) to look for the logits of the next launch, which no CTA
+writes -- a flag that nothing sets.  Every CTA
 gives up after a short limit, drains its copies in flight and exits; the
 forward's stream and the context stay usable, moe_check reports the error
 and resets the kernel's counters, and the next forward gives the same result
@@ -15,7 +16,7 @@ from routed_expert_ffn_forward_b200 import build, moe, synth
 pytestmark = pytest.mark.gpu
 
 
-def test_grid_barrier_wait_runs_out_and_recovers():
+def test_cross_cta_wait_runs_out_and_recovers():
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
@@ -29,7 +30,7 @@ def test_grid_barrier_wait_runs_out_and_recovers():
         want = L.forward(x).clone()
         torch.cuda.synchronize()
         moe.moe_check(L.handle)
-        moe.moe_set_test_hooks(20_000_000, 1)          # 20 ms, barrier never released
+        moe.moe_set_test_hooks(20_000_000, 1)          # 20 ms, logits of a launch that never comes
         try:
             L.forward(x)
             torch.cuda.synchronize()                   # the kernel returns: nothing hangs
