@@ -414,7 +414,7 @@ def measure_resident(args, cfg, rank, world, local_rank, peaks, steps, warmup, e
             "dtype": DTYPE_DECODE if T <= 4 else DTYPE_PREFILL}
 
 
-FEW_ROWS = 64   # the library's default moe_set_few_row_tiles
+FEW_ROWS = 32   # the library's default moe_set_few_row_tiles
 
 
 def tile_split(cfg, ids: np.ndarray, few_rows: int = FEW_ROWS):

@@ -241,7 +241,7 @@ struct GemmArgs {
   unsigned* next;
   int n_rows;                // activation rows P (debug builds)
 };
-constexpr int kMtMaxRows = 64;   // most activation rows of a few-row tile
+constexpr int kMtMaxRows = 32;   // most activation rows of a few-row tile
 size_t prefill_gemm_smem();
 size_t prefill_max_tiles(int n_experts_total, size_t pairs);
 // GEMM tiles of up to 256 rows for the experts with more than small_rows rows

@@ -425,7 +425,8 @@ done:
 // 0-7 are the gate rows of features 8w..8w+7 and rows 8-15 their up rows, so a
 // thread holds g and u of the same (feature, token) and applies SwiGLU in
 // registers; down: output rows 16w..16w+15 -- against every activation row of
-// the tile as up to kMtMaxRows / 8 MMA N tiles.
+// the tile as up to kMtMaxRows / 8 MMA N tiles.  The producer warp issues a
+// stage's activation rows one per lane.
 //
 // K order: the thread at quad position c takes, from each 16-weight half of a
 // 32-weight run, the weights 4c..4c+3: nibbles (0, 2) of its quant word form
@@ -433,7 +434,7 @@ done:
 // the activations are stored within every group of four.
 constexpr int kMtWarps = 16;
 constexpr int kMtThreads = (kMtWarps + 1) * 32;          // + one producer warp
-constexpr int kMtStages = 3;
+constexpr int kMtStages = 4;
 constexpr int kMtWBytes = 2 * kRawBytes;                 // 256 weight rows x 1 super-block
 constexpr int kMtXPitch = 2 * kQK + 32;                  // one activation row's 256 fp16, padded
 constexpr int kMtStageBytes = kMtWBytes + kMtMaxRows * kMtXPitch;
@@ -588,45 +589,54 @@ __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a)
 
   if (warp == kMtWarps) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      ptx::IssueLog log;
-      bool ok = true;
-      while (ok) {
-        const int u = (int)atomicAdd(a.next, 1u);
-        if (u >= n_units) break;
-        const int4 tl = __ldcg(a.tiles + u / ft);   // (expert, n0, count, r0)
-        const int f = u % ft;
-        const int ex = in_range(tl.x, a.n_ex, a.err);
-        const CUtensorMap* wm = a.wmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + ex), a.n_slots, a.err) + 3;
-        const CUtensorMap* m0 = kMode == 0 ? wm : wm + 2;
-        const CUtensorMap* m1 = kMode == 0 ? wm + 1 : wm + 2;
-        const int y0 = kMode == 0 ? f * kGM : f * 2 * kGM;
-        const int y1 = kMode == 0 ? f * kGM : f * 2 * kGM + kGM;
-        const int cnt = min(tl.z, kMtMaxRows);
-        const __half* xr = a.bsrc + (size_t)in_range(tl.w + tl.y, a.n_rows, a.err) * a.b_ld;
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
-            atomicOr(a.err, 16u);
-            ok = false;
-            break;
-          }
+    // lane 0 claims units, waits for free stages and issues the weight
+    // boxes; every lane issues some of the stage's activation-row copies
+    int stage = 0;
+    uint32_t phase = 0;
+    ptx::IssueLog log;
+    bool ok = true;
+    while (ok) {
+      int u = 0;
+      if (lane == 0) u = (int)atomicAdd(a.next, 1u);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (u >= n_units) break;
+      const int4 tl = __ldcg(a.tiles + u / ft);   // (expert, n0, count, r0)
+      const int f = u % ft;
+      const int cnt = min(tl.z, kMtMaxRows);
+      const __half* xr = a.bsrc + (size_t)in_range(tl.w + tl.y, a.n_rows, a.err) * a.b_ld;
+      for (int kb = 0; kb < nkb; ++kb) {
+        int free = 1;
+        if (lane == 0) free = ptx::mbar_wait(&empty[stage], phase ^ 1u) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, free, 0)) {
+          if (lane == 0) atomicOr(a.err, 16u);
+          ok = false;
+          break;
+        }
+        uint8_t* dst = sm + stage * kMtStageBytes;
+        if (lane == 0) {
+          const int ex = in_range(tl.x, a.n_ex, a.err);
+          const CUtensorMap* wm = a.wmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + ex), a.n_slots, a.err) + 3;
+          const CUtensorMap* m0 = kMode == 0 ? wm : wm + 2;
+          const CUtensorMap* m1 = kMode == 0 ? wm + 1 : wm + 2;
+          const int y0 = kMode == 0 ? f * kGM : f * 2 * kGM;
+          const int y1 = kMode == 0 ? f * kGM : f * 2 * kGM + kGM;
           s_unit[stage] = u;
           ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(kMtWBytes + cnt * 2 * kQK));
-          uint8_t* dst = sm + stage * kMtStageBytes;
           ptx::tma_load_2d(dst, m0, kb * 18, y0, &full[stage]);
           ptx::tma_load_2d(dst + kRawBytes, m1, kb * 18, y1, &full[stage]);
-          for (int n = 0; n < cnt; ++n)
-            ptx::bulk_load(dst + kMtWBytes + n * kMtXPitch, xr + (size_t)n * a.b_ld + kb * kQK, 2 * kQK,
-                           &full[stage]);
-          log.note(stage, phase);
-          if (++stage == kMtStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+        }
+        __syncwarp();   // the expected bytes are set before any row copy can complete
+        for (int n = lane; n < cnt; n += 32)
+          ptx::bulk_load(dst + kMtWBytes + n * kMtXPitch, xr + (size_t)n * a.b_ld + kb * kQK, 2 * kQK,
+                         &full[stage]);
+        log.note(stage, phase);
+        if (++stage == kMtStages) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
+    }
+    if (lane == 0) {
       if (ok) {
         // end of work: a stage with unit -1 and no bytes (its earlier issue
         // was consumed, so it leaves the drain list)

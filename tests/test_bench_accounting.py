@@ -49,10 +49,12 @@ def test_few_row_gate_up_bytes():
     assert np.all(np.sort(ids, axis=1)[:, 1:] != np.sort(ids, axis=1)[:, :-1])  # distinct picks per token
     assert int(np.sum(counts > 0)) == 44 and counts.max() == 64
     tiles, rows = 44 + 1, 64 * 9            # + the shared expert's 64 rows
-    assert bench.tile_split(cfg, ids) == (0, rows, tiles)
-    expect = tiles * 2 * gate + rows * 7168 * 2 + rows * 2048 * 4
+    assert bench.tile_split(cfg, ids, few_rows=64) == (0, rows, tiles)
+    # the library's default, 32: expert 0 and the shared expert (64 rows each) take the GEMM
+    assert bench.tile_split(cfg, ids) == (64 + 64, rows - 128, tiles - 2)
+    expect = (tiles - 2) * 2 * gate + (rows - 128) * 7168 * 2 + (rows - 128) * 2048 * 4
     assert bench.few_gate_up_bytes(cfg, ids) == expect
-    assert bench.gate_up_gemm_flops(cfg, ids) == 0.0
+    assert bench.gate_up_gemm_flops(cfg, ids) == 2.0 * 128 * 2 * 2048 * 7168
 
 
 def test_prefill_flops():
@@ -76,8 +78,10 @@ def test_traffic_entry_tracks_its_source():
 def test_tile_split_hand_count():
     # 600 = 256+256+88 (GEMM), 300 = 256 | 44, 64 (few), 65 (GEMM), 1 (few),
     # 513 = 512 | 1, 320 = 256 | 64
-    assert bench.split_rows([600, 300, 64, 65, 1, 513, 320]) == (600 + 256 + 65 + 512 + 256,
-                                                                 44 + 64 + 1 + 1 + 64, 5)
+    assert bench.split_rows([600, 300, 64, 65, 1, 513, 320], few_rows=64) == (600 + 256 + 65 + 512 + 256,
+                                                                              44 + 64 + 1 + 1 + 64, 5)
+    # the library's default, 32: 300 = 256 | 44 and 320 = 256 | 64 stay whole
+    assert bench.split_rows([600, 300, 64, 65, 1, 513, 320]) == (600 + 300 + 64 + 65 + 512 + 320, 1 + 1, 2)
     assert bench.split_rows([600, 300, 64, 65, 1, 513, 320], few_rows=0) == (1863, 0, 0)
     assert bench.split_rows([256, 257], few_rows=1) == (256 + 256, 1, 1)
 

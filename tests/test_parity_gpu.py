@@ -96,18 +96,18 @@ def test_small_every_token(torch, name, T):
     check_against_oracle(cfg, g)
 
 
-@pytest.mark.parametrize("max_rows", [0, 1, 8, 64])
+@pytest.mark.parametrize("max_rows", [0, 1, 8, 32])
 def test_few_row_tile_thresholds(torch, max_rows):
     """The prefill path with the few-row kernel off (GEMM + decode kernels),
     taking only single-row experts, the experts up to 8 rows and the last
-    partial tiles up to 8 rows, or everything up to 64 rows: every token
+    partial tiles up to 8 rows, or everything up to 32 rows: every token
     matches the oracle each way (rows per expert 1..~60 here)."""
     cfg = SMALL["ragged_inter"]
     try:
         moe.moe_set_few_row_tiles(max_rows)
         g = run_gpu(torch, cfg, 200)
     finally:
-        moe.moe_set_few_row_tiles(64)
+        moe.moe_set_few_row_tiles(32)
     check_against_oracle(cfg, g)
 
 
@@ -139,9 +139,9 @@ def prefill_sample(ids: np.ndarray, n_experts: int, tile: int = 256) -> np.ndarr
     """Tokens whose rows reach every kind of work unit of the prefill path:
     the first and last row of every 256-row tile of the three experts with
     the most rows (full GEMM tiles and their last partial tile), one token of
-    every expert with at most 64 rows (few-row tiles), and the last row of
-    every expert whose last partial tile has at most 64 rows (a few-row tile
-    after GEMM tiles).  Rows of an expert are its (token, slot) pairs in
+    every expert with at most 64 rows (few-row tiles up to 32, small GEMM
+    tiles above), and the last row of every expert whose last partial tile
+    has at most 64 rows.  Rows of an expert are its (token, slot) pairs in
     token order."""
     T, k = ids.shape
     counts = np.bincount(ids.ravel(), minlength=n_experts)
