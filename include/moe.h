@@ -113,7 +113,9 @@ typedef struct {
 /* Bytes one expert (gate + up + down, all of type `quant`) occupies in device
  * memory, i.e. one cache slot: its GGUF bytes, except that Q6_K blocks are
  * padded from 210 to 224 bytes and MXFP4 blocks grouped eight at a time from
- * 136 into 144 bytes (16-byte aligned groups for the copy engines).  0 on bad
+ * 136 into 144 bytes (16-byte aligned groups for the copy engines), and each
+ * matrix's rows are padded with zero rows to a multiple of 64 (the device
+ * layout is tile-major: 64-row tiles, stored group after group).  0 on bad
  * args.  Source: LayerStoRm README, "Get a model" (GGUF weights). */
 size_t moe_expert_bytes(int hidden, int inter, moe_quant quant);
 

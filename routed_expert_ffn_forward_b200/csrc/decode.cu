@@ -57,16 +57,14 @@ constexpr int kDnSB = 4;
 constexpr int kDnStages = 4;
 constexpr int kDnStageBytes = kTileRows * kDnSB * kQBytes;  // 36864
 
-// One row's block header and quant chunk c (32 bytes).  Rows sit 144*SB bytes
-// apart, so every 16-byte piece starts on a multiple of 8 banks: lanes of odd
-// row index g read the two halves in the opposite order, which puts the two
-// rows of an 8-lane phase on disjoint banks.
-__device__ __forceinline__ void load_row_block(const uint8_t* blk, int c, int g, uint4& hdr, uint32_t* q) {
+// One row's block header and quant chunk c (32 bytes).  A stage holds its
+// super-blocks one after another, each as 64 rows 144 bytes apart (the
+// tile-major weight layout), so the rows g of an 8-lane phase start 4 banks
+// apart and their 16-byte pieces never share a bank.
+__device__ __forceinline__ void load_row_block(const uint8_t* blk, int c, uint4& hdr, uint32_t* q) {
   hdr = *reinterpret_cast<const uint4*>(blk);
-  const int sw = g & 1;
-  const uint4 a = *reinterpret_cast<const uint4*>(blk + 16 + 32 * c + 16 * sw);
-  const uint4 b = *reinterpret_cast<const uint4*>(blk + 32 + 32 * c - 16 * sw);
-  const uint4 lo = sw ? b : a, hi = sw ? a : b;
+  const uint4 lo = *reinterpret_cast<const uint4*>(blk + 16 + 32 * c);
+  const uint4 hi = *reinterpret_cast<const uint4*>(blk + 32 + 32 * c);
   q[0] = lo.x; q[1] = lo.y; q[2] = lo.z; q[3] = lo.w;
   q[4] = hi.x; q[5] = hi.y; q[6] = hi.z; q[7] = hi.w;
 }
@@ -188,8 +186,8 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
           const int nsb = min(kGuSB, a.nbh - st * kGuSB);  // super-blocks of x this stage needs
           ptx::mbar_arrive_expect_tx(&full[stage], kGuStageBytes + (uint32_t)(cnt * nsb * (2 * kQK + 64)));
           uint8_t* dst = stages + stage * kStride;
-          ptx::tma_load_2d(dst, mg, st * kGuSB * 18, rt * kTileRows, &full[stage]);
-          ptx::tma_load_2d(dst + kGuTileBytes, mg + 1, st * kGuSB * 18, rt * kTileRows, &full[stage]);
+          ptx::tma_load_w(dst, mg, st * kGuSB, rt * kTileRows, &full[stage]);
+          ptx::tma_load_w(dst + kGuTileBytes, mg + 1, st * kGuSB, rt * kTileRows, &full[stage]);
           if (!kStageX) {
 #pragma unroll
             for (int t = 0; t < kMaxTok; ++t) {
@@ -239,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
   // super-block w>>3 of every stage
   const int mat = (warp >> 2) & 1, rbase = (warp & 3) * 16, kp = warp >> 3;
   const int g = lane >> 2, c = lane & 3;
-  const int pitch = kGuSB * kQBytes;
+  const int pitch = kQBytes;                      // rows of one super-block
   int stage = 0;
   uint32_t phase = 0;
   for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
@@ -265,11 +263,11 @@ __global__ void __launch_bounds__(kThreads, 1) gate_up_d1_kernel(DecodeArgs a) {
       const int kb = st * kGuSB + kp;
       if (kb < a.nbh) {
         const uint8_t* sbase = stages + stage * kStride;
-        const uint8_t* blk = sbase + mat * kGuTileBytes + (rbase + g) * pitch + kp * kQBytes;
+        const uint8_t* blk = sbase + mat * kGuTileBytes + kp * kTileRows * kQBytes + (rbase + g) * pitch;
         uint4 h0, h8;
         uint32_t q[8], q8[8];
-        load_row_block(blk, c, g, h0, q);
-        load_row_block(blk + 8 * pitch, c, g, h8, q8);
+        load_row_block(blk, c, h0, q);
+        load_row_block(blk + 8 * pitch, c, h8, q8);
         const RowScales rs = decode_scales(h0, c), rs8 = decode_scales(h8, c);
 #pragma unroll
         for (int t = 0; t < kMaxTok; ++t) {
@@ -394,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) down_d1_kernel(DecodeArgs a) {
             return;
           }
           ptx::mbar_arrive_expect_tx(&full[stage], kDnStageBytes);
-          ptx::tma_load_2d(stages + stage * kDnStageBytes, md, st * kDnSB * 18, rt * kTileRows, &full[stage]);
+          ptx::tma_load_w(stages + stage * kDnStageBytes, md, st * kDnSB, rt * kTileRows, &full[stage]);
           log.note(stage, phase);
           if (++stage == kDnStages) {
             stage = 0;
@@ -441,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1) down_d1_kernel(DecodeArgs a) {
   // consumers: warp w takes rows 16*(w&3).. and super-block w>>2 of every stage
   const int rbase = (warp & 3) * 16, kp = warp >> 2;
   const int g = lane >> 2, c = lane & 3;
-  const int pitch = kDnSB * kQBytes;
+  const int pitch = kQBytes;                      // rows of one super-block
   int stage = 0, slot = 0;
   uint32_t phase = 0, aphase = 0;
   for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
@@ -463,11 +461,11 @@ __global__ void __launch_bounds__(kThreads, 1) down_d1_kernel(DecodeArgs a) {
       }
       const int kb = st * kDnSB + kp;
       if (kb < a.nbi) {
-        const uint8_t* blk = stages + stage * kDnStageBytes + (rbase + g) * pitch + kp * kQBytes;
+        const uint8_t* blk = stages + stage * kDnStageBytes + kp * kTileRows * kQBytes + (rbase + g) * pitch;
         uint4 h0, h8;
         uint32_t q[8], q8[8];
-        load_row_block(blk, c, g, h0, q);
-        load_row_block(blk + 8 * pitch, c, g, h8, q8);
+        load_row_block(blk, c, h0, q);
+        load_row_block(blk + 8 * pitch, c, h8, q8);
         const RowScales rs = decode_scales(h0, c), rs8 = decode_scales(h8, c);
 #pragma unroll
         for (int t = 0; t < kMaxTok; ++t) {

@@ -126,7 +126,6 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
   const FzLayout lay(H, a.act_slot_bytes, a.stages * a.stage_bytes);
   const int n_stages = a.stages, stage_bytes = a.stage_bytes;
   const int gu_box = kFzGuRows * a.sbb_gu, dn_box = kFzDnRows * a.sbb_d;   // bytes of one box
-  const int gu_el = a.sbb_gu / 8, dn_el = a.sbb_d / 8;                    // 8-byte elements per group
   uint8_t* ring = sm;
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + lay.bars);
   uint64_t* empty = full + kFzStages;
@@ -201,8 +200,8 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * nbox * gu_box));
         uint8_t* dst = ring + stage * stage_bytes;
         for (int b = 0; b < nbox; ++b) {
-          ptx::tma_load_2d(dst + b * gu_box, m, (2 * st + b) * gu_el, rt * kFzGuRows, &full[stage]);
-          ptx::tma_load_2d(dst + (2 + b) * gu_box, m + 1, (2 * st + b) * gu_el, rt * kFzGuRows, &full[stage]);
+          ptx::tma_load_w(dst + b * gu_box, m, 2 * st + b, rt * kFzGuRows, &full[stage]);
+          ptx::tma_load_w(dst + (2 + b) * gu_box, m + 1, 2 * st + b, rt * kFzGuRows, &full[stage]);
         }
         issued |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -265,7 +264,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(nbox * dn_box));
         uint8_t* dst = ring + stage * stage_bytes;
         for (int b = 0; b < nbox; ++b)
-          ptx::tma_load_2d(dst + b * dn_box, md, (st * kFzDnSb + b) * dn_el, rt * kFzDnRows, &full[stage]);
+          ptx::tma_load_w(dst + b * dn_box, md, st * kFzDnSb + b, rt * kFzDnRows, &full[stage]);
         issued |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (phase << stage);
         next_stage();

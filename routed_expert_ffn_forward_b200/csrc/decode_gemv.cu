@@ -91,8 +91,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_gate_up_kernel(DecodeArgs 
           }
           ptx::mbar_arrive_expect_tx(&full[stage], kGvStageBytes);
           uint8_t* dst = stages + stage * kGvStageBytes;
-          ptx::tma_load_2d(dst, m, kb * 18, rt * kGvRows, &full[stage]);
-          ptx::tma_load_2d(dst + kGvBox, m + 1, kb * 18, rt * kGvRows, &full[stage]);
+          ptx::tma_load_w(dst, m, kb, rt * kGvRows, &full[stage]);
+          ptx::tma_load_w(dst + kGvBox, m + 1, kb, rt * kGvRows, &full[stage]);
           log.note(stage, phase);
           if (++stage == kGvStages) {
             stage = 0;
@@ -264,8 +264,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_down_kernel(DecodeArgs a) 
           ptx::mbar_arrive_expect_tx(&full[stage], kGvStageBytes);
           uint8_t* dst = stages + stage * kGvStageBytes;
           // a second box past the last super-block reads zeros (never used)
-          ptx::tma_load_2d(dst, md, (2 * st) * 18, rt * kGvRows, &full[stage]);
-          ptx::tma_load_2d(dst + kGvBox, md, (2 * st + 1) * 18, rt * kGvRows, &full[stage]);
+          ptx::tma_load_w(dst, md, 2 * st, rt * kGvRows, &full[stage]);
+          ptx::tma_load_w(dst + kGvBox, md, 2 * st + 1, rt * kGvRows, &full[stage]);
           log.note(stage, phase);
           if (++stage == kGvStages) {
             stage = 0;

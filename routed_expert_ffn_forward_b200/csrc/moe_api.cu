@@ -99,6 +99,7 @@ struct Cache {
   size_t slot_bytes = 0;
   int n_slots = 0;
   uint8_t* arena = nullptr;
+  uint8_t* staging = nullptr;   // one matrix in row-major device rows, before retiling (slot_bytes)
   std::vector<Slot> slots;
   std::list<int> lru;  // front = most recently used
   std::unordered_map<uint64_t, int> where;
@@ -154,6 +155,7 @@ void cache_free(Cache* c) {
     if (s.used) cudaEventDestroy(s.used);
   }
   if (c->arena) cudaFree(c->arena);
+  if (c->staging) cudaFree(c->staging);
   if (c->copy) cudaStreamDestroy(c->copy);
   delete c;
 }
@@ -331,6 +333,7 @@ moe_status ensure_cache(int device, size_t slot_bytes) {
   c->slot_bytes = slot_bytes;
   c->n_slots = (int)n;
   cudaError_t e = cudaMalloc(&c->arena, n * slot_bytes);
+  if (e == cudaSuccess) e = cudaMalloc(&c->staging, slot_bytes);
   if (e != cudaSuccess) {
     cache_free(c);
     return fail(MOE_ERR_OOM, "cache arena of %zu slots x %zu B: %s", n, slot_bytes, cudaGetErrorString(e));
@@ -416,9 +419,11 @@ moe_status cache_fetch(moe_layer* L, int e, uint64_t pin_epoch, bool prefetch, i
     uint8_t* dst = c->arena + (size_t)s * c->slot_bytes;
     const uint8_t* const* hp = &L->host[3 * (size_t)e];
     const Shape& sh = L->s;
-    CUDA_TRY(copy_matrix_h2d(dst, hp[0], sh.I, sh.qgu, sh.hrow_gu, sh.drow_gu, c->copy));
-    CUDA_TRY(copy_matrix_h2d(dst + L->gate_bytes, hp[1], sh.I, sh.qgu, sh.hrow_gu, sh.drow_gu, c->copy));
-    CUDA_TRY(copy_matrix_h2d(dst + 2 * L->gate_bytes, hp[2], sh.H, sh.qd, sh.hrow_d, sh.drow_d, c->copy));
+    CUDA_TRY(upload_matrix(dst, hp[0], sh.I, sh.qgu, sh.hrow_gu, sh.drow_gu, sh.nbh, sh.sbb_gu, c->staging, c->copy));
+    CUDA_TRY(upload_matrix(dst + L->gate_bytes, hp[1], sh.I, sh.qgu, sh.hrow_gu, sh.drow_gu, sh.nbh, sh.sbb_gu,
+                           c->staging, c->copy));
+    CUDA_TRY(upload_matrix(dst + 2 * L->gate_bytes, hp[2], sh.H, sh.qd, sh.hrow_d, sh.drow_d, sh.nbi, sh.sbb_d,
+                           c->staging, c->copy));
     CUDA_TRY(cudaEventRecord(sl.ready, c->copy));
     sl.ready_rec = true;
     sl.key = key;
@@ -853,7 +858,7 @@ size_t moe_expert_bytes(int hidden, int inter, moe_quant quant) {
   if (!dev_sb_bytes(q) || hidden <= 0 || inter <= 0 || hidden % kQK) return 0;
   if (host_block_elems(q) != kQK && inter % kQK) return 0;
   const size_t nbh = hidden / kQK, nbi = (inter + kQK - 1) / kQK;
-  return 2 * (size_t)inter * nbh * dev_sb_bytes(q) + (size_t)hidden * nbi * dev_sb_bytes(q);
+  return 2 * tiled_matrix_bytes(inter, nbh * dev_sb_bytes(q)) + tiled_matrix_bytes(hidden, nbi * dev_sb_bytes(q));
 }
 
 moe_status moe_layer_create(int hidden, int inter, int n_experts, int top_k, int n_shared,
@@ -898,8 +903,8 @@ moe_status moe_layer_create_mixed(int hidden, int inter, int n_experts, int top_
   s.hrow_d = (size_t)((inter + host_block_elems(qd) - 1) / host_block_elems(qd)) * host_block_bytes(qd);
   s.drow_gu = (size_t)s.nbh * s.sbb_gu;
   s.drow_d = (size_t)s.nbi * s.sbb_d;
-  L->gate_bytes = (size_t)inter * s.drow_gu;
-  L->down_bytes = (size_t)hidden * s.drow_d;
+  L->gate_bytes = tiled_matrix_bytes(inter, s.drow_gu);
+  L->down_bytes = tiled_matrix_bytes(hidden, s.drow_d);
   L->expert_bytes = 2 * L->gate_bytes + L->down_bytes;
   L->host_expert_bytes = 2 * (size_t)inter * s.hrow_gu + (size_t)hidden * s.hrow_d;
   cudaError_t e = cudaGetDevice(&L->device);
@@ -1036,15 +1041,23 @@ moe_status moe_set_experts(moe_layer_t L, const void* const* gate, const void* c
   if (budget == SIZE_MAX) {
     // resident: one device copy of every expert, uploaded now
     if (!L->d_resident) CUDA_TRY(cudaMalloc(&L->d_resident, (size_t)n * L->expert_bytes));
-    for (int e = 0; e < n; ++e) {
+    uint8_t* staging = nullptr;   // one matrix before retiling, freed once the uploads are done
+    CUDA_TRY(cudaMalloc(&staging, std::max(L->gate_bytes, L->down_bytes)));
+    cudaError_t ue = cudaSuccess;
+    for (int e = 0; e < n && ue == cudaSuccess; ++e) {
       uint8_t* dst = L->d_resident + (size_t)e * L->expert_bytes;
       const size_t off[3] = {0, L->gate_bytes, 2 * L->gate_bytes};
       const int rows[3] = {L->s.I, L->s.I, L->s.H}, q[3] = {L->s.qgu, L->s.qgu, L->s.qd};
+      const int nb[3] = {L->s.nbh, L->s.nbh, L->s.nbi}, sbb[3] = {L->s.sbb_gu, L->s.sbb_gu, L->s.sbb_d};
       const size_t hrow[3] = {L->s.hrow_gu, L->s.hrow_gu, L->s.hrow_d}, drow[3] = {L->s.drow_gu, L->s.drow_gu, L->s.drow_d};
-      for (int m = 0; m < 3; ++m)
-        CUDA_TRY(copy_matrix_h2d(dst + off[m], L->host[3 * (size_t)e + m], rows[m], q[m], hrow[m], drow[m], L->copy));
+      for (int m = 0; m < 3 && ue == cudaSuccess; ++m)
+        ue = upload_matrix(dst + off[m], L->host[3 * (size_t)e + m], rows[m], q[m], hrow[m], drow[m], nb[m], sbb[m],
+                           staging, L->copy);
     }
-    CUDA_TRY(cudaStreamSynchronize(L->copy));
+    const cudaError_t se = cudaStreamSynchronize(L->copy);
+    cudaFree(staging);
+    CUDA_TRY(ue);
+    CUDA_TRY(se);
     MOE_TRY(build_maps(L, L->d_resident, L->expert_bytes, (size_t)n));
     std::vector<int> ident(n);
     for (int e = 0; e < n; ++e) ident[e] = e;

@@ -187,6 +187,16 @@ cudaError_t launch_decode1_fused(const FusedArgs& a, int n_sm, cudaStream_t st);
 constexpr int kMapsPerSlot = 9;
 struct Shape;
 cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, const Shape& s);
+// Weight matrices live in device memory tile-major (tiles of kWTile rows; see
+// tmap.cu): bytes of a matrix of `rows` rows of drow device bytes.
+constexpr int kWTile = 64;
+inline size_t tiled_matrix_bytes(int rows, size_t drow) { return (size_t)((rows + kWTile - 1) / kWTile) * kWTile * drow; }
+// Upload one matrix: its GGUF host rows into `staging` (row-major device
+// rows, copy_matrix_h2d), then a kernel rewrites them tile-major into `dst`;
+// both on `st`, so `staging` is free again once `st` has reached the next
+// upload.  drow = nb * sbb.
+cudaError_t upload_matrix(uint8_t* dst, const uint8_t* src, int rows, int q, size_t hrow, size_t drow, int nb,
+                          int sbb, uint8_t* staging, cudaStream_t st);
 // Copy one weight matrix of `rows` rows from its GGUF host bytes into the
 // device layout of its type (dev_sb_bytes), asynchronously on `st`.
 cudaError_t copy_matrix_h2d(uint8_t* dst, const uint8_t* src, int rows, int q, size_t hrow, size_t drow,

@@ -243,8 +243,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) q4k_gemm_kernel(const __grid_
             goto raw_drain;
           }
           ptx::mbar_arrive_expect_tx(&raw_full[rs], 2 * kRawBytes);
-          ptx::tma_load_2d(s_rawbuf + (2 * rs) * kRawBytes, m0, kb * 18, y0, &raw_full[rs]);
-          ptx::tma_load_2d(s_rawbuf + (2 * rs + 1) * kRawBytes, m1, kb * 18, y1, &raw_full[rs]);
+          ptx::tma_load_w(s_rawbuf + (2 * rs) * kRawBytes, m0, kb, y0, &raw_full[rs]);
+          ptx::tma_load_w(s_rawbuf + (2 * rs + 1) * kRawBytes, m1, kb, y1, &raw_full[rs]);
           issued |= 1u << rs;
           last_ph = (last_ph & ~(1u << rs)) | (rph << rs);
           if (++rs == kNR) { rs = 0; rph ^= 1u; }
@@ -622,8 +622,8 @@ __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a)
           const int y1 = kMode == 0 ? f * kGM : f * 2 * kGM + kGM;
           s_unit[stage] = u;
           ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(kMtWBytes + cnt * 2 * kQK));
-          ptx::tma_load_2d(dst, m0, kb * 18, y0, &full[stage]);
-          ptx::tma_load_2d(dst + kRawBytes, m1, kb * 18, y1, &full[stage]);
+          ptx::tma_load_w(dst, m0, kb, y0, &full[stage]);
+          ptx::tma_load_w(dst + kRawBytes, m1, kb, y1, &full[stage]);
         }
         __syncwarp();   // the expected bytes are set before any row copy can complete
         for (int n = lane; n < cnt; n += 32)

@@ -148,6 +148,15 @@ struct IssueLog {
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
+// One box of a tile-major weight matrix (tmap.cu): groups from sb0 and tiles
+// from row0 / 64 (row0 a multiple of 64), as many as the map's box holds.
+__device__ __forceinline__ void tma_load_w(void* smem_dst, const CUtensorMap* map, int sb0, int row0, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(0), "r"(sb0), "r"(row0 >> 6),
+        "r"(smem_u32(bar))
+      : "memory");
+}
 // Bring box (x, y) of `map` into L2 (no shared memory, no completion to wait for).
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"

@@ -44,6 +44,7 @@ def test_every_declared_symbol_is_exported(lib):
 def test_expert_bytes():
     assert moe.moe_expert_bytes(7168, 2048) == 24_772_608
     assert moe.moe_expert_bytes(256, 128) == 2 * 128 * 144 + 256 * 1 * 144
+    assert moe.moe_expert_bytes(256, 100) == 2 * 128 * 144 + 256 * 1 * 144   # rows padded to 64
     assert moe.moe_expert_bytes(300, 128) == 0          # hidden not a multiple of 256
     assert moe.moe_expert_bytes(256, 128, 2) == 0       # not Q4_K
 
