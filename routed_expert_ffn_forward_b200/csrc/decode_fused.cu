@@ -400,10 +400,14 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
     }
   }
 
-  // (2) x as 16-bit fixed point per 32-element run (each CTA its own copy)
-  {
+  // (2) x as 16-bit fixed point per 32-element run (each CTA its own copy),
+  // by warps w0 .. 15: all of them before this CTA's shared-expert units,
+  // else warps 1-15 while warp 0 polls the logits
+  int n_sh = 0;   // this CTA's shared gate/up units (the producer skips the same ones)
+  for (int u = blockIdx.x; u < n_gu_sh; u += gridDim.x) n_sh += ep_owned(E + u / gu_tiles, a.ep_rank, a.ep_world);
+  auto quant_x = [&](int w0) {
     const __nv_bfloat16* s_x = reinterpret_cast<const __nv_bfloat16*>(s_uni);
-    for (int run = warp; run < H / 32; run += kFzWarps) {
+    for (int run = warp - w0; run < H / 32; run += kFzWarps - w0) {
       float2 rsc;
       int8_t xh;
       uint8_t xl;
@@ -412,6 +416,9 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
       s_xl[run * 32 + lane] = xl;
       if (lane == 0) s_xsc[run] = rsc;
     }
+  };
+  if (n_sh > 0) {
+    quant_x(0);
     cbar();
   }
 
@@ -424,7 +431,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
       // a test hook that makes the wait run out), copied to shared memory
       const uint32_t want = (uint32_t)(s_epoch + 1u + (uint64_t)a.hold);
       const uint64_t* lg = reinterpret_cast<const uint64_t*>(sync + kSyncLogits);
-      float* s_lg = reinterpret_cast<float*>(s_uni);   // x (bf16) is no longer needed there
+      float* s_lg = s_part;   // free: no unit is in progress
       const uint64_t t0 = ptx::globaltimer();
       while (true) {
         bool mine = true;
@@ -438,13 +445,14 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
           break;
         }
         if (ptx::globaltimer() - t0 > lim) break;
-        __nanosleep(32);
       }
       if (!got && lane == 0) fail(kErrFzGrid);
       __syncwarp();
+    } else if (n_sh == 0) {
+      quant_x(1);
     }
     if (got) {
-      warp_topk_gate<PL, false>(reinterpret_cast<const float*>(s_uni), E, k, a.gating, a.forced, s_ids, s_w);
+      warp_topk_gate<PL, false>(s_part, E, k, a.gating, a.forced, s_ids, s_w);
       __syncwarp();
       if (lane < S) {
         s_ids[k + lane] = E + lane;
@@ -479,8 +487,6 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
   // units and down units as claimed.  The routing is needed from the first
   // unit after the shared ones on.
   {
-    int n_sh = 0;   // this CTA's shared gate/up units (the producer skips the same ones)
-    for (int u = blockIdx.x; u < n_gu_sh; u += gridDim.x) n_sh += ep_owned(E + u / gu_tiles, a.ep_rank, a.ep_world);
     const int g_row = (warp & 1) * 32 + lane, g_sb = (warp >> 1) & 1, g_c = warp >> 2;   // gate/up: row, column, chunk
     const int r0 = lane, sb = warp >> 2, c = warp & 3;                                    // down: rows r0, r0 + 32
     const int I_pad = a.I_pad;

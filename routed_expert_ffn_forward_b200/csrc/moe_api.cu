@@ -99,7 +99,14 @@ struct Cache {
   size_t slot_bytes = 0;
   int n_slots = 0;
   uint8_t* arena = nullptr;
-  uint8_t* staging = nullptr;   // one matrix in row-major device rows, before retiling (slot_bytes)
+  // Uploads: the copy engine writes a matrix's host rows into staging[b] on
+  // `copy` while the previous matrix is retiled from staging[b ^ 1] into its
+  // slot on `retile`; events keep each buffer's two users in order.
+  uint8_t* staging[2] = {nullptr, nullptr};   // slot_bytes each
+  cudaStream_t retile = nullptr;
+  cudaEvent_t copied[2] = {nullptr, nullptr}, retiled[2] = {nullptr, nullptr};
+  bool retiled_rec[2] = {false, false};
+  uint64_t uploads = 0;
   std::vector<Slot> slots;
   std::list<int> lru;  // front = most recently used
   std::unordered_map<uint64_t, int> where;
@@ -155,8 +162,13 @@ void cache_free(Cache* c) {
     if (s.used) cudaEventDestroy(s.used);
   }
   if (c->arena) cudaFree(c->arena);
-  if (c->staging) cudaFree(c->staging);
+  for (int b = 0; b < 2; ++b) {
+    if (c->staging[b]) cudaFree(c->staging[b]);
+    if (c->copied[b]) cudaEventDestroy(c->copied[b]);
+    if (c->retiled[b]) cudaEventDestroy(c->retiled[b]);
+  }
   if (c->copy) cudaStreamDestroy(c->copy);
+  if (c->retile) cudaStreamDestroy(c->retile);
   delete c;
 }
 
@@ -333,12 +345,17 @@ moe_status ensure_cache(int device, size_t slot_bytes) {
   c->slot_bytes = slot_bytes;
   c->n_slots = (int)n;
   cudaError_t e = cudaMalloc(&c->arena, n * slot_bytes);
-  if (e == cudaSuccess) e = cudaMalloc(&c->staging, slot_bytes);
+  for (int b = 0; b < 2 && e == cudaSuccess; ++b) {
+    e = cudaMalloc(&c->staging[b], slot_bytes);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->copied[b], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->retiled[b], cudaEventDisableTiming);
+  }
   if (e != cudaSuccess) {
     cache_free(c);
     return fail(MOE_ERR_OOM, "cache arena of %zu slots x %zu B: %s", n, slot_bytes, cudaGetErrorString(e));
   }
   e = cudaStreamCreateWithFlags(&c->copy, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->retile, cudaStreamNonBlocking);
   c->slots.resize(n);
   for (size_t i = 0; i < n && e == cudaSuccess; ++i) {
     e = cudaEventCreateWithFlags(&c->slots[i].ready, cudaEventDisableTiming);
@@ -415,16 +432,26 @@ moe_status cache_fetch(moe_layer* L, int e, uint64_t pin_epoch, bool prefetch, i
       c->where.erase(sl.key);
       g_stats.evictions++;
     }
-    if (sl.used_rec) CUDA_TRY(cudaStreamWaitEvent(c->copy, sl.used, 0));
+    // the slot's last reader has finished before the retile writes it
+    if (sl.used_rec) CUDA_TRY(cudaStreamWaitEvent(c->retile, sl.used, 0));
     uint8_t* dst = c->arena + (size_t)s * c->slot_bytes;
     const uint8_t* const* hp = &L->host[3 * (size_t)e];
     const Shape& sh = L->s;
-    CUDA_TRY(upload_matrix(dst, hp[0], sh.I, sh.qgu, sh.hrow_gu, sh.drow_gu, sh.nbh, sh.sbb_gu, c->staging, c->copy));
-    CUDA_TRY(upload_matrix(dst + L->gate_bytes, hp[1], sh.I, sh.qgu, sh.hrow_gu, sh.drow_gu, sh.nbh, sh.sbb_gu,
-                           c->staging, c->copy));
-    CUDA_TRY(upload_matrix(dst + 2 * L->gate_bytes, hp[2], sh.H, sh.qd, sh.hrow_d, sh.drow_d, sh.nbi, sh.sbb_d,
-                           c->staging, c->copy));
-    CUDA_TRY(cudaEventRecord(sl.ready, c->copy));
+    const size_t off[3] = {0, L->gate_bytes, 2 * L->gate_bytes};
+    const int rows[3] = {sh.I, sh.I, sh.H}, q[3] = {sh.qgu, sh.qgu, sh.qd};
+    const int nb[3] = {sh.nbh, sh.nbh, sh.nbi}, sbb[3] = {sh.sbb_gu, sh.sbb_gu, sh.sbb_d};
+    const size_t hrow[3] = {sh.hrow_gu, sh.hrow_gu, sh.hrow_d}, drow[3] = {sh.drow_gu, sh.drow_gu, sh.drow_d};
+    for (int m = 0; m < 3; ++m) {
+      const int b = (int)(c->uploads++ & 1u);
+      if (c->retiled_rec[b]) CUDA_TRY(cudaStreamWaitEvent(c->copy, c->retiled[b], 0));   // staging[b] read
+      CUDA_TRY(copy_matrix_h2d(c->staging[b], hp[m], rows[m], q[m], hrow[m], drow[m], c->copy));
+      CUDA_TRY(cudaEventRecord(c->copied[b], c->copy));
+      CUDA_TRY(cudaStreamWaitEvent(c->retile, c->copied[b], 0));
+      CUDA_TRY(launch_retile(c->staging[b], dst + off[m], rows[m], nb[m], sbb[m], c->retile));
+      CUDA_TRY(cudaEventRecord(c->retiled[b], c->retile));
+      c->retiled_rec[b] = true;
+    }
+    CUDA_TRY(cudaEventRecord(sl.ready, c->retile));
     sl.ready_rec = true;
     sl.key = key;
     c->where[key] = s;

@@ -197,6 +197,9 @@ inline size_t tiled_matrix_bytes(int rows, size_t drow) { return (size_t)((rows 
 // upload.  drow = nb * sbb.
 cudaError_t upload_matrix(uint8_t* dst, const uint8_t* src, int rows, int q, size_t hrow, size_t drow, int nb,
                           int sbb, uint8_t* staging, cudaStream_t st);
+// The second half of upload_matrix alone: row-major device rows in `staging`
+// rewritten tile-major into `dst` on `st`.
+cudaError_t launch_retile(const uint8_t* staging, uint8_t* dst, int rows, int nb, int sbb, cudaStream_t st);
 // Copy one weight matrix of `rows` rows from its GGUF host bytes into the
 // device layout of its type (dev_sb_bytes), asynchronously on `st`.
 cudaError_t copy_matrix_h2d(uint8_t* dst, const uint8_t* src, int rows, int q, size_t hrow, size_t drow,

@@ -93,15 +93,19 @@ __global__ void __launch_bounds__(256) retile_kernel(const uint4* __restrict__ s
 
 }  // namespace
 
-cudaError_t upload_matrix(uint8_t* dst, const uint8_t* src, int rows, int q, size_t hrow, size_t drow, int nb,
-                          int sbb, uint8_t* staging, cudaStream_t st) {
-  if (drow != (size_t)nb * sbb || sbb % 16) return cudaErrorInvalidValue;
-  cudaError_t e = copy_matrix_h2d(staging, src, rows, q, hrow, drow, st);
-  if (e != cudaSuccess) return e;
+cudaError_t launch_retile(const uint8_t* staging, uint8_t* dst, int rows, int nb, int sbb, cudaStream_t st) {
+  if (sbb % 16 || rows <= 0 || nb <= 0) return cudaErrorInvalidValue;
   const int tiles = (rows + kWTile - 1) / kWTile;
   retile_kernel<<<tiles * nb, 256, 0, st>>>(reinterpret_cast<const uint4*>(staging), reinterpret_cast<uint4*>(dst),
                                             rows, nb, sbb);
   return cudaGetLastError();
+}
+
+cudaError_t upload_matrix(uint8_t* dst, const uint8_t* src, int rows, int q, size_t hrow, size_t drow, int nb,
+                          int sbb, uint8_t* staging, cudaStream_t st) {
+  if (drow != (size_t)nb * sbb) return cudaErrorInvalidValue;
+  cudaError_t e = copy_matrix_h2d(staging, src, rows, q, hrow, drow, st);
+  return e == cudaSuccess ? launch_retile(staging, dst, rows, nb, sbb, st) : e;
 }
 
 cudaError_t copy_matrix_h2d(uint8_t* dst, const uint8_t* src, int rows, int q, size_t hrow, size_t drow,
