@@ -221,7 +221,8 @@ moe_status moe_set_cache_policy(int policy);
  * block, whatever the row count.  Both compute the same fp16 products with
  * fp32 accumulation; the rounding order differs.  0 = off: all tiles on the
  * GEMM and experts with <= 4 rows on the decode kernels.
- * Default 32; errors: INVALID_ARG outside 0..32.
+ * Up to 32 rows the kernel keeps 4 stages in flight, above 3.
+ * Default 32; errors: INVALID_ARG outside 0..64.
  * Source: LayerStoRm README, "Notes" (decode and prefill throughput measured
  * on the boot-verified configuration: both paths are the product). */
 moe_status moe_set_few_row_tiles(int max_rows);

@@ -82,7 +82,7 @@ size_t g_cache_bytes = SIZE_MAX;
 int g_cache_policy = MOE_CACHE_LRU;
 uint64_t g_hook_wait_ns = 0;  // moe_set_test_hooks
 int g_hook_hold = 0;
-int g_mt_rows = kMtMaxRows;    // moe_set_few_row_tiles
+int g_mt_rows = kMtDefaultRows;   // moe_set_few_row_tiles
 uint32_t g_next_layer_id = 1;
 
 struct Slot {
@@ -829,7 +829,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     gm.bsrc = wk.x16;
     gm.b_ld = s.H;
     gm.next = wk.mt_next;
-    if (mt_rows) MOE_KERNEL(MOE_K_FEW_GATE_UP, launch_prefill_mt(0, gm, s.n_sm, st));
+    if (mt_rows) MOE_KERNEL(MOE_K_FEW_GATE_UP, launch_prefill_mt(0, gm, s.n_sm, st, mt_rows));
     if (split_small) MOE_KERNEL(MOE_K_SMALL, launch_gate_up_d1(da, kD1MaxTok, s.n_sm, st));
     MOE_KERNEL(MOE_K_PREP, launch_convert_h(wk, P, s.I, s.I_pad, st));
     ga.ft = s.H / 256;
@@ -848,7 +848,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     gm.bsrc = wk.h16;
     gm.b_ld = s.I_pad;
     gm.next = wk.mt_next + 1;
-    if (mt_rows) MOE_KERNEL(MOE_K_FEW_DOWN, launch_prefill_mt(1, gm, s.n_sm, st));
+    if (mt_rows) MOE_KERNEL(MOE_K_FEW_DOWN, launch_prefill_mt(1, gm, s.n_sm, st, mt_rows));
     if (split_small) MOE_KERNEL(MOE_K_SMALL, launch_down_d1(da, kD1MaxTok, s.n_sm, st));
     MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true, partial, L->ep_rank, L->ep_world));
   }

@@ -254,7 +254,8 @@ struct GemmArgs {
   unsigned* next;
   int n_rows;                // activation rows P (debug builds)
 };
-constexpr int kMtMaxRows = 32;   // most activation rows of a few-row tile
+constexpr int kMtMaxRows = 64;   // most activation rows of a few-row tile (builds for 32 and 64)
+constexpr int kMtDefaultRows = 32;
 size_t prefill_gemm_smem();
 size_t prefill_max_tiles(int n_experts_total, size_t pairs);
 // GEMM tiles of up to 256 rows for the experts with more than small_rows rows
@@ -269,7 +270,7 @@ cudaError_t launch_convert_h(const Work& wk, int P, int I, int I_pad, cudaStream
 cudaError_t launch_prefill_gemm(int mode, const CUtensorMap& bmap, const GemmArgs& a, int n_sm, cudaStream_t st);
 // The few-row tiles (a.tiles / a.n_tiles = the mtiles list) of mode 0 (gate/up)
 // or 1 (down), same outputs as the GEMM.
-cudaError_t launch_prefill_mt(int mode, const GemmArgs& a, int n_sm, cudaStream_t st);
+cudaError_t launch_prefill_mt(int mode, const GemmArgs& a, int n_sm, cudaStream_t st, int max_rows);
 size_t route_decode_smem(int H, int T, int E, int k, int S);
 
 struct Shape {

@@ -434,13 +434,17 @@ done:
 // the activations are stored within every group of four.
 constexpr int kMtWarps = 16;
 constexpr int kMtThreads = (kMtWarps + 1) * 32;          // + one producer warp
-constexpr int kMtStages = 4;
 constexpr int kMtWBytes = 2 * kRawBytes;                 // 256 weight rows x 1 super-block
 constexpr int kMtXPitch = 2 * kQK + 32;                  // one activation row's 256 fp16, padded
-constexpr int kMtStageBytes = kMtWBytes + kMtMaxRows * kMtXPitch;
-constexpr size_t kMtSmem = 1024 + (size_t)kMtStages * kMtStageBytes + 16 * kMtStages + 16 * kMtStages;
-static_assert(kMtSmem <= 227 * 1024, "few-row kernel shared memory");
-static_assert(kMtStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
+// Two builds: tiles of at most 32 rows with 4 stages, at most 64 with 3
+template <int kRows>
+struct MtCfg {
+  static constexpr int kStages = kRows <= 32 ? 4 : 3;
+  static constexpr int kStageBytes = kMtWBytes + kRows * kMtXPitch;
+  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 32 * kStages;
+  static_assert(kSmem <= 227 * 1024, "few-row kernel shared memory");
+  static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
+};
 
 struct MtRows {
   int boxA, boxB, rowA, rowB;   // the 128-row box and row in it of M-tile rows g and g + 8
@@ -449,7 +453,7 @@ struct MtRows {
 // One work unit of the few-row kernel for one consumer warp: nkb stages of
 // MMAs into NT N tiles, then the epilogue.  Returns false if a stage never
 // arrived (error flag set).
-template <int kMode, int NT>
+template <int kMode, int kRows, int NT>
 __device__ __forceinline__ bool mt_unit(const GemmArgs& a, const uint8_t* sm, uint64_t* full, uint64_t* empty,
                                         int& stage, uint32_t& phase, const int4 tl, int f, int warp, int lane,
                                         const MtRows& rw) {
@@ -459,7 +463,8 @@ __device__ __forceinline__ bool mt_unit(const GemmArgs& a, const uint8_t* sm, ui
   const __half2 off_lo = __float2half2_rn(1024.f), off_hi = __float2half2_rn(64.f);
   const __half2 kNeg2 = __float2half2_rn(-1.f);
   const int ex = in_range(tl.x, a.n_ex, a.err);
-  const int cnt = min(tl.z, kMtMaxRows);
+  using C = MtCfg<kRows>;
+  const int cnt = min(tl.z, kRows);
   // weight rows of this thread and their 2^k scales
   const int8_t* wx = a.wexp + (size_t)ex * a.wexp_stride;
   int wrA, wrB, oA, oB;   // wexp rows; output columns
@@ -485,7 +490,7 @@ __device__ __forceinline__ bool mt_unit(const GemmArgs& a, const uint8_t* sm, ui
       atomicOr(a.err, 64u);
       return false;
     }
-    const uint32_t st = ptx::smem_u32(sm) + (uint32_t)(stage * kMtStageBytes);
+    const uint32_t st = ptx::smem_u32(sm) + (uint32_t)(stage * C::kStageBytes);
     const uint32_t rA = st + offA, rB = st + offB;
     const uint32_t xs = st + kMtWBytes + g * kMtXPitch + 8 * c4;   // token row g of N tile 0
     const uint4 hA = ptx::lds_v4(rA), hB = ptx::lds_v4(rB);
@@ -534,7 +539,7 @@ __device__ __forceinline__ bool mt_unit(const GemmArgs& a, const uint8_t* sm, ui
     }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(&empty[stage]);
-    if (++stage == kMtStages) {
+    if (++stage == C::kStages) {
       stage = 0;
       phase ^= 1u;
     }
@@ -566,8 +571,10 @@ __device__ __forceinline__ bool mt_unit(const GemmArgs& a, const uint8_t* sm, ui
   return true;
 }
 
-template <int kMode>
+template <int kMode, int kRows>
 __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a) {
+  using C = MtCfg<kRows>;
+  constexpr int kMtStages = C::kStages, kMtStageBytes = C::kStageBytes;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + kMtStages * kMtStageBytes);
@@ -602,7 +609,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a)
       if (u >= n_units) break;
       const int4 tl = __ldcg(a.tiles + u / ft);   // (expert, n0, count, r0)
       const int f = u % ft;
-      const int cnt = min(tl.z, kMtMaxRows);
+      const int cnt = min(tl.z, kRows);
       const __half* xr = a.bsrc + (size_t)in_range(tl.w + tl.y, a.n_rows, a.err) * a.b_ld;
       for (int kb = 0; kb < nkb; ++kb) {
         int free = 1;
@@ -674,17 +681,17 @@ __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a)
     if (u < 0) break;
     const int4 tl = __ldcg(a.tiles + u / ft);
     const int f = u % ft;
-    const int nt = (min(tl.z, kMtMaxRows) + 7) >> 3;
+    const int nt = (min(tl.z, kRows) + 7) >> 3;
     // one instantiation per N-tile count: no MMA is issued for an empty N tile
     switch (nt) {
-      case 1: ok = mt_unit<kMode, 1>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
-      case 2: ok = mt_unit<kMode, 2>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
-      case 3: ok = mt_unit<kMode, 3>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
-      case 4: ok = mt_unit<kMode, 4>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
-      case 5: ok = mt_unit<kMode, 5>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
-      case 6: ok = mt_unit<kMode, 6>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
-      case 7: ok = mt_unit<kMode, 7>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
-      default: ok = mt_unit<kMode, 8>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 1: ok = mt_unit<kMode, kRows, (1 <= kRows / 8 ? 1 : kRows / 8)>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 2: ok = mt_unit<kMode, kRows, (2 <= kRows / 8 ? 2 : kRows / 8)>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 3: ok = mt_unit<kMode, kRows, (3 <= kRows / 8 ? 3 : kRows / 8)>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 4: ok = mt_unit<kMode, kRows, (4 <= kRows / 8 ? 4 : kRows / 8)>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 5: ok = mt_unit<kMode, kRows, (5 <= kRows / 8 ? 5 : kRows / 8)>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 6: ok = mt_unit<kMode, kRows, (6 <= kRows / 8 ? 6 : kRows / 8)>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      case 7: ok = mt_unit<kMode, kRows, (7 <= kRows / 8 ? 7 : kRows / 8)>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
+      default: ok = mt_unit<kMode, kRows, kRows / 8>(a, sm, full, empty, stage, phase, tl, f, warp, lane, rw); break;
     }
     if (!ok) break;
   }
@@ -972,19 +979,24 @@ cudaError_t launch_convert_h(const Work& wk, int P, int I, int I_pad, cudaStream
                     wk.hinv);
 }
 
-cudaError_t launch_prefill_mt(int mode, const GemmArgs& a, int n_sm, cudaStream_t st) {
-  static uint64_t attr_done[2] = {0, 0};  // per mode, one bit per device
+cudaError_t launch_prefill_mt(int mode, const GemmArgs& a, int n_sm, cudaStream_t st, int max_rows) {
+  static uint64_t attr_done[4] = {0, 0, 0, 0};  // per (mode, build), one bit per device
+  if (max_rows < 1 || max_rows > kMtMaxRows) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
-  auto kern = mode == 0 ? q4k_mt_kernel<0> : q4k_mt_kernel<1>;
-  if (!(attr_done[mode & 1] & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMtSmem);
+  const bool wide = max_rows > 32;
+  const int v = (mode & 1) * 2 + (wide ? 1 : 0);
+  void (*kern)(const GemmArgs) = wide ? (mode == 0 ? q4k_mt_kernel<0, 64> : q4k_mt_kernel<1, 64>)
+                                      : (mode == 0 ? q4k_mt_kernel<0, 32> : q4k_mt_kernel<1, 32>);
+  const size_t smem = wide ? MtCfg<64>::kSmem : MtCfg<32>::kSmem;
+  if (!(attr_done[v] & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attr_done[mode & 1] |= bit;
+    attr_done[v] |= bit;
   }
-  return launch_pdl(kern, dim3(n_sm), dim3(kMtThreads), kMtSmem, st, a);
+  return launch_pdl(kern, dim3(n_sm), dim3(kMtThreads), smem, st, a);
 }
 
 cudaError_t launch_prefill_gemm(int mode, const CUtensorMap& bmap, const GemmArgs& a, int n_sm, cudaStream_t st) {

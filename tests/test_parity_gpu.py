@@ -96,11 +96,12 @@ def test_small_every_token(torch, name, T):
     check_against_oracle(cfg, g)
 
 
-@pytest.mark.parametrize("max_rows", [0, 1, 8, 32])
+@pytest.mark.parametrize("max_rows", [0, 1, 8, 32, 64])
 def test_few_row_tile_thresholds(torch, max_rows):
     """The prefill path with the few-row kernel off (GEMM + decode kernels),
     taking only single-row experts, the experts up to 8 rows and the last
-    partial tiles up to 8 rows, or everything up to 32 rows: every token
+    partial tiles up to 8 rows, or everything up to 32 or 64 rows (the two
+    builds of the kernel): every token
     matches the oracle each way (rows per expert 1..~60 here)."""
     cfg = SMALL["ragged_inter"]
     try:
