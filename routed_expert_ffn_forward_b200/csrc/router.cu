@@ -64,21 +64,35 @@ __global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int 
                      ids + (size_t)t * k, w + (size_t)t * k);
 }
 
-// One block per token: the block sums the token's logits over the K splits in
-// split order and adds the bias (writing them to `logits` and shared memory),
-// then warp 0 selects and gates.
-constexpr int kSumThreads = 128;
+// One block per token: four groups of 256 threads each sum a quarter of the
+// K splits (in split order) for every expert, the quarters are added in
+// order and the bias after them (writing the logits to `logits` and shared
+// memory), then warp 0 selects and gates.  Splitting the sum puts four times
+// as many of the partial-logit loads in flight (at T = 64 there are 112
+// splits).
+constexpr int kSumThreads = 1024, kSumGroups = 4, kSumGroup = kSumThreads / kSumGroups;
 template <int PL>
 __global__ void __launch_bounds__(kSumThreads)
     topk_sum_kernel(float* __restrict__ logits, int E, int k, int gating, const int* __restrict__ forced,
                     int* __restrict__ ids, float* __restrict__ w, const float* __restrict__ part, int nsplit,
                     size_t split_stride, const float* __restrict__ bias) {
   __shared__ float s_l[32 * PL];
+  __shared__ float s_q[kSumGroups][32 * PL];
   const int t = blockIdx.x;
-  for (int e = threadIdx.x; e < E; e += kSumThreads) {
+  const int q = threadIdx.x / kSumGroup, lt = threadIdx.x - q * kSumGroup;
+  const int s0 = q * nsplit / kSumGroups, s1 = (q + 1) * nsplit / kSumGroups;
+  for (int e = lt; e < E; e += kSumGroup) {
     const float* p = part + (size_t)t * E + e;
-    float v = p[0];
-    for (int s = 1; s < nsplit; ++s) v += p[(size_t)s * split_stride];
+    float v = 0.f;
+#pragma unroll 8
+    for (int s = s0; s < s1; ++s) v += p[(size_t)s * split_stride];
+    s_q[q][e] = v;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kSumThreads) {
+    float v = s_q[0][e];
+#pragma unroll
+    for (int g = 1; g < kSumGroups; ++g) v += s_q[g][e];
     v += bias ? bias[e] : 0.f;
     logits[(size_t)t * E + e] = v;
     s_l[e] = v;
