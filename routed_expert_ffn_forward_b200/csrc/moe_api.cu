@@ -259,7 +259,7 @@ moe_status ensure_scratch(moe_layer* L, int T, cudaStream_t st) {
                o_hq = take(P * s.I_pad * 2), o_hsc = take(P * (s.I_pad / 32) * 8), o_act1 = take(ES * 4),
                o_act2 = take(ES * 4), o_nact1 = take(4), o_nact2 = take(4),
                o_err = take(4), o_tiles = take(prefill_max_tiles((int)ES, P) * 16), o_ntiles = take(4),
-               o_mtiles = take(ES * 16), o_nmtiles = take(4), o_nmtwide = take(4), o_mtnext = take(16),
+               o_mtiles = take(ES * 16), o_nmtiles = take(4), o_mtnext = take(8),
                o_x16 = take(P * s.H * 2), o_rinv = take(P * 4), o_h16 = take(P * s.I_pad * 2), o_hinv = take(P * 4),
                o_rpart = take(router_part_floats(cap, s.E, s.n_sm) * 4), o_sync = take(kSyncWords * 4);
   if (L->scratch) {
@@ -305,7 +305,6 @@ moe_status ensure_scratch(moe_layer* L, int T, cudaStream_t st) {
   L->wk.n_tiles = reinterpret_cast<int*>(b + o_ntiles);
   L->wk.mtiles = reinterpret_cast<int4*>(b + o_mtiles);
   L->wk.n_mtiles = reinterpret_cast<int*>(b + o_nmtiles);
-  L->wk.n_mt_wide = reinterpret_cast<int*>(b + o_nmtwide);
   L->wk.mt_next = reinterpret_cast<unsigned*>(b + o_mtnext);
   L->wk.x16 = reinterpret_cast<__half*>(b + o_x16);
   L->wk.rinv = reinterpret_cast<float*>(b + o_rinv);
@@ -824,28 +823,13 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     ga.n_slots = (int)L->n_tmap_slots;
     ga.n_rows = P;
     MOE_KERNEL(MOE_K_GATE_UP, launch_prefill_gemm(0, L->x16_map, ga, s.n_sm, st));
-    // the few-row tiles: those of more than 32 rows (listed first) on the
-    // 64-row build, the rest on the 32-row build, each launch claiming its
-    // own units
-    auto few = [&](int mode, GemmArgs g, int kid) -> moe_status {
-      g.tiles = wk.mtiles;
-      if (mt_rows > 32) {
-        GemmArgs gw = g;
-        gw.n_tiles = wk.n_mt_wide;
-        gw.tile_begin = nullptr;
-        gw.next = wk.mt_next + 2 * mode + 1;
-        MOE_KERNEL(kid, launch_prefill_mt(mode, gw, s.n_sm, st, 64));
-        g.tile_begin = wk.n_mt_wide;
-      }
-      g.n_tiles = wk.n_mtiles;
-      g.next = wk.mt_next + 2 * mode;
-      MOE_KERNEL(kid, launch_prefill_mt(mode, g, s.n_sm, st, 32));
-      return MOE_OK;
-    };
-    GemmArgs gm = ga;
+    GemmArgs gm = ga;   // the few-row tiles
+    gm.tiles = wk.mtiles;
+    gm.n_tiles = wk.n_mtiles;
     gm.bsrc = wk.x16;
     gm.b_ld = s.H;
-    if (mt_rows) MOE_TRY(few(0, gm, MOE_K_FEW_GATE_UP));
+    gm.next = wk.mt_next;
+    if (mt_rows) MOE_KERNEL(MOE_K_FEW_GATE_UP, launch_prefill_mt(0, gm, s.n_sm, st, mt_rows));
     if (split_small) MOE_KERNEL(MOE_K_SMALL, launch_gate_up_d1(da, kD1MaxTok, s.n_sm, st));
     MOE_KERNEL(MOE_K_PREP, launch_convert_h(wk, P, s.I, s.I_pad, st));
     ga.ft = s.H / 256;
@@ -863,7 +847,8 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     gm.out_rows = ga.out_rows;
     gm.bsrc = wk.h16;
     gm.b_ld = s.I_pad;
-    if (mt_rows) MOE_TRY(few(1, gm, MOE_K_FEW_DOWN));
+    gm.next = wk.mt_next + 1;
+    if (mt_rows) MOE_KERNEL(MOE_K_FEW_DOWN, launch_prefill_mt(1, gm, s.n_sm, st, mt_rows));
     if (split_small) MOE_KERNEL(MOE_K_SMALL, launch_down_d1(da, kD1MaxTok, s.n_sm, st));
     MOE_KERNEL(MOE_K_COMBINE, launch_combine(wk, T, s, static_cast<__nv_bfloat16*>(out), st, true, partial, L->ep_rank, L->ep_world));
   }

@@ -67,8 +67,7 @@ struct Work {
   int* n_tiles;
   int4* mtiles;       // [E+S] few-row tiles (expert, n0, count <= kMtMaxRows, r0)
   int* n_mtiles;
-  int* n_mt_wide;     // [1] few-row tiles with more than 32 rows (listed first)
-  unsigned* mt_next;  // [4] unit counters of the few-row kernels (gate/up, down) x (<= 32 rows, wider)
+  unsigned* mt_next;  // [2] unit counters of the few-row kernels (gate/up, down)
   __half* x16;        // [P_cap, H] activations of each row, fp16 scaled by 1/rinv, K order (0,2,1,3)
   float* rinv;        // [P]
   __half* h16;        // [P_cap, I_pad] SwiGLU output, fp16 scaled by 1/hinv, same K order
@@ -253,7 +252,6 @@ struct GemmArgs {
   const __half* bsrc;
   int b_ld;
   unsigned* next;
-  const int* tile_begin;     // few-row kernel: first tile of its range (null: 0); the range ends at *n_tiles
   int n_rows;                // activation rows P (debug builds)
 };
 constexpr int kMtMaxRows = 64;   // most activation rows of a few-row tile (builds for 32 and 64)
@@ -270,9 +268,8 @@ cudaError_t launch_quant_x(const __nv_bfloat16* x, const Work& wk, int T, int H,
 cudaError_t launch_gather_rows(const __nv_bfloat16* x, const Work& wk, int P, int kS, int H, cudaStream_t st);
 cudaError_t launch_convert_h(const Work& wk, int P, int I, int I_pad, cudaStream_t st);
 cudaError_t launch_prefill_gemm(int mode, const CUtensorMap& bmap, const GemmArgs& a, int n_sm, cudaStream_t st);
-// The few-row tiles (a.tiles = the mtiles list, tiles [*a.tile_begin,
-// *a.n_tiles)) of mode 0 (gate/up) or 1 (down), same outputs as the GEMM;
-// max_rows 32 or 64 picks the build (4 or 3 stages).
+// The few-row tiles (a.tiles / a.n_tiles = the mtiles list) of mode 0 (gate/up)
+// or 1 (down), same outputs as the GEMM.
 cudaError_t launch_prefill_mt(int mode, const GemmArgs& a, int n_sm, cudaStream_t st, int max_rows);
 size_t route_decode_smem(int H, int T, int E, int k, int S);
 

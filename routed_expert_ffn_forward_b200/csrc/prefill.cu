@@ -592,8 +592,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a)
   ptx::pdl_wait();  // tiles, counters and activation rows of the previous kernels
   ptx::pdl_launch_dependents();
   const int ft = a.ft, nkb = a.nkb;
-  const int t0 = a.tile_begin ? __ldcg(a.tile_begin) : 0;   // this launch's tiles: [t0, *n_tiles)
-  const int n_units = max(0, __ldcg(a.n_tiles) - t0) * ft;
+  const int n_units = __ldcg(a.n_tiles) * ft;
 
   if (warp == kMtWarps) {
     // ------------------------------------------------------------ producer
@@ -608,7 +607,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a)
       if (lane == 0) u = (int)atomicAdd(a.next, 1u);
       u = __shfl_sync(0xffffffffu, u, 0);
       if (u >= n_units) break;
-      const int4 tl = __ldcg(a.tiles + t0 + u / ft);   // (expert, n0, count, r0)
+      const int4 tl = __ldcg(a.tiles + u / ft);   // (expert, n0, count, r0)
       const int f = u % ft;
       const int cnt = min(tl.z, kRows);
       const __half* xr = a.bsrc + (size_t)in_range(tl.w + tl.y, a.n_rows, a.err) * a.b_ld;
@@ -680,7 +679,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) q4k_mt_kernel(const GemmArgs a)
       break;
     }
     if (u < 0) break;
-    const int4 tl = __ldcg(a.tiles + t0 + u / ft);
+    const int4 tl = __ldcg(a.tiles + u / ft);
     const int f = u % ft;
     const int nt = (min(tl.z, kRows) + 7) >> 3;
     // one instantiation per N-tile count: no MMA is issued for an empty N tile
@@ -740,8 +739,7 @@ __global__ void __launch_bounds__(1024) build_tiles_kernel(const int* __restrict
                                                            int* __restrict__ n_tiles, int small_rows,
                                                            int* __restrict__ small, int* __restrict__ n_small,
                                                            int mt_rows, int4* __restrict__ mtiles,
-                                                           int* __restrict__ n_mtiles, int* __restrict__ n_mt_wide,
-                                                           unsigned* __restrict__ mt_next,
+                                                           int* __restrict__ n_mtiles, unsigned* __restrict__ mt_next,
                                                            int ep_rank, int ep_world) {
   constexpr int kNB = kMtMaxRows / 8 + 1;   // N-tile counts 0..8 (0: not a few-row tile)
   __shared__ int s_warp[32];
@@ -779,8 +777,8 @@ __global__ void __launch_bounds__(1024) build_tiles_kernel(const int* __restrict
     *n_tiles = base;
     *n_small = sbase;
     *n_mtiles = run;
-    *n_mt_wide = s_base[kMtMaxRows / 16];   // the tiles of more than 4 N tiles come first
-    for (int i = 0; i < 4; ++i) mt_next[i] = 0u;
+    mt_next[0] = 0u;
+    mt_next[1] = 0u;
   }
   __syncthreads();
   if (mt_rows == 0) return;
@@ -961,7 +959,7 @@ cudaError_t launch_build_tiles(const Work& wk, int small_rows, int mt_rows, cuda
   if (mt_rows < 0 || mt_rows > kMtMaxRows) return cudaErrorInvalidValue;
   return launch_pdl(build_tiles_kernel, dim3(1), dim3(1024), 0, st, (const int*)wk.act, (const int*)wk.n_act,
                     (const int*)wk.counts, (const int*)wk.offsets, wk.tiles, wk.n_tiles, small_rows, wk.act1,
-                    wk.n_act1, mt_rows, wk.mtiles, wk.n_mtiles, wk.n_mt_wide, wk.mt_next, ep_rank, ep_world);
+                    wk.n_act1, mt_rows, wk.mtiles, wk.n_mtiles, wk.mt_next, ep_rank, ep_world);
 }
 
 cudaError_t launch_quant_x(const __nv_bfloat16* x, const Work& wk, int T, int H, cudaStream_t st) {
@@ -983,7 +981,7 @@ cudaError_t launch_convert_h(const Work& wk, int P, int I, int I_pad, cudaStream
 
 cudaError_t launch_prefill_mt(int mode, const GemmArgs& a, int n_sm, cudaStream_t st, int max_rows) {
   static uint64_t attr_done[4] = {0, 0, 0, 0};  // per (mode, build), one bit per device
-  if (max_rows != 32 && max_rows != 64) return cudaErrorInvalidValue;
+  if (max_rows < 1 || max_rows > kMtMaxRows) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
