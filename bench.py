@@ -414,10 +414,12 @@ def measure_resident(args, cfg, rank, world, local_rank, peaks, steps, warmup, e
             "dtype": DTYPE_DECODE if T <= 4 else DTYPE_PREFILL}
 
 
-FEW_ROWS = 32   # the library's default moe_set_few_row_tiles
+def few_rows_default(T: int) -> int:
+    """The library's default moe_set_few_row_tiles for a batch of T tokens."""
+    return 64 if T <= 256 else 32
 
 
-def tile_split(cfg, ids: np.ndarray, few_rows: int = FEW_ROWS):
+def tile_split(cfg, ids: np.ndarray, few_rows: int | None = None):
     """How the prefill path splits this routing (as the library's tile
     builder does): (rows on the tensor-memory GEMM, rows on few-row tiles,
     number of few-row tiles).  An expert with at most few_rows rows is one
@@ -425,10 +427,11 @@ def tile_split(cfg, ids: np.ndarray, few_rows: int = FEW_ROWS):
     last partial tile of at most few_rows rows, which becomes a few-row tile."""
     T = ids.shape[0]
     counts = np.bincount(ids.ravel(), minlength=cfg.n_experts)
-    return split_rows([int(c) for c in counts if c > 0] + [T] * cfg.n_shared, few_rows)
+    few = few_rows_default(T) if few_rows is None else few_rows
+    return split_rows([int(c) for c in counts if c > 0] + [T] * cfg.n_shared, few)
 
 
-def split_rows(rows, few_rows: int = FEW_ROWS):
+def split_rows(rows, few_rows: int = 32):
     """tile_split on a list of rows per active expert."""
     gemm = few = n_few = 0
     for c in rows:

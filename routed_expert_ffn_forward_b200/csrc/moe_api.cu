@@ -82,7 +82,7 @@ size_t g_cache_bytes = SIZE_MAX;
 int g_cache_policy = MOE_CACHE_LRU;
 uint64_t g_hook_wait_ns = 0;  // moe_set_test_hooks
 int g_hook_hold = 0;
-int g_mt_rows = kMtDefaultRows;   // moe_set_few_row_tiles
+int g_mt_rows = -1;   // moe_set_few_row_tiles (-1: default_few_rows(T))
 uint32_t g_next_layer_id = 1;
 
 struct Slot {
@@ -571,7 +571,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     prof = g_profiling;
     hook_wait_ns = g_hook_wait_ns;
     hook_hold = g_hook_hold;
-    mt_rows = g_mt_rows;
+    mt_rows = g_mt_rows < 0 ? default_few_rows(T) : g_mt_rows;
     if (prof)
       for (int i = 0; i < 2 * kProfRanges; ++i) pr.ev[i] = prof_event();
   }
@@ -1131,8 +1131,8 @@ moe_status moe_set_test_hooks(uint64_t wait_limit_ns, int hold_barrier) {
 
 moe_status moe_set_few_row_tiles(int max_rows) {
   g_err.clear();
-  if (max_rows < 0 || max_rows > kMtMaxRows)
-    return fail(MOE_ERR_INVALID_ARG, "max_rows=%d outside 0..%d", max_rows, kMtMaxRows);
+  if (max_rows < -1 || max_rows > kMtMaxRows)
+    return fail(MOE_ERR_INVALID_ARG, "max_rows=%d outside -1..%d", max_rows, kMtMaxRows);
   std::lock_guard<std::mutex> lk(g_mu);
   g_mt_rows = max_rows;
   return MOE_OK;

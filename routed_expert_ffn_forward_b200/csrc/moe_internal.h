@@ -255,7 +255,11 @@ struct GemmArgs {
   int n_rows;                // activation rows P (debug builds)
 };
 constexpr int kMtMaxRows = 64;   // most activation rows of a few-row tile (builds for 32 and 64)
-constexpr int kMtDefaultRows = 32;
+// The default row limit: 64 for batches of at most kMtWideMaxT tokens (their
+// experts have a few to a few dozen rows), 32 above (there the 3-stage build
+// slows the many small tiles more than it gains on the 33-64-row ones).
+constexpr int kMtWideMaxT = 256;
+inline int default_few_rows(int T) { return T <= kMtWideMaxT ? 64 : 32; }
 size_t prefill_gemm_smem();
 size_t prefill_max_tiles(int n_experts_total, size_t pairs);
 // GEMM tiles of up to 256 rows for the experts with more than small_rows rows

@@ -75,10 +75,10 @@ def test_null_arguments(lib):
 
 
 def test_process_wide_settings_validate_on_the_host(lib):
-    for bad in (-1, 65):
+    for bad in (-2, 65):
         assert lib.moe_set_few_row_tiles(bad) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_set_cache_policy(7) == moe.MOE_ERR_INVALID_ARG
-    for ok in (0, 64, 32):
+    for ok in (0, 64, -1):
         assert lib.moe_set_few_row_tiles(ok) == moe.MOE_OK
 
 

@@ -49,12 +49,14 @@ def test_few_row_gate_up_bytes():
     assert np.all(np.sort(ids, axis=1)[:, 1:] != np.sort(ids, axis=1)[:, :-1])  # distinct picks per token
     assert int(np.sum(counts > 0)) == 44 and counts.max() == 64
     tiles, rows = 44 + 1, 64 * 9            # + the shared expert's 64 rows
-    assert bench.tile_split(cfg, ids, few_rows=64) == (0, rows, tiles)
-    # the library's default, 32: expert 0 and the shared expert (64 rows each) take the GEMM
-    assert bench.tile_split(cfg, ids) == (64 + 64, rows - 128, tiles - 2)
-    expect = (tiles - 2) * 2 * gate + (rows - 128) * 7168 * 2 + (rows - 128) * 2048 * 4
+    # the library's default at T = 64 is 64 rows: every tile is a few-row tile
+    assert bench.tile_split(cfg, ids) == bench.tile_split(cfg, ids, few_rows=64) == (0, rows, tiles)
+    # with 32, expert 0 and the shared expert (64 rows each) take the GEMM
+    assert bench.tile_split(cfg, ids, few_rows=32) == (64 + 64, rows - 128, tiles - 2)
+    expect = tiles * 2 * gate + rows * 7168 * 2 + rows * 2048 * 4
     assert bench.few_gate_up_bytes(cfg, ids) == expect
-    assert bench.gate_up_gemm_flops(cfg, ids) == 2.0 * 128 * 2 * 2048 * 7168
+    assert bench.gate_up_gemm_flops(cfg, ids) == 0.0
+    assert bench.few_rows_default(64) == 64 and bench.few_rows_default(4096) == 32
 
 
 def test_prefill_flops():

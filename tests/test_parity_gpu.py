@@ -108,7 +108,7 @@ def test_few_row_tile_thresholds(torch, max_rows):
         moe.moe_set_few_row_tiles(max_rows)
         g = run_gpu(torch, cfg, 200)
     finally:
-        moe.moe_set_few_row_tiles(32)
+        moe.moe_set_few_row_tiles(-1)
     check_against_oracle(cfg, g)
 
 
