@@ -64,18 +64,19 @@ __global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int 
                      ids + (size_t)t * k, w + (size_t)t * k);
 }
 
-// One block per token: four groups of 256 threads each sum a quarter of the
-// K splits (in split order) for every expert, the quarters are added in
-// order and the bias after them (writing the logits to `logits` and shared
-// memory), then warp 0 selects and gates.  Splitting the sum puts four times
-// as many of the partial-logit loads in flight (at T = 64 there are 112
-// splits).
-constexpr int kSumThreads = 1024, kSumGroups = 4, kSumGroup = kSumThreads / kSumGroups;
-template <int PL>
-__global__ void __launch_bounds__(kSumThreads)
+// One block per token: G groups of 128 threads each sum a G-th of the K
+// splits (in split order) for every expert, the parts are added in order and
+// the bias after them (writing the logits to `logits` and shared memory),
+// then warp 0 selects and gates.  With many splits (112 at T = 64) four
+// groups put four times as many partial-logit loads in flight; with few
+// (4 at T = 4096) one group keeps the blocks small.
+constexpr int kSumGroup = 128;
+template <int PL, int G>
+__global__ void __launch_bounds__(kSumGroup * G)
     topk_sum_kernel(float* __restrict__ logits, int E, int k, int gating, const int* __restrict__ forced,
                     int* __restrict__ ids, float* __restrict__ w, const float* __restrict__ part, int nsplit,
                     size_t split_stride, const float* __restrict__ bias) {
+  constexpr int kSumGroups = G, kSumThreads = kSumGroup * G;
   __shared__ float s_l[32 * PL];
   __shared__ float s_q[kSumGroups][32 * PL];
   const int t = blockIdx.x;
@@ -117,12 +118,11 @@ cudaError_t launch_topk(float* logits, int T, int E, int k, int gating, const in
                         const float* bias) {
   const int pl = (E + 31) / 32;
   if (part) {
-    if (pl <= 8)
-      topk_sum_kernel<8><<<T, kSumThreads, 0, st>>>(logits, E, k, gating, forced, ids, w, part, nsplit,
-                                                    split_stride, bias);
-    else
-      topk_sum_kernel<32><<<T, kSumThreads, 0, st>>>(logits, E, k, gating, forced, ids, w, part, nsplit,
-                                                     split_stride, bias);
+    const bool wide = nsplit >= 16;
+    auto kern = pl <= 8 ? (wide ? topk_sum_kernel<8, 4> : topk_sum_kernel<8, 1>)
+                        : (wide ? topk_sum_kernel<32, 4> : topk_sum_kernel<32, 1>);
+    kern<<<T, kSumGroup * (wide ? 4 : 1), 0, st>>>(logits, E, k, gating, forced, ids, w, part, nsplit, split_stride,
+                                                   bias);
     return cudaGetLastError();
   }
   const int warps = 8;
