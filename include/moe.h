@@ -221,6 +221,8 @@ moe_status moe_set_cache_policy(int policy);
  * block, whatever the row count.  Both compute the same fp16 products with
  * fp32 accumulation; the rounding order differs.  0 = off: all tiles on the
  * GEMM and experts with <= 4 rows on the decode kernels.
+ * With T <= max_rows every expert is a single few-row tile and the GEMM
+ * kernels are not launched.
  * Up to 32 rows the kernel keeps 4 stages in flight, above 3.  -1 (the
  * default) = 64 for batches of at most 256 tokens, 32 above (measured: at
  * T = 64, 0.55 ms with 64 against 0.58 with 32; at T = 4096, 5.6 ms with 32

@@ -187,22 +187,27 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
         phase ^= 1u;
       }
     };
+    // the image of pick j's expert (tile-major: 64-row tiles one after another, each
+    // tile its groups one after another, a group 64 rows x its group bytes)
+    auto image_of = [&](int j) {
+      return a.warena + a.wstride * (size_t)in_range(__ldcg(a.slot_of + expert_of(j)), a.n_slots, a.err);
+    };
     // the stages of gate/up unit u: per stage two super-blocks (columns) of the
-    // unit's 64 gate rows and 64 up rows, one box each
+    // unit's 64 gate rows and 64 up rows.  In the tile-major image those are
+    // one contiguous run per matrix, so each is one bulk copy.
     auto issue_gu = [&](int u) -> bool {
       const int jj = u / gu_tiles, rt = u - jj * gu_tiles;
       const int j = jj < S ? k + jj : jj - S;
-      const CUtensorMap* m = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + expert_of(j)), a.n_slots, a.err) + 7;
+      const uint8_t* wg = image_of(j) + (size_t)rt * a.nbh * gu_box;   // tile rt of gate
+      const uint8_t* wu = wg + a.gate_bytes;                            // tile rt of up
       for (int st = 0; st < n_gst; ++st) {
         if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, lim)) return false;
-        const int nbox = min(2, a.nbh - 2 * st);
+        const uint32_t run = (uint32_t)(min(2, a.nbh - 2 * st) * gu_box);
         s_unit[stage] = u;
-        ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * nbox * gu_box));
+        ptx::mbar_arrive_expect_tx(&full[stage], 2u * run);
         uint8_t* dst = ring + stage * stage_bytes;
-        for (int b = 0; b < nbox; ++b) {
-          ptx::tma_load_w(dst + b * gu_box, m, 2 * st + b, rt * kFzGuRows, &full[stage]);
-          ptx::tma_load_w(dst + (2 + b) * gu_box, m + 1, 2 * st + b, rt * kFzGuRows, &full[stage]);
-        }
+        ptx::bulk_load(dst, wg + (size_t)2 * st * gu_box, run, &full[stage]);
+        ptx::bulk_load(dst + 2 * gu_box, wu + (size_t)2 * st * gu_box, run, &full[stage]);
         issued |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (phase << stage);
         next_stage();
@@ -253,18 +258,17 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
       const int jj = u / dn_tiles, rt = u - jj * dn_tiles;
       const int j = jj < S ? k + jj : jj - S;
       if (!ep_owned(expert_of(j), a.ep_rank, a.ep_world)) continue;   // the slot stays free for the next claim
-      const CUtensorMap* md = a.tmaps + kMapsPerSlot * in_range(__ldcg(a.slot_of + expert_of(j)), a.n_slots, a.err) + 6;
+      // tile rt of down: per stage up to kFzDnSb groups, one contiguous run
+      const uint8_t* wd = image_of(j) + 2 * a.gate_bytes + (size_t)rt * a.nbi * dn_box;
       for (int st = 0; st < n_dst; ++st) {
         if (st > 0 && !ptx::mbar_wait(&empty[stage], phase ^ 1u, lim)) {
           ok = false;
           break;
         }
-        const int nbox = min(kFzDnSb, a.nbi - st * kFzDnSb);
+        const uint32_t run = (uint32_t)(min(kFzDnSb, a.nbi - st * kFzDnSb) * dn_box);
         s_unit[stage] = n_gu + u;
-        ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(nbox * dn_box));
-        uint8_t* dst = ring + stage * stage_bytes;
-        for (int b = 0; b < nbox; ++b)
-          ptx::tma_load_w(dst + b * dn_box, md, st * kFzDnSb + b, rt * kFzDnRows, &full[stage]);
+        ptx::mbar_arrive_expect_tx(&full[stage], run);
+        ptx::bulk_load(ring + stage * stage_bytes, wd + (size_t)st * kFzDnSb * dn_box, run, &full[stage]);
         issued |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (phase << stage);
         next_stage();

@@ -198,6 +198,8 @@ struct moe_layer {
   int8_t* d_wexp = nullptr;             // [E+S][2I + H] prefill weight-scale exponents per weight row
   CUtensorMap* d_tmaps = nullptr;       // [slots][kMapsPerSlot] TMA maps (resident: one slot per expert)
   size_t n_tmap_slots = 0;
+  const uint8_t* w_arena = nullptr;     // the images the maps cover: slot i at w_arena + i * w_stride
+  size_t w_stride = 0;
   int* d_slot_of = nullptr;             // [E+S] expert -> slot of d_tmaps
   uint64_t cache_gen = 0;               // streaming: cache arena the maps point into
   cudaStream_t copy = nullptr;          // resident uploads
@@ -488,6 +490,8 @@ moe_status build_maps(moe_layer* L, const uint8_t* arena, size_t stride, size_t 
     L->n_tmap_slots = n_slots;
   }
   CUDA_TRY(cudaMemcpy(L->d_tmaps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice));
+  L->w_arena = arena;
+  L->w_stride = stride;
   return MOE_OK;
 }
 
@@ -649,7 +653,9 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
       MOE_TRY(resolve_experts(L, hid, T * s.k, st, &used));
     }
     FusedArgs fa{};
-    fa.tmaps = L->d_tmaps;
+    fa.warena = L->w_arena;
+    fa.wstride = L->w_stride;
+    fa.gate_bytes = L->gate_bytes;
     fa.slot_of = L->d_slot_of;
     fa.W = L->d_W;
     fa.b = L->d_b;
@@ -799,6 +805,9 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     // kernels instead, which do not dequantise
     const int kS = s.k + s.S, P = T * kS;
     const bool split_small = mt_rows == 0 && down_d1_smem(kD1MaxTok, act_slot) <= kMaxDecodeSmem;
+    // an expert has at most T rows, so with T <= mt_rows every one is a
+    // single few-row tile and the GEMM tile lists are empty: skip the GEMMs
+    const bool gemms = !(mt_rows > 0 && T <= mt_rows);
     MOE_KERNEL(MOE_K_PERMUTE, launch_permute(wk.ids, T, s, wk, st));
     MOE_KERNEL(MOE_K_PERMUTE,
                launch_build_tiles(wk, split_small ? kD1MaxTok : 0, mt_rows, st, L->ep_rank, L->ep_world));
@@ -822,7 +831,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     ga.n_ex = s.E + s.S;
     ga.n_slots = (int)L->n_tmap_slots;
     ga.n_rows = P;
-    MOE_KERNEL(MOE_K_GATE_UP, launch_prefill_gemm(0, L->x16_map, ga, s.n_sm, st));
+    if (gemms) MOE_KERNEL(MOE_K_GATE_UP, launch_prefill_gemm(0, L->x16_map, ga, s.n_sm, st));
     GemmArgs gm = ga;   // the few-row tiles
     gm.tiles = wk.mtiles;
     gm.n_tiles = wk.n_mtiles;
@@ -838,7 +847,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
     ga.out = wk.y;
     ga.out_ld = s.H;
     ga.out_rows = s.H;
-    MOE_KERNEL(MOE_K_DOWN, launch_prefill_gemm(1, L->h16_map, ga, s.n_sm, st));
+    if (gemms) MOE_KERNEL(MOE_K_DOWN, launch_prefill_gemm(1, L->h16_map, ga, s.n_sm, st));
     gm.ft = ga.ft;
     gm.nkb = ga.nkb;
     gm.rinv = ga.rinv;

@@ -106,7 +106,7 @@ cudaError_t launch_stage_in(const void* src, void* dst, size_t bytes, cudaStream
 
 // Arguments of the decode expert kernels.
 struct DecodeArgs {
-  const CUtensorMap* tmaps;  // [slots][kMapsPerSlot] maps of gate, up, down (2-D, 8-byte elements)
+  const CUtensorMap* tmaps;  // [slots][kMapsPerSlot] maps of gate, up, down (4-D, 8-byte elements)
   const int* slot_of;        // [E+S] expert -> slot
   const int* act;            // experts this kernel handles
   const int* n_act;
@@ -143,7 +143,8 @@ size_t gemv_down_smem(size_t act_slot_bytes);
 // T = 1 as one persistent kernel: router, top-k, gate/up + SwiGLU, down and
 // combine (one CTA per SM; steps meet through counters in `sync`).
 struct FusedArgs {
-  const CUtensorMap* tmaps;  // [slots][kMapsPerSlot]
+  const uint8_t* warena;     // expert images (tile-major gate, up, down), slot s at warena + s * wstride
+  size_t wstride, gate_bytes;  // bytes from one slot to the next; of one gate (= up) matrix
   const int* slot_of;        // [E+S] expert -> slot
   const __nv_bfloat16* x;    // [H]
   const float* W;            // router [E, H]
@@ -179,12 +180,12 @@ inline void decode1_ring(int sbb_gu, int sbb_d, int* stages, int* stage_bytes) {
 size_t decode1_fused_smem(int H, size_t act_slot_bytes, int ring_bytes);
 cudaError_t launch_decode1_fused(const FusedArgs& a, int n_sm, cudaStream_t st);
 
-// Tensor maps of one expert's Q4_K matrices at `base`, kMapsPerSlot of them:
-// [0..2] gate, up, down with boxes of 64 rows x 2 (gate/up) or 4 (down)
-// super-blocks (decode kernels); [3..5] gate, up, down with boxes of 128 rows x
-// 1 super-block (single-token GEMVs and prefill GEMMs); [6..8] down, gate, up
-// with boxes of 64 rows x 1 super-block (the fused single-token kernel).
-constexpr int kMapsPerSlot = 9;
+// Tensor maps of one expert's matrices at `base` (tile-major), kMapsPerSlot of
+// them: [0..2] gate, up, down with boxes of 64 rows x 2 (gate/up) or 4 (down)
+// groups (decode kernels); [3..5] gate, up, down with boxes of 128 rows x 1
+// group (single-token GEMVs, prefill GEMMs and the few-row kernel).  The
+// fused single-token kernel reads the images with plain bulk copies.
+constexpr int kMapsPerSlot = 6;
 struct Shape;
 cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, const Shape& s);
 // Weight matrices live in device memory tile-major (tiles of kWTile rows; see

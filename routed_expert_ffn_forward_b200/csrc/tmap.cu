@@ -70,8 +70,6 @@ cudaError_t encode_expert_maps(CUtensorMap* maps, const uint8_t* base, const Sha
   for (int m = 0; m < 3 && e == cudaSuccess; ++m)
     e = encode_q4k(&maps[m], mats[m], rows[m], nb[m], m < 2 ? 2 : 4, kTileRows, sbb[m]);
   for (int m = 0; m < 3 && e == cudaSuccess; ++m) e = encode_q4k(&maps[3 + m], mats[m], rows[m], nb[m], 1, 128, sbb[m]);
-  if (e == cudaSuccess) e = encode_q4k(&maps[6], mats[2], rows[2], nb[2], 1, 64, sbb[2]);
-  for (int m = 0; m < 2 && e == cudaSuccess; ++m) e = encode_q4k(&maps[7 + m], mats[m], rows[m], nb[m], 1, 64, sbb[m]);
   return e;
 }
 
