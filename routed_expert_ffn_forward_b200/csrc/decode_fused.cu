@@ -430,12 +430,15 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
   bool routed = false;
   auto route = [&]() {
     bool got = false;
+    // warps 0-1 may still be reading the last unit's partials in s_part,
+    // which warp 0 is about to reuse for the logits
+    cbar();
     if (warp == 0) {
       // every logit of this launch, polled until all carry its tag (+ hold,
       // a test hook that makes the wait run out), copied to shared memory
       const uint32_t want = (uint32_t)(s_epoch + 1u + (uint64_t)a.hold);
       const uint64_t* lg = reinterpret_cast<const uint64_t*>(sync + kSyncLogits);
-      float* s_lg = s_part;   // free: no unit is in progress
+      float* s_lg = s_part;   // free: every consumer warp has passed the barrier above
       const uint64_t t0 = ptx::globaltimer();
       while (true) {
         bool mine = true;
@@ -538,19 +541,25 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
           next_stage();
         }
         if (!ok) fail(kErrFzConsumer);
-        cbar();
+        // the unit's partial sums go to the buffer the unit before last used
+        // (double-buffered like the down units'), so the two warps that run
+        // the SwiGLU may lag the others by a unit
+        float* sp = s_part + buf * (kFzWarps * kFzDnRows);
+        sp[(g_sb * 4 + g_c) * kFzGuRows + g_row] = acc[0];
+        sp[(8 + g_sb * 4 + g_c) * kFzGuRows + g_row] = acc[1];
+        cbar();                          // every warp, every unit: the partials are complete
         if (s_flag[0]) return;
-        s_part[(g_sb * 4 + g_c) * kFzGuRows + g_row] = acc[0];
-        s_part[(8 + g_sb * 4 + g_c) * kFzGuRows + g_row] = acc[1];
-        cbar();
-        // SwiGLU (the 8 parts of each row summed in a fixed order) -> h_j, warps 0-1
+        // SwiGLU (the 8 parts of each row summed in a fixed order) -> h_j,
+        // warps 0-1; then one thread publishes the features (release,
+        // cumulative over the two warps' stores; the ready counters are
+        // zeroed before the routing)
         if (warp < 2) {
           const int f = warp * 32 + lane;
-          float g = s_part[f], up = s_part[8 * kFzGuRows + f];
+          float g = sp[f], up = sp[8 * kFzGuRows + f];
 #pragma unroll
           for (int p = 1; p < 8; ++p) {
-            g += s_part[p * kFzGuRows + f];
-            up += s_part[(8 + p) * kFzGuRows + f];
+            g += sp[p * kFzGuRows + f];
+            up += sp[(8 + p) * kFzGuRows + f];
           }
           float2 rsc;
           int8_t hh;
@@ -561,13 +570,13 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode1_fused_kernel(const Fuse
           a.hq[o] = hh;
           reinterpret_cast<uint8_t*>(a.hq + a.hq_plane)[o] = hl;
           if (lane == 0) a.hsc[(size_t)j * (I_pad / 32) + feat / 32] = rsc;
+          ptx::named_barrier_sync(2, 64);
+          if (tid == 0) {
+            ptx::fence_proxy_async_global();
+            ptx::red_add_release_gpu(sync + kSyncReady + 64 * (int)(s_epoch & 1u) + j, 1u);
+          }
         }
-        cbar();
-        // publish the features (the ready counters are zeroed before the barrier)
-        if (tid == 0) {
-          ptx::fence_proxy_async_global();
-          ptx::red_add_release_gpu(sync + kSyncReady + 64 * (int)(s_epoch & 1u) + j, 1u);
-        }
+        buf ^= 1;
         continue;
       }
       // ---- down unit: 64 output rows of pick j.  Its 64 rows of y_j are
