@@ -746,6 +746,7 @@ __global__ void __launch_bounds__(1024) build_tiles_kernel(const int* __restrict
   __shared__ int s_bw[kNB][32];             // per count, per warp: tiles, then their first position
   __shared__ int s_base[kNB];               // per count: first position in the list (all chunks)
   ptx::pdl_wait();
+  ptx::pdl_launch_dependents();   // the next kernel waits for this one's end before reading
   const int na = __ldcg(n_act);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
@@ -867,6 +868,7 @@ __global__ void __launch_bounds__(kRowThreads) gather_rows_kernel(const __nv_bfl
                                                                   float* __restrict__ rinv) {
   __shared__ float s_red[kRowThreads / 32];
   ptx::pdl_wait();
+  ptx::pdl_launch_dependents();
   const int r = blockIdx.x;
   const uint2* src = reinterpret_cast<const uint2*>(x + (size_t)(__ldg(perm + r) / kS) * H);
   uint2 v[kRowMaxVec];
@@ -913,12 +915,14 @@ __global__ void __launch_bounds__(kConvWarps * 32) convert_h_kernel(const float*
                                                                     int P, __half* __restrict__ h16,
                                                                     float* __restrict__ hinv) {
   ptx::pdl_wait();
+  ptx::pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int r = blockIdx.x * kConvWarps + (threadIdx.x >> 5);
   if (r >= P) return;
   const float4* src = reinterpret_cast<const float4*>(h + (size_t)r * I_pad);
   const int nv = I_pad / 4;
   float m = 0.f;
+#pragma unroll 4
   for (int c = lane; c < nv; c += 32) {
     const float4 f = h_quad(src, c, I);
     m = fmaxf(m, fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w))));
@@ -928,6 +932,7 @@ __global__ void __launch_bounds__(kConvWarps * 32) convert_h_kernel(const float*
   float inv;
   const float sc = row_scale(m, &inv);
   uint2* dst = reinterpret_cast<uint2*>(h16 + (size_t)r * I_pad);
+#pragma unroll 4
   for (int c = lane; c < nv; c += 32) {
     const float4 f = h_quad(src, c, I);
     dst[c] = pack4_swz(f.x * sc, f.y * sc, f.z * sc, f.w * sc);
