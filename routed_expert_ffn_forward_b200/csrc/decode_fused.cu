@@ -53,7 +53,7 @@ constexpr int kFzConsumers = kFzWarps * 32;
 constexpr int kFzGuRows = 64;                      // gate/up unit: weight rows of gate and of up
 constexpr int kFzDnRows = 64;                      // down unit: output rows
 constexpr int kFzDnSb = 4;                         // 256-weight groups per down stage
-constexpr int kFzStages = 4;                       // at most; a stage is 256 x the group size (Q4_K: 36,864 B)
+constexpr int kFzStages = kFusedMaxStages;         // at most; a stage is 256 x the group size (Q4_K: 36,864 B)
 constexpr uint64_t kFzLimitNs = 2000000000ull;
 
 // error bits (moe_check): which wait gave up
@@ -77,11 +77,11 @@ struct FzLayout {
   uint32_t bars, unit, ids, w, flags, part, xh, xl, xsc, uni, total;
   __host__ __device__ FzLayout(int H, size_t act_slot, int ring_bytes) {
     auto up16 = [](uint32_t v) { return (v + 15u) & ~15u; };
-    bars = (uint32_t)ring_bytes;                      // full[4] empty[4] afull[2] aempty[2] route[1]
-    unit = bars + 13 * 8;                             // int [kFzStages]
-    ids = unit + kFzStages * 4;                       // int [40]
+    bars = (uint32_t)ring_bytes;                      // full[S] empty[S] afull[2] aempty[2] route[1]
+    unit = bars + (2 * kFzStages + 5) * 8;            // int [kFzStages]
+    ids = up16(unit + kFzStages * 4);                 // int [40]
     w = ids + 40 * 4;                                 // float [40]
-    flags = w + 40 * 4;                               // int [4], then u64 barrier target
+    flags = up16(w + 40 * 4);                         // int [4], then the u64 launch index (8-byte aligned)
     part = up16(flags + 24);                          // float [2][1024]
     xh = part + 2048 * 4;                             // u8 [H]
     xl = xh + (uint32_t)H;                            // u8 [H]

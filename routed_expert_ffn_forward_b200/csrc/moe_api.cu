@@ -606,7 +606,7 @@ moe_status forward_impl(moe_layer* L, const void* x, void* out, int T, const int
   // Layers with other block types than Q4_K run every token this way.
   const size_t act1 = 2 * (size_t)s.I_pad + (size_t)(s.I_pad / 32) * 8;
   int ring_stages = 0, ring_stage_bytes = 0;
-  decode1_ring(s.sbb_gu, s.sbb_d, &ring_stages, &ring_stage_bytes);
+  decode1_ring(s.sbb_gu, s.sbb_d, s.H, act1, &ring_stages, &ring_stage_bytes);
   const bool fused_ok = s.k + s.S <= 40 && s.H % 64 == 0 &&
                         decode1_fused_smem(s.H, act1, ring_stages * ring_stage_bytes) <= kMaxDecodeSmem;
   const bool q4k = s.qgu == kQ4_K && s.qd == kQ4_K;

@@ -172,12 +172,17 @@ struct FusedArgs {
   int ep_rank, ep_world;     // expert parallelism: work only for owned experts
   float* partial;            // non-null: write the owned experts' unrounded sum here instead of out
 };
-// Weight-ring geometry of the single-token kernel for these group sizes.
-inline void decode1_ring(int sbb_gu, int sbb_d, int* stages, int* stage_bytes) {
-  *stage_bytes = 256 * std::max(sbb_gu, sbb_d);
-  *stages = std::min(4, 147456 / *stage_bytes);
-}
 size_t decode1_fused_smem(int H, size_t act_slot_bytes, int ring_bytes);
+constexpr int kFusedMaxStages = 5;
+// Weight-ring geometry of the single-token kernel for these group sizes: as
+// many stages (2 .. kFusedMaxStages, at most 180 KB) as fit in shared memory
+// beside the kernel's other arrays for this H and activation slot size.
+inline void decode1_ring(int sbb_gu, int sbb_d, int H, size_t act_slot_bytes, int* stages, int* stage_bytes) {
+  *stage_bytes = 256 * std::max(sbb_gu, sbb_d);
+  int n = std::max(2, std::min(kFusedMaxStages, 184320 / *stage_bytes));
+  while (n > 2 && decode1_fused_smem(H, act_slot_bytes, n * *stage_bytes) > kMaxDecodeSmem) --n;
+  *stages = n;
+}
 cudaError_t launch_decode1_fused(const FusedArgs& a, int n_sm, cudaStream_t st);
 
 // Tensor maps of one expert's matrices at `base` (tile-major), kMapsPerSlot of
